@@ -1,0 +1,438 @@
+#!/usr/bin/env python
+"""Benchmark: paged GQA decode on B200 -- effective KV-read HBM GB/s and decode steps/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload llama]
+                    [--partition P] [--impl reference]
+
+One step = the whole decode hot path for one layer over one batch: slot
+computation and cache write of every sequence's new token, split-K paged
+decode attention, log-sum-exp merge.  The default workload is the
+Llama-3-8B-shaped batch (32 sequences x 4096 tokens, 32 query / 8 KV heads,
+head_dim 128, bf16, 16-token blocks in a randomly permuted 8192-block pool).
+
+value    = KV bytes read per step x steps / device time, inputs resident in HBM;
+e2e      = the same metric through the binding with pinned host buffers: each
+           step copies q, the new K/V rows, the block table and context lengths
+           host->device and the output device->host inside the timed region;
+roofline = the decode call (split + merge kernels) timed live with CUDA events
+           on its stream, against the measured HBM copy bandwidth;
+cpu_baseline = the double-precision CPU oracle on a bounded sample (rank 0).
+``--impl reference`` times that oracle alone as the reference arm.
+With N > 1 (torchrun), every rank runs an independent replica on its own GPU
+(the workload needs no exchange); value is the sum over ranks / the slowest rank.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workloads import WORKLOADS, make_inputs, storage_view  # noqa: E402
+
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama_b32x4k.md")
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_401_b200", "csrc", "decode.cu")
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    return (int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)),
+            int(os.environ.get("WORLD_SIZE", 1)))
+
+
+def dist_init(world: int, backend: str, device=None):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        kw = {"backend": backend, "timeout": datetime.timedelta(seconds=120)}
+        if device is not None and backend == "nccl":
+            kw["device_id"] = device
+        dist.init_process_group(**kw)
+
+
+def reduce_over_ranks(x: float, op: str, device=None) -> float:
+    """max/sum of a scalar over ranks (identity when not distributed)."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None:
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+def gpu_id(device) -> str:
+    """nvidia-smi id of a torch device (its UUID, robust to CUDA_VISIBLE_DEVICES)."""
+    uuid = getattr(torch.cuda.get_device_properties(device), "uuid", None)
+    if uuid is not None:
+        u = str(uuid)
+        return u if u.startswith("GPU-") else "GPU-" + u
+    return str(device.index)
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None or not os.path.exists(self.path):
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i in range(4)
+                          if r[i + 1].lower() == "active"})
+        return {"sm_mhz": float(np.median([r[0] for r in rows])),
+                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- workload bytes
+def kv_bytes_per_step(inp) -> int:
+    """Algorithmic KV bytes one decode step reads: every context token's K and V
+    row of every KV head (plus the fp32 per-row scales of an FP8 cache)."""
+    spec = inp.spec
+    tokens = int(inp.context_lens.astype(np.int64).sum())
+    elem = {"f32": 4, "bf16": 2, "fp8": 1}[spec.kv_dtype]
+    per_row = spec.head_dim * elem + (4 if spec.kv_dtype == "fp8" else 0)
+    return tokens * spec.num_kv_heads * 2 * per_row
+
+
+def describe(inp, partition: int) -> dict:
+    spec = inp.spec
+    return {"workload": f"{spec.name}: paged GQA decode, batch {inp.q.shape[0]}, "
+                        f"{spec.num_q_heads} q / {spec.num_kv_heads} kv heads, head_dim "
+                        f"{spec.head_dim}, {spec.kv_dtype} KV, block 16, "
+                        f"context {int(inp.context_lens.min())}..{int(inp.context_lens.max())}",
+            "batch": int(inp.q.shape[0]), "max_context_len": inp.max_context_len,
+            "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads,
+            "head_dim": spec.head_dim, "block_size": 16, "num_blocks": inp.num_blocks,
+            "kv_dtype": spec.kv_dtype, "partition_tokens": partition,
+            "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush"
+            if kv_bytes_per_step(inp) > 126e6 else "inputs fit in L2, not flushed",
+            "parallelism": "replicas: one independent decode per GPU"}
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def profiled_traffic():
+    """ncu DRAM bytes per decode call, if the committed summary was taken on the
+    current decode kernel source (else None: the kernel changed since)."""
+    if not os.path.exists(PROFILE_SUMMARY):
+        return None
+    kv = {}
+    for line in open(PROFILE_SUMMARY, encoding="utf-8"):
+        if ":" in line and line.lstrip().startswith("- "):
+            k, _, v = line.strip()[2:].partition(":")
+            kv[k.strip()] = v.strip().strip("`")
+    sha = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
+    if kv.get("decode_source_sha256") != sha:
+        return None
+    try:
+        return int(kv["dram_bytes_per_decode_call"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ---------------------------------------------------------------- oracle (CPU) timing
+def time_oracle(inp, max_seqs: int, repeats: int = 1):
+    """Time the CPU oracle on the first `max_seqs` sequences; returns (GB/s, s, desc, cores)."""
+    import oracle
+    spec = inp.spec
+    n = min(max_seqs, inp.q.shape[0])
+    seqs = np.arange(n)
+    q = storage_view(inp.q)[seqs]
+    lens = inp.context_lens[seqs]
+    args = dict(seq_offsets=inp.seq_offsets[seqs], lens=lens, scale=spec.scale,
+                num_kv_heads=spec.num_kv_heads, q_dtype=spec.q_dtype)
+    if spec.kv_dtype == "fp8":
+        rows = slice(int(inp.seq_offsets[0]), int(inp.seq_offsets[n - 1] + lens[-1]))
+        kc, ks = oracle.quantize_rows(inp.k[rows].float().numpy())
+        vc, vs = oracle.quantize_rows(inp.v[rows].float().numpy())
+        kv = dict(k=kc, v=vc, kv_dtype="fp8", k_scale=ks, v_scale=vs)
+    else:
+        kv = dict(k=storage_view(inp.k), v=storage_view(inp.v), kv_dtype=spec.kv_dtype)
+    t0 = time.perf_counter()
+    for _ in range(repeats):
+        oracle.decode_attention(q, **kv, **args)
+    dt = (time.perf_counter() - t0) / repeats
+    elem = {"f32": 4, "bf16": 2, "fp8": 1}[spec.kv_dtype]
+    per_row = spec.head_dim * elem + (4 if spec.kv_dtype == "fp8" else 0)
+    nbytes = int(lens.astype(np.int64).sum()) * spec.num_kv_heads * 2 * per_row
+    desc = (f"oracle (C, double, OpenMP) over {n} of {inp.q.shape[0]} sequences "
+            f"({int(lens.sum())} tokens, {nbytes / 2**20:.0f} MiB of KV) x {repeats}")
+    return nbytes / dt / 1e9, dt, desc, oracle.num_threads()
+
+
+def run_reference(args, inp):
+    rank, _, _ = dist_env()
+    if rank != 0:
+        return
+    # calibrate: one sequence, then as many as fit ~90 s for the whole run
+    _, t1, _, _ = time_oracle(inp, 1)
+    budget = 90.0 / (args.steps + args.warmup)
+    sample = int(max(1, min(inp.q.shape[0], budget // max(t1, 1e-6))))
+    for _ in range(args.warmup):
+        time_oracle(inp, sample)
+    vals = []
+    for _ in range(args.steps):
+        v, dt, desc, cores = time_oracle(inp, sample)
+        vals.append((v, dt))
+    gbs = float(np.mean([v for v, _ in vals]))
+    ms = float(np.mean([dt for _, dt in vals])) * 1e3
+    line = {"metric": "paged GQA decode: effective KV-read HBM GB/s (% of peak), decode steps/s",
+            "value": round(gbs, 3), "unit": "GB/s", "impl": "reference",
+            "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": describe(inp, 0),
+            "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": cores,
+                             "kind": "oracle", "sample": desc},
+            "e2e": {"value": round(gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- GPU arm
+def stage_on_device(inp, device):
+    """Fill the paged pool with every sequence's history through the library."""
+    from paged_kv_cache_401_b200.cache import PagedKVCache
+    spec = inp.spec
+    cache = PagedKVCache(inp.num_blocks, spec.num_kv_heads, spec.head_dim, spec.kv_dtype,
+                         device)
+    bt = torch.from_numpy(inp.block_table).to(device)
+    chunk = 1 << 17
+    for c0 in range(0, len(inp.fill_rows), chunk):
+        c1 = min(len(inp.fill_rows), c0 + chunk)
+        rows = torch.from_numpy(inp.fill_rows[c0:c1])
+        cache.append(bt, torch.from_numpy(inp.fill_seq_ids[c0:c1]).to(device),
+                     torch.from_numpy(inp.fill_positions[c0:c1]).to(device),
+                     inp.k[rows].to(device), inp.v[rows].to(device))
+    torch.cuda.synchronize(device)
+    return cache, bt
+
+
+def run_gpu(args, inp):
+    import paged_kv_cache_401_b200 as pk
+    rank, local, world = dist_env()
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    dist_init(world, "nccl", device)
+    spec = inp.spec
+    B = inp.q.shape[0]
+    cache, bt = stage_on_device(inp, device)
+    lens = torch.from_numpy(inp.context_lens).to(device)
+    q = inp.q.to(device)
+    app = torch.from_numpy(inp.append_rows)
+    k_new, v_new = inp.k[app].to(device), inp.v[app].to(device)
+    seq_ids = torch.arange(B, dtype=torch.int32, device=device)
+    positions = torch.from_numpy(inp.append_positions).to(device)
+    slots = torch.empty(B, dtype=torch.int64, device=device)
+    out = torch.empty_like(q)
+    P = args.partition or pk.paged_decode_default_partition(cache.desc, B, spec.num_q_heads,
+                                                            inp.max_context_len)
+    ws = cache.alloc_workspace(B, spec.num_q_heads, inp.max_context_len, P)
+    stream = torch.cuda.current_stream(device)
+    max_parts = -(-inp.max_context_len // P)
+    launches_per_step = 3 + (1 if max_parts > 1 else 0)
+
+    def append():
+        cache.append(bt, seq_ids, positions, k_new, v_new, slots=slots)
+
+    def decode():
+        cache.decode(q, bt, lens, inp.max_context_len, spec.scale, out=out,
+                     partition_tokens=P, workspace=ws)
+
+    for _ in range(args.warmup):
+        append()
+        decode()
+    torch.cuda.synchronize(device)
+    err0 = cache.errors()
+
+    # ---- timed region: K steps, decode calls bracketed by events ----
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(gpu_id(device)) as clk:
+        barrier(device)
+        torch.cuda.synchronize(device)
+        time.sleep(0.25)  # let the clock sampler see the loaded region start
+        start.record(stream)
+        for i in range(args.steps):
+            append()
+            ev[i][0].record(stream)
+            decode()
+            ev[i][1].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+    elapsed_ms = start.elapsed_time(end)
+    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    errs = cache.errors()
+
+    # ---- e2e: host buffers, copies inside the timed region ----
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    h_q, h_k, h_v = pin(inp.q), pin(inp.k[app]), pin(inp.v[app])
+    h_bt, h_lens = pin(torch.from_numpy(inp.block_table)), pin(torch.from_numpy(inp.context_lens))
+    h_out = torch.empty_like(h_q).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_bt, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        k_new.copy_(h_k, non_blocking=True)
+        v_new.copy_(h_v, non_blocking=True)
+        bt.copy_(h_bt, non_blocking=True)
+        lens.copy_(h_lens, non_blocking=True)
+        append()
+        decode()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = e0.elapsed_time(e1)
+    barrier(device)
+
+    nbytes = kv_bytes_per_step(inp)
+    max_ms = reduce_over_ranks(elapsed_ms, "max", device)
+    max_e2e_ms = reduce_over_ranks(e2e_ms, "max", device)
+    max_decode_ms = reduce_over_ranks(decode_ms, "max", device)
+    total_bytes = reduce_over_ranks(nbytes * args.steps, "sum", device)
+    value = total_bytes / (max_ms * 1e-3) / 1e9
+    e2e_value = total_bytes / (max_e2e_ms * 1e-3) / 1e9
+    clocks = clk.summary()
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        _, t1, _, _ = time_oracle(inp, 1)      # calibrate to ~10 s of CPU work
+        reps = int(max(1, min(5, 10.0 // max(t1 * args.reference_seqs, 1e-6))))
+        gbs, dt, desc, cores = time_oracle(inp, args.reference_seqs, reps)
+        cpu = {"value": round(gbs, 3), "unit": "GB/s", "cores": cores, "kind": "oracle",
+               "sample": desc}
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peak()
+    achieved = nbytes / (max_decode_ms * 1e-3) / 1e9
+    line = {
+        "metric": "paged GQA decode: effective KV-read HBM GB/s (% of peak), decode steps/s",
+        "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(max_ms / args.steps, 5),
+        "steps_per_s": round(args.steps / (max_ms * 1e-3), 1),
+        "pct_of_peak": round(100 * value / world / peak, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": spec.kv_dtype if spec.kv_dtype != "fp8" else "fp8_e4m3",
+        "data": "synthetic (seeded N(0,1) q/K/V, random block permutation)",
+        "config": describe(inp, P),
+        "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h,
+                "ms_per_step": round(max_e2e_ms / args.steps, 5)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                     "unit": "GB/s", "frac": round(achieved / peak, 4),
+                     "traffic": profiled_traffic(), "kernel": "paged_decode_attention "
+                     "(split + merge kernels, one call)", "peak_kind": peak_kind,
+                     "algorithmic_bytes_per_launch": nbytes,
+                     "ms_per_launch": round(max_decode_ms, 5)},
+        "cpu_baseline": cpu,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks,
+        "device_errors": {"warmup": err0, "timed": errs},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="llama", choices=sorted(WORKLOADS))
+    ap.add_argument("--partition", type=int, default=0, help="split-K partition (0 = library)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--reference-seqs", type=int, default=8,
+                    help="sequences in the oracle's bounded sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, reported as run
+    inp = make_inputs(args.workload)
+    if args.impl == "reference":
+        run_reference(args, inp)
+    else:
+        run_gpu(args, inp)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * paged_kv.h -- C ABI of libpagedkv.so: single-token GQA decode attention
+ * over a PagedAttention KV cache, for NVIDIA B200 (sm_100a).
+ *
+ * The method (the four web pages on KV caching it follows):
+ *  - "KV Cache 深度解析：显存黑洞、PagedAttention 与三路省内存方案" (d7kj.com):
+ *    §一 decode attends the new token's q to every cached K/V with
+ *    softmax(q·Kᵀ/√d)·V; §三 the cache is cut into fixed 16-token blocks and
+ *    a block table maps each sequence's logical blocks to physical blocks
+ *    scattered in a pool ("逻辑连续、物理离散"), several sequences may share a
+ *    physical block; §四 GQA (query heads share KV heads) and fp8 E4M3 KV
+ *    with per-token scales.
+ *  - "llm-inference-optimization" notes (qingdujian.com): §二 the paged
+ *    cache's append (new block when the last one is full, write at the next
+ *    offset); §三 the tiled online-softmax update (running max, running sum,
+ *    rescaled running output).
+ *  - k1-blog daily note 2026-07-13, "PagedAttention 與 vLLM": the attention
+ *    kernel must be rewritten to read non-contiguous memory.
+ *
+ * Conventions for every entry point:
+ *  - Every device buffer is owned by the caller.  The library allocates no
+ *    device memory, keeps no state between calls and never synchronises:
+ *    work is enqueued on the caller's stream (NULL = legacy default stream).
+ *  - Device pointers must be 16-byte aligned; contiguous row-major layouts.
+ *  - Argument errors found on the host return KV_ERR_INVALID_ARGUMENT or
+ *    KV_ERR_UNSUPPORTED before anything is enqueued; a failed launch returns
+ *    KV_ERR_CUDA.  Nothing throws, nothing aborts the process.
+ *  - Data errors found on the device (a slot or block id out of range, a bad
+ *    context length, a bounded wait that ran out) never trap: the kernel skips
+ *    the offending work and ORs a KV_DEVERR_* bit into *dev_error when
+ *    dev_error is non-NULL (an int32 in device memory the caller zeroes).
+ */
+#ifndef PAGED_KV_H
+#define PAGED_KV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define KV_API __attribute__((visibility("default")))
+#else
+#define KV_API
+#endif
+
+/* The CUDA stream type (identical to cudaStream_t / CUstream). */
+struct CUstream_st;
+typedef struct CUstream_st* kv_stream_t;
+
+typedef enum {
+    KV_OK = 0,
+    KV_ERR_INVALID_ARGUMENT = 1,
+    KV_ERR_UNSUPPORTED = 2,
+    KV_ERR_CUDA = 3
+} kv_status;
+
+typedef enum {
+    KV_F32 = 0,        /* IEEE binary32 */
+    KV_BF16 = 1,       /* bfloat16 */
+    KV_FP8_E4M3 = 2    /* OCP FP8 E4M3 codes (KV pools only) with fp32 row scales */
+} kv_dtype;
+
+/* Bits ORed into *dev_error by the kernels. */
+#define KV_DEVERR_BAD_SLOT        0x1  /* slot >= num_blocks * block_size: write skipped */
+#define KV_DEVERR_BAD_CONTEXT_LEN 0x2  /* context_lens[b] < 1 or > max_context_len: out[b] = 0 */
+#define KV_DEVERR_BAD_BLOCK_ID    0x4  /* block id outside [0, num_blocks): block skipped */
+#define KV_DEVERR_TIMEOUT         0x8  /* a bounded wait on staged data ran out: output invalid */
+#define KV_DEVERR_BAD_POSITION    0x10 /* slot mapping: position outside the block table */
+
+/*
+ * Geometry of one layer's K pool and V pool (plain data, owns nothing).
+ *
+ * Layout of each pool, row-major: [num_blocks][num_kv_heads][block_size][head_dim]
+ * so the 16 tokens of one (physical block, kv head) pair are one contiguous
+ * span of block_size*head_dim elements.  FP8 pools have a matching fp32 scale
+ * pool per K and V laid out [num_blocks][num_kv_heads][block_size].
+ */
+typedef struct {
+    int32_t num_blocks;
+    int32_t block_size;      /* tokens per block; 16 */
+    int32_t num_kv_heads;
+    int32_t head_dim;        /* 64 or 128 */
+    int32_t dtype;           /* kv_dtype */
+    int32_t elem_bytes;      /* 4, 2 or 1 */
+    uint64_t kv_bytes;       /* bytes of ONE pool (K or V) */
+    uint64_t scale_bytes;    /* bytes of ONE scale pool (FP8 only, else 0) */
+    int64_t stride_block;    /* elements between consecutive physical blocks */
+    int64_t stride_head;     /* elements between consecutive kv heads of a block */
+    int64_t stride_slot;     /* elements between consecutive tokens of a block */
+} kv_pool_desc;
+
+/*
+ * Fill *out with the geometry of a pool (host only, no device work).
+ * Errors: KV_ERR_INVALID_ARGUMENT for out == NULL or non-positive sizes;
+ * KV_ERR_UNSUPPORTED for block_size != 16, head_dim not in {64, 128},
+ * num_kv_heads > 256 or an unknown dtype.
+ */
+KV_API kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                         int32_t head_dim, kv_dtype dtype, kv_pool_desc* out);
+
+/*
+ * Slot of each token to append ("KV Cache 深度解析" §三; "llm-inference-
+ * optimization" notes §二): token i is position positions[i] of sequence
+ * seq_ids[i]; its slot is
+ *     block_table[seq][pos / block_size] * block_size + pos % block_size.
+ *   block_table  : device int32 [batch][max_blocks_per_seq]
+ *   seq_ids      : device int32 [num_tokens], each in [0, batch)
+ *   positions    : device int32 [num_tokens]
+ *   slot_mapping : device int64 [num_tokens] (written)
+ * A position outside [0, max_blocks_per_seq*block_size) or a seq id outside
+ * [0, batch) gives slot -1 (padding, skipped by reshape_and_cache) and
+ * KV_DEVERR_BAD_POSITION.  num_tokens == 0 enqueues nothing.
+ */
+KV_API kv_status compute_slot_mapping(const int32_t* block_table, int32_t batch,
+                               int32_t max_blocks_per_seq, int32_t block_size,
+                               const int32_t* seq_ids, const int32_t* positions,
+                               int32_t num_tokens, int64_t* slot_mapping,
+                               int32_t* dev_error, kv_stream_t stream);
+
+/*
+ * Cache write ("KV Cache 深度解析" §一: decode computes only the new token's
+ * K/V and appends it to the cache).  For token t and kv head h with
+ * s = slot_mapping[t] >= 0:
+ *     pool[s / 16][h][s % 16][:] = row(t, h)
+ *   k_new, v_new : device [num_tokens][num_kv_heads][head_dim] in src_dtype
+ *   slot_mapping : device int64 [num_tokens]; s < 0 is padding (skipped);
+ *                  s >= num_blocks*16 is skipped with KV_DEVERR_BAD_SLOT
+ * F32 / BF16 pools: src_dtype must equal the pool dtype; the copy is exact.
+ * FP8 pools ("KV Cache 深度解析" §四): src_dtype F32 or BF16; for each row
+ *     a = max |x| (fp32),  scale = a / 448 (IEEE fp32 division),
+ *     code = E4M3(x / scale) (IEEE division, round to nearest even,
+ *            saturating to ±448),  and scale = 0, codes 0x00 when a == 0;
+ *   k_scales, v_scales : device fp32 scale pools [num_blocks][num_kv_heads][16]
+ *   (must be NULL for non-FP8 pools).  Rows must be finite.
+ * Two tokens given the same slot race (last writer unspecified).
+ */
+KV_API kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool,
+                            float* k_scales, float* v_scales,
+                            const void* k_new, const void* v_new, kv_dtype src_dtype,
+                            const int64_t* slot_mapping, int32_t num_tokens,
+                            int32_t* dev_error, kv_stream_t stream);
+
+/*
+ * Sequence-partition (split-K) size the library uses when
+ * paged_decode_attention is given partition_tokens == 0: a multiple of 16
+ * chosen from the batch, the longest context and the SM count of the current
+ * device (148 when no device can be queried).  Host only.
+ */
+KV_API int32_t paged_decode_default_partition(const kv_pool_desc* pool, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_context_len);
+
+/*
+ * Bytes of device workspace paged_decode_attention needs for these sizes
+ * (partial maxima, sums and outputs of every sequence partition).  Host only;
+ * partition_tokens as for paged_decode_attention.  0 means none is needed.
+ */
+KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
+                                    int32_t num_q_heads, int32_t max_context_len,
+                                    int32_t partition_tokens);
+
+/*
+ * Single-token GQA decode attention over the paged cache ("KV Cache 深度解析"
+ * §一, §三, §四; "llm-inference-optimization" notes §三).  For sequence b,
+ * query head h, kv head g = h / (num_q_heads / num_kv_heads) and the
+ * L = context_lens[b] tokens of logical positions 0..L-1 (token p stored in
+ * physical block block_table[b][p / 16], slot p % 16):
+ *     s_p = scale * q[b,h,:] . K_p[g,:]
+ *     out[b,h,:] = sum_p softmax(s)_p * V_p[g,:]
+ * computed exactly up to fp32 rounding with an online softmax; the sequence
+ * is cut into partitions of partition_tokens tokens (0 = library default),
+ * each partition's (max, sum, output) is merged by log-sum-exp.
+ *   out          : device [batch][num_q_heads][head_dim] in q_dtype
+ *   q            : device [batch][num_q_heads][head_dim], q_dtype F32 or BF16
+ *   k_pool/v_pool: device pools (layout above)
+ *   k_scales/v_scales : device fp32 scale pools, non-NULL iff the pool is FP8
+ *   block_table  : device int32 [batch][max_blocks_per_seq]; entries past
+ *                  ceil(L/16) are never read
+ *   context_lens : device int32 [batch], each in [1, max_context_len]
+ *   max_context_len : upper bound of context_lens, <= max_blocks_per_seq*16
+ *   workspace    : device buffer of >= paged_decode_workspace_bytes(...) bytes
+ *                  (may be NULL when that size is 0)
+ * Host checks: num_q_heads % num_kv_heads == 0 with a group size of 1, 2, 4
+ * or 8 (else KV_ERR_UNSUPPORTED); partition_tokens a multiple of 16;
+ * max_context_len <= max_blocks_per_seq * 16; pointer alignment; workspace
+ * size.  Device errors: KV_DEVERR_BAD_CONTEXT_LEN (that sequence's output is
+ * zero), KV_DEVERR_BAD_BLOCK_ID (that block's tokens are skipped),
+ * KV_DEVERR_TIMEOUT.
+ */
+KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
+                                 kv_dtype q_dtype, const void* k_pool, const void* v_pool,
+                                 const float* k_scales, const float* v_scales,
+                                 const int32_t* block_table, int32_t max_blocks_per_seq,
+                                 const int32_t* context_lens, int32_t batch,
+                                 int32_t num_q_heads, int32_t max_context_len, float scale,
+                                 int32_t partition_tokens, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_error,
+                                 kv_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+KV_API const char* kv_status_string(kv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_KV_H */

@@ -81,9 +81,19 @@ uint8_t oracle_e4m3_encode(float x) {
     sign = signbit(x) ? 0x80 : 0x00;
     a = fabsf(x);
     if (a >= 448.0f) return (uint8_t)(sign | 0x7E);
-    /* largest code c (0..0x7D) with value(c) <= a */
-    c = 0;
-    while (c < 0x7E && oracle_e4m3_decode((uint8_t)(c + 1)) <= (double)a) c++;
+    /* largest code c (0..0x7D) with value(c) <= a: the positive codes 0..0x7E
+       decode to increasing magnitudes, so bisect over them */
+    {
+        int lo = 0, hi = 0x7E;                   /* value(lo) <= a < value(hi) */
+        while (hi - lo > 1) {
+            int mid = (lo + hi) / 2;
+            if (oracle_e4m3_decode((uint8_t)mid) <= (double)a)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        c = lo;
+    }
     if (c < 0x7E) {
         double lo = oracle_e4m3_decode((uint8_t)c);
         double hi = oracle_e4m3_decode((uint8_t)(c + 1));
@@ -104,8 +114,8 @@ uint8_t oracle_e4m3_encode(float x) {
  */
 void oracle_quantize_rows(const float* x, int64_t rows, int32_t d,
                           uint8_t* codes, float* scales) {
-    int64_t r;
-    for (r = 0; r < rows; ++r) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
         const float* xr = x + r * d;
         float a = 0.0f, s;
         int32_t i;

@@ -1,0 +1,193 @@
+"""Python binding of libpagedkv.so: paged GQA decode attention on B200.
+
+Argument marshalling only.  Every step of the decode path (slot computation,
+cache write, split-K decode, log-sum-exp merge, FP8 quantise/dequantise) runs
+in the library's CUDA kernels; PyTorch supplies device memory and streams.
+The functions carry the C ABI's names (include/paged_kv.h) and raise
+``KvError`` on a non-OK status.  There is no fallback: if the compiled
+library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
+
+KV_F32, KV_BF16, KV_FP8_E4M3 = 0, 1, 2
+KV_OK, KV_ERR_INVALID_ARGUMENT, KV_ERR_UNSUPPORTED, KV_ERR_CUDA = 0, 1, 2, 3
+KV_DEVERR_BAD_SLOT = 0x1
+KV_DEVERR_BAD_CONTEXT_LEN = 0x2
+KV_DEVERR_BAD_BLOCK_ID = 0x4
+KV_DEVERR_TIMEOUT = 0x8
+KV_DEVERR_BAD_POSITION = 0x10
+BLOCK_SIZE = 16
+
+EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
+            "paged_decode_default_partition", "paged_decode_workspace_bytes",
+            "paged_decode_attention", "kv_status_string")
+
+
+class KvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {kv_status_string(status)} ({status})")
+        self.status = status
+
+
+class KvPoolDesc(ctypes.Structure):
+    """Mirror of kv_pool_desc (plain data; owns nothing)."""
+    _fields_ = [("num_blocks", ctypes.c_int32), ("block_size", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("elem_bytes", ctypes.c_int32),
+                ("kv_bytes", ctypes.c_uint64), ("scale_bytes", ctypes.c_uint64),
+                ("stride_block", ctypes.c_int64), ("stride_head", ctypes.c_int64),
+                ("stride_slot", ctypes.c_int64)]
+
+
+_lib = None
+_P, _I32, _I64, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+
+
+def _load() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m paged_kv_cache_401_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        desc_p = ctypes.POINTER(KvPoolDesc)
+        sig = {
+            "kv_pool_create": (_I32, [_I32, _I32, _I32, _I32, _I32, desc_p]),
+            "compute_slot_mapping": (_I32, [_P, _I32, _I32, _I32, _P, _P, _I32, _P, _P, _P]),
+            "reshape_and_cache": (_I32, [desc_p, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
+            "paged_decode_default_partition": (_I32, [desc_p, _I32, _I32, _I32]),
+            "paged_decode_workspace_bytes": (_SZ, [desc_p, _I32, _I32, _I32, _I32]),
+            "paged_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _I32, _P,
+                                              _I32, _I32, _I32, ctypes.c_float, _I32, _P, _SZ,
+                                              _P, _P]),
+            "kv_status_string": (ctypes.c_char_p, [_I32]),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(lib, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = lib
+    return _lib
+
+
+def library() -> ctypes.CDLL:
+    """The loaded libpagedkv.so (raises if it has not been built)."""
+    return _load()
+
+
+def kv_dtype_of(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return KV_F32
+    if t.dtype == torch.bfloat16:
+        return KV_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return KV_FP8_E4M3
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libpagedkv must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _check(fn: str, status: int) -> None:
+    if status != KV_OK:
+        raise KvError(fn, status)
+
+
+def kv_status_string(status: int) -> str:
+    return _load().kv_status_string(int(status)).decode()
+
+
+def kv_pool_create(num_blocks: int, block_size: int, num_kv_heads: int, head_dim: int,
+                   dtype: int) -> KvPoolDesc:
+    desc = KvPoolDesc()
+    _check("kv_pool_create", _load().kv_pool_create(num_blocks, block_size, num_kv_heads,
+                                                    head_dim, dtype, ctypes.byref(desc)))
+    return desc
+
+
+def empty_pool(desc: KvPoolDesc, device, fill: float | int | None = None):
+    """Allocate (k_pool, v_pool, k_scales, v_scales) tensors for a descriptor
+    (scales None unless FP8).  ``fill`` poisons every element (NaN, or a byte)."""
+    shape = (desc.num_blocks, desc.num_kv_heads, desc.block_size, desc.head_dim)
+    dt = {KV_F32: torch.float32, KV_BF16: torch.bfloat16, KV_FP8_E4M3: torch.uint8}[desc.dtype]
+    k = torch.empty(shape, dtype=dt, device=device)
+    v = torch.empty(shape, dtype=dt, device=device)
+    ks = vs = None
+    if desc.dtype == KV_FP8_E4M3:
+        ks = torch.empty(shape[:3], dtype=torch.float32, device=device)
+        vs = torch.empty(shape[:3], dtype=torch.float32, device=device)
+    if fill is not None:
+        for t in (k, v):
+            t.fill_(fill)
+        for t in (ks, vs):
+            if t is not None:
+                t.fill_(float("nan"))
+    return k, v, ks, vs
+
+
+def compute_slot_mapping(block_table: torch.Tensor, seq_ids: torch.Tensor,
+                         positions: torch.Tensor, slot_mapping: torch.Tensor,
+                         block_size: int = BLOCK_SIZE, dev_error: torch.Tensor | None = None,
+                         stream=None) -> torch.Tensor:
+    batch, max_blocks = block_table.shape
+    _check("compute_slot_mapping", _load().compute_slot_mapping(
+        _ptr(block_table), batch, max_blocks, block_size, _ptr(seq_ids), _ptr(positions),
+        seq_ids.numel(), _ptr(slot_mapping), _ptr(dev_error), _stream(stream)))
+    return slot_mapping
+
+
+def reshape_and_cache(pool: KvPoolDesc, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                      k_scales: torch.Tensor | None, v_scales: torch.Tensor | None,
+                      k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
+                      dev_error: torch.Tensor | None = None, stream=None) -> None:
+    _check("reshape_and_cache", _load().reshape_and_cache(
+        ctypes.byref(pool), _ptr(k_pool), _ptr(v_pool), _ptr(k_scales), _ptr(v_scales),
+        _ptr(k_new), _ptr(v_new), kv_dtype_of(k_new), _ptr(slot_mapping), k_new.shape[0],
+        _ptr(dev_error), _stream(stream)))
+
+
+def paged_decode_default_partition(pool: KvPoolDesc, batch: int, num_q_heads: int,
+                                   max_context_len: int) -> int:
+    return int(_load().paged_decode_default_partition(ctypes.byref(pool), batch, num_q_heads,
+                                                      max_context_len))
+
+
+def paged_decode_workspace_bytes(pool: KvPoolDesc, batch: int, num_q_heads: int,
+                                 max_context_len: int, partition_tokens: int = 0) -> int:
+    return int(_load().paged_decode_workspace_bytes(ctypes.byref(pool), batch, num_q_heads,
+                                                    max_context_len, partition_tokens))
+
+
+def paged_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
+                           k_pool: torch.Tensor, v_pool: torch.Tensor,
+                           k_scales: torch.Tensor | None, v_scales: torch.Tensor | None,
+                           block_table: torch.Tensor, context_lens: torch.Tensor,
+                           max_context_len: int, scale: float, partition_tokens: int = 0,
+                           workspace: torch.Tensor | None = None,
+                           dev_error: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    batch, num_q_heads, _ = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("paged_decode_attention", _load().paged_decode_attention(
+        ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool), _ptr(v_pool),
+        _ptr(k_scales), _ptr(v_scales), _ptr(block_table), block_table.shape[1],
+        _ptr(context_lens), batch, num_q_heads, max_context_len, float(scale),
+        partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream)))
+    return out

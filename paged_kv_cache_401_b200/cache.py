@@ -1,0 +1,73 @@
+"""PagedKVCache: one layer's paged K/V pool plus the calls a decode step makes.
+
+A thin convenience layer over the binding: it allocates the pools with torch
+(device memory is PyTorch's job here) and forwards to the C ABI.  Per step, a
+caller appends each sequence's new token (``append``: slot computation and
+cache write) and then runs ``decode`` (split-K paged attention + merge).
+"""
+from __future__ import annotations
+
+import torch
+
+from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, compute_slot_mapping, empty_pool,
+               kv_pool_create, paged_decode_attention, paged_decode_workspace_bytes,
+               reshape_and_cache)
+
+_DTYPES = {"f32": KV_F32, "bf16": KV_BF16, "fp8": KV_FP8_E4M3}
+
+
+class PagedKVCache:
+    def __init__(self, num_blocks: int, num_kv_heads: int, head_dim: int, dtype: str,
+                 device="cuda", poison: bool = False):
+        self.kv_dtype = dtype
+        self.device = torch.device(device)
+        self.desc = kv_pool_create(num_blocks, BLOCK_SIZE, num_kv_heads, head_dim, _DTYPES[dtype])
+        fill = None
+        if poison:
+            fill = 0x7F if dtype == "fp8" else float("nan")
+        self.k_pool, self.v_pool, self.k_scales, self.v_scales = empty_pool(self.desc,
+                                                                            self.device, fill)
+        self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
+
+    # ---- a1 + a2/a3: slots and cache write ---------------------------------------
+    def append(self, block_table: torch.Tensor, seq_ids: torch.Tensor, positions: torch.Tensor,
+               k_new: torch.Tensor, v_new: torch.Tensor, slots: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        if slots is None:
+            slots = torch.empty(seq_ids.numel(), dtype=torch.int64, device=self.device)
+        compute_slot_mapping(block_table, seq_ids, positions, slots, BLOCK_SIZE, self.dev_error,
+                             stream)
+        reshape_and_cache(self.desc, self.k_pool, self.v_pool, self.k_scales, self.v_scales,
+                          k_new, v_new, slots, self.dev_error, stream)
+        return slots
+
+    # ---- a4..a10: paged split-K decode + merge --------------------------------------
+    def workspace_bytes(self, batch: int, num_q_heads: int, max_context_len: int,
+                        partition_tokens: int = 0) -> int:
+        return paged_decode_workspace_bytes(self.desc, batch, num_q_heads, max_context_len,
+                                            partition_tokens)
+
+    def alloc_workspace(self, batch: int, num_q_heads: int, max_context_len: int,
+                        partition_tokens: int = 0) -> torch.Tensor | None:
+        n = self.workspace_bytes(batch, num_q_heads, max_context_len, partition_tokens)
+        return torch.empty(n, dtype=torch.uint8, device=self.device) if n else None
+
+    def decode(self, q: torch.Tensor, block_table: torch.Tensor, context_lens: torch.Tensor,
+               max_context_len: int, scale: float, out: torch.Tensor | None = None,
+               partition_tokens: int = 0, workspace: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty_like(q)
+        if workspace is None:
+            workspace = self.alloc_workspace(q.shape[0], q.shape[1], max_context_len,
+                                             partition_tokens)
+        return paged_decode_attention(self.desc, out, q, self.k_pool, self.v_pool, self.k_scales,
+                                      self.v_scales, block_table, context_lens, max_context_len,
+                                      scale, partition_tokens, workspace, self.dev_error, stream)
+
+    def errors(self) -> int:
+        """The device error word (KV_DEVERR_* bits); synchronises."""
+        return int(self.dev_error.item())
+
+    def clear_errors(self) -> None:
+        self.dev_error.zero_()

@@ -1,0 +1,228 @@
+// C ABI of libpagedkv.so (declared in include/paged_kv.h): host-side argument
+// checks, geometry, the split-K partition heuristic and kernel launches.
+#include <cmath>
+
+#include "kernels.cuh"
+
+namespace {
+
+using pkv::kBlockTokens;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t elem_bytes(int32_t dtype) {
+    switch (dtype) {
+        case KV_F32: return 4;
+        case KV_BF16: return 2;
+        case KV_FP8_E4M3: return 1;
+        default: return 0;
+    }
+}
+
+// SM count of the current device; 148 (B200) when no device can be queried.
+int32_t current_sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) {
+        cudaGetLastError();  // clear the sticky "no device" error of the query
+        return 148;
+    }
+    return n;
+}
+
+bool valid_pool(const kv_pool_desc* d) {
+    return d != nullptr && d->num_blocks > 0 && d->block_size == kBlockTokens &&
+           d->num_kv_heads > 0 && (d->head_dim == 64 || d->head_dim == 128) &&
+           elem_bytes(d->dtype) == d->elem_bytes;
+}
+
+int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
+
+}  // namespace
+
+extern "C" {
+
+kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
+                         int32_t head_dim, kv_dtype dtype, kv_pool_desc* out) {
+    if (out == nullptr || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (block_size != kBlockTokens || (head_dim != 64 && head_dim != 128) || num_kv_heads > 256 ||
+        elem_bytes(dtype) == 0)
+        return KV_ERR_UNSUPPORTED;
+    kv_pool_desc d{};
+    d.num_blocks = num_blocks;
+    d.block_size = block_size;
+    d.num_kv_heads = num_kv_heads;
+    d.head_dim = head_dim;
+    d.dtype = dtype;
+    d.elem_bytes = elem_bytes(dtype);
+    d.stride_slot = head_dim;
+    d.stride_head = static_cast<int64_t>(block_size) * head_dim;
+    d.stride_block = d.stride_head * num_kv_heads;
+    d.kv_bytes = static_cast<uint64_t>(d.stride_block) * num_blocks * d.elem_bytes;
+    d.scale_bytes = dtype == KV_FP8_E4M3
+                        ? static_cast<uint64_t>(num_blocks) * num_kv_heads * block_size * 4u
+                        : 0u;
+    *out = d;
+    return KV_OK;
+}
+
+kv_status compute_slot_mapping(const int32_t* block_table, int32_t batch,
+                               int32_t max_blocks_per_seq, int32_t block_size,
+                               const int32_t* seq_ids, const int32_t* positions,
+                               int32_t num_tokens, int64_t* slot_mapping, int32_t* dev_error,
+                               kv_stream_t stream) {
+    if (num_tokens < 0 || batch < 0 || max_blocks_per_seq < 0) return KV_ERR_INVALID_ARGUMENT;
+    if (block_size != kBlockTokens) return KV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return KV_OK;
+    if (block_table == nullptr || seq_ids == nullptr || positions == nullptr ||
+        slot_mapping == nullptr)
+        return KV_ERR_INVALID_ARGUMENT;
+    cudaError_t e = pkv::launch_slot_mapping(block_table, batch, max_blocks_per_seq, seq_ids,
+                                             positions, num_tokens, slot_mapping, dev_error,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool,
+                            float* k_scales, float* v_scales, const void* k_new,
+                            const void* v_new, kv_dtype src_dtype, const int64_t* slot_mapping,
+                            int32_t num_tokens, int32_t* dev_error, kv_stream_t stream) {
+    if (!valid_pool(pool) || num_tokens < 0) return KV_ERR_INVALID_ARGUMENT;
+    if (num_tokens == 0) return KV_OK;
+    if (k_pool == nullptr || v_pool == nullptr || k_new == nullptr || v_new == nullptr ||
+        slot_mapping == nullptr)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(k_new) || !aligned16(v_new))
+        return KV_ERR_INVALID_ARGUMENT;
+    const int64_t num_slots = static_cast<int64_t>(pool->num_blocks) * kBlockTokens;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    if (pool->dtype == KV_FP8_E4M3) {
+        if (src_dtype != KV_F32 && src_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
+        if (k_scales == nullptr || v_scales == nullptr) return KV_ERR_INVALID_ARGUMENT;
+        e = pkv::launch_cache_fp8(src_dtype, pool->head_dim, k_pool, v_pool, k_scales, v_scales,
+                                  k_new, v_new, slot_mapping, num_tokens, pool->num_kv_heads,
+                                  num_slots, dev_error, s);
+    } else {
+        if (src_dtype != pool->dtype) return KV_ERR_UNSUPPORTED;
+        if (k_scales != nullptr || v_scales != nullptr) return KV_ERR_INVALID_ARGUMENT;
+        e = pkv::launch_cache_copy(k_pool, v_pool, k_new, v_new, slot_mapping, num_tokens,
+                                   pool->num_kv_heads, pool->head_dim * pool->elem_bytes,
+                                   num_slots, current_sm_count(), dev_error, s);
+    }
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+int32_t paged_decode_default_partition(const kv_pool_desc* pool, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_context_len) {
+    (void)num_q_heads;
+    if (!valid_pool(pool) || batch <= 0 || max_context_len <= 0) return 512;
+    // Enough thread blocks for several waves over the SMs (a decode block keeps
+    // 32-64 KB of tiles in flight; ~3 fit per SM), each partition long enough
+    // that its partial (m, l, o) write stays a few percent of the KV it reads.
+    const int64_t pairs = static_cast<int64_t>(batch) * pool->num_kv_heads;
+    const int64_t want = 8ll * current_sm_count() * 3;
+    int32_t P = 1024;
+    while (P > 256 && pairs * ceil_div(max_context_len, P) < want) P /= 2;
+    return P;
+}
+
+size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
+                                    int32_t num_q_heads, int32_t max_context_len,
+                                    int32_t partition_tokens) {
+    if (!valid_pool(pool) || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
+    const int32_t P = partition_tokens > 0
+                          ? partition_tokens
+                          : paged_decode_default_partition(pool, batch, num_q_heads,
+                                                           max_context_len);
+    const int32_t parts = ceil_div(max_context_len, P);
+    if (parts <= 1) return 0;
+    const size_t rows = static_cast<size_t>(batch) * num_q_heads * parts;
+    size_t ml = rows * sizeof(float2);
+    ml = (ml + 255) & ~static_cast<size_t>(255);
+    return ml + rows * pool->head_dim * sizeof(float);
+}
+
+kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
+                                 kv_dtype q_dtype, const void* k_pool, const void* v_pool,
+                                 const float* k_scales, const float* v_scales,
+                                 const int32_t* block_table, int32_t max_blocks_per_seq,
+                                 const int32_t* context_lens, int32_t batch,
+                                 int32_t num_q_heads, int32_t max_context_len, float scale,
+                                 int32_t partition_tokens, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_error,
+                                 kv_stream_t stream) {
+    if (!valid_pool(pool) || batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (q_dtype != KV_F32 && q_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
+    if (num_q_heads % pool->num_kv_heads != 0) return KV_ERR_INVALID_ARGUMENT;
+    const int32_t group = num_q_heads / pool->num_kv_heads;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return KV_ERR_UNSUPPORTED;
+    if (batch == 0) return KV_OK;
+    if (max_context_len <= 0 ||
+        static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (partition_tokens < 0 || partition_tokens % kBlockTokens != 0 || partition_tokens > 8192)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (!std::isfinite(scale)) return KV_ERR_INVALID_ARGUMENT;
+    if (out == nullptr || q == nullptr || k_pool == nullptr || v_pool == nullptr ||
+        block_table == nullptr || context_lens == nullptr)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
+        return KV_ERR_INVALID_ARGUMENT;
+    const bool fp8 = pool->dtype == KV_FP8_E4M3;
+    if (fp8 != (k_scales != nullptr) || fp8 != (v_scales != nullptr))
+        return KV_ERR_INVALID_ARGUMENT;
+    if (fp8 && (!aligned16(k_scales) || !aligned16(v_scales))) return KV_ERR_INVALID_ARGUMENT;
+
+    const int32_t P = partition_tokens > 0
+                          ? partition_tokens
+                          : paged_decode_default_partition(pool, batch, num_q_heads,
+                                                           max_context_len);
+    const size_t need =
+        paged_decode_workspace_bytes(pool, batch, num_q_heads, max_context_len, P);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+        return KV_ERR_INVALID_ARGUMENT;
+
+    pkv::DecodeParams p{};
+    p.out = out;
+    p.q = q;
+    p.k_pool = static_cast<const uint8_t*>(k_pool);
+    p.v_pool = static_cast<const uint8_t*>(v_pool);
+    p.k_scales = k_scales;
+    p.v_scales = v_scales;
+    p.block_table = block_table;
+    p.context_lens = context_lens;
+    p.dev_error = dev_error;
+    p.batch = batch;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = pool->num_kv_heads;
+    p.num_blocks = pool->num_blocks;
+    p.max_blocks = max_blocks_per_seq;
+    p.max_context_len = max_context_len;
+    p.partition_tokens = P;
+    p.max_parts = ceil_div(max_context_len, P);
+    p.scale_log2 = scale * 1.4426950408889634f;
+    if (need > 0) {
+        const size_t rows = static_cast<size_t>(batch) * num_q_heads * p.max_parts;
+        size_t ml = (rows * sizeof(float2) + 255) & ~static_cast<size_t>(255);
+        p.ws_ml = static_cast<float2*>(workspace);
+        p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ml);
+    }
+    cudaError_t e = pkv::launch_paged_decode(p, pool->dtype, q_dtype, pool->head_dim, group,
+                                             reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+const char* kv_status_string(kv_status status) {
+    switch (status) {
+        case KV_OK: return "KV_OK";
+        case KV_ERR_INVALID_ARGUMENT: return "KV_ERR_INVALID_ARGUMENT";
+        case KV_ERR_UNSUPPORTED: return "KV_ERR_UNSUPPORTED";
+        case KV_ERR_CUDA: return "KV_ERR_CUDA";
+        default: return "KV_STATUS_UNKNOWN";
+    }
+}
+
+}  // extern "C"

@@ -1,0 +1,170 @@
+// Slot computation and cache write ("KV Cache 深度解析" §一/§三/§四;
+// "llm-inference-optimization" notes §二 PagedKVCache.append_token).
+//
+// Pool layout [num_blocks][num_kv_heads][16][head_dim]: the new token's row of
+// kv head h goes to block slot/16, row slot%16.  HBM-bound scatter: every
+// thread moves one 16-byte vector (bf16/fp32) or one warp quantises one row
+// (FP8), so loads and stores are full 32-byte sectors.
+#include "kernels.cuh"
+
+namespace pkv {
+
+__global__ void slot_mapping_kernel(const int32_t* __restrict__ block_table, int32_t batch,
+                                    int32_t max_blocks, const int32_t* __restrict__ seq_ids,
+                                    const int32_t* __restrict__ positions, int32_t num_tokens,
+                                    int64_t* __restrict__ slots, int32_t* dev_error) {
+    const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= num_tokens) return;
+    const int32_t s = seq_ids[i];
+    const int32_t p = positions[i];
+    if (s < 0 || s >= batch || p < 0 || p >= max_blocks * kBlockTokens) {
+        slots[i] = -1;
+        report(dev_error, KV_DEVERR_BAD_POSITION);
+        return;
+    }
+    const int64_t blk = block_table[static_cast<int64_t>(s) * max_blocks + p / kBlockTokens];
+    slots[i] = blk * kBlockTokens + p % kBlockTokens;
+}
+
+// Exact copy: one 16-byte vector per thread, K and V.
+__global__ void cache_copy_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
+                                  const uint8_t* __restrict__ k_new,
+                                  const uint8_t* __restrict__ v_new,
+                                  const int64_t* __restrict__ slots, int32_t num_tokens,
+                                  int32_t num_kv_heads, int32_t row_bytes, int64_t num_slots,
+                                  int32_t* dev_error) {
+    const int32_t vecs_per_row = row_bytes / 16;
+    const int64_t per_token = static_cast<int64_t>(num_kv_heads) * vecs_per_row;
+    const int64_t total = per_token * num_tokens;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t t = i / per_token;
+        const int64_t rem = i - t * per_token;
+        const int32_t h = static_cast<int32_t>(rem / vecs_per_row);
+        const int32_t v = static_cast<int32_t>(rem - static_cast<int64_t>(h) * vecs_per_row);
+        const int64_t slot = slots[t];
+        if (slot < 0) continue;
+        if (slot >= num_slots) {
+            if (h == 0 && v == 0) report(dev_error, KV_DEVERR_BAD_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / kBlockTokens, off = slot % kBlockTokens;
+        const int64_t src = (t * num_kv_heads + h) * row_bytes + v * 16;
+        const int64_t dst = ((blk * num_kv_heads + h) * kBlockTokens + off) * row_bytes + v * 16;
+        const uint4 kv = *reinterpret_cast<const uint4*>(k_new + src);
+        const uint4 vv = *reinterpret_cast<const uint4*>(v_new + src);
+        *reinterpret_cast<uint4*>(k_pool + dst) = kv;
+        *reinterpret_cast<uint4*>(v_pool + dst) = vv;
+    }
+}
+
+// FP8 quantising write: one warp per (token, kv head, K|V) row of D elements.
+//   a = max|x|; scale = a / 448 (IEEE fp32 division); code = E4M3(x / scale)
+//   (IEEE division, RNE, saturating); a == 0 -> scale 0 and codes 0.
+template <int SRC_T, int D>
+__global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
+                                 float* __restrict__ k_scales, float* __restrict__ v_scales,
+                                 const void* __restrict__ k_new, const void* __restrict__ v_new,
+                                 const int64_t* __restrict__ slots, int32_t num_tokens,
+                                 int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error) {
+    constexpr int kPer = D / 32;  // elements per lane (4 or 2)
+    const int32_t lane = threadIdx.x & 31;
+    const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t rows = 2ll * num_tokens * num_kv_heads;
+    if (row >= rows) return;
+    const int32_t which = static_cast<int32_t>(row & 1);  // 0 = K, 1 = V
+    const int64_t th = row >> 1;                          // token * heads + head
+    const int64_t t = th / num_kv_heads;
+    const int32_t h = static_cast<int32_t>(th - t * num_kv_heads);
+    const int64_t slot = slots[t];
+    if (slot < 0) return;
+    if (slot >= num_slots) {
+        if (lane == 0 && h == 0 && which == 0) report(dev_error, KV_DEVERR_BAD_SLOT);
+        return;
+    }
+    float x[kPer];
+    const void* src = which ? v_new : k_new;
+    if constexpr (SRC_T == KV_F32) {
+        const float* p = static_cast<const float*>(src) + th * D + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) x[e] = p[e];
+    } else {
+        const uint16_t* p = static_cast<const uint16_t*>(src) + th * D + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) x[e] = __uint_as_float(static_cast<uint32_t>(p[e]) << 16);
+    }
+    float a = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) a = fmaxf(a, fabsf(x[e]));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+    const float s = __fdiv_rn(a, 448.0f);
+    uint32_t codes = 0;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2) {
+        uint32_t pair = 0;
+        if (a != 0.0f) pair = float2_to_e4m3x2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s));
+        codes |= pair << (8 * e);
+    }
+    const int64_t blk = slot / kBlockTokens, off = slot % kBlockTokens;
+    const int64_t rowi = (blk * num_kv_heads + h) * kBlockTokens + off;
+    uint8_t* dst = (which ? v_pool : k_pool) + rowi * D + lane * kPer;
+    if constexpr (kPer == 4) {
+        *reinterpret_cast<uint32_t*>(dst) = codes;
+    } else {
+        *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(codes);
+    }
+    if (lane == 0) (which ? v_scales : k_scales)[rowi] = (a == 0.0f) ? 0.0f : s;
+}
+
+// ---- launchers ------------------------------------------------------------------
+cudaError_t launch_slot_mapping(const int32_t* block_table, int32_t batch, int32_t max_blocks,
+                                const int32_t* seq_ids, const int32_t* positions,
+                                int32_t num_tokens, int64_t* slots, int32_t* dev_error,
+                                cudaStream_t stream) {
+    const int threads = 256;
+    const int blocks = (num_tokens + threads - 1) / threads;
+    slot_mapping_kernel<<<blocks, threads, 0, stream>>>(block_table, batch, max_blocks, seq_ids,
+                                                        positions, num_tokens, slots, dev_error);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, const void* v_new,
+                              const int64_t* slots, int32_t num_tokens, int32_t num_kv_heads,
+                              int32_t row_bytes, int64_t num_slots, int32_t num_sms,
+                              int32_t* dev_error, cudaStream_t stream) {
+    const int threads = 256;
+    const int64_t vecs = static_cast<int64_t>(num_tokens) * num_kv_heads * (row_bytes / 16);
+    int64_t blocks = (vecs + threads - 1) / threads;
+    const int64_t cap = static_cast<int64_t>(num_sms) * 16;
+    if (blocks > cap) blocks = cap;
+    cache_copy_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
+        static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool),
+        static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), slots,
+        num_tokens, num_kv_heads, row_bytes, num_slots, dev_error);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, void* v_pool,
+                             float* k_scales, float* v_scales, const void* k_new,
+                             const void* v_new, const int64_t* slots, int32_t num_tokens,
+                             int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
+                             cudaStream_t stream) {
+    const int threads = 256;
+    const int64_t rows = 2ll * num_tokens * num_kv_heads;
+    const int64_t blocks = (rows * 32 + threads - 1) / threads;
+    auto* kp = static_cast<uint8_t*>(k_pool);
+    auto* vp = static_cast<uint8_t*>(v_pool);
+#define PKV_FP8_LAUNCH(ST, DD)                                                               \
+    cache_fp8_kernel<ST, DD><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(         \
+        kp, vp, k_scales, v_scales, k_new, v_new, slots, num_tokens, num_kv_heads, num_slots, \
+        dev_error)
+    if (src_dtype == KV_F32 && head_dim == 128) PKV_FP8_LAUNCH(KV_F32, 128);
+    else if (src_dtype == KV_F32 && head_dim == 64) PKV_FP8_LAUNCH(KV_F32, 64);
+    else if (src_dtype == KV_BF16 && head_dim == 128) PKV_FP8_LAUNCH(KV_BF16, 128);
+    else PKV_FP8_LAUNCH(KV_BF16, 64);
+#undef PKV_FP8_LAUNCH
+    return cudaGetLastError();
+}
+
+}  // namespace pkv

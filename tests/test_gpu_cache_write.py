@@ -1,0 +1,103 @@
+"""GPU: slot computation and cache write are bit-exact against the oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import paged_kv_cache_401_b200 as pk
+from paged_kv_cache_401_b200.cache import PagedKVCache
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _bits(t: torch.Tensor) -> np.ndarray:
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float32:
+        return t.view(torch.int32).numpy()
+    return t.numpy()
+
+
+def test_slot_mapping_bitexact_and_bad_positions():
+    rng = np.random.default_rng(1)
+    B, MB = 7, 9
+    table = rng.permutation(200)[:B * MB].reshape(B, MB).astype(np.int32)
+    sids = rng.integers(0, B, 500).astype(np.int32)
+    poss = rng.integers(0, MB * 16, 500).astype(np.int32)
+    expect = oracle.slot_mapping(table, sids, poss, 16)
+    bad = np.array([[0, MB * 16], [B, 3], [-1, 0], [2, -5]], dtype=np.int32)
+    sids_all = np.r_[sids, bad[:, 0]]
+    poss_all = np.r_[poss, bad[:, 1]]
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    slots = torch.empty(len(sids_all), dtype=torch.int64, device=DEV)
+    pk.compute_slot_mapping(torch.from_numpy(table).to(DEV), torch.from_numpy(sids_all).to(DEV),
+                            torch.from_numpy(poss_all).to(DEV), slots, 16, err)
+    got = slots.cpu().numpy()
+    assert (got[:500] == expect).all()
+    assert (got[500:] == -1).all()
+    assert err.item() == pk.KV_DEVERR_BAD_POSITION
+
+
+@pytest.mark.parametrize("dtype,D", [("f32", 64), ("f32", 128), ("bf16", 64), ("bf16", 128)])
+def test_cache_copy_bitexact(dtype, D):
+    rng = np.random.default_rng(2)
+    NB, Hkv, T = 40, 3, 300
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16}[dtype]
+    cache = PagedKVCache(NB, Hkv, D, dtype, DEV, poison=True)
+    k = torch.randn(T, Hkv, D, dtype=torch.float32).to(tdt)
+    v = torch.randn(T, Hkv, D, dtype=torch.float32).to(tdt)
+    slots = rng.permutation(NB * 16)[:T].astype(np.int64)
+    slots[5] = -1                       # padding
+    slots[6] = NB * 16 + 3              # out of range: skipped, reported
+    pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, None, None, k.to(DEV),
+                         v.to(DEV), torch.from_numpy(slots).to(DEV), cache.dev_error)
+    slots_ok = slots.copy()
+    slots_ok[6] = -1
+    for pool, src in ((cache.k_pool, k), (cache.v_pool, v)):
+        poison = np.full(tuple(pool.shape), np.nan, dtype=np.float32)
+        poison = torch.from_numpy(poison).to(tdt)
+        want = oracle.scatter_to_pool(_bits(poison), _bits(src), slots_ok)
+        assert (_bits(pool) == want).all()
+    assert cache.errors() == pk.KV_DEVERR_BAD_SLOT
+
+
+def _fp8_rows(rng, T, Hkv, D):
+    x = rng.normal(size=(T, Hkv, D)).astype(np.float32)
+    x[0] = 0.0                                   # zero rows: scale 0, codes 0
+    x[1, 0, :] = 0.0
+    x[1, 0, 7] = 1e-3                            # a single non-zero element
+    x[2] *= 1e-4                                 # small magnitudes
+    x[3, :, ::7] *= 50.0                         # outlier channels: subnormal codes elsewhere
+    x[4] *= 3e4                                  # large magnitudes
+    x[5, 1, :] = np.linspace(-1, 1, D)           # ties are likely on a regular grid
+    return x
+
+
+@pytest.mark.parametrize("src", ["f32", "bf16"])
+@pytest.mark.parametrize("D", [64, 128])
+def test_cache_fp8_bitexact(src, D):
+    rng = np.random.default_rng(3 + D)
+    NB, Hkv, T = 50, 2, 400
+    x_k = _fp8_rows(rng, T, Hkv, D)
+    x_v = rng.normal(size=(T, Hkv, D)).astype(np.float32)
+    tdt = {"f32": torch.float32, "bf16": torch.bfloat16}[src]
+    k = torch.from_numpy(x_k).to(tdt)
+    v = torch.from_numpy(x_v).to(tdt)
+    slots = rng.permutation(NB * 16)[:T].astype(np.int64)
+    slots[9] = -1
+    cache = PagedKVCache(NB, Hkv, D, "fp8", DEV, poison=True)
+    pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, cache.k_scales,
+                         cache.v_scales, k.to(DEV), v.to(DEV), torch.from_numpy(slots).to(DEV),
+                         cache.dev_error)
+    for pool, spool, src_t in ((cache.k_pool, cache.k_scales, k),
+                               (cache.v_pool, cache.v_scales, v)):
+        codes, scales = oracle.quantize_rows(src_t.float().numpy())
+        want_codes = oracle.scatter_to_pool(np.full(tuple(pool.shape), 0x7F, np.uint8), codes,
+                                            slots)
+        nan_scales = np.full(tuple(spool.shape), np.nan, np.float32)
+        want_scales = oracle.scatter_scales_to_pool(nan_scales, scales, slots)
+        assert (pool.cpu().numpy() == want_codes).all()
+        assert (_bits(spool) == want_scales.view(np.int32)).all()
+    assert cache.errors() == 0

@@ -1,0 +1,186 @@
+"""Host-side checks of libpagedkv.so that need no GPU.
+
+The library loads, exports every entry point include/paged_kv.h declares, and
+its host logic (geometry, argument validation, workspace sizing, partition
+heuristic) behaves as documented.  No call here enqueues device work: every
+call is rejected on the host before any launch, or is host-only.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+import paged_kv_cache_401_b200 as pk
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "paged_kv.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from paged_kv_cache_401_b200 import build
+    build.build()
+
+
+def _declared():
+    text = open(HEADER, encoding="utf-8").read()
+    return re.findall(r"KV_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)
+
+
+def test_header_declares_the_binding_names():
+    assert sorted(_declared()) == sorted(pk.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(pk.LIB_PATH)
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_library_exports_nothing_else():
+    out = os.popen(f"nm -D --defined-only {pk.LIB_PATH}").read().split("\n")
+    text_syms = {ln.split()[-1] for ln in out if " T " in ln}
+    assert text_syms == set(_declared())
+
+
+def test_status_strings():
+    assert pk.kv_status_string(0) == "KV_OK"
+    assert pk.kv_status_string(3) == "KV_ERR_CUDA"
+    assert pk.kv_status_string(99) == "KV_STATUS_UNKNOWN"
+
+
+def test_pool_geometry_llama_shape():
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
+    assert (d.stride_slot, d.stride_head, d.stride_block) == (128, 16 * 128, 8 * 16 * 128)
+    assert d.kv_bytes == 8192 * 8 * 16 * 128 * 2 == 256 * 2**20
+    assert d.scale_bytes == 0 and d.elem_bytes == 2
+    f = pk.kv_pool_create(100, 16, 8, 64, pk.KV_FP8_E4M3)
+    assert f.kv_bytes == 100 * 8 * 16 * 64 and f.scale_bytes == 100 * 8 * 16 * 4
+
+
+@pytest.mark.parametrize("args,status", [
+    ((0, 16, 8, 128, pk.KV_BF16), pk.KV_ERR_INVALID_ARGUMENT),
+    ((10, 32, 8, 128, pk.KV_BF16), pk.KV_ERR_UNSUPPORTED),
+    ((10, 16, 8, 96, pk.KV_BF16), pk.KV_ERR_UNSUPPORTED),
+    ((10, 16, 8, 128, 7), pk.KV_ERR_UNSUPPORTED),
+    ((10, 16, 0, 128, pk.KV_BF16), pk.KV_ERR_INVALID_ARGUMENT),
+])
+def test_pool_create_rejects(args, status):
+    with pytest.raises(pk.KvError) as e:
+        pk.kv_pool_create(*args)
+    assert e.value.status == status
+
+
+def test_workspace_bytes_and_partition():
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
+    # one partition: no workspace
+    assert pk.paged_decode_workspace_bytes(d, 32, 32, 4096, 4096) == 0
+    # 8 partitions of 512: (m, l) pairs padded to 256 B, then fp32 partial outputs
+    rows = 32 * 32 * 8
+    ml = (rows * 8 + 255) // 256 * 256
+    assert pk.paged_decode_workspace_bytes(d, 32, 32, 4096, 512) == ml + rows * 128 * 4
+    p = pk.paged_decode_default_partition(d, 32, 32, 4096)
+    assert p % 16 == 0 and 256 <= p <= 1024
+
+
+class _FakeTensor:
+    """Stands in for a device tensor in calls the host rejects before launching."""
+
+    def __init__(self, addr, shape, dtype="bf16"):
+        self.addr, self.shape, self._dt = addr, shape, dtype
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return self.addr
+
+    def numel(self):
+        n = 1
+        for s in self.shape:
+            n *= s
+        return n
+
+    def element_size(self):
+        return 1
+
+
+def _call_decode(desc, **kw):
+    lib = pk.library()
+    args = dict(out=4096, q=8192, q_dtype=pk.KV_BF16, k_pool=1 << 20, v_pool=2 << 20,
+                k_scales=None, v_scales=None, block_table=3 << 20, max_blocks=256,
+                context_lens=4 << 20, batch=32, num_q_heads=32, max_context_len=4096,
+                scale=0.088, partition=512, workspace=5 << 20, workspace_bytes=1 << 30,
+                dev_error=None, stream=None)
+    args.update(kw)
+    return lib.paged_decode_attention(
+        ctypes.byref(desc), args["out"], args["q"], args["q_dtype"], args["k_pool"],
+        args["v_pool"], args["k_scales"], args["v_scales"], args["block_table"],
+        args["max_blocks"], args["context_lens"], args["batch"], args["num_q_heads"],
+        args["max_context_len"], args["scale"], args["partition"], args["workspace"],
+        args["workspace_bytes"], args["dev_error"], args["stream"])
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_q_heads=24), pk.KV_ERR_UNSUPPORTED),                 # group 3
+    (dict(num_q_heads=30), pk.KV_ERR_INVALID_ARGUMENT),            # not a multiple of Hkv
+    (dict(num_q_heads=128), pk.KV_ERR_UNSUPPORTED),                # group 16
+    (dict(q_dtype=pk.KV_FP8_E4M3), pk.KV_ERR_UNSUPPORTED),
+    (dict(max_context_len=4097), pk.KV_ERR_INVALID_ARGUMENT),      # beyond the table
+    (dict(max_context_len=0), pk.KV_ERR_INVALID_ARGUMENT),
+    (dict(partition=500), pk.KV_ERR_INVALID_ARGUMENT),             # not a multiple of 16
+    (dict(partition=16384), pk.KV_ERR_INVALID_ARGUMENT),
+    (dict(q=8192 + 8), pk.KV_ERR_INVALID_ARGUMENT),                # misaligned
+    (dict(k_pool=None), pk.KV_ERR_INVALID_ARGUMENT),
+    (dict(k_scales=6 << 20, v_scales=7 << 20), pk.KV_ERR_INVALID_ARGUMENT),  # scales on bf16
+    (dict(workspace_bytes=100), pk.KV_ERR_INVALID_ARGUMENT),       # too small
+    (dict(workspace=None), pk.KV_ERR_INVALID_ARGUMENT),
+    (dict(scale=float("nan")), pk.KV_ERR_INVALID_ARGUMENT),
+])
+def test_decode_host_validation(kw, status):
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
+    assert _call_decode(d, **kw) == status
+
+
+def test_decode_fp8_pool_requires_scales():
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_FP8_E4M3)
+    assert _call_decode(d) == pk.KV_ERR_INVALID_ARGUMENT
+    assert _call_decode(d, k_scales=6 << 20) == pk.KV_ERR_INVALID_ARGUMENT
+
+
+def test_decode_empty_batch_is_a_no_op():
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
+    assert _call_decode(d, batch=0) == pk.KV_OK
+
+
+def test_cache_write_host_validation():
+    lib = pk.library()
+    d = pk.kv_pool_create(64, 16, 8, 128, pk.KV_BF16)
+    f = pk.kv_pool_create(64, 16, 8, 128, pk.KV_FP8_E4M3)
+    ok = dict(kp=1 << 20, vp=2 << 20, ks=None, vs=None, kn=3 << 20, vn=4 << 20,
+              src=pk.KV_BF16, slots=5 << 20, n=4)
+
+    def call(desc, **kw):
+        a = dict(ok)
+        a.update(kw)
+        return lib.reshape_and_cache(ctypes.byref(desc), a["kp"], a["vp"], a["ks"], a["vs"],
+                                     a["kn"], a["vn"], a["src"], a["slots"], a["n"], None, None)
+
+    assert call(d, n=0) == pk.KV_OK                                   # nothing to do
+    assert call(d, src=pk.KV_F32) == pk.KV_ERR_UNSUPPORTED            # no conversion on copy
+    assert call(d, kn=(3 << 20) + 4) == pk.KV_ERR_INVALID_ARGUMENT    # misaligned
+    assert call(d, ks=6 << 20) == pk.KV_ERR_INVALID_ARGUMENT          # scales on a bf16 pool
+    assert call(d, n=-1) == pk.KV_ERR_INVALID_ARGUMENT
+    assert call(f) == pk.KV_ERR_INVALID_ARGUMENT                      # fp8 needs scales
+    assert call(f, ks=6 << 20, vs=7 << 20, src=pk.KV_FP8_E4M3) == pk.KV_ERR_UNSUPPORTED
+
+
+def test_slot_mapping_host_validation():
+    lib = pk.library()
+    assert lib.compute_slot_mapping(1 << 20, 2, 4, 16, 2 << 20, 3 << 20, 0, 4 << 20, None,
+                                    None) == pk.KV_OK
+    assert lib.compute_slot_mapping(1 << 20, 2, 4, 32, 2 << 20, 3 << 20, 5, 4 << 20, None,
+                                    None) == pk.KV_ERR_UNSUPPORTED
+    assert lib.compute_slot_mapping(None, 2, 4, 16, 2 << 20, 3 << 20, 5, 4 << 20, None,
+                                    None) == pk.KV_ERR_INVALID_ARGUMENT

@@ -8,12 +8,13 @@ Recipe (all draws from one ``torch.Generator`` on the CPU, seeded per
 workload with 401 + the workload's index in ``WORKLOADS``):
   1. context lengths (fixed, or integers uniform in an inclusive range);
   2. q ~ N(0, 1), [B][Hq][D];
-  3. K ~ N(0, 1) then V ~ N(0, 1), each as one contiguous [tokens][Hkv][D]
+  3. outlier channels of K, where a workload has them (a seeded choice of
+     channels per KV head, multiplied by 20 before rounding);
+  4. K ~ N(0, 1) then V ~ N(0, 1), each as one contiguous [tokens][Hkv][D]
      array holding every sequence's tokens in logical order (sequence b at
-     rows seq_offsets[b] .. + L_b); a shared prefix, where a workload has
-     one, is drawn once and copied into each sharing sequence;
-  4. outlier channels of K, where a workload has them (a seeded choice of
-     channels per KV head, multiplied by 20);
+     rows seq_offsets[b] .. + L_b), drawn sequence by sequence in chunks of
+     65536 rows; a shared prefix, where a workload has one, is drawn first
+     and copied into each sharing sequence;
   5. a random permutation of the physical block ids, dealt to the sequences'
      logical blocks in order (shared prefix blocks first).
 Values are rounded to the stored dtype (fp32 or bf16, round to nearest even)
@@ -169,39 +170,34 @@ def make_inputs(name_or_spec, batch: int | None = None, lens_override=None) -> I
     sdt = _dtype(spec.source_dtype)
     # 2. q
     q = _randn(gen, (B, Hq, D), _dtype(spec.q_dtype))
-    # 3. K, V (shared prefix drawn once, first)
+    # 3. outlier channels of K (a seeded choice per KV head)
+    chans = None
+    if spec.outlier_channels:
+        chans = [torch.randperm(D, generator=gen)[:spec.outlier_channels] for _ in range(Hkv)]
+    # 4. K then V: the shared prefix (drawn once), then every sequence's own rows
     P = spec.shared_prefix_tokens if nshare else 0
     seq_offsets = np.zeros(B, dtype=np.int64)
     seq_offsets[1:] = np.cumsum(lens.astype(np.int64))[:-1]
     total = int(lens.astype(np.int64).sum())
     k = torch.empty((total, Hkv, D), dtype=sdt)
     v = torch.empty((total, Hkv, D), dtype=sdt)
-    if P:
-        kp = _randn(gen, (P, Hkv, D), torch.float32)
-        vp = _randn(gen, (P, Hkv, D), torch.float32)
-    own_k = _randn(gen, (total - nshare * P, Hkv, D), torch.float32) if total else None
-    own_v = _randn(gen, (total - nshare * P, Hkv, D), torch.float32) if total else None
-    # 4. outliers in K
-    if spec.outlier_channels:
-        chans = torch.stack([torch.randperm(D, generator=gen)[:spec.outlier_channels]
-                             for _ in range(Hkv)])
-        for h in range(Hkv):
-            own_k[:, h, chans[h]] *= spec.outlier_factor
-            if P:
-                kp[:, h, chans[h]] *= spec.outlier_factor
-    r = 0
-    for s in range(B):
-        o, n = int(seq_offsets[s]), int(lens[s])
-        if s < nshare:
-            k[o:o + P] = kp.to(sdt)
-            v[o:o + P] = vp.to(sdt)
-            k[o + P:o + n] = own_k[r:r + n - P].to(sdt)
-            v[o + P:o + n] = own_v[r:r + n - P].to(sdt)
-            r += n - P
-        else:
-            k[o:o + n] = own_k[r:r + n].to(sdt)
-            v[o:o + n] = own_v[r:r + n].to(sdt)
-            r += n
+    for dst, outliers in ((k, chans), (v, None)):
+        def draw(rows, _out=outliers):
+            x = torch.randn((rows, Hkv, D), generator=gen, dtype=torch.float32)
+            if _out is not None:
+                for h in range(Hkv):
+                    x[:, h, _out[h]] *= spec.outlier_factor
+            return x.to(sdt)
+        prefix = draw(P) if P else None
+        for s in range(B):
+            o, n = int(seq_offsets[s]), int(lens[s])
+            start = 0
+            if s < nshare:
+                dst[o:o + P] = prefix
+                start = P
+            for r0 in range(start, n, 1 << 16):
+                r1 = min(n, r0 + (1 << 16))
+                dst[o + r0:o + r1] = draw(r1 - r0)
     # 5. block table from a permutation of physical blocks
     nblk = (lens.astype(np.int64) + BLOCK_SIZE - 1) // BLOCK_SIZE
     shared_blocks = P // BLOCK_SIZE
