@@ -51,14 +51,14 @@ def test_cache_copy_bitexact(dtype, D):
     slots = rng.permutation(NB * 16)[:T].astype(np.int64)
     slots[5] = -1                       # padding
     slots[6] = NB * 16 + 3              # out of range: skipped, reported
+    before = {id(cache.k_pool): _bits(cache.k_pool), id(cache.v_pool): _bits(cache.v_pool)}
     pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, None, None, k.to(DEV),
                          v.to(DEV), torch.from_numpy(slots).to(DEV), cache.dev_error)
     slots_ok = slots.copy()
     slots_ok[6] = -1
     for pool, src in ((cache.k_pool, k), (cache.v_pool, v)):
-        poison = np.full(tuple(pool.shape), np.nan, dtype=np.float32)
-        poison = torch.from_numpy(poison).to(tdt)
-        want = oracle.scatter_to_pool(_bits(poison), _bits(src), slots_ok)
+        # expected: the pool's poisoned bits as filled, with the written rows replaced
+        want = oracle.scatter_to_pool(before[id(pool)], _bits(src), slots_ok)
         assert (_bits(pool) == want).all()
     assert cache.errors() == pk.KV_DEVERR_BAD_SLOT
 
