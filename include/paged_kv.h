@@ -199,6 +199,47 @@ KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, con
                                  size_t workspace_bytes, int32_t* dev_error,
                                  kv_stream_t stream);
 
+/*
+ * Bytes of device memory the library holds on every GPU that loads it, for
+ * paged_decode_attention_static_workspace (16 MiB: enough for the partials
+ * of e.g. 32 sequences x 32 query heads x 64 partitions of 128-wide heads).
+ */
+#define KV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
+
+/*
+ * paged_decode_attention for callers that cannot allocate device memory.
+ * The pages have no counterpart to this entry point: it exists for callers
+ * that have no way to obtain a workspace buffer -- an engine that reserved
+ * all device memory for its KV pool at start-up, a plugin inside another
+ * runtime that owns the allocator and gives plugins no allocation hook, a
+ * latency-bound loop that cannot take cudaMalloc's implicit synchronisation.
+ *
+ * Same arguments, layouts and results as paged_decode_attention, without
+ * workspace / workspace_bytes: the split-K partials go to a fixed array of
+ * KV_STATIC_WORKSPACE_BYTES in the library's own device memory, which every
+ * GPU that loads the library holds until the process exits.  The caller
+ * still passes q, the pools, the tables and out.  Nothing is allocated: no
+ * cudaMalloc, cudaFree or allocating library routine is called.
+ *  - Sizes whose workspace (paged_decode_workspace_bytes for the same
+ *    arguments) exceeds KV_STATIC_WORKSPACE_BYTES return
+ *    KV_ERR_INVALID_ARGUMENT before anything is enqueued; a larger
+ *    partition_tokens needs less workspace.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.  A failed look-up returns KV_ERR_CUDA.
+ *  - All calls on a device share the one array, which keeps the last call's
+ *    contents: calls that may overlap on the GPU (on different streams, or
+ *    from different host threads without ordering) race and must be
+ *    serialised by the caller.  Each call writes every partial it reads, so
+ *    nothing has to be cleared between calls.
+ */
+KV_API kv_status paged_decode_attention_static_workspace(
+    const kv_pool_desc* pool, void* out, const void* q, kv_dtype q_dtype, const void* k_pool,
+    const void* v_pool, const float* k_scales, const float* v_scales, const int32_t* block_table,
+    int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t max_context_len, float scale, int32_t partition_tokens, int32_t* dev_error,
+    kv_stream_t stream);
+
 /* Static, human-readable name of a status code. */
 KV_API const char* kv_status_string(kv_status status);
 

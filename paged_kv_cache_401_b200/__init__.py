@@ -28,7 +28,9 @@ BLOCK_SIZE = 16
 
 EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
             "paged_decode_default_partition", "paged_decode_workspace_bytes",
-            "paged_decode_attention", "kv_status_string")
+            "paged_decode_attention", "paged_decode_attention_static_workspace",
+            "kv_status_string")
+KV_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 
 class KvError(RuntimeError):
@@ -68,6 +70,9 @@ def _load() -> ctypes.CDLL:
             "paged_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _I32, _P,
                                               _I32, _I32, _I32, ctypes.c_float, _I32, _P, _SZ,
                                               _P, _P]),
+            "paged_decode_attention_static_workspace": (
+                _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
+                       ctypes.c_float, _I32, _P, _P]),
             "kv_status_string": (ctypes.c_char_p, [_I32]),
         }
         for name, (res, args) in sig.items():
@@ -190,4 +195,23 @@ def paged_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
         _ptr(k_scales), _ptr(v_scales), _ptr(block_table), block_table.shape[1],
         _ptr(context_lens), batch, num_q_heads, max_context_len, float(scale),
         partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream)))
+    return out
+
+
+def paged_decode_attention_static_workspace(
+        pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
+        v_pool: torch.Tensor, k_scales: torch.Tensor | None, v_scales: torch.Tensor | None,
+        block_table: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
+        scale: float, partition_tokens: int = 0, dev_error: torch.Tensor | None = None,
+        stream=None) -> torch.Tensor:
+    """paged_decode_attention without a caller workspace (for callers that cannot
+    allocate device memory): the partials live in the library's fixed
+    KV_STATIC_WORKSPACE_BYTES device array, shared by every call on the device."""
+    batch, num_q_heads, _ = q.shape
+    _check("paged_decode_attention_static_workspace",
+           _load().paged_decode_attention_static_workspace(
+               ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool),
+               _ptr(v_pool), _ptr(k_scales), _ptr(v_scales), _ptr(block_table),
+               block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
+               float(scale), partition_tokens, _ptr(dev_error), _stream(stream)))
     return out

@@ -1,0 +1,78 @@
+// paged_decode_attention_static_workspace: the split-K decode for callers that
+// cannot allocate device memory.
+//
+// Some callers have no way to obtain device memory for the split-K workspace:
+// an engine that reserved all of HBM for its KV pool up front (a cudaMalloc would
+// fail, or fragment the pool), a plugin inside another runtime that owns the
+// allocator and hands plugins no allocation hook, or a latency-bound loop that
+// cannot take cudaMalloc's implicit device synchronisation.  For them the
+// partial (max, sum, output) of every sequence partition lives in a fixed array
+// in this library's device image instead of a caller buffer.
+//
+// The array is file-scope device memory: every GPU that loads the library holds
+// KV_STATIC_WORKSPACE_BYTES of it until the process exits, and every call on a
+// device shares it.  Host code cannot use the array's name as a device address
+// (on the host it names a stand-in object), so the device address is looked up
+// once per device with cudaGetSymbolAddress, with that device current, on the
+// first call made on it.
+#include "kernels.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) static uint8_t g_static_workspace[KV_STATIC_WORKSPACE_BYTES];
+
+// Device address of g_static_workspace on each device, filled on first use.
+void* g_workspace_addr[kMaxDevices] = {};
+
+// Returns the array's device address on the current device, or nullptr with *err set.
+void* static_workspace_address(cudaError_t* err) {
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= kMaxDevices) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    if (g_workspace_addr[dev] == nullptr) {  // benign race: every caller finds the same address
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_static_workspace);
+        if (*err != cudaSuccess) return nullptr;
+        g_workspace_addr[dev] = p;
+    }
+    return g_workspace_addr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+KV_API kv_status paged_decode_attention_static_workspace(
+    const kv_pool_desc* pool, void* out, const void* q, kv_dtype q_dtype, const void* k_pool,
+    const void* v_pool, const float* k_scales, const float* v_scales, const int32_t* block_table,
+    int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+    int32_t max_context_len, float scale, int32_t partition_tokens, int32_t* dev_error,
+    kv_stream_t stream) {
+    // size check first, on the host: a request needing more than the array holds is refused
+    const size_t need = paged_decode_workspace_bytes(pool, batch, num_q_heads, max_context_len,
+                                                     partition_tokens);
+    if (need > KV_STATIC_WORKSPACE_BYTES) return KV_ERR_INVALID_ARGUMENT;
+    void* ws = nullptr;
+    if (need > 0) {
+        cudaError_t err = cudaSuccess;
+        ws = static_workspace_address(&err);
+        if (ws == nullptr) {
+            cudaGetLastError();
+            return KV_ERR_CUDA;
+        }
+    }
+    // Every partial the merge reads is written earlier in the same call, so
+    // nothing in the array needs clearing between calls.
+    return paged_decode_attention(pool, out, q, q_dtype, k_pool, v_pool, k_scales, v_scales,
+                                  block_table, max_blocks_per_seq, context_lens, batch,
+                                  num_q_heads, max_context_len, scale, partition_tokens, ws,
+                                  need > 0 ? KV_STATIC_WORKSPACE_BYTES : 0, dev_error, stream);
+}
+
+}  // extern "C"
