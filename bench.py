@@ -14,7 +14,7 @@ value    = KV bytes read per step x steps / device time, inputs resident in HBM;
 e2e      = the same metric through the binding with pinned host buffers: each
            step copies q, the new K/V rows, the block table and context lengths
            host->device and the output device->host inside the timed region;
-roofline = the decode call (split + merge kernels) timed live with CUDA events
+roofline = the decode call (decode + merge kernels) timed live with CUDA events
            on its stream, against the measured HBM copy bandwidth;
 cpu_baseline = the double-precision CPU oracle on a bounded sample (rank 0).
 ``--impl reference`` times that oracle alone as the reference arm.
@@ -164,7 +164,8 @@ def describe(inp, partition: int) -> dict:
             "batch": int(inp.q.shape[0]), "max_context_len": inp.max_context_len,
             "num_q_heads": spec.num_q_heads, "num_kv_heads": spec.num_kv_heads,
             "head_dim": spec.head_dim, "block_size": 16, "num_blocks": inp.num_blocks,
-            "kv_dtype": spec.kv_dtype, "partition_tokens": partition,
+            "kv_dtype": spec.kv_dtype,
+            "partition_tokens": partition if partition else "0 (balanced over all SMs)",
             "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush"
             if kv_bytes_per_step(inp) > 126e6 else "inputs fit in L2, not flushed",
             "parallelism": "replicas: one independent decode per GPU"}
@@ -292,12 +293,11 @@ def run_gpu(args, inp):
     positions = torch.from_numpy(inp.append_positions).to(device)
     slots = torch.empty(B, dtype=torch.int64, device=device)
     out = torch.empty_like(q)
-    P = args.partition or pk.paged_decode_default_partition(cache.desc, B, spec.num_q_heads,
-                                                            inp.max_context_len)
+    P = args.partition
+    ranges = pk.paged_decode_num_ranges(cache.desc, B, spec.num_q_heads, inp.max_context_len, P)
     ws = cache.alloc_workspace(B, spec.num_q_heads, inp.max_context_len, P)
     stream = torch.cuda.current_stream(device)
-    max_parts = -(-inp.max_context_len // P)
-    launches_per_step = 3 + (1 if max_parts > 1 else 0)
+    launches_per_step = 4   # slot mapping, cache write, decode, merge
 
     def append():
         cache.append(bt, seq_ids, positions, k_new, v_new, slots=slots)
@@ -396,14 +396,14 @@ def run_gpu(args, inp):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": spec.kv_dtype if spec.kv_dtype != "fp8" else "fp8_e4m3",
         "data": "synthetic (seeded N(0,1) q/K/V, random block permutation)",
-        "config": describe(inp, P),
+        "config": dict(describe(inp, P), num_ranges=ranges),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(max_e2e_ms / args.steps, 5)},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
                      "traffic": profiled_traffic(), "kernel": "paged_decode_attention "
-                     "(split + merge kernels, one call)", "peak_kind": peak_kind,
+                     "(decode + merge kernels, one call)", "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": nbytes,
                      "ms_per_launch": round(max_decode_ms, 5)},
         "cpu_baseline": cpu,
@@ -420,7 +420,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="llama", choices=sorted(WORKLOADS))
-    ap.add_argument("--partition", type=int, default=0, help="split-K partition (0 = library)")
+    ap.add_argument("--partition", type=int, default=0,
+                    help="max tokens per consumer range (0 = balanced over all SMs)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--reference-seqs", type=int, default=8,
                     help="sequences in the oracle's bounded sample")

@@ -144,22 +144,31 @@ KV_API kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void*
                             int32_t* dev_error, kv_stream_t stream);
 
 /*
- * Sequence-partition (split-K) size the library uses when
- * paged_decode_attention is given partition_tokens == 0: a multiple of 16
- * chosen from the batch, the longest context and the SM count of the current
- * device (148 when no device can be queried).  Host only.
+ * Number of consumer ranges the decode cuts its work into (host only).
+ * The decode lays the (sequence, kv head) pairs end to end as one list of
+ * 16-token tiles and cuts it into this many equal contiguous ranges, one per
+ * consumer warp.  partition_tokens == 0: as many ranges as the current
+ * device runs consumer warps at once (148 SMs assumed when no device can be
+ * queried), so every SM streams the same number of bytes; partition_tokens >
+ * 0 (a multiple of 16): ranges of at most that many tokens over the longest
+ * possible list (batch * kv heads * ceil(max_context_len / 16) tiles).
+ * Returns 0 for invalid arguments.
  */
-KV_API int32_t paged_decode_default_partition(const kv_pool_desc* pool, int32_t batch,
-                                       int32_t num_q_heads, int32_t max_context_len);
+KV_API int32_t paged_decode_num_ranges(const kv_pool_desc* pool, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_context_len,
+                                       int32_t partition_tokens);
 
 /*
  * Bytes of device workspace paged_decode_attention needs for these sizes
- * (partial maxima, sums and outputs of every sequence partition).  Host only;
- * partition_tokens as for paged_decode_attention.  0 means none is needed.
+ * (host only; partition_tokens as above; 0 for invalid arguments):
+ * (batch + 1) int32 sequence starts, then, for each of
+ * batch * num_kv_heads + num_ranges pieces, the partial (max, sum) and
+ * head_dim-wide partial output of every query head of the group.  Its
+ * contents need no initialisation.
  */
 KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
-                                    int32_t num_q_heads, int32_t max_context_len,
-                                    int32_t partition_tokens);
+                                           int32_t num_q_heads, int32_t max_context_len,
+                                           int32_t partition_tokens);
 
 /*
  * Single-token GQA decode attention over the paged cache ("KV Cache 深度解析"
@@ -169,9 +178,10 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  * physical block block_table[b][p / 16], slot p % 16):
  *     s_p = scale * q[b,h,:] . K_p[g,:]
  *     out[b,h,:] = sum_p softmax(s)_p * V_p[g,:]
- * computed exactly up to fp32 rounding with an online softmax; the sequence
- * is cut into partitions of partition_tokens tokens (0 = library default),
- * each partition's (max, sum, output) is merged by log-sum-exp.
+ * computed exactly up to fp32 rounding with an online softmax.  The
+ * (sequence, kv head) pairs are split over paged_decode_num_ranges(...)
+ * consumer ranges; a pair split over several ranges has its pieces' (max,
+ * sum, output) merged by log-sum-exp in a second kernel.
  *   out          : device [batch][num_q_heads][head_dim] in q_dtype
  *   q            : device [batch][num_q_heads][head_dim], q_dtype F32 or BF16
  *   k_pool/v_pool: device pools (layout above)
@@ -180,12 +190,14 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  *                  ceil(L/16) are never read
  *   context_lens : device int32 [batch], each in [1, max_context_len]
  *   max_context_len : upper bound of context_lens, <= max_blocks_per_seq*16
+ *   partition_tokens : 0 (balanced over the GPU) or a multiple of 16, see
+ *                  paged_decode_num_ranges
  *   workspace    : device buffer of >= paged_decode_workspace_bytes(...) bytes
- *                  (may be NULL when that size is 0)
  * Host checks: num_q_heads % num_kv_heads == 0 with a group size of 1, 2, 4
  * or 8 (else KV_ERR_UNSUPPORTED); partition_tokens a multiple of 16;
- * max_context_len <= max_blocks_per_seq * 16; pointer alignment; workspace
- * size.  Device errors: KV_DEVERR_BAD_CONTEXT_LEN (that sequence's output is
+ * max_context_len <= max_blocks_per_seq * 16; batch * num_kv_heads *
+ * ceil(max_context_len / 16) < 2^31 (else KV_ERR_UNSUPPORTED); pointer
+ * alignment; workspace size.  Device errors: KV_DEVERR_BAD_CONTEXT_LEN (that sequence's output is
  * zero), KV_DEVERR_BAD_BLOCK_ID (that block's tokens are skipped),
  * KV_DEVERR_TIMEOUT.
  */
@@ -201,8 +213,9 @@ KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, con
 
 /*
  * Bytes of device memory the library holds on every GPU that loads it, for
- * paged_decode_attention_static_workspace (16 MiB: enough for the partials
- * of e.g. 32 sequences x 32 query heads x 64 partitions of 128-wide heads).
+ * paged_decode_attention_static_workspace (16 MiB: enough for the default
+ * split of e.g. 256 sequences x 8 kv heads x 4 query heads per group at
+ * head_dim 128 on a 148-SM GPU, about 8 MB).
  */
 #define KV_STATIC_WORKSPACE_BYTES (16u * 1024u * 1024u)
 

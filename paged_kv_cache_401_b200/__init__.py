@@ -27,7 +27,7 @@ KV_DEVERR_BAD_POSITION = 0x10
 BLOCK_SIZE = 16
 
 EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
-            "paged_decode_default_partition", "paged_decode_workspace_bytes",
+            "paged_decode_num_ranges", "paged_decode_workspace_bytes",
             "paged_decode_attention", "paged_decode_attention_static_workspace",
             "kv_status_string")
 KV_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
@@ -65,7 +65,7 @@ def _load() -> ctypes.CDLL:
             "kv_pool_create": (_I32, [_I32, _I32, _I32, _I32, _I32, desc_p]),
             "compute_slot_mapping": (_I32, [_P, _I32, _I32, _I32, _P, _P, _I32, _P, _P, _P]),
             "reshape_and_cache": (_I32, [desc_p, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
-            "paged_decode_default_partition": (_I32, [desc_p, _I32, _I32, _I32]),
+            "paged_decode_num_ranges": (_I32, [desc_p, _I32, _I32, _I32, _I32]),
             "paged_decode_workspace_bytes": (_SZ, [desc_p, _I32, _I32, _I32, _I32]),
             "paged_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _I32, _P,
                                               _I32, _I32, _I32, ctypes.c_float, _I32, _P, _SZ,
@@ -169,10 +169,10 @@ def reshape_and_cache(pool: KvPoolDesc, k_pool: torch.Tensor, v_pool: torch.Tens
         _ptr(dev_error), _stream(stream)))
 
 
-def paged_decode_default_partition(pool: KvPoolDesc, batch: int, num_q_heads: int,
-                                   max_context_len: int) -> int:
-    return int(_load().paged_decode_default_partition(ctypes.byref(pool), batch, num_q_heads,
-                                                      max_context_len))
+def paged_decode_num_ranges(pool: KvPoolDesc, batch: int, num_q_heads: int,
+                            max_context_len: int, partition_tokens: int = 0) -> int:
+    return int(_load().paged_decode_num_ranges(ctypes.byref(pool), batch, num_q_heads,
+                                               max_context_len, partition_tokens))
 
 
 def paged_decode_workspace_bytes(pool: KvPoolDesc, batch: int, num_q_heads: int,

@@ -1,5 +1,6 @@
 // C ABI of libpagedkv.so (declared in include/paged_kv.h): host-side argument
-// checks, geometry, the split-K partition heuristic and kernel launches.
+// checks, geometry, the split of the tile list into consumer ranges, the
+// workspace layout and kernel launches.
 #include <cmath>
 
 #include "kernels.cuh"
@@ -114,34 +115,51 @@ kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
-int32_t paged_decode_default_partition(const kv_pool_desc* pool, int32_t batch,
-                                       int32_t num_q_heads, int32_t max_context_len) {
-    (void)num_q_heads;
-    if (!valid_pool(pool) || batch <= 0 || max_context_len <= 0) return 512;
-    // Enough thread blocks for several waves over the SMs (a decode block keeps
-    // 32-64 KB of tiles in flight; ~3 fit per SM), each partition long enough
-    // that its partial (m, l, o) write stays a few percent of the KV it reads.
-    const int64_t pairs = static_cast<int64_t>(batch) * pool->num_kv_heads;
-    const int64_t want = 8ll * current_sm_count() * 3;
-    int32_t P = 1024;
-    while (P > 256 && pairs * ceil_div(max_context_len, P) < want) P /= 2;
-    return P;
+int32_t paged_decode_num_ranges(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
+                                int32_t max_context_len, int32_t partition_tokens) {
+    if (!valid_pool(pool) || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0 ||
+        num_q_heads % pool->num_kv_heads != 0 || partition_tokens < 0 ||
+        partition_tokens % kBlockTokens != 0)
+        return 0;
+    const int32_t group = num_q_heads / pool->num_kv_heads;
+    if (partition_tokens == 0) {
+        // persistent: one range per consumer warp of every CTA the GPU holds at once
+        return current_sm_count() * pkv::decode_ctas_per_sm(pool->dtype, pool->head_dim, group) * 4;
+    }
+    // ranges of at most partition_tokens tokens over the largest possible tile list
+    const int64_t max_tiles = static_cast<int64_t>(batch) * pool->num_kv_heads *
+                              ceil_div(max_context_len, kBlockTokens);
+    const int64_t per = partition_tokens / kBlockTokens;
+    const int64_t n = (max_tiles + per - 1) / per;
+    return static_cast<int32_t>(n < 1 ? 1 : (n > (1 << 28) ? (1 << 28) : n));
 }
+
+namespace {
+// Workspace layout: [B + 1] int32 sequence starts | [pieces][G] float2 (m, l) |
+// [pieces][G][D] float partial outputs; pieces = B * Hkv + num_ranges.
+struct WsLayout {
+    size_t ml_off, o_off, total;
+};
+WsLayout ws_layout(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
+                   int32_t num_ranges) {
+    auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t group = static_cast<size_t>(num_q_heads / pool->num_kv_heads);
+    const size_t pieces = static_cast<size_t>(batch) * pool->num_kv_heads + num_ranges;
+    WsLayout w{};
+    w.ml_off = up(sizeof(int32_t) * (static_cast<size_t>(batch) + 1));
+    w.o_off = w.ml_off + up(pieces * group * sizeof(float2));
+    w.total = w.o_off + pieces * group * pool->head_dim * sizeof(float);
+    return w;
+}
+}  // namespace
 
 size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
                                     int32_t num_q_heads, int32_t max_context_len,
                                     int32_t partition_tokens) {
-    if (!valid_pool(pool) || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0) return 0;
-    const int32_t P = partition_tokens > 0
-                          ? partition_tokens
-                          : paged_decode_default_partition(pool, batch, num_q_heads,
-                                                           max_context_len);
-    const int32_t parts = ceil_div(max_context_len, P);
-    if (parts <= 1) return 0;
-    const size_t rows = static_cast<size_t>(batch) * num_q_heads * parts;
-    size_t ml = rows * sizeof(float2);
-    ml = (ml + 255) & ~static_cast<size_t>(255);
-    return ml + rows * pool->head_dim * sizeof(float);
+    const int32_t ranges =
+        paged_decode_num_ranges(pool, batch, num_q_heads, max_context_len, partition_tokens);
+    if (ranges <= 0) return 0;
+    return ws_layout(pool, batch, num_q_heads, ranges).total;
 }
 
 kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
@@ -163,8 +181,12 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     if (max_context_len <= 0 ||
         static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens)
         return KV_ERR_INVALID_ARGUMENT;
-    if (partition_tokens < 0 || partition_tokens % kBlockTokens != 0 || partition_tokens > 8192)
+    if (partition_tokens < 0 || partition_tokens % kBlockTokens != 0)
         return KV_ERR_INVALID_ARGUMENT;
+    // the tile list (and its int32 per-sequence starts) must stay below 2^31 tiles
+    if (static_cast<int64_t>(batch) * pool->num_kv_heads *
+            ceil_div(max_context_len, kBlockTokens) >= (int64_t{1} << 31))
+        return KV_ERR_UNSUPPORTED;
     if (!std::isfinite(scale)) return KV_ERR_INVALID_ARGUMENT;
     if (out == nullptr || q == nullptr || k_pool == nullptr || v_pool == nullptr ||
         block_table == nullptr || context_lens == nullptr)
@@ -176,13 +198,11 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
         return KV_ERR_INVALID_ARGUMENT;
     if (fp8 && (!aligned16(k_scales) || !aligned16(v_scales))) return KV_ERR_INVALID_ARGUMENT;
 
-    const int32_t P = partition_tokens > 0
-                          ? partition_tokens
-                          : paged_decode_default_partition(pool, batch, num_q_heads,
-                                                           max_context_len);
-    const size_t need =
-        paged_decode_workspace_bytes(pool, batch, num_q_heads, max_context_len, P);
-    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace)))
+    const int32_t ranges =
+        paged_decode_num_ranges(pool, batch, num_q_heads, max_context_len, partition_tokens);
+    if (ranges <= 0) return KV_ERR_INVALID_ARGUMENT;
+    const WsLayout wl = ws_layout(pool, batch, num_q_heads, ranges);
+    if (workspace == nullptr || workspace_bytes < wl.total || !aligned16(workspace))
         return KV_ERR_INVALID_ARGUMENT;
 
     pkv::DecodeParams p{};
@@ -201,15 +221,12 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     p.num_blocks = pool->num_blocks;
     p.max_blocks = max_blocks_per_seq;
     p.max_context_len = max_context_len;
-    p.partition_tokens = P;
-    p.max_parts = ceil_div(max_context_len, P);
+    p.num_ranges = ranges;
     p.scale_log2 = scale * 1.4426950408889634f;
-    if (need > 0) {
-        const size_t rows = static_cast<size_t>(batch) * num_q_heads * p.max_parts;
-        size_t ml = (rows * sizeof(float2) + 255) & ~static_cast<size_t>(255);
-        p.ws_ml = static_cast<float2*>(workspace);
-        p.ws_o = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + ml);
-    }
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    p.ws_seq_start = reinterpret_cast<int32_t*>(ws);
+    p.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
+    p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
     cudaError_t e = pkv::launch_paged_decode(p, pool->dtype, q_dtype, pool->head_dim, group,
                                              reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;

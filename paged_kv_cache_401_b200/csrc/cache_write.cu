@@ -13,6 +13,8 @@ __global__ void slot_mapping_kernel(const int32_t* __restrict__ block_table, int
                                     int32_t max_blocks, const int32_t* __restrict__ seq_ids,
                                     const int32_t* __restrict__ positions, int32_t num_tokens,
                                     int64_t* __restrict__ slots, int32_t* dev_error) {
+    pdl_wait();
+    pdl_trigger();
     const int32_t i = blockIdx.x * blockDim.x + threadIdx.x;
     if (i >= num_tokens) return;
     const int32_t s = seq_ids[i];
@@ -33,6 +35,8 @@ __global__ void cache_copy_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restr
                                   const int64_t* __restrict__ slots, int32_t num_tokens,
                                   int32_t num_kv_heads, int32_t row_bytes, int64_t num_slots,
                                   int32_t* dev_error) {
+    pdl_wait();
+    pdl_trigger();
     const int32_t vecs_per_row = row_bytes / 16;
     const int64_t per_token = static_cast<int64_t>(num_kv_heads) * vecs_per_row;
     const int64_t total = per_token * num_tokens;
@@ -68,6 +72,8 @@ __global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restri
                                  const int64_t* __restrict__ slots, int32_t num_tokens,
                                  int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error) {
     constexpr int kPer = D / 32;  // elements per lane (4 or 2)
+    pdl_wait();
+    pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
     const int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
     const int64_t rows = 2ll * num_tokens * num_kv_heads;
@@ -124,9 +130,8 @@ cudaError_t launch_slot_mapping(const int32_t* block_table, int32_t batch, int32
                                 cudaStream_t stream) {
     const int threads = 256;
     const int blocks = (num_tokens + threads - 1) / threads;
-    slot_mapping_kernel<<<blocks, threads, 0, stream>>>(block_table, batch, max_blocks, seq_ids,
-                                                        positions, num_tokens, slots, dev_error);
-    return cudaGetLastError();
+    return launch_pdl(slot_mapping_kernel, dim3(blocks), dim3(threads), 0, stream, block_table,
+                      batch, max_blocks, seq_ids, positions, num_tokens, slots, dev_error);
 }
 
 cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, const void* v_new,
@@ -138,11 +143,10 @@ cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, con
     int64_t blocks = (vecs + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
-    cache_copy_kernel<<<static_cast<unsigned>(blocks), threads, 0, stream>>>(
-        static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool),
-        static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new), slots,
-        num_tokens, num_kv_heads, row_bytes, num_slots, dev_error);
-    return cudaGetLastError();
+    return launch_pdl(cache_copy_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+                      stream, static_cast<uint8_t*>(k_pool), static_cast<uint8_t*>(v_pool),
+                      static_cast<const uint8_t*>(k_new), static_cast<const uint8_t*>(v_new),
+                      slots, num_tokens, num_kv_heads, row_bytes, num_slots, dev_error);
 }
 
 cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, void* v_pool,
@@ -155,16 +159,15 @@ cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, 
     const int64_t blocks = (rows * 32 + threads - 1) / threads;
     auto* kp = static_cast<uint8_t*>(k_pool);
     auto* vp = static_cast<uint8_t*>(v_pool);
-#define PKV_FP8_LAUNCH(ST, DD)                                                               \
-    cache_fp8_kernel<ST, DD><<<static_cast<unsigned>(blocks), threads, 0, stream>>>(         \
-        kp, vp, k_scales, v_scales, k_new, v_new, slots, num_tokens, num_kv_heads, num_slots, \
-        dev_error)
-    if (src_dtype == KV_F32 && head_dim == 128) PKV_FP8_LAUNCH(KV_F32, 128);
-    else if (src_dtype == KV_F32 && head_dim == 64) PKV_FP8_LAUNCH(KV_F32, 64);
-    else if (src_dtype == KV_BF16 && head_dim == 128) PKV_FP8_LAUNCH(KV_BF16, 128);
-    else PKV_FP8_LAUNCH(KV_BF16, 64);
-#undef PKV_FP8_LAUNCH
-    return cudaGetLastError();
+    auto go = [&](auto kernel) {
+        return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
+                          kp, vp, k_scales, v_scales, k_new, v_new, slots, num_tokens,
+                          num_kv_heads, num_slots, dev_error);
+    };
+    if (src_dtype == KV_F32 && head_dim == 128) return go(cache_fp8_kernel<KV_F32, 128>);
+    if (src_dtype == KV_F32 && head_dim == 64) return go(cache_fp8_kernel<KV_F32, 64>);
+    if (src_dtype == KV_BF16 && head_dim == 128) return go(cache_fp8_kernel<KV_BF16, 128>);
+    return go(cache_fp8_kernel<KV_BF16, 64>);
 }
 
 }  // namespace pkv

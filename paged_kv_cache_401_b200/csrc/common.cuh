@@ -82,6 +82,17 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
         : "memory");
 }
 
+// ---- programmatic dependent launch -------------------------------------------
+// Every kernel of the library waits for the grid before it in the stream to
+// finish (and its writes to be visible) before touching global memory, then
+// lets the next grid start launching: with the launch attribute set, a
+// kernel's launch and prologue overlap its predecessor's tail; without it both
+// instructions are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- error word --------------------------------------------------------------
 __device__ __forceinline__ void report(int32_t* dev_error, int32_t bits) {
     if (dev_error != nullptr) atomicOr(dev_error, bits);

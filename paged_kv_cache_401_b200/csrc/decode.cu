@@ -1,27 +1,40 @@
-// Split-K paged GQA decode attention and its log-sum-exp merge (sm_100a).
+// Paged GQA decode attention: persistent split-K ("stream-K") kernel and its
+// log-sum-exp merge (sm_100a).
 //
 // Method ("KV Cache 深度解析" §一/§三/§四; "llm-inference-optimization" notes
-// §三 Flash Attention; k1-blog 2026-07-13, "PagedAttention 與 vLLM"):
-// one thread block per (sequence partition, kv head, sequence).  Its tokens are
-// read once from HBM, block by block through the block table, and shared by
-// the G query heads of the GQA group.  A running max m, running sum l and
-// rescaled running output o per query head implement the online softmax, so
-// no score ever leaves the chip.  Partitions of one sequence are combined by
-// their log-sum-exp in a second, small kernel.
+// §三 Flash Attention; k1-blog 2026-07-13, "PagedAttention 與 vLLM"): for each
+// sequence b and kv head g, the G query heads of the group attend to the
+// L_b cached tokens, read block by block through the block table, with an
+// online softmax (running max m, running sum l, rescaled running output o)
+// so no score leaves the chip.  Partial (m, l, o) of pieces of one sequence
+// are combined by their log-sum-exp.
+//
+// Work decomposition.  The (sequence, kv head) pairs are laid end to end as
+// one list of 16-token tiles, T tiles in all (a pair with L tokens has
+// ceil(L/16)).  The list is cut into num_ranges equal contiguous ranges, one
+// per consumer warp: every warp streams the same number of bytes whatever
+// the mix of context lengths, so ragged batches and a handful of very long
+// sequences keep every SM busy.  A warp's range may start or end inside a
+// pair; such a "piece" writes its (m, l, o) to the workspace and the merge
+// kernel combines the pieces of each pair.  A pair entirely inside one range
+// is finished by its warp, which writes the output directly.
 //
 // B200 design:
-//  * one producer warp stages each (block, kv head) K and V tile (a contiguous
-//    16*D-element span in the pool) into shared memory with 1-D bulk async
-//    copies (the TMA engine, no multicast) completing on mbarriers, through a
-//    ring of kStages stages;
-//  * four consumer warps take the ring's tiles round-robin, each keeping its
-//    own (m, l, o), and are combined through shared memory at the end;
-//  * q·K: every lane multiplies 16-byte chunks of 8 lanes-per-row against q
-//    held in registers with packed fp32x2 FMAs, then a shuffle reduce-scatter
-//    leaves each score on one lane; P·V: every lane owns D/32 output columns;
-//  * scores are in base-2 units (q pre-scaled by scale*log2 e) and exp2 is used.
-// Every wait is bounded; bad block ids and context lengths are reported through
-// the error word and never dereferenced.
+//  * a CTA is one producer warp and four consumer warps; by default the grid
+//    is exactly the number of CTAs resident on the GPU (persistent), so the
+//    tile stream never stalls between work items;
+//  * the producer's lane 0 walks the four consumer warps' ranges and stages
+//    each (block, kv head) K and V tile -- one contiguous 16*D span of the
+//    pool -- into a shared-memory ring with 1-D bulk async copies (the TMA
+//    engine, no multicast) completing on mbarriers; block ids are fetched 8
+//    tiles ahead so table-lookup latency never gaps the stream;
+//  * stage s of the ring always feeds consumer warp s % 4; a consumer warp
+//    computes q.K with packed fp32x2 FMAs on 16-byte chunks (8 lanes per
+//    row) and a shuffle reduce-scatter, the online softmax with exp2 on
+//    scores pre-scaled by scale*log2(e), and P.V with each lane owning D/32
+//    output columns, all in fp32;
+//  * every wait is bounded; bad block ids and context lengths are reported
+//    through the error word and never dereferenced.
 #include "kernels.cuh"
 
 namespace pkv {
@@ -62,22 +75,21 @@ struct Cfg {
     static constexpr int kDPL = D / 32;                                      // output cols per lane
     static constexpr int kSMLanes = (kBlockTokens * G) < 32 ? kBlockTokens * G : 32;
     static constexpr int kSPL = kBlockTokens * G / kSMLanes;                 // softmax vals/lane
-    // shared memory
+    // shared memory: the ring, per-consumer-warp scratch, per-stage flags, barriers
     static constexpr int kRingBytes = kStages * kStageBytes;
-    static constexpr int kEpiBytes = kConsumerWarps * G * (D * 4 + 8);
-    static constexpr int kBodyBytes = kRingBytes > kEpiBytes ? kRingBytes : kEpiBytes;
     // per consumer warp: p pairs [16][G] float2, scores [16][G], corrections [G];
     // rounded to 16 bytes so every warp's region (and its float2 array) is aligned
-    static constexpr int kWarpScratch = (kBlockTokens * G * 8 + kBlockTokens * G * 4 + G * 4 + 15) / 16 * 16;
-    static constexpr int kMaxIds = 512;                                      // partition <= 8192
+    static constexpr int kWarpScratch =
+        (kBlockTokens * G * 8 + kBlockTokens * G * 4 + G * 4 + 15) / 16 * 16;
+    static constexpr int kFlagsBytes = (2 * kStages * 4 + 16 + 15) / 16 * 16;  // ok, issued, abort
     static constexpr int kSmemBytes =
-        kBodyBytes + kConsumerWarps * kWarpScratch + kMaxIds * 4 + 2 * kStages * 8 + 16;
+        kRingBytes + kConsumerWarps * kWarpScratch + kFlagsBytes + 2 * kStages * 8;
     // resident blocks per SM the register budget is sized for (G = 8 needs the
     // whole register file of one block's worth of q and accumulators)
     static constexpr int kMinBlocks = G >= 8 ? 1 : 3;
-    static_assert(kStages % kConsumerWarps == 0, "stage ring must split evenly across warps");
-    static_assert(kStageBytes % 16 == 0 && kBodyBytes % 16 == 0, "bulk copies need 16-B alignment");
-    static_assert((kBodyBytes + kConsumerWarps * kWarpScratch + kMaxIds * 4) % 8 == 0,
+    static_assert(kStages % kConsumerWarps == 0, "stage s feeds consumer warp s % 4");
+    static_assert(kStageBytes % 16 == 0 && kRingBytes % 16 == 0, "bulk copies need 16-B alignment");
+    static_assert((kRingBytes + kConsumerWarps * kWarpScratch + kFlagsBytes) % 8 == 0,
                   "mbarriers need 8-B alignment");
     static_assert(kQPL % 2 == 0 && kDPL % 2 == 0, "pairs for fp32x2 FMA");
 };
@@ -190,77 +202,246 @@ __device__ __forceinline__ float load_q(const void* q, int64_t i) {
     }
 }
 
+
+// ---- tile list bookkeeping ----------------------------------------------------------
+// Tiles of a sequence with context length L: ceil(L/16), or 0 when L is invalid.
+__device__ __forceinline__ int32_t seq_tiles(int32_t L, int32_t max_context_len) {
+    return (L >= 1 && L <= max_context_len) ? (L + kBlockTokens - 1) / kBlockTokens : 0;
+}
+
+// First tile of consumer range W (ranges are equal cuts of the T-tile list).
+__device__ __forceinline__ int64_t range_begin(int64_t W, int64_t T, int32_t num_ranges) {
+    return W >= num_ranges ? T : (W * T) / num_ranges;
+}
+
+// The range holding tile x < T: the largest W with range_begin(W) <= x, i.e.
+// the largest W with W*T < (x+1)*num_ranges.
+__device__ __forceinline__ int64_t range_of(int64_t x, int64_t T, int32_t num_ranges) {
+    const int64_t W = ((x + 1) * num_ranges - 1) / T;
+    return W < num_ranges - 1 ? W : num_ranges - 1;
+}
+
+__device__ __forceinline__ int64_t warp_sum_i64(int64_t x) {
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
+
+// Total tiles T over the batch (computed by every warp that needs it).
+__device__ int64_t total_tiles(const DecodeParams& p, int lane) {
+    int64_t t = 0;
+    for (int b = lane; b < p.batch; b += 32)
+        t += static_cast<int64_t>(p.num_kv_heads) * seq_tiles(p.context_lens[b], p.max_context_len);
+    return warp_sum_i64(t);
+}
+
+// Position of one tile in the list: sequence b, kv head, block index jb in
+// the sequence, the sequence's tile count nt and length L, and the list
+// index of the pair's first tile.
+struct Cursor {
+    int32_t b, kvh, jb, nt, L;
+    int64_t seg_start;
+};
+
+// Warp-cooperative search for the pair holding tile x (< T).  When `prefix`
+// is non-null the warp also writes every sequence's first tile (and T at
+// [batch]) there for the merge kernel.
+__device__ Cursor locate_tile(const DecodeParams& p, int64_t x, int lane, int32_t* prefix,
+                              int64_t T) {
+    Cursor c{p.batch, 0, 0, 0, 0, T};
+    bool found = false;
+    int64_t base = 0;
+    for (int b0 = 0; b0 < p.batch; b0 += 32) {
+        const int b = b0 + lane;
+        const int32_t L = b < p.batch ? p.context_lens[b] : 0;
+        const int32_t nt = b < p.batch ? seq_tiles(L, p.max_context_len) : 0;
+        const int64_t cnt = static_cast<int64_t>(p.num_kv_heads) * nt;
+        int64_t incl = cnt;
+#pragma unroll
+        for (int m = 1; m < 32; m <<= 1) {
+            const int64_t y = __shfl_up_sync(0xffffffffu, incl, m);
+            if (lane >= m) incl += y;
+        }
+        const int64_t excl = base + incl - cnt;
+        if (prefix != nullptr && b < p.batch) prefix[b] = static_cast<int32_t>(excl);
+        const uint32_t hit = __ballot_sync(0xffffffffu, !found && cnt > 0 && x >= excl && x < excl + cnt);
+        if (hit != 0u && !found) {
+            const int src = __ffs(hit) - 1;
+            const int64_t e = __shfl_sync(0xffffffffu, excl, src);
+            const int32_t n = __shfl_sync(0xffffffffu, nt, src);
+            const int32_t l = __shfl_sync(0xffffffffu, L, src);
+            const int64_t off = x - e;
+            c.b = b0 + src;
+            c.nt = n;
+            c.L = l;
+            c.kvh = static_cast<int32_t>(off / n);
+            c.jb = static_cast<int32_t>(off % n);
+            c.seg_start = e + static_cast<int64_t>(c.kvh) * n;
+            found = true;
+            if (prefix == nullptr) break;
+        }
+        base += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (prefix != nullptr && lane == 0) prefix[p.batch] = static_cast<int32_t>(T);
+    return c;
+}
+
+// Move a cursor to the next tile of the list (single thread or warp-uniform).
+__device__ __forceinline__ void advance(Cursor& c, const DecodeParams& p) {
+    if (++c.jb < c.nt) return;
+    c.seg_start += c.nt;
+    c.jb = 0;
+    if (++c.kvh < p.num_kv_heads) return;
+    c.kvh = 0;
+    do {
+        ++c.b;
+        c.L = c.b < p.batch ? p.context_lens[c.b] : 0;
+        c.nt = c.b < p.batch ? seq_tiles(c.L, p.max_context_len) : 0;
+    } while (c.b < p.batch && c.nt == 0);
+}
+
 // ======================================================================================
-// Split kernel: grid (max_parts, Hkv, B), kThreads threads.
+// Decode kernel: grid ceil(num_ranges / 4) CTAs of kThreads threads.
 // ======================================================================================
 template <int KV_T, int Q_T, int D, int G>
 __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kMinBlocks)
-    paged_decode_split_kernel(const DecodeParams p) {
+    paged_decode_kernel(const DecodeParams p) {
     using C = Cfg<KV_T, D, G>;
     using OutT = typename QType<Q_T>::T;
     extern __shared__ __align__(128) uint8_t smem[];
 
-    const int32_t part = blockIdx.x;
-    const int32_t kvh = blockIdx.y;
-    const int32_t b = blockIdx.z;
     const int32_t warp = threadIdx.x >> 5;
     const int32_t lane = threadIdx.x & 31;
-    const int32_t L = p.context_lens[b];
-    const int32_t hq0 = kvh * G;  // first query head of the group
-
-    if (L < 1 || L > p.max_context_len) {
-        // invalid length: the first partition writes zeros and reports
-        if (part == 0) {
-            OutT* out = static_cast<OutT*>(p.out);
-            for (int i = threadIdx.x; i < G * D; i += C::kThreads)
-                out[(static_cast<int64_t>(b) * p.num_q_heads + hq0) * D + i] = out_cast<OutT>(0.0f);
-            if (threadIdx.x == 0) report(p.dev_error, KV_DEVERR_BAD_CONTEXT_LEN);
-        }
-        return;
-    }
-    const int32_t P = p.partition_tokens;
-    const int32_t nparts = (L + P - 1) / P;
-    if (part >= nparts) return;
-    const int32_t tok0 = part * P;
-    const int32_t tok1 = min(tok0 + P, L);
-    const int32_t blk0 = tok0 / kBlockTokens;
-    const int32_t nblk = (tok1 - tok0 + kBlockTokens - 1) / kBlockTokens;
-
     uint8_t* ring = smem;
-    uint8_t* scratch = smem + C::kBodyBytes;
-    int32_t* ids = reinterpret_cast<int32_t*>(scratch + C::kConsumerWarps * C::kWarpScratch);
-    uint64_t* full = reinterpret_cast<uint64_t*>(ids + C::kMaxIds);
+    uint8_t* scratch = smem + C::kRingBytes;
+    int32_t* stage_ok = reinterpret_cast<int32_t*>(scratch + C::kConsumerWarps * C::kWarpScratch);
+    int32_t* issued_round = stage_ok + C::kStages;
+    volatile int32_t* abort_flag = issued_round + C::kStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage_ok) + C::kFlagsBytes);
     uint64_t* empty = full + C::kStages;
-    volatile int32_t* abort_flag = reinterpret_cast<volatile int32_t*>(empty + C::kStages);
 
-    // ---- prologue: block ids (producer warp), q (consumer warps), barriers -------
-    float2 q2[G][C::kQPL / 2];
-    const int32_t c = lane % C::kLPR;   // chunk column of this lane
-    const int32_t r0 = lane / C::kLPR;  // first row of this lane
+    pdl_wait();
+    pdl_trigger();
+    const int64_t T = total_tiles(p, lane);
+    const int64_t W0 = static_cast<int64_t>(blockIdx.x) * C::kConsumerWarps;
+
     if (warp == C::kConsumerWarps) {
-        const int32_t* bt = p.block_table + static_cast<int64_t>(b) * p.max_blocks + blk0;
-        for (int k = lane; k < nblk; k += 32) {
-            int32_t id = bt[k];
-            if (id < 0 || id >= p.num_blocks) {
-                report(p.dev_error, KV_DEVERR_BAD_BLOCK_ID);
-                id = -1;
-            }
-            ids[k] = id;
+        // ================= producer warp =================
+        Cursor cur[C::kConsumerWarps];
+        int32_t cnt[C::kConsumerWarps];
+        int32_t kmax = 0;
+#pragma unroll
+        for (int w = 0; w < C::kConsumerWarps; ++w) {
+            const int64_t lo = range_begin(W0 + w, T, p.num_ranges);
+            const int64_t hi = range_begin(W0 + w + 1, T, p.num_ranges);
+            cnt[w] = static_cast<int32_t>(hi - lo);
+            // the first CTA also publishes every sequence's first tile for the merge
+            int32_t* prefix = (blockIdx.x == 0 && w == 0) ? p.ws_seq_start : nullptr;
+            if (cnt[w] > 0 || prefix != nullptr) cur[w] = locate_tile(p, lo, lane, prefix, T);
+            kmax = max(kmax, C::kConsumerWarps * cnt[w]);
         }
         if (lane == 0) {
             for (int s = 0; s < C::kStages; ++s) {
                 mbar_init(&full[s], 1);
                 mbar_init(&empty[s], 1);
+                issued_round[s] = -1;
             }
             *abort_flag = 0;
             mbar_init_fence();
         }
-    } else {
-        const int64_t qbase = (static_cast<int64_t>(b) * p.num_q_heads + hq0) * D;
+        __syncthreads();
+        if (lane != 0) return;
+
+        // slot k feeds consumer warp k % 4 with its (k / 4)-th tile, through
+        // stage k % kStages; block ids are loaded kLook slots ahead
+        constexpr int kLook = 8;
+        int32_t q_id[kLook];
+        int32_t q_head[kLook];
+        bool q_valid[kLook];
+        auto fetch = [&](int k, int i) {
+            const int w = i % C::kConsumerWarps;  // == k % 4: i == k % kLook
+            q_valid[i] = k < kmax && (k / C::kConsumerWarps) < cnt[w];
+            if (q_valid[i]) {
+                const Cursor& c = cur[w];
+                q_id[i] = p.block_table[static_cast<int64_t>(c.b) * p.max_blocks + c.jb];
+                q_head[i] = c.kvh;
+                advance(cur[w], p);
+            }
+        };
 #pragma unroll
-        for (int g = 0; g < G; ++g) {
+        for (int i = 0; i < kLook; ++i) fetch(i, i);
+        const int64_t tile_elems = static_cast<int64_t>(kBlockTokens) * D;
+        for (int k0 = 0; k0 < kmax; k0 += kLook) {
 #pragma unroll
-            for (int k = 0; k < C::kNCH; ++k) {
+            for (int i = 0; i < kLook; ++i) {
+                const int k = k0 + i;
+                if (q_valid[i] && !*abort_flag) {
+                    const int s = k % C::kStages;
+                    const int round = k / C::kStages;
+                    if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
+                        report(p.dev_error, KV_DEVERR_TIMEOUT);
+                        *abort_flag = 1;
+                    } else {
+                        const int32_t id = q_id[i];
+                        const bool ok = id >= 0 && id < p.num_blocks;
+                        stage_ok[s] = ok;
+                        issued_round[s] = round;
+                        if (ok) {
+                            const int64_t tile = static_cast<int64_t>(id) * p.num_kv_heads + q_head[i];
+                            uint8_t* st = ring + s * C::kStageBytes;
+                            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+                            bulk_copy_g2s(st, p.k_pool + tile * tile_elems * C::kElem, C::kTileBytes,
+                                          &full[s]);
+                            bulk_copy_g2s(st + C::kTileBytes, p.v_pool + tile * tile_elems * C::kElem,
+                                          C::kTileBytes, &full[s]);
+                            if constexpr (KV_T == KV_FP8_E4M3) {
+                                bulk_copy_g2s(st + 2 * C::kTileBytes, p.k_scales + tile * kBlockTokens,
+                                              C::kScaleBytes, &full[s]);
+                                bulk_copy_g2s(st + 2 * C::kTileBytes + C::kScaleBytes,
+                                              p.v_scales + tile * kBlockTokens, C::kScaleBytes,
+                                              &full[s]);
+                            }
+                        } else {
+                            report(p.dev_error, KV_DEVERR_BAD_BLOCK_ID);
+                            mbar_arrive(&full[s]);  // nothing to copy: the consumer skips it
+                        }
+                    }
+                }
+                fetch(k + kLook, i);
+            }
+        }
+        if (*abort_flag) {
+            // drain: wait (bounded) until no copy issued by this block is in flight
+            for (int s = 0; s < C::kStages; ++s)
+                if (issued_round[s] >= 0) mbar_wait_bounded(&full[s], issued_round[s] & 1);
+        }
+        return;
+    }
+
+    // ================= consumer warps =================
+    const int64_t W = W0 + warp;
+    const int64_t lo = range_begin(W, T, p.num_ranges);
+    const int32_t n = static_cast<int32_t>(range_begin(W + 1, T, p.num_ranges) - lo);
+    Cursor cur{};
+    if (n > 0) cur = locate_tile(p, lo, lane, nullptr, T);
+    __syncthreads();
+    if (n <= 0) return;
+
+    float2* p_buf = reinterpret_cast<float2*>(scratch + warp * C::kWarpScratch);  // [16][G]
+    float* s_buf = reinterpret_cast<float*>(p_buf + kBlockTokens * G);            // [16][G]
+    float* c_buf = s_buf + kBlockTokens * G;                                       // [G]
+    const int32_t c = lane % C::kLPR;   // chunk column of this lane in a K row
+    const int32_t r0 = lane / C::kLPR;  // first K row of this lane
+    const int32_t sm_lane = lane % C::kSMLanes;
+    const int32_t sm_g = sm_lane % G;   // query head this lane's softmax values belong to
+
+    float2 q2[G][C::kQPL / 2];
+    auto load_q_group = [&]() {
+        const int64_t qbase = (static_cast<int64_t>(cur.b) * p.num_q_heads + cur.kvh * G) * D;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int k = 0; k < C::kNCH; ++k)
 #pragma unroll
                 for (int e = 0; e < C::kChunkElems; e += 2) {
                     const int64_t col = (c + k * C::kLPR) * C::kChunkElems + e;
@@ -268,83 +449,37 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
                         make_float2(load_q<Q_T>(p.q, qbase + g * D + col) * p.scale_log2,
                                     load_q<Q_T>(p.q, qbase + g * D + col + 1) * p.scale_log2);
                 }
-            }
-        }
-    }
-    __syncthreads();
-
-    // ---- producer: stream the partition's tiles through the ring -----------------
-    if (warp == C::kConsumerWarps) {
-        if (lane == 0) {
-            const int64_t tile_elems = static_cast<int64_t>(kBlockTokens) * D;
-            int issued = 0;
-            for (int k = 0; k < nblk; ++k) {
-                const int s = k % C::kStages;
-                const int round = k / C::kStages;
-                if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
-                    report(p.dev_error, KV_DEVERR_TIMEOUT);
-                    *abort_flag = 1;
-                }
-                if (*abort_flag) break;
-                const int32_t id = ids[k];
-                uint8_t* st = ring + s * C::kStageBytes;
-                if (id >= 0) {
-                    const int64_t tile = static_cast<int64_t>(id) * p.num_kv_heads + kvh;
-                    mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                    bulk_copy_g2s(st, p.k_pool + tile * tile_elems * C::kElem, C::kTileBytes,
-                                  &full[s]);
-                    bulk_copy_g2s(st + C::kTileBytes, p.v_pool + tile * tile_elems * C::kElem,
-                                  C::kTileBytes, &full[s]);
-                    if constexpr (KV_T == KV_FP8_E4M3) {
-                        bulk_copy_g2s(st + 2 * C::kTileBytes, p.k_scales + tile * kBlockTokens,
-                                      C::kScaleBytes, &full[s]);
-                        bulk_copy_g2s(st + 2 * C::kTileBytes + C::kScaleBytes,
-                                      p.v_scales + tile * kBlockTokens, C::kScaleBytes,
-                                      &full[s]);
-                    }
-                } else {
-                    mbar_arrive(&full[s]);  // skipped block: nothing to wait for
-                }
-                issued = k + 1;
-            }
-            if (*abort_flag) {
-                // drain: wait (bounded) until no copy issued by this block is in flight
-                for (int k = (issued > C::kStages ? issued - C::kStages : 0); k < issued; ++k)
-                    mbar_wait_bounded(&full[k % C::kStages], (k / C::kStages) & 1);
-            }
-        }
-        return;
-    }
-
-    // ---- consumers ------------------------------------------------------------------
-    float2* p_buf = reinterpret_cast<float2*>(scratch + warp * C::kWarpScratch);  // [16][G]
-    float* s_buf = reinterpret_cast<float*>(p_buf + kBlockTokens * G);            // [16][G]
-    float* c_buf = s_buf + kBlockTokens * G;                                       // [G]
-
-    const int32_t sm_lane = lane % C::kSMLanes;
-    const int32_t sm_g = sm_lane % G;
-    float m_run = -INFINITY;  // running max of this lane's head (base-2 units)
-    float l_run = 0.0f;       // this lane's share of the running sum
+    };
+    float m_run, l_run;
     float2 o2[G][C::kDPL / 2];
+    auto reset = [&]() {
+        m_run = -INFINITY;  // running max of this lane's head (base-2 units)
+        l_run = 0.0f;       // this lane's share of the running sum
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+        for (int g = 0; g < G; ++g)
 #pragma unroll
-        for (int i = 0; i < C::kDPL / 2; ++i) o2[g][i] = make_float2(0.0f, 0.0f);
+            for (int i = 0; i < C::kDPL / 2; ++i) o2[g][i] = make_float2(0.0f, 0.0f);
+    };
+    load_q_group();
+    reset();
+    int64_t piece_start = lo;
 
-    for (int k = warp; k < nblk; k += C::kConsumerWarps) {
+    for (int j = 0; j < n; ++j) {
+        const int k = j * C::kConsumerWarps + warp;
         const int s = k % C::kStages;
-        const bool arrived = __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (k / C::kStages) & 1));
+        const bool arrived =
+            __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (k / C::kStages) & 1));
         if (!arrived) {
             if (lane == 0) report(p.dev_error, KV_DEVERR_TIMEOUT);
             *abort_flag = 1;
         }
-        if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-        if (ids[k] >= 0) {
+        if (__any_sync(0xffffffffu, *abort_flag != 0)) return;  // output invalid (reported)
+        if (stage_ok[s]) {
             const uint8_t* kt = ring + s * C::kStageBytes;
             const uint8_t* vt = kt + C::kTileBytes;
             const float* ksc = reinterpret_cast<const float*>(kt + 2 * C::kTileBytes);
             const float* vsc = ksc + kBlockTokens;
-            const int32_t nvalid = min(kBlockTokens, tok1 - (tok0 + k * kBlockTokens));
+            const int32_t nvalid = min(kBlockTokens, cur.L - cur.jb * kBlockTokens);
 
             // scores: partial dot products over this lane's columns, then reduce-scatter
             float acc[C::kNV];
@@ -380,14 +515,14 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
             }
             __syncwarp();
 
-            // online softmax: lane handles head sm_g, tokens sm_lane/G + j*(kSMLanes/G)
+            // online softmax: lane handles head sm_g, tokens sm_lane/G + i*(kSMLanes/G)
             float sv[C::kSPL];
             float tmax = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < C::kSPL; ++j) {
-                const int t = sm_lane / G + j * (C::kSMLanes / G);
-                sv[j] = (t < nvalid) ? s_buf[t * G + sm_g] : -INFINITY;
-                tmax = fmaxf(tmax, sv[j]);
+            for (int i = 0; i < C::kSPL; ++i) {
+                const int t = sm_lane / G + i * (C::kSMLanes / G);
+                sv[i] = (t < nvalid) ? s_buf[t * G + sm_g] : -INFINITY;
+                tmax = fmaxf(tmax, sv[i]);
             }
 #pragma unroll
             for (int m = G; m < C::kSMLanes; m <<= 1)
@@ -396,9 +531,9 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
             const float corr = exp2f(m_run - m_new);
             l_run *= corr;
 #pragma unroll
-            for (int j = 0; j < C::kSPL; ++j) {
-                const int t = sm_lane / G + j * (C::kSMLanes / G);
-                const float pr = exp2f(sv[j] - m_new);
+            for (int i = 0; i < C::kSPL; ++i) {
+                const int t = sm_lane / G + i * (C::kSMLanes / G);
+                const float pr = exp2f(sv[i] - m_new);
                 l_run += pr;
                 float pv = pr;
                 if constexpr (KV_T == KV_FP8_E4M3) pv *= vsc[t];
@@ -408,7 +543,7 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
             if (lane < G) c_buf[lane] = corr;
             __syncwarp();
 
-            // P·V: this lane's kDPL output columns for every head of the group
+            // P.V: this lane's kDPL output columns for every head of the group
 #pragma unroll
             for (int g = 0; g < G; ++g) {
                 const float cg = c_buf[g];
@@ -443,92 +578,146 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
-    }
 
-    // ---- combine the consumer warps of this block ---------------------------------------
-    // full sum of l over the lanes sharing this lane's head
+        // ---- end of a piece: at the end of a (sequence, kv head) pair or of the range
+        const bool seg_end = cur.jb + 1 == cur.nt;
+        if (seg_end || j == n - 1) {
+            float l = l_run;  // sum of l over the lanes that share this lane's head
 #pragma unroll
-    for (int m = G; m < C::kSMLanes; m <<= 1) l_run += __shfl_xor_sync(0xffffffffu, l_run, m);
-    asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
-    if (*abort_flag) return;  // output invalid, reported as KV_DEVERR_TIMEOUT
-    float* wo = reinterpret_cast<float*>(ring);                                  // [W][G][D]
-    float2* wml = reinterpret_cast<float2*>(ring + C::kConsumerWarps * G * D * 4);  // [W][G]
-    if (lane < G) wml[warp * G + lane] = make_float2(m_run, l_run);
+            for (int m = G; m < C::kSMLanes; m <<= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
+            const int64_t bh0 = static_cast<int64_t>(cur.b) * p.num_q_heads + cur.kvh * G;
+            if (seg_end && piece_start == cur.seg_start) {
+                // the whole pair was this warp's: write the output
 #pragma unroll
-    for (int g = 0; g < G; ++g)
+                for (int g = 0; g < G; ++g) {
+                    const float lg = __shfl_sync(0xffffffffu, l, g);
+                    OutT* o = static_cast<OutT*>(p.out) + (bh0 + g) * D + lane * C::kDPL;
 #pragma unroll
-        for (int i = 0; i < C::kDPL / 2; ++i)
-            *reinterpret_cast<float2*>(&wo[(warp * G + g) * D + lane * C::kDPL + 2 * i]) = o2[g][i];
-    asm volatile("bar.sync 1, %0;" ::"n"(C::kConsumerWarps * 32) : "memory");
-
-    const int32_t tid = threadIdx.x;  // 0 .. 127
-    for (int idx = tid; idx < G * D; idx += C::kConsumerWarps * 32) {
-        const int g = idx / D, d = idx % D;
-        float M = -INFINITY;
+                    for (int i = 0; i < C::kDPL / 2; ++i) {
+                        o[2 * i] = out_cast<OutT>(lg > 0.0f ? o2[g][i].x / lg : 0.0f);
+                        o[2 * i + 1] = out_cast<OutT>(lg > 0.0f ? o2[g][i].y / lg : 0.0f);
+                    }
+                }
+            } else {
+                // a piece of the pair: partial (m, l, o) for the merge kernel
+                const int64_t pid = static_cast<int64_t>(cur.b) * p.num_kv_heads + cur.kvh + W;
+                if (lane < G) p.ws_ml[pid * G + lane] = make_float2(m_run, l);
 #pragma unroll
-        for (int w = 0; w < C::kConsumerWarps; ++w) M = fmaxf(M, wml[w * G + g].x);
-        float o = 0.0f, l = 0.0f;
-        if (M != -INFINITY) {
+                for (int g = 0; g < G; ++g)
 #pragma unroll
-            for (int w = 0; w < C::kConsumerWarps; ++w) {
-                const float2 ml = wml[w * G + g];
-                const float f = exp2f(ml.x - M);
-                o += f * wo[(w * G + g) * D + d];
-                l += f * ml.y;
+                    for (int i = 0; i < C::kDPL / 2; ++i)
+                        *reinterpret_cast<float2*>(&p.ws_o[(pid * G + g) * D + lane * C::kDPL + 2 * i]) =
+                            o2[g][i];
             }
-        }
-        const int64_t bh = static_cast<int64_t>(b) * p.num_q_heads + hq0 + g;
-        if (nparts == 1) {
-            static_cast<OutT*>(p.out)[bh * D + d] = out_cast<OutT>(l > 0.0f ? o / l : 0.0f);
+            if (j + 1 < n) {
+                advance(cur, p);  // next pair (the range goes on)
+                piece_start = lo + j + 1;
+                load_q_group();
+                reset();
+            }
         } else {
-            p.ws_o[(bh * p.max_parts + part) * D + d] = o;
-            if (d == 0) p.ws_ml[bh * p.max_parts + part] = make_float2(M, l);
+            ++cur.jb;
         }
     }
 }
 
 // ======================================================================================
-// Merge kernel: one warp per (sequence, query head) with more than one partition.
-//   M = max_p m_p;  w_p = 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p l_p
+// Merge kernel: one warp per (sequence, query head).  Pairs split over several
+// consumer ranges are combined:  M = max_p m_p;  w_p = 2^(m_p - M);
+// out = sum_p w_p o_p / sum_p w_p l_p.  Pairs of invalid length get zeros.
 // ======================================================================================
 template <int Q_T, int D>
 __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p) {
     using OutT = typename QType<Q_T>::T;
     constexpr int kDPL = D / 32;
+    constexpr int kBatch = 8;  // pieces whose loads are in flight together
+    pdl_wait();
+    pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
     const int64_t bh = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
     if (bh >= static_cast<int64_t>(p.batch) * p.num_q_heads) return;
     const int32_t b = static_cast<int32_t>(bh / p.num_q_heads);
-    const int32_t L = p.context_lens[b];
-    if (L < 1 || L > p.max_context_len) return;
-    const int32_t n = (L + p.partition_tokens - 1) / p.partition_tokens;
-    if (n <= 1) return;
-    const float2* ml = p.ws_ml + bh * p.max_parts;
+    const int32_t h = static_cast<int32_t>(bh % p.num_q_heads);
+    const int32_t G = p.num_q_heads / p.num_kv_heads;
+    const int32_t kvh = h / G, g = h % G;
+    const int32_t nt = seq_tiles(p.context_lens[b], p.max_context_len);
+    OutT* out = static_cast<OutT*>(p.out) + bh * D + lane * kDPL;
+    if (nt == 0) {
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) out[j] = out_cast<OutT>(0.0f);
+        if (lane == 0 && g == 0 && kvh == 0) report(p.dev_error, KV_DEVERR_BAD_CONTEXT_LEN);
+        return;
+    }
+    const int64_t T = p.ws_seq_start[p.batch];
+    const int64_t a = static_cast<int64_t>(p.ws_seq_start[b]) + static_cast<int64_t>(kvh) * nt;
+    const int64_t w_first = range_of(a, T, p.num_ranges);
+    const int64_t w_last = range_of(a + nt - 1, T, p.num_ranges);
+    if (w_first == w_last) return;  // the pair was one range's: written by the decode kernel
+    const int64_t s = static_cast<int64_t>(b) * p.num_kv_heads + kvh;
+    const int32_t npieces = static_cast<int32_t>(w_last - w_first + 1);
+    // pieces are (pair s, range W) for the non-empty ranges W in [w_first, w_last];
+    // piece id s + W (see the decode kernel)
+    auto piece_id = [&](int32_t i) -> int64_t {
+        const int64_t W = w_first + i;
+        return range_begin(W, T, p.num_ranges) < range_begin(W + 1, T, p.num_ranges) ? s + W : -1;
+    };
     float M = -INFINITY;
-    for (int i = lane; i < n; i += 32) M = fmaxf(M, ml[i].x);
+    for (int i = lane; i < npieces; i += 32) {
+        const int64_t pid = piece_id(i);
+        if (pid >= 0) M = fmaxf(M, p.ws_ml[pid * G + g].x);
+    }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
     float o[kDPL];
 #pragma unroll
-    for (int i = 0; i < kDPL; ++i) o[i] = 0.0f;
+    for (int j = 0; j < kDPL; ++j) o[j] = 0.0f;
     float l = 0.0f;
     if (M != -INFINITY) {
-        const float* ob = p.ws_o + bh * p.max_parts * D + lane * kDPL;
-        for (int i = 0; i < n; ++i) {
-            const float2 mli = ml[i];
-            const float w = exp2f(mli.x - M);
-            l += w * mli.y;
+        for (int i0 = 0; i0 < npieces; i0 += 32) {
+            // lane i holds piece i0+i's id and weight; the warp then folds the pieces
+            // in kBatch at a time with all their loads issued before the first FMA
+            const int64_t pl = (i0 + lane < npieces) ? piece_id(i0 + lane) : -1;
+            float wl = 0.0f;
+            if (pl >= 0) {
+                const float2 ml = p.ws_ml[pl * G + g];
+                wl = exp2f(ml.x - M);
+                l += wl * ml.y;
+            }
+            const int cnt = min(32, npieces - i0);
+            for (int i1 = 0; i1 < cnt; i1 += kBatch) {
+                float v[kBatch][kDPL];
+                float w[kBatch];
 #pragma unroll
-            for (int j = 0; j < kDPL; ++j) o[j] += w * ob[static_cast<int64_t>(i) * D + j];
+                for (int u = 0; u < kBatch; ++u) {
+                    const int i = (i1 + u) & 31;
+                    w[u] = __shfl_sync(0xffffffffu, wl, i);
+                    const int64_t pid = __shfl_sync(0xffffffffu, pl, i);
+                    const bool use = i1 + u < cnt && pid >= 0;
+                    const float* src = p.ws_o + ((use ? pid : 0) * G + g) * D + lane * kDPL;
+#pragma unroll
+                    for (int j = 0; j < kDPL; ++j) v[u][j] = use ? src[j] : 0.0f;
+                    if (!use) w[u] = 0.0f;
+                }
+#pragma unroll
+                for (int u = 0; u < kBatch; ++u)
+#pragma unroll
+                    for (int j = 0; j < kDPL; ++j) o[j] = fmaf(w[u], v[u][j], o[j]);
+            }
         }
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
     }
-    OutT* out = static_cast<OutT*>(p.out) + bh * D + lane * kDPL;
 #pragma unroll
     for (int j = 0; j < kDPL; ++j) out[j] = out_cast<OutT>(l > 0.0f ? o[j] / l : 0.0f);
 }
 
-// ---- dispatch ---------------------------------------------------------------------------
+// ---- launch ------------------------------------------------------------------------------
 constexpr int kMaxDevices = 64;
+
+template <int KV_T, int D, int G>
+int32_t resident_ctas_per_sm() {
+    return Cfg<KV_T, D, G>::kMinBlocks;
+}
 
 template <int KV_T, int Q_T, int D, int G>
 static cudaError_t launch_one(const DecodeParams& p, cudaStream_t stream) {
@@ -538,18 +727,19 @@ static cudaError_t launch_one(const DecodeParams& p, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= kMaxDevices || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(paged_decode_split_kernel<KV_T, Q_T, D, G>,
+        e = cudaFuncSetAttribute(paged_decode_kernel<KV_T, Q_T, D, G>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) attr_set[dev] = true;
     }
-    const dim3 grid(p.max_parts, p.num_kv_heads, p.batch);
-    paged_decode_split_kernel<KV_T, Q_T, D, G><<<grid, C::kThreads, C::kSmemBytes, stream>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess || p.max_parts <= 1) return e;
+    const unsigned grid = static_cast<unsigned>((p.num_ranges + C::kConsumerWarps - 1) /
+                                                C::kConsumerWarps);
+    e = launch_pdl(paged_decode_kernel<KV_T, Q_T, D, G>, dim3(grid), dim3(C::kThreads),
+                   C::kSmemBytes, stream, p);
+    if (e != cudaSuccess) return e;
     const int64_t warps = static_cast<int64_t>(p.batch) * p.num_q_heads;
-    paged_decode_merge_kernel<Q_T, D><<<static_cast<unsigned>((warps + 3) / 4), 128, 0, stream>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(paged_decode_merge_kernel<Q_T, D>, dim3(static_cast<unsigned>((warps + 3) / 4)),
+                      dim3(128), 0, stream, p);
 }
 
 template <int KV_T, int Q_T, int D>
@@ -583,6 +773,12 @@ cudaError_t launch_paged_decode(const DecodeParams& p, int32_t kv_dtype, int32_t
         case KV_BF16: return dispatch_q<KV_BF16>(p, q_dtype, head_dim, group, stream);
         default: return dispatch_q<KV_FP8_E4M3>(p, q_dtype, head_dim, group, stream);
     }
+}
+
+int32_t decode_ctas_per_sm(int32_t kv_dtype, int32_t head_dim, int32_t group) {
+    (void)kv_dtype;
+    (void)head_dim;
+    return group >= 8 ? 1 : 3;
 }
 
 }  // namespace pkv

@@ -1,9 +1,28 @@
 // Launchers of the paged-KV kernels, called by the C ABI layer (api.cu).
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace pkv {
+
+// Launch with programmatic stream serialisation (see pdl_wait / pdl_trigger).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 cudaError_t launch_slot_mapping(const int32_t* block_table, int32_t batch, int32_t max_blocks,
                                 const int32_t* seq_ids, const int32_t* positions,
@@ -21,7 +40,7 @@ cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, 
                              int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
                              cudaStream_t stream);
 
-// Everything the split-K decode and its merge need for one launch.
+// Everything the decode kernel and its merge need for one launch.
 struct DecodeParams {
     void* out;                    // [B][Hq][D] in q dtype
     const void* q;                // [B][Hq][D]
@@ -31,13 +50,18 @@ struct DecodeParams {
     const float* v_scales;
     const int32_t* block_table;   // [B][max_blocks]
     const int32_t* context_lens;  // [B]
-    float2* ws_ml;                // [B][Hq][max_parts] (running max in log2 units, sum)
-    float* ws_o;                  // [B][Hq][max_parts][D]
+    int32_t* ws_seq_start;        // [B + 1]: first tile of each sequence, total tiles at [B]
+    float2* ws_ml;                // [pieces][G]: (running max in base-2 units, running sum)
+    float* ws_o;                  // [pieces][G][D]: unnormalised partial outputs
     int32_t* dev_error;
     int32_t batch, num_q_heads, num_kv_heads, num_blocks, max_blocks;
-    int32_t max_context_len, partition_tokens, max_parts;
+    int32_t max_context_len;
+    int32_t num_ranges;           // consumer-warp ranges the tile list is cut into
     float scale_log2;             // scale * log2(e): scores are kept in base-2 units
 };
+
+// Resident decode CTAs per SM the kernels are built for (their register budget).
+int32_t decode_ctas_per_sm(int32_t kv_dtype, int32_t head_dim, int32_t group);
 
 // kv_dtype, q_dtype, head_dim and group size select the kernel instantiation.
 cudaError_t launch_paged_decode(const DecodeParams& p, int32_t kv_dtype, int32_t q_dtype,

@@ -1,8 +1,8 @@
 """Host-side checks of libpagedkv.so that need no GPU.
 
 The library loads, exports every entry point include/paged_kv.h declares, and
-its host logic (geometry, argument validation, workspace sizing, partition
-heuristic) behaves as documented.  No call here enqueues device work: every
+its host logic (geometry, argument validation, workspace sizing, the split
+into consumer ranges) behaves as documented.  No call here enqueues device work: every
 call is rejected on the host before any launch, or is host-only.
 """
 import ctypes
@@ -72,38 +72,21 @@ def test_pool_create_rejects(args, status):
     assert e.value.status == status
 
 
-def test_workspace_bytes_and_partition():
+def test_workspace_bytes_and_ranges():
     d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
-    # one partition: no workspace
-    assert pk.paged_decode_workspace_bytes(d, 32, 32, 4096, 4096) == 0
-    # 8 partitions of 512: (m, l) pairs padded to 256 B, then fp32 partial outputs
-    rows = 32 * 32 * 8
-    ml = (rows * 8 + 255) // 256 * 256
-    assert pk.paged_decode_workspace_bytes(d, 32, 32, 4096, 512) == ml + rows * 128 * 4
-    p = pk.paged_decode_default_partition(d, 32, 32, 4096)
-    assert p % 16 == 0 and 256 <= p <= 1024
-
-
-class _FakeTensor:
-    """Stands in for a device tensor in calls the host rejects before launching."""
-
-    def __init__(self, addr, shape, dtype="bf16"):
-        self.addr, self.shape, self._dt = addr, shape, dtype
-
-    def is_contiguous(self):
-        return True
-
-    def data_ptr(self):
-        return self.addr
-
-    def numel(self):
-        n = 1
-        for s in self.shape:
-            n *= s
-        return n
-
-    def element_size(self):
-        return 1
+    # balanced default: one range per consumer warp of 3 CTAs x 4 warps on each of 148 SMs
+    assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 0) == 148 * 3 * 4
+    # group 8 kernels keep one CTA per SM
+    assert pk.paged_decode_num_ranges(d, 32, 64, 4096, 0) == 148 * 4
+    # explicit partition: ranges of at most 512 tokens over 32 x 8 x 256 tiles
+    assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 512) == 32 * 8 * 256 // 32
+    assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 500) == 0
+    ranges = 148 * 12
+    pieces = 32 * 8 + ranges
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    want = up(4 * 33) + up(pieces * 4 * 8) + pieces * 4 * 128 * 4
+    assert pk.paged_decode_workspace_bytes(d, 32, 32, 4096, 0) == want
+    assert pk.paged_decode_workspace_bytes(d, 32, 30, 4096, 0) == 0
 
 
 def _call_decode(desc, **kw):
@@ -130,7 +113,8 @@ def _call_decode(desc, **kw):
     (dict(max_context_len=4097), pk.KV_ERR_INVALID_ARGUMENT),      # beyond the table
     (dict(max_context_len=0), pk.KV_ERR_INVALID_ARGUMENT),
     (dict(partition=500), pk.KV_ERR_INVALID_ARGUMENT),             # not a multiple of 16
-    (dict(partition=16384), pk.KV_ERR_INVALID_ARGUMENT),
+    (dict(max_blocks=1 << 24, max_context_len=1 << 28, batch=2048),
+     pk.KV_ERR_UNSUPPORTED),                                        # tile list >= 2^31
     (dict(q=8192 + 8), pk.KV_ERR_INVALID_ARGUMENT),                # misaligned
     (dict(k_pool=None), pk.KV_ERR_INVALID_ARGUMENT),
     (dict(k_scales=6 << 20, v_scales=7 << 20), pk.KV_ERR_INVALID_ARGUMENT),  # scales on bf16
@@ -147,6 +131,12 @@ def test_decode_fp8_pool_requires_scales():
     d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_FP8_E4M3)
     assert _call_decode(d) == pk.KV_ERR_INVALID_ARGUMENT
     assert _call_decode(d, k_scales=6 << 20) == pk.KV_ERR_INVALID_ARGUMENT
+
+
+def test_decode_needs_a_workspace_even_for_one_range():
+    d = pk.kv_pool_create(64, 16, 1, 64, pk.KV_F32)
+    assert _call_decode(d, q_dtype=pk.KV_F32, batch=1, num_q_heads=4, max_blocks=4,
+                        max_context_len=20, workspace=None) == pk.KV_ERR_INVALID_ARGUMENT
 
 
 def test_decode_empty_batch_is_a_no_op():
