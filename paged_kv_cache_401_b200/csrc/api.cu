@@ -1,6 +1,8 @@
 // C ABI of libpagedkv.so (declared in include/paged_kv.h): host-side argument
 // checks, geometry, the split of the tile list into consumer ranges, the
 // workspace layout and kernel launches.
+#include <cudaTypedefs.h>
+
 #include <cmath>
 
 #include "kernels.cuh"
@@ -38,6 +40,43 @@ bool valid_pool(const kv_pool_desc* d) {
 }
 
 int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
+
+// The driver's tensor-map encoder, looked up once through the runtime (no libcuda link).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess) {
+            cudaGetLastError();
+            return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+        }
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }();
+    return fn;
+}
+
+// A pool as a 2-D tensor [num_blocks*Hkv*16 rows][head_dim], 16-row x 128-byte
+// boxes, 128-byte swizzle.  Returns a kv_status.
+kv_status encode_pool_map(CUtensorMap* map, const void* base, const kv_pool_desc* pool) {
+    const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (encode == nullptr) return KV_ERR_CUDA;
+    const cuuint64_t rows = static_cast<cuuint64_t>(pool->num_blocks) * pool->num_kv_heads *
+                            kBlockTokens;
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pool->head_dim), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pool->head_dim) * pool->elem_bytes};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / pool->elem_bytes),
+                               static_cast<cuuint32_t>(kBlockTokens)};
+    const cuuint32_t elem_strides[2] = {1, 1};
+    const CUtensorMapDataType type = pool->dtype == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                            : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+    const CUresult r = encode(map, type, 2, const_cast<void*>(base), dims, strides, box,
+                              elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? KV_OK : KV_ERR_INVALID_ARGUMENT;
+}
 
 }  // namespace
 
@@ -227,8 +266,18 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     p.ws_seq_start = reinterpret_cast<int32_t*>(ws);
     p.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
     p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
-    cudaError_t e = pkv::launch_paged_decode(p, pool->dtype, q_dtype, pool->head_dim, group,
-                                             reinterpret_cast<cudaStream_t>(stream));
+    pkv::TmaMaps maps{};
+    if (pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim)) {
+        // TMA row coordinates are 32-bit
+        if (static_cast<int64_t>(pool->num_blocks) * pool->num_kv_heads * kBlockTokens >=
+            (int64_t{1} << 31))
+            return KV_ERR_UNSUPPORTED;
+        kv_status st = encode_pool_map(&maps.k, k_pool, pool);
+        if (st == KV_OK) st = encode_pool_map(&maps.v, v_pool, pool);
+        if (st != KV_OK) return st;
+    }
+    cudaError_t e = pkv::launch_paged_decode(p, maps, pool->dtype, q_dtype, pool->head_dim,
+                                             group, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 

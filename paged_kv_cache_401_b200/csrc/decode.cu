@@ -21,18 +21,23 @@
 //
 // B200 design:
 //  * a CTA is one producer warp and four consumer warps; by default the grid
-//    is exactly the number of CTAs resident on the GPU (persistent), so the
-//    tile stream never stalls between work items;
+//    is the number of CTAs resident on the GPU (persistent), so the tile
+//    stream never stalls between work items;
 //  * the producer's lane 0 walks the four consumer warps' ranges and stages
-//    each (block, kv head) K and V tile -- one contiguous 16*D span of the
-//    pool -- into a shared-memory ring with 1-D bulk async copies (the TMA
-//    engine, no multicast) completing on mbarriers; block ids are fetched 8
-//    tiles ahead so table-lookup latency never gaps the stream;
-//  * stage s of the ring always feeds consumer warp s % 4; a consumer warp
-//    computes q.K with packed fp32x2 FMAs on 16-byte chunks (8 lanes per
-//    row) and a shuffle reduce-scatter, the online softmax with exp2 on
-//    scores pre-scaled by scale*log2(e), and P.V with each lane owning D/32
-//    output columns, all in fp32;
+//    each (block, kv head) K and V tile -- one contiguous 16-row span of the
+//    pool -- into a shared-memory ring through the TMA engine (no multicast),
+//    completing on mbarriers; block ids are fetched 8 tiles ahead;
+//  * stage s of the ring always feeds consumer warp s % 4;
+//  * the per-tile arithmetic is a policy:
+//      MmaMath  (bf16 or FP8 KV, head_dim 128, bf16 q): tiles land in shared
+//               memory 128-byte swizzled by 2-D TMA tensor copies; the group's
+//               scores S = Q.K^T come from mma.m16n8k16 (query heads as rows,
+//               fp32 accumulate), the softmax runs on the accumulator
+//               fragments, and P feeds O^T = V^T.P^T straight from registers;
+//               FP8 codes are widened to f16 in registers (exact);
+//      SimtMath (every other shape and fp32): 1-D bulk copies; q.K with
+//               packed fp32x2 FMAs and a shuffle reduce-scatter, P.V with each
+//               lane owning D/32 output columns, all in fp32;
 //  * every wait is bounded; bad block ids and context lengths are reported
 //    through the error word and never dereferenced.
 #include "kernels.cuh"
@@ -52,46 +57,6 @@ struct KvElem<KV_BF16> {
 template <>
 struct KvElem<KV_FP8_E4M3> {
     static constexpr int kBytes = 1;
-};
-
-template <int KV_T, int D, int G>
-struct Cfg {
-    static constexpr int kElem = KvElem<KV_T>::kBytes;
-    static constexpr int kTileBytes = kBlockTokens * D * kElem;              // K or V tile
-    static constexpr int kScaleBytes = (KV_T == KV_FP8_E4M3) ? kBlockTokens * 4 : 0;
-    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kScaleBytes;
-    static constexpr int kConsumerWarps = 4;
-    static constexpr int kThreads = (kConsumerWarps + 1) * 32;
-    static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
-    static constexpr int kChunkElems = 16 / kElem;                           // per 16-byte load
-    static constexpr int kRowChunks = D / kChunkElems;
-    static constexpr int kLPR = kRowChunks >= 8 ? 8 : kRowChunks;           // lanes per row
-    static constexpr int kNCH = kRowChunks / kLPR;                           // chunks per lane/row
-    static constexpr int kRPI = 32 / kLPR;                                   // rows per load step
-    static constexpr int kNR = kBlockTokens / kRPI;                          // rows per lane
-    static constexpr int kQPL = kNCH * kChunkElems;                          // q elems per lane/head
-    static constexpr int kNV = kNR * G;                                      // partial scores/lane
-    static constexpr int kVPL = kNV >= kLPR ? kNV / kLPR : 1;                // scores/lane after RS
-    static constexpr int kDPL = D / 32;                                      // output cols per lane
-    static constexpr int kSMLanes = (kBlockTokens * G) < 32 ? kBlockTokens * G : 32;
-    static constexpr int kSPL = kBlockTokens * G / kSMLanes;                 // softmax vals/lane
-    // shared memory: the ring, per-consumer-warp scratch, per-stage flags, barriers
-    static constexpr int kRingBytes = kStages * kStageBytes;
-    // per consumer warp: p pairs [16][G] float2, scores [16][G], corrections [G];
-    // rounded to 16 bytes so every warp's region (and its float2 array) is aligned
-    static constexpr int kWarpScratch =
-        (kBlockTokens * G * 8 + kBlockTokens * G * 4 + G * 4 + 15) / 16 * 16;
-    static constexpr int kFlagsBytes = (2 * kStages * 4 + 16 + 15) / 16 * 16;  // ok, issued, abort
-    static constexpr int kSmemBytes =
-        kRingBytes + kConsumerWarps * kWarpScratch + kFlagsBytes + 2 * kStages * 8;
-    // resident blocks per SM the register budget is sized for (G = 8 needs the
-    // whole register file of one block's worth of q and accumulators)
-    static constexpr int kMinBlocks = G >= 8 ? 1 : 3;
-    static_assert(kStages % kConsumerWarps == 0, "stage s feeds consumer warp s % 4");
-    static_assert(kStageBytes % 16 == 0 && kRingBytes % 16 == 0, "bulk copies need 16-B alignment");
-    static_assert((kRingBytes + kConsumerWarps * kWarpScratch + kFlagsBytes) % 8 == 0,
-                  "mbarriers need 8-B alignment");
-    static_assert(kQPL % 2 == 0 && kDPL % 2 == 0, "pairs for fp32x2 FMA");
 };
 
 // ---- small vector helpers --------------------------------------------------------
@@ -194,7 +159,7 @@ struct QType<KV_BF16> {
 };
 
 template <int Q_T>
-__device__ __forceinline__ float load_q(const void* q, int64_t i) {
+__device__ __forceinline__ float load_q_elem(const void* q, int64_t i) {
     if constexpr (Q_T == KV_F32) {
         return static_cast<const float*>(q)[i];
     } else {
@@ -202,6 +167,70 @@ __device__ __forceinline__ float load_q(const void* q, int64_t i) {
     }
 }
 
+
+
+// ---- tensor-core and TMA helpers --------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// d += A(16x16, row) * B(16x8, col), fp32 accumulate; bf16 or f16 operands.
+template <bool F16>
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+    if constexpr (F16) {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    } else {
+        asm volatile(
+            "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+            "{%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+    }
+}
+
+// Two fp32 -> packed pair (low half = first argument), round to nearest even.
+template <bool F16>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    uint32_t r;
+    if constexpr (F16)
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    else
+        asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+// Two E4M3 codes (low 16 bits) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w16) {
+    uint32_t h2;
+    asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
+        : "=r"(h2)
+        : "r"(w16));
+    return h2;
+}
+
+// 2-D TMA tile load (no multicast) completing on an mbarrier; x is the
+// innermost coordinate in elements (always 0 or a multiple of 16 bytes here).
+__device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
+                                            int32_t y, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, "
+        "{%2, %3}], [%4];" ::"r"(smem_addr(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar))
+        : "memory");
+}
 
 // ---- tile list bookkeeping ----------------------------------------------------------
 // Tiles of a sequence with context length L: ceil(L/16), or 0 when L is invalid.
@@ -300,48 +329,564 @@ __device__ __forceinline__ void advance(Cursor& c, const DecodeParams& p) {
     } while (c.b < p.batch && c.nt == 0);
 }
 
+
 // ======================================================================================
-// Decode kernel: grid ceil(num_ranges / 4) CTAs of kThreads threads.
+// SimtMath: fp32 CUDA-core tile arithmetic (any KV dtype, head_dim 64 or 128).
 // ======================================================================================
 template <int KV_T, int Q_T, int D, int G>
-__global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kMinBlocks)
-    paged_decode_kernel(const DecodeParams p) {
-    using C = Cfg<KV_T, D, G>;
+struct SimtMath {
     using OutT = typename QType<Q_T>::T;
-    extern __shared__ __align__(128) uint8_t smem[];
+    static constexpr int kElem = KvElem<KV_T>::kBytes;
+    static constexpr int kTileBytes = kBlockTokens * D * kElem;              // K or V tile
+    static constexpr int kScaleBytes = (KV_T == KV_FP8_E4M3) ? kBlockTokens * 4 : 0;
+    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kScaleBytes;
+    static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
+    static constexpr int kRingAlign = 128;
+    static constexpr int kChunkElems = 16 / kElem;                           // per 16-byte load
+    static constexpr int kRowChunks = D / kChunkElems;
+    static constexpr int kLPR = kRowChunks >= 8 ? 8 : kRowChunks;           // lanes per row
+    static constexpr int kNCH = kRowChunks / kLPR;                           // chunks per lane/row
+    static constexpr int kRPI = 32 / kLPR;                                   // rows per load step
+    static constexpr int kNR = kBlockTokens / kRPI;                          // rows per lane
+    static constexpr int kQPL = kNCH * kChunkElems;                          // q elems per lane/head
+    static constexpr int kNV = kNR * G;                                      // partial scores/lane
+    static constexpr int kVPL = kNV >= kLPR ? kNV / kLPR : 1;                // scores/lane after RS
+    static constexpr int kDPL = D / 32;                                      // output cols per lane
+    static constexpr int kSMLanes = (kBlockTokens * G) < 32 ? kBlockTokens * G : 32;
+    static constexpr int kSPL = kBlockTokens * G / kSMLanes;                 // softmax vals/lane
+    // per consumer warp: p pairs [16][G] float2, scores [16][G], corrections [G]
+    static constexpr int kWarpScratch =
+        (kBlockTokens * G * 8 + kBlockTokens * G * 4 + G * 4 + 15) / 16 * 16;
+    // resident blocks per SM the register budget is sized for (G = 8 needs the
+    // whole register file of one block's worth of q and accumulators)
+    static constexpr int kMinBlocks = G >= 8 ? 1 : 3;
+    static_assert(kStageBytes % 16 == 0, "bulk copies need 16-B alignment");
+    static_assert(kQPL % 2 == 0 && kDPL % 2 == 0, "pairs for fp32x2 FMA");
+
+    // ---- producer side: one stage = K tile, V tile (+ FP8 row scales), 1-D bulk copies
+    __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
+                                 const TmaMaps&) {
+        const int64_t off = tile * kTileBytes;
+        mbar_arrive_expect_tx(bar, kStageBytes);
+        bulk_copy_g2s(st, p.k_pool + off, kTileBytes, bar);
+        bulk_copy_g2s(st + kTileBytes, p.v_pool + off, kTileBytes, bar);
+        if constexpr (KV_T == KV_FP8_E4M3) {
+            bulk_copy_g2s(st + 2 * kTileBytes, p.k_scales + tile * kBlockTokens, kScaleBytes, bar);
+            bulk_copy_g2s(st + 2 * kTileBytes + kScaleBytes, p.v_scales + tile * kBlockTokens,
+                          kScaleBytes, bar);
+        }
+    }
+
+    // ---- consumer side
+    int32_t lane, c, r0, sm_lane, sm_g;
+    float2* p_buf;  // [16][G]
+    float* s_buf;   // [16][G]
+    float* c_buf;   // [G]
+    float2 q2[G][kQPL / 2];
+    float m_run, l_run;
+    float2 o2[G][kDPL / 2];
+
+    __device__ void init(int32_t lane_, uint8_t* scratch) {
+        lane = lane_;
+        c = lane % kLPR;    // chunk column of this lane in a K row
+        r0 = lane / kLPR;   // first K row of this lane
+        sm_lane = lane % kSMLanes;
+        sm_g = sm_lane % G; // query head this lane's softmax values belong to
+        p_buf = reinterpret_cast<float2*>(scratch);
+        s_buf = reinterpret_cast<float*>(p_buf + kBlockTokens * G);
+        c_buf = s_buf + kBlockTokens * G;
+    }
+
+    __device__ void load_q(const DecodeParams& p, int32_t b, int32_t kvh) {
+        const int64_t qbase = (static_cast<int64_t>(b) * p.num_q_heads + kvh * G) * D;
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int k = 0; k < kNCH; ++k)
+#pragma unroll
+                for (int e = 0; e < kChunkElems; e += 2) {
+                    const int64_t col = (c + k * kLPR) * kChunkElems + e;
+                    q2[g][(k * kChunkElems + e) / 2] =
+                        make_float2(load_q_elem<Q_T>(p.q, qbase + g * D + col) * p.scale_log2,
+                                    load_q_elem<Q_T>(p.q, qbase + g * D + col + 1) * p.scale_log2);
+                }
+    }
+
+    __device__ void reset() {
+        m_run = -INFINITY;  // running max of this lane's head (base-2 units)
+        l_run = 0.0f;       // this lane's share of the running sum
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+#pragma unroll
+            for (int i = 0; i < kDPL / 2; ++i) o2[g][i] = make_float2(0.0f, 0.0f);
+    }
+
+    __device__ void tile(const uint8_t* kt, int32_t nvalid, const DecodeParams&) {
+        const uint8_t* vt = kt + kTileBytes;
+        const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
+        const float* vsc = ksc + kBlockTokens;
+
+        // scores: partial dot products over this lane's columns, then reduce-scatter
+        float acc[kNV];
+#pragma unroll
+        for (int i = 0; i < kNR; ++i) {
+            const int row = r0 + kRPI * i;
+            float2 ap[G];
+#pragma unroll
+            for (int g = 0; g < G; ++g) ap[g] = make_float2(0.0f, 0.0f);
+#pragma unroll
+            for (int kk = 0; kk < kNCH; ++kk) {
+                const uint4 chunk =
+                    *reinterpret_cast<const uint4*>(kt + row * (D * kElem) + (c + kk * kLPR) * 16);
+                float2 kv[kChunkElems / 2];
+                decode_chunk<KV_T>(chunk, kv);
+#pragma unroll
+                for (int g = 0; g < G; ++g)
+#pragma unroll
+                    for (int e = 0; e < kChunkElems / 2; ++e)
+                        ap[g] = ffma2(q2[g][kk * kChunkElems / 2 + e], kv[e], ap[g]);
+            }
+#pragma unroll
+            for (int g = 0; g < G; ++g) acc[i * G + g] = ap[g].x + ap[g].y;
+        }
+        reduce_scatter<kNV, kLPR / 2>(acc, lane);
+#pragma unroll
+        for (int v = 0; v < kVPL; ++v) {
+            const int idx = (kNV >= kLPR) ? c * kVPL + v : c / (kLPR / kNV);
+            const int t = r0 + kRPI * (idx / G);
+            float sc = acc[v];
+            if constexpr (KV_T == KV_FP8_E4M3) sc *= ksc[t];
+            s_buf[t * G + (idx % G)] = sc;
+        }
+        __syncwarp();
+
+        // online softmax: lane handles head sm_g, tokens sm_lane/G + i*(kSMLanes/G)
+        float sv[kSPL];
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kSPL; ++i) {
+            const int t = sm_lane / G + i * (kSMLanes / G);
+            sv[i] = (t < nvalid) ? s_buf[t * G + sm_g] : -INFINITY;
+            tmax = fmaxf(tmax, sv[i]);
+        }
+#pragma unroll
+        for (int m = G; m < kSMLanes; m <<= 1)
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
+        const float m_new = fmaxf(m_run, tmax);
+        const float corr = exp2f(m_run - m_new);
+        l_run *= corr;
+#pragma unroll
+        for (int i = 0; i < kSPL; ++i) {
+            const int t = sm_lane / G + i * (kSMLanes / G);
+            const float pr = exp2f(sv[i] - m_new);
+            l_run += pr;
+            float pv = pr;
+            if constexpr (KV_T == KV_FP8_E4M3) pv *= vsc[t];
+            if (lane < kSMLanes) p_buf[t * G + sm_g] = make_float2(pv, pv);
+        }
+        m_run = m_new;
+        if (lane < G) c_buf[lane] = corr;
+        __syncwarp();
+
+        // P.V: this lane's kDPL output columns for every head of the group
+#pragma unroll
+        for (int g = 0; g < G; ++g) {
+            const float cg = c_buf[g];
+#pragma unroll
+            for (int i = 0; i < kDPL / 2; ++i) o2[g][i] = __fmul2_rn(o2[g][i], make_float2(cg, cg));
+        }
+        const uint8_t* vrow = vt + lane * kDPL * kElem;
+        if (nvalid == kBlockTokens) {
+#pragma unroll
+            for (int t = 0; t < kBlockTokens; ++t) {
+                float2 vv[kDPL / 2];
+                load_v<KV_T, kDPL>(vrow + t * D * kElem, vv);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float2 pp = p_buf[t * G + g];
+#pragma unroll
+                    for (int i = 0; i < kDPL / 2; ++i) o2[g][i] = ffma2(pp, vv[i], o2[g][i]);
+                }
+            }
+        } else {
+            for (int t = 0; t < nvalid; ++t) {
+                float2 vv[kDPL / 2];
+                load_v<KV_T, kDPL>(vrow + t * D * kElem, vv);
+#pragma unroll
+                for (int g = 0; g < G; ++g) {
+                    const float2 pp = p_buf[t * G + g];
+#pragma unroll
+                    for (int i = 0; i < kDPL / 2; ++i) o2[g][i] = ffma2(pp, vv[i], o2[g][i]);
+                }
+            }
+        }
+    }
+
+    // End of a piece: the whole pair's output, or a partial (m, l, o) for the merge.
+    __device__ void finish(const DecodeParams& p, int32_t b, int32_t kvh, bool whole,
+                           int64_t pid) {
+        float l = l_run;  // sum of l over the lanes that share this lane's head
+#pragma unroll
+        for (int m = G; m < kSMLanes; m <<= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
+        const int64_t bh0 = static_cast<int64_t>(b) * p.num_q_heads + kvh * G;
+        if (whole) {
+#pragma unroll
+            for (int g = 0; g < G; ++g) {
+                const float lg = __shfl_sync(0xffffffffu, l, g);
+                OutT* o = static_cast<OutT*>(p.out) + (bh0 + g) * D + lane * kDPL;
+#pragma unroll
+                for (int i = 0; i < kDPL / 2; ++i) {
+                    o[2 * i] = out_cast<OutT>(lg > 0.0f ? o2[g][i].x / lg : 0.0f);
+                    o[2 * i + 1] = out_cast<OutT>(lg > 0.0f ? o2[g][i].y / lg : 0.0f);
+                }
+            }
+        } else {
+            if (lane < G) p.ws_ml[pid * G + lane] = make_float2(m_run, l);
+#pragma unroll
+            for (int g = 0; g < G; ++g)
+#pragma unroll
+                for (int i = 0; i < kDPL / 2; ++i)
+                    *reinterpret_cast<float2*>(&p.ws_o[(pid * G + g) * D + lane * kDPL + 2 * i]) =
+                        o2[g][i];
+        }
+    }
+};
+
+// ======================================================================================
+// MmaMath: tensor-core tile arithmetic for bf16 or FP8 KV, head_dim 128, bf16 q.
+//
+// A tile is 16 tokens x 128 dims.  K and V land in shared memory as [16 rows]
+// x [128-byte] boxes written by TMA with the 128-byte swizzle (16-byte chunk
+// c of row r stored at chunk c ^ (r & 7)), so every ldmatrix row set hits 32
+// distinct banks.  Per tile and warp (gid = lane / 4, tig = lane % 4):
+//   S   = Q.K^T      m16n8k16, rows = query heads of the group (G <= 8 real),
+//                    2 token tiles x 8 dim steps; fp32 accumulators.
+//   softmax on the accumulator fragments: row gid holds tokens 2tig,2tig+1
+//                    and 8+2tig,9+2tig; max/sum across the 4 lanes of a row.
+//   O^T += V^T.P^T   m16n8k16, rows = 16 head dims, columns = 8 heads; the P
+//                    fragment of the score accumulators is exactly the B
+//                    operand, so P never leaves registers.
+// bf16 KV: bf16 MMAs, P rounded to bf16.  FP8 KV: codes widened to f16 in
+// registers (exact), f16 MMAs with q rounded to f16 and P (times the V row
+// scale) rounded to f16; the K row scale multiplies the scores.  Element
+// orders inside a k-step are permuted consistently between the two operands
+// (a dot product does not depend on the order of its terms), which is what
+// lets FP8 rows be read with 16-bit ldmatrix.
+// ======================================================================================
+template <int KV_T, int G>
+struct MmaMath {
+    static_assert(KV_T == KV_BF16 || KV_T == KV_FP8_E4M3, "bf16 or FP8 KV");
+    static_assert(G <= 8, "one m16n8 column per query head");
+    using OutT = uint16_t;                                        // bf16 output
+    static constexpr bool kF16 = KV_T == KV_FP8_E4M3;
+    static constexpr int D = 128;
+    static constexpr int kElem = KvElem<KV_T>::kBytes;
+    static constexpr int kRowBytes = D * kElem;                   // 256 (bf16) / 128 (fp8)
+    static constexpr int kBoxCols = 128 / kElem;                  // elements per 128-byte box row
+    static constexpr int kBoxes = kRowBytes / 128;
+    static constexpr int kBoxBytes = kBlockTokens * 128;
+    static constexpr int kTileBytes = kBlockTokens * kRowBytes;
+    static constexpr int kScaleBytes = kF16 ? kBlockTokens * 4 : 0;
+    static constexpr int kStageBytes = (2 * kTileBytes + 2 * kScaleBytes + 1023) / 1024 * 1024;
+    static constexpr int kStages = kF16 ? 12 : 8;                 // multiple of 4
+    static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
+    static constexpr int kWarpScratch = 0;
+    static constexpr int kMinBlocks = 3;
+
+    // ---- producer side: TMA boxes of K and V (+ FP8 row scales by bulk copy)
+    __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
+                                 const TmaMaps& maps) {
+        const int32_t row = static_cast<int32_t>(tile * kBlockTokens);
+        mbar_arrive_expect_tx(bar, 2 * kTileBytes + 2 * kScaleBytes);
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) {
+            tma_load_2d(st + bx * kBoxBytes, &maps.k, bx * kBoxCols, row, bar);
+            tma_load_2d(st + kTileBytes + bx * kBoxBytes, &maps.v, bx * kBoxCols, row, bar);
+        }
+        if constexpr (kF16) {
+            bulk_copy_g2s(st + 2 * kTileBytes, p.k_scales + tile * kBlockTokens, kScaleBytes, bar);
+            bulk_copy_g2s(st + 2 * kTileBytes + kScaleBytes, p.v_scales + tile * kBlockTokens,
+                          kScaleBytes, bar);
+        }
+    }
+
+    // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile.
+    __device__ static __forceinline__ uint32_t swz(int32_t row, int32_t chunk) {
+        return (chunk >> 3) * kBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
+    }
+
+    // head-dim of row r (0..15) of output m-tile mi: FP8 tiles interleave even/odd dims
+    __device__ static __forceinline__ int32_t dim_of(int32_t mi, int32_t r) {
+        if constexpr (kF16) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
+        return 16 * mi + r;
+    }
+
+    // ---- consumer side
+    int32_t lane, gid, tig;
+    uint32_t qa[8][2];  // A fragments of q per 16-dim k-step: rows gid (< G), cols {lo, hi}
+    float o[8][4];      // O^T: m-tile mi = 16 dims; c0,c1 = (dim row gid, heads 2tig, 2tig+1)
+    float m_run, l_run; // running max (base 2) and this lane's part of the sum, row gid
+
+    __device__ void init(int32_t lane_, uint8_t*) {
+        lane = lane_;
+        gid = lane >> 2;
+        tig = lane & 3;
+    }
+
+    __device__ void load_q(const DecodeParams& p, int32_t b, int32_t kvh) {
+        const uint16_t* q = static_cast<const uint16_t*>(p.q) +
+                            (static_cast<int64_t>(b) * p.num_q_heads + kvh * G + gid) * D;
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            if (gid >= G) {
+                qa[ks][0] = qa[ks][1] = 0u;
+            } else if constexpr (!kF16) {
+                // k index 2tig+{0,1} -> dim 16ks+2tig+{0,1}; 8+2tig+{0,1} -> dim 16ks+8+2tig+{0,1}
+                qa[ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
+                qa[ks][1] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 8 + 2 * tig);
+            } else {
+                // FP8 rows are read 4 codes per lane: k 2tig+{0,1} -> dim 16ks+4tig+{0,1},
+                // k 8+2tig+{0,1} -> dim 16ks+4tig+{2,3}
+                const uint2 w = *reinterpret_cast<const uint2*>(q + 16 * ks + 4 * tig);
+                qa[ks][0] = pack2<true>(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
+                qa[ks][1] = pack2<true>(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+            }
+        }
+    }
+
+    __device__ void reset() {
+        m_run = -INFINITY;
+        l_run = 0.0f;
+#pragma unroll
+        for (int mi = 0; mi < 8; ++mi)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) o[mi][j] = 0.0f;
+    }
+
+    __device__ void tile(const uint8_t* kt, int32_t nvalid, const DecodeParams& p) {
+        const uint32_t k_s = smem_addr(kt);
+        const uint32_t v_s = k_s + kTileBytes;
+        const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
+        const float* vsc = ksc + kBlockTokens;
+        const int32_t mtx = lane >> 3, r = lane & 7;  // ldmatrix: matrix and row this lane addresses
+
+        // ---- S = Q.K^T: s[nt] holds rows gid (c0, c1) and gid + 8 (c2, c3, unused)
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        if constexpr (!kF16) {
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                uint32_t b[4];  // {nt0 dims lo, nt0 dims hi, nt1 dims lo, nt1 dims hi}
+                ldsm_x4(b, k_s + swz(8 * (mtx >> 1) + r, 2 * ks + (mtx & 1)));
+                mma_16816<false>(s[0], qa[ks][0], 0u, qa[ks][1], 0u, b[0], b[1]);
+                mma_16816<false>(s[1], qa[ks][0], 0u, qa[ks][1], 0u, b[2], b[3]);
+            }
+        } else {
+#pragma unroll
+            for (int kq = 0; kq < 4; ++kq) {
+                uint32_t w[4];  // {(ks 2kq, nt0), (2kq+1, nt0), (2kq, nt1), (2kq+1, nt1)}
+                ldsm_x4(w, k_s + swz(8 * (mtx >> 1) + r, 2 * kq + (mtx & 1)));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int ks = 2 * kq + h;
+                    mma_16816<true>(s[0], qa[ks][0], 0u, qa[ks][1], 0u, e4m3x2_to_f16x2(w[h] & 0xffffu),
+                                    e4m3x2_to_f16x2(w[h] >> 16));
+                    mma_16816<true>(s[1], qa[ks][0], 0u, qa[ks][1], 0u,
+                                    e4m3x2_to_f16x2(w[2 + h] & 0xffffu), e4m3x2_to_f16x2(w[2 + h] >> 16));
+                }
+            }
+        }
+
+        // ---- online softmax on row gid: tokens 8nt + 2tig + j
+        float mx = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int t = 8 * nt + 2 * tig + j;
+                float v = s[nt][j] * p.scale_log2;
+                if constexpr (kF16) v *= ksc[t];
+                s[nt][j] = (t < nvalid) ? v : -INFINITY;
+                mx = fmaxf(mx, s[nt][j]);
+            }
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+        const float m_new = fmaxf(m_run, mx);
+        const float corr = exp2f(m_run - m_new);
+        float pr[2][2];
+        float psum = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                pr[nt][j] = exp2f(s[nt][j] - m_new);
+                psum += pr[nt][j];
+            }
+        l_run = l_run * corr + psum;
+        m_run = m_new;
+
+        // rescale O^T columns (heads 2tig, 2tig+1): head h's factor is on lanes gid == h
+        const float ca = __shfl_sync(0xffffffffu, corr, 8 * tig);
+        const float cb = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
+        if (__any_sync(0xffffffffu, ca != 1.0f || cb != 1.0f)) {
+#pragma unroll
+            for (int mi = 0; mi < 8; ++mi) {
+                o[mi][0] *= ca;
+                o[mi][1] *= cb;
+                o[mi][2] *= ca;
+                o[mi][3] *= cb;
+            }
+        }
+
+        // ---- P^T fragment (B operand: k = token, n = head gid).  Tokens past the
+        // context end have p = 0; their V rows and scales may hold anything (NaN
+        // included), so they are removed by select, never multiplied.
+        if constexpr (kF16) {
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int t = 8 * nt + 2 * tig + j;
+                    pr[nt][j] = (t < nvalid) ? pr[nt][j] * vsc[t] : 0.0f;
+                }
+        }
+        const uint32_t pb0 = pack2<kF16>(pr[0][0], pr[0][1]);
+        const uint32_t pb1 = pack2<kF16>(pr[1][0], pr[1][1]);
+        // V^T fragment halves of tokens 2tig, 2tig+1 (mask_a) and 8+2tig, 9+2tig (mask_b)
+        const bool partial = nvalid < kBlockTokens;
+        const uint32_t mask_a = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+        const uint32_t mask_b = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
+
+        // ---- O^T += V^T.P^T over 8 m-tiles of 16 head dims
+        if constexpr (!kF16) {
+#pragma unroll
+            for (int mi = 0; mi < 8; ++mi) {
+                uint32_t a[4];  // {tok 0-7 dims lo, tok 0-7 dims hi, tok 8-15 lo, tok 8-15 hi}
+                ldsm_x4_trans(a, v_s + swz(8 * (mtx >> 1) + r, 2 * mi + (mtx & 1)));
+                if (partial) {
+                    a[0] &= mask_a;
+                    a[1] &= mask_a;
+                    a[2] &= mask_b;
+                    a[3] &= mask_b;
+                }
+                mma_16816<false>(o[mi], a[0], a[1], a[2], a[3], pb0, pb1);
+            }
+        } else {
+#pragma unroll
+            for (int mq = 0; mq < 4; ++mq) {
+                uint32_t w[4];  // {(tok 0-7, mt 2mq), (tok 8-15, 2mq), (tok 0-7, 2mq+1), (tok 8-15, 2mq+1)}
+                ldsm_x4_trans(w, v_s + swz(8 * (mtx & 1) + r, 2 * mq + (mtx >> 1)));
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    // bytes of w: [t0 d2g, t0 d2g+1, t1 d2g, t1 d2g+1]; row gid <- even dim,
+                    // row gid + 8 <- odd dim
+                    uint32_t lo0 = e4m3x2_to_f16x2(__byte_perm(w[2 * h], 0u, 0x4420));
+                    uint32_t hi0 = e4m3x2_to_f16x2(__byte_perm(w[2 * h], 0u, 0x4431));
+                    uint32_t lo1 = e4m3x2_to_f16x2(__byte_perm(w[2 * h + 1], 0u, 0x4420));
+                    uint32_t hi1 = e4m3x2_to_f16x2(__byte_perm(w[2 * h + 1], 0u, 0x4431));
+                    if (partial) {
+                        lo0 &= mask_a;
+                        hi0 &= mask_a;
+                        lo1 &= mask_b;
+                        hi1 &= mask_b;
+                    }
+                    mma_16816<true>(o[2 * mq + h], lo0, hi0, lo1, hi1, pb0, pb1);
+                }
+            }
+        }
+    }
+
+    __device__ void finish(const DecodeParams& p, int32_t b, int32_t kvh, bool whole,
+                           int64_t pid) {
+        float l = l_run;  // row gid's sum over its 4 lanes
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        const float la = __shfl_sync(0xffffffffu, l, 8 * tig);      // head 2tig
+        const float lb = __shfl_sync(0xffffffffu, l, 8 * tig + 4);  // head 2tig + 1
+        const int64_t bh0 = static_cast<int64_t>(b) * p.num_q_heads + kvh * G;
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int h = 2 * tig + j;
+            if (h >= G) continue;
+            const float lh = j ? lb : la;
+            if (whole) {
+                uint16_t* out = static_cast<uint16_t*>(p.out) + (bh0 + h) * D;
+#pragma unroll
+                for (int mi = 0; mi < 8; ++mi) {
+                    out[dim_of(mi, gid)] = out_cast<uint16_t>(lh > 0.0f ? o[mi][j] / lh : 0.0f);
+                    out[dim_of(mi, gid + 8)] = out_cast<uint16_t>(lh > 0.0f ? o[mi][2 + j] / lh : 0.0f);
+                }
+            } else {
+                float* ws = p.ws_o + (pid * G + h) * D;
+#pragma unroll
+                for (int mi = 0; mi < 8; ++mi) {
+                    ws[dim_of(mi, gid)] = o[mi][j];
+                    ws[dim_of(mi, gid + 8)] = o[mi][2 + j];
+                }
+            }
+        }
+        if (!whole && gid < G && tig == 0) p.ws_ml[pid * G + gid] = make_float2(m_run, l);
+    }
+};
+
+// ======================================================================================
+// Decode kernel: grid ceil(num_ranges / 4) CTAs of 160 threads.
+// ======================================================================================
+constexpr int kConsumerWarps = 4;
+constexpr int kThreads = (kConsumerWarps + 1) * 32;
+
+template <class M>
+struct Smem {
+    static constexpr int kRingBytes = M::kStages * M::kStageBytes;
+    static constexpr int kScratch = kConsumerWarps * M::kWarpScratch;
+    static constexpr int kFlags = (2 * M::kStages * 4 + 16 + 15) / 16 * 16;  // ok, issued, abort
+    static constexpr int kBars = 2 * M::kStages * 8;
+    // dynamic shared memory is only guaranteed 16-byte aligned: pad for the ring's alignment
+    static constexpr int kBytes = M::kRingAlign + kRingBytes + kScratch + kFlags + kBars;
+    static_assert(M::kStages % kConsumerWarps == 0, "stage s feeds consumer warp s % 4");
+    static_assert(M::kStageBytes % M::kRingAlign == 0, "stages keep the ring's alignment");
+    static_assert((kRingBytes + kScratch + kFlags) % 8 == 0, "mbarriers need 8-B alignment");
+    static_assert(kBytes <= 227 * 1024, "shared memory per block");
+};
+
+template <class M, int Q_T>
+__global__ void __launch_bounds__(kThreads, M::kMinBlocks)
+    paged_decode_kernel(const DecodeParams p, const __grid_constant__ TmaMaps maps) {
+    using S = Smem<M>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + M::kRingAlign - 1) &
+        ~static_cast<uintptr_t>(M::kRingAlign - 1));
+    uint8_t* scratch = ring + S::kRingBytes;
+    int32_t* stage_ok = reinterpret_cast<int32_t*>(scratch + S::kScratch);
+    int32_t* issued_round = stage_ok + M::kStages;
+    volatile int32_t* abort_flag = issued_round + M::kStages;
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage_ok) + S::kFlags);
+    uint64_t* empty = full + M::kStages;
 
     const int32_t warp = threadIdx.x >> 5;
     const int32_t lane = threadIdx.x & 31;
-    uint8_t* ring = smem;
-    uint8_t* scratch = smem + C::kRingBytes;
-    int32_t* stage_ok = reinterpret_cast<int32_t*>(scratch + C::kConsumerWarps * C::kWarpScratch);
-    int32_t* issued_round = stage_ok + C::kStages;
-    volatile int32_t* abort_flag = issued_round + C::kStages;
-    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage_ok) + C::kFlagsBytes);
-    uint64_t* empty = full + C::kStages;
-
     pdl_wait();
     pdl_trigger();
     const int64_t T = total_tiles(p, lane);
-    const int64_t W0 = static_cast<int64_t>(blockIdx.x) * C::kConsumerWarps;
+    const int64_t W0 = static_cast<int64_t>(blockIdx.x) * kConsumerWarps;
 
-    if (warp == C::kConsumerWarps) {
+    if (warp == kConsumerWarps) {
         // ================= producer warp =================
-        Cursor cur[C::kConsumerWarps];
-        int32_t cnt[C::kConsumerWarps];
+        Cursor cur[kConsumerWarps];
+        int32_t cnt[kConsumerWarps];
         int32_t kmax = 0;
 #pragma unroll
-        for (int w = 0; w < C::kConsumerWarps; ++w) {
+        for (int w = 0; w < kConsumerWarps; ++w) {
             const int64_t lo = range_begin(W0 + w, T, p.num_ranges);
             const int64_t hi = range_begin(W0 + w + 1, T, p.num_ranges);
             cnt[w] = static_cast<int32_t>(hi - lo);
             // the first CTA also publishes every sequence's first tile for the merge
             int32_t* prefix = (blockIdx.x == 0 && w == 0) ? p.ws_seq_start : nullptr;
             if (cnt[w] > 0 || prefix != nullptr) cur[w] = locate_tile(p, lo, lane, prefix, T);
-            kmax = max(kmax, C::kConsumerWarps * cnt[w]);
+            kmax = max(kmax, kConsumerWarps * cnt[w]);
         }
         if (lane == 0) {
-            for (int s = 0; s < C::kStages; ++s) {
+            for (int s = 0; s < M::kStages; ++s) {
                 mbar_init(&full[s], 1);
                 mbar_init(&empty[s], 1);
                 issued_round[s] = -1;
@@ -359,8 +904,8 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
         int32_t q_head[kLook];
         bool q_valid[kLook];
         auto fetch = [&](int k, int i) {
-            const int w = i % C::kConsumerWarps;  // == k % 4: i == k % kLook
-            q_valid[i] = k < kmax && (k / C::kConsumerWarps) < cnt[w];
+            const int w = i % kConsumerWarps;  // == k % 4: i == k % kLook
+            q_valid[i] = k < kmax && (k / kConsumerWarps) < cnt[w];
             if (q_valid[i]) {
                 const Cursor& c = cur[w];
                 q_id[i] = p.block_table[static_cast<int64_t>(c.b) * p.max_blocks + c.jb];
@@ -370,14 +915,13 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
         };
 #pragma unroll
         for (int i = 0; i < kLook; ++i) fetch(i, i);
-        const int64_t tile_elems = static_cast<int64_t>(kBlockTokens) * D;
         for (int k0 = 0; k0 < kmax; k0 += kLook) {
 #pragma unroll
             for (int i = 0; i < kLook; ++i) {
                 const int k = k0 + i;
                 if (q_valid[i] && !*abort_flag) {
-                    const int s = k % C::kStages;
-                    const int round = k / C::kStages;
+                    const int s = k % M::kStages;
+                    const int round = k / M::kStages;
                     if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
                         report(p.dev_error, KV_DEVERR_TIMEOUT);
                         *abort_flag = 1;
@@ -387,20 +931,9 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
                         stage_ok[s] = ok;
                         issued_round[s] = round;
                         if (ok) {
-                            const int64_t tile = static_cast<int64_t>(id) * p.num_kv_heads + q_head[i];
-                            uint8_t* st = ring + s * C::kStageBytes;
-                            mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-                            bulk_copy_g2s(st, p.k_pool + tile * tile_elems * C::kElem, C::kTileBytes,
-                                          &full[s]);
-                            bulk_copy_g2s(st + C::kTileBytes, p.v_pool + tile * tile_elems * C::kElem,
-                                          C::kTileBytes, &full[s]);
-                            if constexpr (KV_T == KV_FP8_E4M3) {
-                                bulk_copy_g2s(st + 2 * C::kTileBytes, p.k_scales + tile * kBlockTokens,
-                                              C::kScaleBytes, &full[s]);
-                                bulk_copy_g2s(st + 2 * C::kTileBytes + C::kScaleBytes,
-                                              p.v_scales + tile * kBlockTokens, C::kScaleBytes,
-                                              &full[s]);
-                            }
+                            M::issue(ring + s * M::kStageBytes,
+                                     static_cast<int64_t>(id) * p.num_kv_heads + q_head[i], &full[s],
+                                     p, maps);
                         } else {
                             report(p.dev_error, KV_DEVERR_BAD_BLOCK_ID);
                             mbar_arrive(&full[s]);  // nothing to copy: the consumer skips it
@@ -412,7 +945,7 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
         }
         if (*abort_flag) {
             // drain: wait (bounded) until no copy issued by this block is in flight
-            for (int s = 0; s < C::kStages; ++s)
+            for (int s = 0; s < M::kStages; ++s)
                 if (issued_round[s] >= 0) mbar_wait_bounded(&full[s], issued_round[s] & 1);
         }
         return;
@@ -427,193 +960,38 @@ __global__ void __launch_bounds__(Cfg<KV_T, D, G>::kThreads, Cfg<KV_T, D, G>::kM
     __syncthreads();
     if (n <= 0) return;
 
-    float2* p_buf = reinterpret_cast<float2*>(scratch + warp * C::kWarpScratch);  // [16][G]
-    float* s_buf = reinterpret_cast<float*>(p_buf + kBlockTokens * G);            // [16][G]
-    float* c_buf = s_buf + kBlockTokens * G;                                       // [G]
-    const int32_t c = lane % C::kLPR;   // chunk column of this lane in a K row
-    const int32_t r0 = lane / C::kLPR;  // first K row of this lane
-    const int32_t sm_lane = lane % C::kSMLanes;
-    const int32_t sm_g = sm_lane % G;   // query head this lane's softmax values belong to
-
-    float2 q2[G][C::kQPL / 2];
-    auto load_q_group = [&]() {
-        const int64_t qbase = (static_cast<int64_t>(cur.b) * p.num_q_heads + cur.kvh * G) * D;
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int k = 0; k < C::kNCH; ++k)
-#pragma unroll
-                for (int e = 0; e < C::kChunkElems; e += 2) {
-                    const int64_t col = (c + k * C::kLPR) * C::kChunkElems + e;
-                    q2[g][(k * C::kChunkElems + e) / 2] =
-                        make_float2(load_q<Q_T>(p.q, qbase + g * D + col) * p.scale_log2,
-                                    load_q<Q_T>(p.q, qbase + g * D + col + 1) * p.scale_log2);
-                }
-    };
-    float m_run, l_run;
-    float2 o2[G][C::kDPL / 2];
-    auto reset = [&]() {
-        m_run = -INFINITY;  // running max of this lane's head (base-2 units)
-        l_run = 0.0f;       // this lane's share of the running sum
-#pragma unroll
-        for (int g = 0; g < G; ++g)
-#pragma unroll
-            for (int i = 0; i < C::kDPL / 2; ++i) o2[g][i] = make_float2(0.0f, 0.0f);
-    };
-    load_q_group();
-    reset();
+    M math;
+    math.init(lane, scratch + warp * M::kWarpScratch);
+    math.load_q(p, cur.b, cur.kvh);
+    math.reset();
     int64_t piece_start = lo;
 
     for (int j = 0; j < n; ++j) {
-        const int k = j * C::kConsumerWarps + warp;
-        const int s = k % C::kStages;
+        const int k = j * kConsumerWarps + warp;
+        const int s = k % M::kStages;
         const bool arrived =
-            __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (k / C::kStages) & 1));
+            __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (k / M::kStages) & 1));
         if (!arrived) {
             if (lane == 0) report(p.dev_error, KV_DEVERR_TIMEOUT);
             *abort_flag = 1;
         }
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return;  // output invalid (reported)
-        if (stage_ok[s]) {
-            const uint8_t* kt = ring + s * C::kStageBytes;
-            const uint8_t* vt = kt + C::kTileBytes;
-            const float* ksc = reinterpret_cast<const float*>(kt + 2 * C::kTileBytes);
-            const float* vsc = ksc + kBlockTokens;
-            const int32_t nvalid = min(kBlockTokens, cur.L - cur.jb * kBlockTokens);
-
-            // scores: partial dot products over this lane's columns, then reduce-scatter
-            float acc[C::kNV];
-#pragma unroll
-            for (int i = 0; i < C::kNR; ++i) {
-                const int row = r0 + C::kRPI * i;
-                float2 ap[G];
-#pragma unroll
-                for (int g = 0; g < G; ++g) ap[g] = make_float2(0.0f, 0.0f);
-#pragma unroll
-                for (int kk = 0; kk < C::kNCH; ++kk) {
-                    const uint4 chunk = *reinterpret_cast<const uint4*>(
-                        kt + row * (D * C::kElem) + (c + kk * C::kLPR) * 16);
-                    float2 kv[C::kChunkElems / 2];
-                    decode_chunk<KV_T>(chunk, kv);
-#pragma unroll
-                    for (int g = 0; g < G; ++g)
-#pragma unroll
-                        for (int e = 0; e < C::kChunkElems / 2; ++e)
-                            ap[g] = ffma2(q2[g][kk * C::kChunkElems / 2 + e], kv[e], ap[g]);
-                }
-#pragma unroll
-                for (int g = 0; g < G; ++g) acc[i * G + g] = ap[g].x + ap[g].y;
-            }
-            reduce_scatter<C::kNV, C::kLPR / 2>(acc, lane);
-#pragma unroll
-            for (int v = 0; v < C::kVPL; ++v) {
-                const int idx = (C::kNV >= C::kLPR) ? c * C::kVPL + v : c / (C::kLPR / C::kNV);
-                const int t = r0 + C::kRPI * (idx / G);
-                float sc = acc[v];
-                if constexpr (KV_T == KV_FP8_E4M3) sc *= ksc[t];
-                s_buf[t * G + (idx % G)] = sc;
-            }
-            __syncwarp();
-
-            // online softmax: lane handles head sm_g, tokens sm_lane/G + i*(kSMLanes/G)
-            float sv[C::kSPL];
-            float tmax = -INFINITY;
-#pragma unroll
-            for (int i = 0; i < C::kSPL; ++i) {
-                const int t = sm_lane / G + i * (C::kSMLanes / G);
-                sv[i] = (t < nvalid) ? s_buf[t * G + sm_g] : -INFINITY;
-                tmax = fmaxf(tmax, sv[i]);
-            }
-#pragma unroll
-            for (int m = G; m < C::kSMLanes; m <<= 1)
-                tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, m));
-            const float m_new = fmaxf(m_run, tmax);
-            const float corr = exp2f(m_run - m_new);
-            l_run *= corr;
-#pragma unroll
-            for (int i = 0; i < C::kSPL; ++i) {
-                const int t = sm_lane / G + i * (C::kSMLanes / G);
-                const float pr = exp2f(sv[i] - m_new);
-                l_run += pr;
-                float pv = pr;
-                if constexpr (KV_T == KV_FP8_E4M3) pv *= vsc[t];
-                if (lane < C::kSMLanes) p_buf[t * G + sm_g] = make_float2(pv, pv);
-            }
-            m_run = m_new;
-            if (lane < G) c_buf[lane] = corr;
-            __syncwarp();
-
-            // P.V: this lane's kDPL output columns for every head of the group
-#pragma unroll
-            for (int g = 0; g < G; ++g) {
-                const float cg = c_buf[g];
-#pragma unroll
-                for (int i = 0; i < C::kDPL / 2; ++i) o2[g][i] = __fmul2_rn(o2[g][i], make_float2(cg, cg));
-            }
-            const uint8_t* vrow = vt + lane * C::kDPL * C::kElem;
-            if (nvalid == kBlockTokens) {
-#pragma unroll
-                for (int t = 0; t < kBlockTokens; ++t) {
-                    float2 vv[C::kDPL / 2];
-                    load_v<KV_T, C::kDPL>(vrow + t * D * C::kElem, vv);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const float2 pp = p_buf[t * G + g];
-#pragma unroll
-                        for (int i = 0; i < C::kDPL / 2; ++i) o2[g][i] = ffma2(pp, vv[i], o2[g][i]);
-                    }
-                }
-            } else {
-                for (int t = 0; t < nvalid; ++t) {
-                    float2 vv[C::kDPL / 2];
-                    load_v<KV_T, C::kDPL>(vrow + t * D * C::kElem, vv);
-#pragma unroll
-                    for (int g = 0; g < G; ++g) {
-                        const float2 pp = p_buf[t * G + g];
-#pragma unroll
-                        for (int i = 0; i < C::kDPL / 2; ++i) o2[g][i] = ffma2(pp, vv[i], o2[g][i]);
-                    }
-                }
-            }
-        }
+        if (stage_ok[s])
+            math.tile(ring + s * M::kStageBytes, min(kBlockTokens, cur.L - cur.jb * kBlockTokens), p);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
         // ---- end of a piece: at the end of a (sequence, kv head) pair or of the range
         const bool seg_end = cur.jb + 1 == cur.nt;
         if (seg_end || j == n - 1) {
-            float l = l_run;  // sum of l over the lanes that share this lane's head
-#pragma unroll
-            for (int m = G; m < C::kSMLanes; m <<= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
-            const int64_t bh0 = static_cast<int64_t>(cur.b) * p.num_q_heads + cur.kvh * G;
-            if (seg_end && piece_start == cur.seg_start) {
-                // the whole pair was this warp's: write the output
-#pragma unroll
-                for (int g = 0; g < G; ++g) {
-                    const float lg = __shfl_sync(0xffffffffu, l, g);
-                    OutT* o = static_cast<OutT*>(p.out) + (bh0 + g) * D + lane * C::kDPL;
-#pragma unroll
-                    for (int i = 0; i < C::kDPL / 2; ++i) {
-                        o[2 * i] = out_cast<OutT>(lg > 0.0f ? o2[g][i].x / lg : 0.0f);
-                        o[2 * i + 1] = out_cast<OutT>(lg > 0.0f ? o2[g][i].y / lg : 0.0f);
-                    }
-                }
-            } else {
-                // a piece of the pair: partial (m, l, o) for the merge kernel
-                const int64_t pid = static_cast<int64_t>(cur.b) * p.num_kv_heads + cur.kvh + W;
-                if (lane < G) p.ws_ml[pid * G + lane] = make_float2(m_run, l);
-#pragma unroll
-                for (int g = 0; g < G; ++g)
-#pragma unroll
-                    for (int i = 0; i < C::kDPL / 2; ++i)
-                        *reinterpret_cast<float2*>(&p.ws_o[(pid * G + g) * D + lane * C::kDPL + 2 * i]) =
-                            o2[g][i];
-            }
+            const bool whole = seg_end && piece_start == cur.seg_start;
+            const int64_t pid = static_cast<int64_t>(cur.b) * p.num_kv_heads + cur.kvh + W;
+            math.finish(p, cur.b, cur.kvh, whole, pid);
             if (j + 1 < n) {
                 advance(cur, p);  // next pair (the range goes on)
                 piece_start = lo + j + 1;
-                load_q_group();
-                reset();
+                math.load_q(p, cur.b, cur.kvh);
+                math.reset();
             }
         } else {
             ++cur.jb;
@@ -714,71 +1092,83 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
 // ---- launch ------------------------------------------------------------------------------
 constexpr int kMaxDevices = 64;
 
-template <int KV_T, int D, int G>
-int32_t resident_ctas_per_sm() {
-    return Cfg<KV_T, D, G>::kMinBlocks;
-}
-
-template <int KV_T, int Q_T, int D, int G>
-static cudaError_t launch_one(const DecodeParams& p, cudaStream_t stream) {
-    using C = Cfg<KV_T, D, G>;
+template <class M, int Q_T, int D>
+static cudaError_t launch_one(const DecodeParams& p, const TmaMaps& maps, cudaStream_t stream) {
+    using S = Smem<M>;
     static bool attr_set[kMaxDevices] = {};  // benign race: every caller sets the same value
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= kMaxDevices || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(paged_decode_kernel<KV_T, Q_T, D, G>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+        e = cudaFuncSetAttribute(paged_decode_kernel<M, Q_T>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
         if (e != cudaSuccess) return e;
         if (dev < kMaxDevices) attr_set[dev] = true;
     }
-    const unsigned grid = static_cast<unsigned>((p.num_ranges + C::kConsumerWarps - 1) /
-                                                C::kConsumerWarps);
-    e = launch_pdl(paged_decode_kernel<KV_T, Q_T, D, G>, dim3(grid), dim3(C::kThreads),
-                   C::kSmemBytes, stream, p);
+    const unsigned grid =
+        static_cast<unsigned>((p.num_ranges + kConsumerWarps - 1) / kConsumerWarps);
+    e = launch_pdl(paged_decode_kernel<M, Q_T>, dim3(grid), dim3(kThreads), S::kBytes, stream, p,
+                   maps);
     if (e != cudaSuccess) return e;
     const int64_t warps = static_cast<int64_t>(p.batch) * p.num_q_heads;
-    return launch_pdl(paged_decode_merge_kernel<Q_T, D>, dim3(static_cast<unsigned>((warps + 3) / 4)),
-                      dim3(128), 0, stream, p);
+    return launch_pdl(paged_decode_merge_kernel<Q_T, D>,
+                      dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, stream, p);
 }
 
 template <int KV_T, int Q_T, int D>
-static cudaError_t dispatch_g(const DecodeParams& p, int32_t group, cudaStream_t s) {
+static cudaError_t dispatch_g(const DecodeParams& p, const TmaMaps& maps, int32_t group,
+                              cudaStream_t s) {
     switch (group) {
-        case 1: return launch_one<KV_T, Q_T, D, 1>(p, s);
-        case 2: return launch_one<KV_T, Q_T, D, 2>(p, s);
-        case 4: return launch_one<KV_T, Q_T, D, 4>(p, s);
-        default: return launch_one<KV_T, Q_T, D, 8>(p, s);
+        case 1: return launch_one<SimtMath<KV_T, Q_T, D, 1>, Q_T, D>(p, maps, s);
+        case 2: return launch_one<SimtMath<KV_T, Q_T, D, 2>, Q_T, D>(p, maps, s);
+        case 4: return launch_one<SimtMath<KV_T, Q_T, D, 4>, Q_T, D>(p, maps, s);
+        default: return launch_one<SimtMath<KV_T, Q_T, D, 8>, Q_T, D>(p, maps, s);
+    }
+}
+
+template <int KV_T>
+static cudaError_t dispatch_mma(const DecodeParams& p, const TmaMaps& maps, int32_t group,
+                                cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_one<MmaMath<KV_T, 1>, KV_BF16, 128>(p, maps, s);
+        case 2: return launch_one<MmaMath<KV_T, 2>, KV_BF16, 128>(p, maps, s);
+        case 4: return launch_one<MmaMath<KV_T, 4>, KV_BF16, 128>(p, maps, s);
+        default: return launch_one<MmaMath<KV_T, 8>, KV_BF16, 128>(p, maps, s);
     }
 }
 
 template <int KV_T, int Q_T>
-static cudaError_t dispatch_d(const DecodeParams& p, int32_t head_dim, int32_t group,
-                              cudaStream_t s) {
-    return head_dim == 128 ? dispatch_g<KV_T, Q_T, 128>(p, group, s)
-                           : dispatch_g<KV_T, Q_T, 64>(p, group, s);
+static cudaError_t dispatch_d(const DecodeParams& p, const TmaMaps& maps, int32_t head_dim,
+                              int32_t group, cudaStream_t s) {
+    return head_dim == 128 ? dispatch_g<KV_T, Q_T, 128>(p, maps, group, s)
+                           : dispatch_g<KV_T, Q_T, 64>(p, maps, group, s);
 }
 
 template <int KV_T>
-static cudaError_t dispatch_q(const DecodeParams& p, int32_t q_dtype, int32_t head_dim,
-                              int32_t group, cudaStream_t s) {
-    return q_dtype == KV_F32 ? dispatch_d<KV_T, KV_F32>(p, head_dim, group, s)
-                             : dispatch_d<KV_T, KV_BF16>(p, head_dim, group, s);
+static cudaError_t dispatch_q(const DecodeParams& p, const TmaMaps& maps, int32_t q_dtype,
+                              int32_t head_dim, int32_t group, cudaStream_t s) {
+    return q_dtype == KV_F32 ? dispatch_d<KV_T, KV_F32>(p, maps, head_dim, group, s)
+                             : dispatch_d<KV_T, KV_BF16>(p, maps, head_dim, group, s);
 }
 
-cudaError_t launch_paged_decode(const DecodeParams& p, int32_t kv_dtype, int32_t q_dtype,
-                                int32_t head_dim, int32_t group, cudaStream_t stream) {
+bool decode_uses_tensor_cores(int32_t kv_dtype, int32_t q_dtype, int32_t head_dim) {
+    return (kv_dtype == KV_BF16 || kv_dtype == KV_FP8_E4M3) && q_dtype == KV_BF16 &&
+           head_dim == 128;
+}
+
+cudaError_t launch_paged_decode(const DecodeParams& p, const TmaMaps& maps, int32_t kv_dtype,
+                                int32_t q_dtype, int32_t head_dim, int32_t group,
+                                cudaStream_t stream) {
+    if (decode_uses_tensor_cores(kv_dtype, q_dtype, head_dim))
+        return kv_dtype == KV_BF16 ? dispatch_mma<KV_BF16>(p, maps, group, stream)
+                                   : dispatch_mma<KV_FP8_E4M3>(p, maps, group, stream);
     switch (kv_dtype) {
-        case KV_F32: return dispatch_q<KV_F32>(p, q_dtype, head_dim, group, stream);
-        case KV_BF16: return dispatch_q<KV_BF16>(p, q_dtype, head_dim, group, stream);
-        default: return dispatch_q<KV_FP8_E4M3>(p, q_dtype, head_dim, group, stream);
+        case KV_F32: return dispatch_q<KV_F32>(p, maps, q_dtype, head_dim, group, stream);
+        case KV_BF16: return dispatch_q<KV_BF16>(p, maps, q_dtype, head_dim, group, stream);
+        default: return dispatch_q<KV_FP8_E4M3>(p, maps, q_dtype, head_dim, group, stream);
     }
 }
 
-int32_t decode_ctas_per_sm(int32_t kv_dtype, int32_t head_dim, int32_t group) {
-    (void)kv_dtype;
-    (void)head_dim;
-    return group >= 8 ? 1 : 3;
-}
+int32_t decode_ctas_per_sm(int32_t, int32_t, int32_t) { return 3; }
 
 }  // namespace pkv

@@ -1,6 +1,8 @@
 // Launchers of the paged-KV kernels, called by the C ABI layer (api.cu).
 #pragma once
 
+#include <cuda.h>
+
 #include <utility>
 
 #include "common.cuh"
@@ -60,11 +62,22 @@ struct DecodeParams {
     float scale_log2;             // scale * log2(e): scores are kept in base-2 units
 };
 
+// TMA descriptors of the K and V pools as 2-D tensors [num_blocks*Hkv*16 rows][head_dim],
+// boxes of 16 rows x 128 bytes with the 128-byte swizzle (tensor-core path only).
+struct TmaMaps {
+    CUtensorMap k;
+    CUtensorMap v;
+};
+
 // Resident decode CTAs per SM the kernels are built for (their register budget).
 int32_t decode_ctas_per_sm(int32_t kv_dtype, int32_t head_dim, int32_t group);
 
+// Whether this shape runs the tensor-core tile arithmetic (and needs TmaMaps).
+bool decode_uses_tensor_cores(int32_t kv_dtype, int32_t q_dtype, int32_t head_dim);
+
 // kv_dtype, q_dtype, head_dim and group size select the kernel instantiation.
-cudaError_t launch_paged_decode(const DecodeParams& p, int32_t kv_dtype, int32_t q_dtype,
-                                int32_t head_dim, int32_t group, cudaStream_t stream);
+cudaError_t launch_paged_decode(const DecodeParams& p, const TmaMaps& maps, int32_t kv_dtype,
+                                int32_t q_dtype, int32_t head_dim, int32_t group,
+                                cudaStream_t stream);
 
 }  // namespace pkv
