@@ -23,11 +23,11 @@
 //  * a CTA is one producer warp and four consumer warps; by default the grid
 //    is the number of CTAs resident on the GPU (persistent), so the tile
 //    stream never stalls between work items;
-//  * the producer's lane 0 walks the four consumer warps' ranges and stages
-//    each (block, kv head) K and V tile -- one contiguous 16-row span of the
-//    pool -- into a shared-memory ring through the TMA engine (no multicast),
-//    completing on mbarriers; block ids are fetched 8 tiles ahead;
-//  * stage s of the ring always feeds consumer warp s % 4;
+//  * producer lane w walks consumer warp w's range and stages each (block,
+//    kv head) K and V tile -- one contiguous 16-row span of the pool -- into
+//    that warp's stages of a shared-memory ring (stage s feeds warp s % 4)
+//    through the TMA engine (no multicast), completing on mbarriers; block
+//    ids are fetched 4 tiles ahead, and no warp's refill waits behind another;
 //  * the per-tile arithmetic is a policy:
 //      MmaMath  (bf16 or FP8 KV, head_dim 128, bf16 q): tiles land in shared
 //               memory 128-byte swizzled by 2-D TMA tensor copies; the group's
@@ -212,13 +212,12 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return r;
 }
 
-// Two E4M3 codes (low 16 bits) -> f16x2, exact.
-__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t w16) {
-    uint32_t h2;
-    asm("{\n\t.reg .b16 lo;\n\tcvt.u16.u32 lo, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, lo;\n\t}"
-        : "=r"(h2)
-        : "r"(w16));
-    return h2;
+// Four E4M3 codes -> two f16x2 (codes 0,1 -> lo; codes 2,3 -> hi), exact.
+__device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 // 2-D TMA tile load (no multicast) completing on an mbarrier; x is the
@@ -688,10 +687,11 @@ struct MmaMath {
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int ks = 2 * kq + h;
-                    mma_16816<true>(s[0], qa[ks][0], 0u, qa[ks][1], 0u, e4m3x2_to_f16x2(w[h] & 0xffffu),
-                                    e4m3x2_to_f16x2(w[h] >> 16));
-                    mma_16816<true>(s[1], qa[ks][0], 0u, qa[ks][1], 0u,
-                                    e4m3x2_to_f16x2(w[2 + h] & 0xffffu), e4m3x2_to_f16x2(w[2 + h] >> 16));
+                    uint32_t b0, b1, b2, b3;
+                    e4m3x4_to_f16x2x2(w[h], b0, b1);
+                    e4m3x4_to_f16x2x2(w[2 + h], b2, b3);
+                    mma_16816<true>(s[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
+                    mma_16816<true>(s[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
                 }
             }
         }
@@ -777,12 +777,11 @@ struct MmaMath {
                 ldsm_x4_trans(w, v_s + swz(8 * (mtx & 1) + r, 2 * mq + (mtx >> 1)));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
-                    // bytes of w: [t0 d2g, t0 d2g+1, t1 d2g, t1 d2g+1]; row gid <- even dim,
-                    // row gid + 8 <- odd dim
-                    uint32_t lo0 = e4m3x2_to_f16x2(__byte_perm(w[2 * h], 0u, 0x4420));
-                    uint32_t hi0 = e4m3x2_to_f16x2(__byte_perm(w[2 * h], 0u, 0x4431));
-                    uint32_t lo1 = e4m3x2_to_f16x2(__byte_perm(w[2 * h + 1], 0u, 0x4420));
-                    uint32_t hi1 = e4m3x2_to_f16x2(__byte_perm(w[2 * h + 1], 0u, 0x4431));
+                    // bytes of w: [t0 d2g, t0 d2g+1, t1 d2g, t1 d2g+1] -> [t0 d2g, t1 d2g,
+                    // t0 d2g+1, t1 d2g+1]; row gid <- even dim, row gid + 8 <- odd dim
+                    uint32_t lo0, hi0, lo1, hi1;
+                    e4m3x4_to_f16x2x2(__byte_perm(w[2 * h], 0u, 0x3120), lo0, hi0);
+                    e4m3x4_to_f16x2x2(__byte_perm(w[2 * h + 1], 0u, 0x3120), lo1, hi1);
                     if (partial) {
                         lo0 &= mask_a;
                         hi0 &= mask_a;
@@ -874,7 +873,6 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
         // ================= producer warp =================
         Cursor cur[kConsumerWarps];
         int32_t cnt[kConsumerWarps];
-        int32_t kmax = 0;
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
             const int64_t lo = range_begin(W0 + w, T, p.num_ranges);
@@ -883,7 +881,6 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
             // the first CTA also publishes every sequence's first tile for the merge
             int32_t* prefix = (blockIdx.x == 0 && w == 0) ? p.ws_seq_start : nullptr;
             if (cnt[w] > 0 || prefix != nullptr) cur[w] = locate_tile(p, lo, lane, prefix, T);
-            kmax = max(kmax, kConsumerWarps * cnt[w]);
         }
         if (lane == 0) {
             for (int s = 0; s < M::kStages; ++s) {
@@ -895,33 +892,39 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
             mbar_init_fence();
         }
         __syncthreads();
-        if (lane != 0) return;
+        if (lane >= kConsumerWarps) return;
 
-        // slot k feeds consumer warp k % 4 with its (k / 4)-th tile, through
-        // stage k % kStages; block ids are loaded kLook slots ahead
-        constexpr int kLook = 8;
+        // Lane w feeds consumer warp w: its j-th tile goes through stage
+        // w + 4 * (j % kPerWarp), so no warp's stage ever waits behind another
+        // warp's; block ids are loaded kLook tiles ahead.
+        constexpr int kPerWarp = M::kStages / kConsumerWarps;
+        constexpr int kLook = 4;
+        Cursor c = cur[0];
+        int32_t count = cnt[0];
+#pragma unroll
+        for (int w = 1; w < kConsumerWarps; ++w)
+            if (lane == w) {
+                c = cur[w];
+                count = cnt[w];
+            }
         int32_t q_id[kLook];
         int32_t q_head[kLook];
-        bool q_valid[kLook];
-        auto fetch = [&](int k, int i) {
-            const int w = i % kConsumerWarps;  // == k % 4: i == k % kLook
-            q_valid[i] = k < kmax && (k / kConsumerWarps) < cnt[w];
-            if (q_valid[i]) {
-                const Cursor& c = cur[w];
+        auto fetch = [&](int j, int i) {
+            if (j < count) {
                 q_id[i] = p.block_table[static_cast<int64_t>(c.b) * p.max_blocks + c.jb];
                 q_head[i] = c.kvh;
-                advance(cur[w], p);
+                advance(c, p);
             }
         };
 #pragma unroll
         for (int i = 0; i < kLook; ++i) fetch(i, i);
-        for (int k0 = 0; k0 < kmax; k0 += kLook) {
+        for (int j0 = 0; j0 < count; j0 += kLook) {
 #pragma unroll
             for (int i = 0; i < kLook; ++i) {
-                const int k = k0 + i;
-                if (q_valid[i] && !*abort_flag) {
-                    const int s = k % M::kStages;
-                    const int round = k / M::kStages;
+                const int j = j0 + i;
+                if (j < count && !*abort_flag) {
+                    const int s = lane + kConsumerWarps * (j % kPerWarp);
+                    const int round = j / kPerWarp;
                     if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
                         report(p.dev_error, KV_DEVERR_TIMEOUT);
                         *abort_flag = 1;
@@ -940,12 +943,12 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
                         }
                     }
                 }
-                fetch(k + kLook, i);
+                fetch(j + kLook, i);
             }
         }
         if (*abort_flag) {
-            // drain: wait (bounded) until no copy issued by this block is in flight
-            for (int s = 0; s < M::kStages; ++s)
+            // drain: wait (bounded) until no copy issued by this lane is in flight
+            for (int s = lane; s < M::kStages; s += kConsumerWarps)
                 if (issued_round[s] >= 0) mbar_wait_bounded(&full[s], issued_round[s] & 1);
         }
         return;
@@ -966,11 +969,11 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
     math.reset();
     int64_t piece_start = lo;
 
+    constexpr int kPerWarp = M::kStages / kConsumerWarps;
     for (int j = 0; j < n; ++j) {
-        const int k = j * kConsumerWarps + warp;
-        const int s = k % M::kStages;
+        const int s = warp + kConsumerWarps * (j % kPerWarp);
         const bool arrived =
-            __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (k / M::kStages) & 1));
+            __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (j / kPerWarp) & 1));
         if (!arrived) {
             if (lane == 0) report(p.dev_error, KV_DEVERR_TIMEOUT);
             *abort_flag = 1;
