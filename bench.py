@@ -155,6 +155,19 @@ def kv_bytes_per_step(inp) -> int:
     return tokens * spec.num_kv_heads * 2 * per_row
 
 
+def unique_kv_bytes_per_step(inp) -> int:
+    """KV bytes of distinct physical blocks read per step: a prefix shared by
+    several sequences is one set of blocks in HBM (later readers may hit L2)."""
+    spec = inp.spec
+    nshare = min(spec.shared_prefix_seqs, inp.q.shape[0])
+    if nshare <= 1:
+        return kv_bytes_per_step(inp)
+    elem = {"f32": 4, "bf16": 2, "fp8": 1}[spec.kv_dtype]
+    per_row = spec.head_dim * elem + (4 if spec.kv_dtype == "fp8" else 0)
+    dup = (nshare - 1) * spec.shared_prefix_tokens
+    return kv_bytes_per_step(inp) - dup * spec.num_kv_heads * 2 * per_row
+
+
 def describe(inp, partition: int) -> dict:
     spec = inp.spec
     return {"workload": f"{spec.name}: paged GQA decode, batch {inp.q.shape[0]}, "
@@ -408,6 +421,9 @@ def run_gpu(args, inp):
                      "ms_per_launch": round(max_decode_ms, 5)},
         "cpu_baseline": cpu,
         "gpu_launches": launches_per_step * args.steps,
+        "unique_kv": {"bytes_per_step": unique_kv_bytes_per_step(inp),
+                      "value": round(unique_kv_bytes_per_step(inp) * args.steps * world
+                                     / (max_ms * 1e-3) / 1e9, 2), "unit": "GB/s"},
         "clocks": clocks,
         "device_errors": {"warmup": err0, "timed": errs},
     }
