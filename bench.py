@@ -14,8 +14,9 @@ value    = KV bytes read per step x steps / device time, inputs resident in HBM;
 e2e      = the same metric through the binding with pinned host buffers: each
            step copies q, the new K/V rows, the block table and context lengths
            host->device and the output device->host inside the timed region;
-roofline = the decode call (decode + merge kernels) timed live with CUDA events
-           on its stream, against the measured HBM copy bandwidth;
+roofline = the decode call (decode + merge kernels): K calls back to back timed
+           with CUDA events on their stream after the steps, against the
+           measured HBM copy bandwidth;
 cpu_baseline = the double-precision CPU oracle on a bounded sample (rank 0).
 ``--impl reference`` times that oracle alone as the reference arm.
 With N > 1 (torchrun), every rank runs an independent replica on its own GPU
@@ -325,25 +326,29 @@ def run_gpu(args, inp):
     torch.cuda.synchronize(device)
     err0 = cache.errors()
 
-    # ---- timed region: K steps, decode calls bracketed by events ----
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for _ in range(args.steps)]
+    # ---- timed region: K whole steps back to back (the kernels of consecutive
+    # calls overlap their launches), then K decode calls alone for the roofline
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with ClockSampler(gpu_id(device)) as clk:
         barrier(device)
         torch.cuda.synchronize(device)
         time.sleep(0.25)  # let the clock sampler see the loaded region start
         start.record(stream)
-        for i in range(args.steps):
+        for _ in range(args.steps):
             append()
-            ev[i][0].record(stream)
             decode()
-            ev[i][1].record(stream)
         end.record(stream)
         torch.cuda.synchronize(device)
         barrier(device)
+        d0.record(stream)
+        for _ in range(args.steps):
+            decode()
+        d1.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
     elapsed_ms = start.elapsed_time(end)
-    decode_ms = float(np.mean([a.elapsed_time(b) for a, b in ev]))
+    decode_ms = d0.elapsed_time(d1) / args.steps
     errs = cache.errors()
 
     # ---- e2e: host buffers, copies inside the timed region ----
@@ -420,7 +425,7 @@ def run_gpu(args, inp):
                      "algorithmic_bytes_per_launch": nbytes,
                      "ms_per_launch": round(max_decode_ms, 5)},
         "cpu_baseline": cpu,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_step * args.steps + 2 * args.steps,
         "unique_kv": {"bytes_per_step": unique_kv_bytes_per_step(inp),
                       "value": round(unique_kv_bytes_per_step(inp) * args.steps * world
                                      / (max_ms * 1e-3) / 1e9, 2), "unit": "GB/s"},

@@ -1011,7 +1011,7 @@ template <int Q_T, int D>
 __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p) {
     using OutT = typename QType<Q_T>::T;
     constexpr int kDPL = D / 32;
-    constexpr int kBatch = 8;  // pieces whose loads are in flight together
+    constexpr int kBatch = 8;  // pieces whose partial outputs are loaded together
     pdl_wait();
     pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
@@ -1021,7 +1021,11 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
     const int32_t h = static_cast<int32_t>(bh % p.num_q_heads);
     const int32_t G = p.num_q_heads / p.num_kv_heads;
     const int32_t kvh = h / G, g = h % G;
-    const int32_t nt = seq_tiles(p.context_lens[b], p.max_context_len);
+    // three independent loads in one round trip
+    const int32_t L = p.context_lens[b];
+    const int64_t T = p.ws_seq_start[p.batch];
+    const int64_t seq0 = p.ws_seq_start[b];
+    const int32_t nt = seq_tiles(L, p.max_context_len);
     OutT* out = static_cast<OutT*>(p.out) + bh * D + lane * kDPL;
     if (nt == 0) {
 #pragma unroll
@@ -1029,65 +1033,80 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
         if (lane == 0 && g == 0 && kvh == 0) report(p.dev_error, KV_DEVERR_BAD_CONTEXT_LEN);
         return;
     }
-    const int64_t T = p.ws_seq_start[p.batch];
-    const int64_t a = static_cast<int64_t>(p.ws_seq_start[b]) + static_cast<int64_t>(kvh) * nt;
+    const int64_t a = seq0 + static_cast<int64_t>(kvh) * nt;
     const int64_t w_first = range_of(a, T, p.num_ranges);
     const int64_t w_last = range_of(a + nt - 1, T, p.num_ranges);
     if (w_first == w_last) return;  // the pair was one range's: written by the decode kernel
     const int64_t s = static_cast<int64_t>(b) * p.num_kv_heads + kvh;
     const int32_t npieces = static_cast<int32_t>(w_last - w_first + 1);
-    // pieces are (pair s, range W) for the non-empty ranges W in [w_first, w_last];
-    // piece id s + W (see the decode kernel)
+    // pieces are (pair s, range W) for the non-empty ranges W in [w_first, w_last],
+    // with piece id s + W (see the decode kernel); ranges are never empty when T >= N
+    const bool all_ranges_full = T >= p.num_ranges;
     auto piece_id = [&](int32_t i) -> int64_t {
         const int64_t W = w_first + i;
+        if (all_ranges_full) return s + W;
         return range_begin(W, T, p.num_ranges) < range_begin(W + 1, T, p.num_ranges) ? s + W : -1;
     };
-    float M = -INFINITY;
-    for (int i = lane; i < npieces; i += 32) {
-        const int64_t pid = piece_id(i);
-        if (pid >= 0) M = fmaxf(M, p.ws_ml[pid * G + g].x);
-    }
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
     float o[kDPL];
 #pragma unroll
     for (int j = 0; j < kDPL; ++j) o[j] = 0.0f;
     float l = 0.0f;
-    if (M != -INFINITY) {
-        for (int i0 = 0; i0 < npieces; i0 += 32) {
-            // lane i holds piece i0+i's id and weight; the warp then folds the pieces
-            // in kBatch at a time with all their loads issued before the first FMA
-            const int64_t pl = (i0 + lane < npieces) ? piece_id(i0 + lane) : -1;
-            float wl = 0.0f;
-            if (pl >= 0) {
-                const float2 ml = p.ws_ml[pl * G + g];
-                wl = exp2f(ml.x - M);
-                l += wl * ml.y;
+    float M = -INFINITY;
+    for (int i0 = 0; i0 < npieces; i0 += 32) {
+        // lane i: piece i0+i's (m, l); every lane: this round's first kBatch partial
+        // outputs -- both sets of loads are in flight together
+        const int64_t pl = (i0 + lane < npieces) ? piece_id(i0 + lane) : -1;
+        const float2 ml = pl >= 0 ? p.ws_ml[pl * G + g] : make_float2(-INFINITY, 0.0f);
+        const int cnt = min(32, npieces - i0);
+        float v[kBatch][kDPL];
+        int64_t pids[kBatch];
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            pids[u] = __shfl_sync(0xffffffffu, pl, u);
+            const bool use = u < cnt && pids[u] >= 0;
+            const float* src = p.ws_o + ((use ? pids[u] : 0) * G + g) * D + lane * kDPL;
+#pragma unroll
+            for (int j = 0; j < kDPL; ++j) v[u][j] = use ? src[j] : 0.0f;
+        }
+        // running max over the pieces seen so far; rescale what is accumulated
+        float mr = ml.x;
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, m));
+        const float M_new = fmaxf(M, mr);
+        if (M_new == -INFINITY) continue;  // nothing but empty pieces so far
+        const float c = exp2f(M - M_new);
+        l *= c;
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) o[j] *= c;
+        M = M_new;
+        const float wl = pl >= 0 ? exp2f(ml.x - M) : 0.0f;
+        l += wl * ml.y;  // lane-partial, reduced at the end
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const float w = __shfl_sync(0xffffffffu, wl, u);
+#pragma unroll
+            for (int j = 0; j < kDPL; ++j) o[j] = fmaf(w, v[u][j], o[j]);
+        }
+        for (int u0 = kBatch; u0 < cnt; u0 += kBatch) {
+#pragma unroll
+            for (int u = 0; u < kBatch; ++u) {
+                const int i = (u0 + u) & 31;
+                pids[u] = __shfl_sync(0xffffffffu, pl, i);
+                const bool use = u0 + u < cnt && pids[u] >= 0;
+                const float* src = p.ws_o + ((use ? pids[u] : 0) * G + g) * D + lane * kDPL;
+#pragma unroll
+                for (int j = 0; j < kDPL; ++j) v[u][j] = use ? src[j] : 0.0f;
             }
-            const int cnt = min(32, npieces - i0);
-            for (int i1 = 0; i1 < cnt; i1 += kBatch) {
-                float v[kBatch][kDPL];
-                float w[kBatch];
 #pragma unroll
-                for (int u = 0; u < kBatch; ++u) {
-                    const int i = (i1 + u) & 31;
-                    w[u] = __shfl_sync(0xffffffffu, wl, i);
-                    const int64_t pid = __shfl_sync(0xffffffffu, pl, i);
-                    const bool use = i1 + u < cnt && pid >= 0;
-                    const float* src = p.ws_o + ((use ? pid : 0) * G + g) * D + lane * kDPL;
+            for (int u = 0; u < kBatch; ++u) {
+                const float w = __shfl_sync(0xffffffffu, wl, (u0 + u) & 31);
 #pragma unroll
-                    for (int j = 0; j < kDPL; ++j) v[u][j] = use ? src[j] : 0.0f;
-                    if (!use) w[u] = 0.0f;
-                }
-#pragma unroll
-                for (int u = 0; u < kBatch; ++u)
-#pragma unroll
-                    for (int j = 0; j < kDPL; ++j) o[j] = fmaf(w[u], v[u][j], o[j]);
+                for (int j = 0; j < kDPL; ++j) o[j] = fmaf(w, v[u][j], o[j]);
             }
         }
-#pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
     }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
 #pragma unroll
     for (int j = 0; j < kDPL; ++j) out[j] = out_cast<OutT>(l > 0.0f ? o[j] / l : 0.0f);
 }

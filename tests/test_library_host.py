@@ -76,8 +76,9 @@ def test_workspace_bytes_and_ranges():
     d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
     # balanced default: one range per consumer warp of 3 CTAs x 4 warps on each of 148 SMs
     assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 0) == 148 * 3 * 4
-    # group 8 kernels keep one CTA per SM
-    assert pk.paged_decode_num_ranges(d, 32, 64, 4096, 0) == 148 * 4
+    # the range count does not depend on the group size or q dtype (the workspace
+    # size must not either); group-8 fp32 kernels, one CTA per SM, run it in waves
+    assert pk.paged_decode_num_ranges(d, 32, 64, 4096, 0) == 148 * 3 * 4
     # explicit partition: ranges of at most 512 tokens over 32 x 8 x 256 tiles
     assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 512) == 32 * 8 * 256 // 32
     assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 500) == 0
