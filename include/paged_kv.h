@@ -75,8 +75,9 @@ typedef enum {
  *
  * Layout of each pool, row-major: [num_blocks][num_kv_heads][block_size][head_dim]
  * so the 16 tokens of one (physical block, kv head) pair are one contiguous
- * span of block_size*head_dim elements.  FP8 pools have a matching fp32 scale
- * pool per K and V laid out [num_blocks][num_kv_heads][block_size].
+ * span of block_size*head_dim elements.  An FP8 cache also has ONE fp32 scale
+ * pool laid out [num_blocks][num_kv_heads][2][block_size]: for each (block,
+ * kv head) the 16 K row scales then the 16 V row scales, 128 contiguous bytes.
  */
 typedef struct {
     int32_t num_blocks;
@@ -86,7 +87,7 @@ typedef struct {
     int32_t dtype;           /* kv_dtype */
     int32_t elem_bytes;      /* 4, 2 or 1 */
     uint64_t kv_bytes;       /* bytes of ONE pool (K or V) */
-    uint64_t scale_bytes;    /* bytes of ONE scale pool (FP8 only, else 0) */
+    uint64_t scale_bytes;    /* bytes of the scale pool (FP8 only, else 0) */
     int64_t stride_block;    /* elements between consecutive physical blocks */
     int64_t stride_head;     /* elements between consecutive kv heads of a block */
     int64_t stride_slot;     /* elements between consecutive tokens of a block */
@@ -133,12 +134,12 @@ KV_API kv_status compute_slot_mapping(const int32_t* block_table, int32_t batch,
  *     a = max |x| (fp32),  scale = a / 448 (IEEE fp32 division),
  *     code = E4M3(x / scale) (IEEE division, round to nearest even,
  *            saturating to ±448),  and scale = 0, codes 0x00 when a == 0;
- *   k_scales, v_scales : device fp32 scale pools [num_blocks][num_kv_heads][16]
- *   (must be NULL for non-FP8 pools).  Rows must be finite.
+ *   scales : device fp32 scale pool [num_blocks][num_kv_heads][2][16] (K row
+ *   scales, then V row scales), NULL for non-FP8 pools.  Rows must be finite.
  * Two tokens given the same slot race (last writer unspecified).
  */
 KV_API kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool,
-                            float* k_scales, float* v_scales,
+                            float* scales,
                             const void* k_new, const void* v_new, kv_dtype src_dtype,
                             const int64_t* slot_mapping, int32_t num_tokens,
                             int32_t* dev_error, kv_stream_t stream);
@@ -185,7 +186,7 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  *   out          : device [batch][num_q_heads][head_dim] in q_dtype
  *   q            : device [batch][num_q_heads][head_dim], q_dtype F32 or BF16
  *   k_pool/v_pool: device pools (layout above)
- *   k_scales/v_scales : device fp32 scale pools, non-NULL iff the pool is FP8
+ *   scales       : device fp32 scale pool (layout above), non-NULL iff the pool is FP8
  *   block_table  : device int32 [batch][max_blocks_per_seq]; entries past
  *                  ceil(L/16) are never read
  *   context_lens : device int32 [batch], each in [1, max_context_len]
@@ -203,7 +204,7 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  */
 KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
                                  kv_dtype q_dtype, const void* k_pool, const void* v_pool,
-                                 const float* k_scales, const float* v_scales,
+                                 const float* scales,
                                  const int32_t* block_table, int32_t max_blocks_per_seq,
                                  const int32_t* context_lens, int32_t batch,
                                  int32_t num_q_heads, int32_t max_context_len, float scale,
@@ -248,7 +249,7 @@ KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, con
  */
 KV_API kv_status paged_decode_attention_static_workspace(
     const kv_pool_desc* pool, void* out, const void* q, kv_dtype q_dtype, const void* k_pool,
-    const void* v_pool, const float* k_scales, const float* v_scales, const int32_t* block_table,
+    const void* v_pool, const float* scales, const int32_t* block_table,
     int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
     int32_t max_context_len, float scale, int32_t partition_tokens, int32_t* dev_error,
     kv_stream_t stream);

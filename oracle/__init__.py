@@ -126,14 +126,16 @@ def scatter_to_pool(pool: np.ndarray, rows: np.ndarray, slots: np.ndarray,
 
 
 def scatter_scales_to_pool(scale_pool: np.ndarray, scales: np.ndarray, slots: np.ndarray,
-                           block_size: int = 16) -> np.ndarray:
-    """Same as scatter_to_pool for the FP8 scale pool [num_blocks][kv_heads][block_size]."""
+                           which: int, block_size: int = 16) -> np.ndarray:
+    """Expected FP8 scale pool after a write: the pool is laid out
+    [num_blocks][kv_heads][2][block_size] (K row scales, then V row scales, of
+    each (block, kv head)); ``which`` is 0 for K, 1 for V.  scales: [T][kv_heads]."""
     out = scale_pool.copy()
     for t, slot in enumerate(slots.tolist()):
         if slot < 0:
             continue
         blk, off = divmod(int(slot), block_size)
-        out[blk, :, off] = scales[t, :]
+        out[blk, :, which, off] = scales[t, :]
     return out
 
 

@@ -64,14 +64,14 @@ def _load() -> ctypes.CDLL:
         sig = {
             "kv_pool_create": (_I32, [_I32, _I32, _I32, _I32, _I32, desc_p]),
             "compute_slot_mapping": (_I32, [_P, _I32, _I32, _I32, _P, _P, _I32, _P, _P, _P]),
-            "reshape_and_cache": (_I32, [desc_p, _P, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
+            "reshape_and_cache": (_I32, [desc_p, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
             "paged_decode_num_ranges": (_I32, [desc_p, _I32, _I32, _I32, _I32]),
             "paged_decode_workspace_bytes": (_SZ, [desc_p, _I32, _I32, _I32, _I32]),
-            "paged_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _I32, _P,
+            "paged_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P,
                                               _I32, _I32, _I32, ctypes.c_float, _I32, _P, _SZ,
                                               _P, _P]),
             "paged_decode_attention_static_workspace": (
-                _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
+                _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
                        ctypes.c_float, _I32, _P, _P]),
             "kv_status_string": (ctypes.c_char_p, [_I32]),
         }
@@ -129,23 +129,24 @@ def kv_pool_create(num_blocks: int, block_size: int, num_kv_heads: int, head_dim
 
 
 def empty_pool(desc: KvPoolDesc, device, fill: float | int | None = None):
-    """Allocate (k_pool, v_pool, k_scales, v_scales) tensors for a descriptor
-    (scales None unless FP8).  ``fill`` poisons every element (NaN, or a byte)."""
+    """Allocate (k_pool, v_pool, scales) tensors for a descriptor: pools
+    [num_blocks][kv_heads][16][head_dim]; scales [num_blocks][kv_heads][2][16]
+    fp32 (K then V row scales) for FP8, else None.  ``fill`` poisons every
+    element (NaN, or a byte; scales get NaN)."""
     shape = (desc.num_blocks, desc.num_kv_heads, desc.block_size, desc.head_dim)
     dt = {KV_F32: torch.float32, KV_BF16: torch.bfloat16, KV_FP8_E4M3: torch.uint8}[desc.dtype]
     k = torch.empty(shape, dtype=dt, device=device)
     v = torch.empty(shape, dtype=dt, device=device)
-    ks = vs = None
+    scales = None
     if desc.dtype == KV_FP8_E4M3:
-        ks = torch.empty(shape[:3], dtype=torch.float32, device=device)
-        vs = torch.empty(shape[:3], dtype=torch.float32, device=device)
+        scales = torch.empty((desc.num_blocks, desc.num_kv_heads, 2, desc.block_size),
+                             dtype=torch.float32, device=device)
     if fill is not None:
         for t in (k, v):
             t.fill_(fill)
-        for t in (ks, vs):
-            if t is not None:
-                t.fill_(float("nan"))
-    return k, v, ks, vs
+        if scales is not None:
+            scales.fill_(float("nan"))
+    return k, v, scales
 
 
 def compute_slot_mapping(block_table: torch.Tensor, seq_ids: torch.Tensor,
@@ -160,11 +161,11 @@ def compute_slot_mapping(block_table: torch.Tensor, seq_ids: torch.Tensor,
 
 
 def reshape_and_cache(pool: KvPoolDesc, k_pool: torch.Tensor, v_pool: torch.Tensor,
-                      k_scales: torch.Tensor | None, v_scales: torch.Tensor | None,
-                      k_new: torch.Tensor, v_new: torch.Tensor, slot_mapping: torch.Tensor,
-                      dev_error: torch.Tensor | None = None, stream=None) -> None:
+                      scales: torch.Tensor | None, k_new: torch.Tensor, v_new: torch.Tensor,
+                      slot_mapping: torch.Tensor, dev_error: torch.Tensor | None = None,
+                      stream=None) -> None:
     _check("reshape_and_cache", _load().reshape_and_cache(
-        ctypes.byref(pool), _ptr(k_pool), _ptr(v_pool), _ptr(k_scales), _ptr(v_scales),
+        ctypes.byref(pool), _ptr(k_pool), _ptr(v_pool), _ptr(scales),
         _ptr(k_new), _ptr(v_new), kv_dtype_of(k_new), _ptr(slot_mapping), k_new.shape[0],
         _ptr(dev_error), _stream(stream)))
 
@@ -183,7 +184,7 @@ def paged_decode_workspace_bytes(pool: KvPoolDesc, batch: int, num_q_heads: int,
 
 def paged_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
                            k_pool: torch.Tensor, v_pool: torch.Tensor,
-                           k_scales: torch.Tensor | None, v_scales: torch.Tensor | None,
+                           scales: torch.Tensor | None,
                            block_table: torch.Tensor, context_lens: torch.Tensor,
                            max_context_len: int, scale: float, partition_tokens: int = 0,
                            workspace: torch.Tensor | None = None,
@@ -192,7 +193,7 @@ def paged_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("paged_decode_attention", _load().paged_decode_attention(
         ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool), _ptr(v_pool),
-        _ptr(k_scales), _ptr(v_scales), _ptr(block_table), block_table.shape[1],
+        _ptr(scales), _ptr(block_table), block_table.shape[1],
         _ptr(context_lens), batch, num_q_heads, max_context_len, float(scale),
         partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream)))
     return out
@@ -200,7 +201,7 @@ def paged_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
 
 def paged_decode_attention_static_workspace(
         pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor, k_pool: torch.Tensor,
-        v_pool: torch.Tensor, k_scales: torch.Tensor | None, v_scales: torch.Tensor | None,
+        v_pool: torch.Tensor, scales: torch.Tensor | None,
         block_table: torch.Tensor, context_lens: torch.Tensor, max_context_len: int,
         scale: float, partition_tokens: int = 0, dev_error: torch.Tensor | None = None,
         stream=None) -> torch.Tensor:
@@ -211,7 +212,7 @@ def paged_decode_attention_static_workspace(
     _check("paged_decode_attention_static_workspace",
            _load().paged_decode_attention_static_workspace(
                ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool),
-               _ptr(v_pool), _ptr(k_scales), _ptr(v_scales), _ptr(block_table),
+               _ptr(v_pool), _ptr(scales), _ptr(block_table),
                block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
                float(scale), partition_tokens, _ptr(dev_error), _stream(stream)))
     return out

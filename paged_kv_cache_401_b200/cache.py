@@ -25,8 +25,7 @@ class PagedKVCache:
         fill = None
         if poison:
             fill = 0x7F if dtype == "fp8" else float("nan")
-        self.k_pool, self.v_pool, self.k_scales, self.v_scales = empty_pool(self.desc,
-                                                                            self.device, fill)
+        self.k_pool, self.v_pool, self.scales = empty_pool(self.desc, self.device, fill)
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
 
     # ---- a1 + a2/a3: slots and cache write ---------------------------------------
@@ -37,8 +36,8 @@ class PagedKVCache:
             slots = torch.empty(seq_ids.numel(), dtype=torch.int64, device=self.device)
         compute_slot_mapping(block_table, seq_ids, positions, slots, BLOCK_SIZE, self.dev_error,
                              stream)
-        reshape_and_cache(self.desc, self.k_pool, self.v_pool, self.k_scales, self.v_scales,
-                          k_new, v_new, slots, self.dev_error, stream)
+        reshape_and_cache(self.desc, self.k_pool, self.v_pool, self.scales, k_new, v_new, slots,
+                          self.dev_error, stream)
         return slots
 
     # ---- a4..a10: paged split-K decode + merge --------------------------------------
@@ -61,8 +60,8 @@ class PagedKVCache:
         if workspace is None:
             workspace = self.alloc_workspace(q.shape[0], q.shape[1], max_context_len,
                                              partition_tokens)
-        return paged_decode_attention(self.desc, out, q, self.k_pool, self.v_pool, self.k_scales,
-                                      self.v_scales, block_table, context_lens, max_context_len,
+        return paged_decode_attention(self.desc, out, q, self.k_pool, self.v_pool, self.scales,
+                                      block_table, context_lens, max_context_len,
                                       scale, partition_tokens, workspace, self.dev_error, stream)
 
     def errors(self) -> int:

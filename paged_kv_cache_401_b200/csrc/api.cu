@@ -101,7 +101,7 @@ kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_
     d.stride_block = d.stride_head * num_kv_heads;
     d.kv_bytes = static_cast<uint64_t>(d.stride_block) * num_blocks * d.elem_bytes;
     d.scale_bytes = dtype == KV_FP8_E4M3
-                        ? static_cast<uint64_t>(num_blocks) * num_kv_heads * block_size * 4u
+                        ? static_cast<uint64_t>(num_blocks) * num_kv_heads * 2u * block_size * 4u
                         : 0u;
     *out = d;
     return KV_OK;
@@ -125,7 +125,7 @@ kv_status compute_slot_mapping(const int32_t* block_table, int32_t batch,
 }
 
 kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool,
-                            float* k_scales, float* v_scales, const void* k_new,
+                            float* scales, const void* k_new,
                             const void* v_new, kv_dtype src_dtype, const int64_t* slot_mapping,
                             int32_t num_tokens, int32_t* dev_error, kv_stream_t stream) {
     if (!valid_pool(pool) || num_tokens < 0) return KV_ERR_INVALID_ARGUMENT;
@@ -140,13 +140,13 @@ kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool
     cudaError_t e;
     if (pool->dtype == KV_FP8_E4M3) {
         if (src_dtype != KV_F32 && src_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
-        if (k_scales == nullptr || v_scales == nullptr) return KV_ERR_INVALID_ARGUMENT;
-        e = pkv::launch_cache_fp8(src_dtype, pool->head_dim, k_pool, v_pool, k_scales, v_scales,
+        if (scales == nullptr) return KV_ERR_INVALID_ARGUMENT;
+        e = pkv::launch_cache_fp8(src_dtype, pool->head_dim, k_pool, v_pool, scales,
                                   k_new, v_new, slot_mapping, num_tokens, pool->num_kv_heads,
                                   num_slots, dev_error, s);
     } else {
         if (src_dtype != pool->dtype) return KV_ERR_UNSUPPORTED;
-        if (k_scales != nullptr || v_scales != nullptr) return KV_ERR_INVALID_ARGUMENT;
+        if (scales != nullptr) return KV_ERR_INVALID_ARGUMENT;
         e = pkv::launch_cache_copy(k_pool, v_pool, k_new, v_new, slot_mapping, num_tokens,
                                    pool->num_kv_heads, pool->head_dim * pool->elem_bytes,
                                    num_slots, current_sm_count(), dev_error, s);
@@ -203,7 +203,7 @@ size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
 
 kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
                                  kv_dtype q_dtype, const void* k_pool, const void* v_pool,
-                                 const float* k_scales, const float* v_scales,
+                                 const float* scales,
                                  const int32_t* block_table, int32_t max_blocks_per_seq,
                                  const int32_t* context_lens, int32_t batch,
                                  int32_t num_q_heads, int32_t max_context_len, float scale,
@@ -233,9 +233,8 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
         return KV_ERR_INVALID_ARGUMENT;
     const bool fp8 = pool->dtype == KV_FP8_E4M3;
-    if (fp8 != (k_scales != nullptr) || fp8 != (v_scales != nullptr))
-        return KV_ERR_INVALID_ARGUMENT;
-    if (fp8 && (!aligned16(k_scales) || !aligned16(v_scales))) return KV_ERR_INVALID_ARGUMENT;
+    if (fp8 != (scales != nullptr)) return KV_ERR_INVALID_ARGUMENT;
+    if (fp8 && !aligned16(scales)) return KV_ERR_INVALID_ARGUMENT;
 
     const int32_t ranges =
         paged_decode_num_ranges(pool, batch, num_q_heads, max_context_len, partition_tokens);
@@ -249,8 +248,7 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     p.q = q;
     p.k_pool = static_cast<const uint8_t*>(k_pool);
     p.v_pool = static_cast<const uint8_t*>(v_pool);
-    p.k_scales = k_scales;
-    p.v_scales = v_scales;
+    p.scales = scales;
     p.block_table = block_table;
     p.context_lens = context_lens;
     p.dev_error = dev_error;

@@ -67,7 +67,7 @@ __global__ void cache_copy_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restr
 //   (IEEE division, RNE, saturating); a == 0 -> scale 0 and codes 0.
 template <int SRC_T, int D>
 __global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
-                                 float* __restrict__ k_scales, float* __restrict__ v_scales,
+                                 float* __restrict__ scales,
                                  const void* __restrict__ k_new, const void* __restrict__ v_new,
                                  const int64_t* __restrict__ slots, int32_t num_tokens,
                                  int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error) {
@@ -120,7 +120,9 @@ __global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restri
     } else {
         *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(codes);
     }
-    if (lane == 0) (which ? v_scales : k_scales)[rowi] = (a == 0.0f) ? 0.0f : s;
+    // scale pool [block][head][K|V][16]: one 128-byte line per (block, head)
+    if (lane == 0)
+        scales[((blk * num_kv_heads + h) * 2 + which) * kBlockTokens + off] = (a == 0.0f) ? 0.0f : s;
 }
 
 // ---- launchers ------------------------------------------------------------------
@@ -150,7 +152,7 @@ cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, con
 }
 
 cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, void* v_pool,
-                             float* k_scales, float* v_scales, const void* k_new,
+                             float* scales, const void* k_new,
                              const void* v_new, const int64_t* slots, int32_t num_tokens,
                              int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
                              cudaStream_t stream) {
@@ -161,7 +163,7 @@ cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, 
     auto* vp = static_cast<uint8_t*>(v_pool);
     auto go = [&](auto kernel) {
         return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
-                          kp, vp, k_scales, v_scales, k_new, v_new, slots, num_tokens,
+                          kp, vp, scales, k_new, v_new, slots, num_tokens,
                           num_kv_heads, num_slots, dev_error);
     };
     if (src_dtype == KV_F32 && head_dim == 128) return go(cache_fp8_kernel<KV_F32, 128>);

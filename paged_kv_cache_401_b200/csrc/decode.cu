@@ -23,6 +23,7 @@
 //  * a CTA is one producer warp and four consumer warps; by default the grid
 //    is the number of CTAs resident on the GPU (persistent), so the tile
 //    stream never stalls between work items;
+//  * FP8 row scales of a tile (16 K then 16 V) are one 128-byte line;
 //  * producer lane w walks consumer warp w's range and stages each (block,
 //    kv head) K and V tile -- one contiguous 16-row span of the pool -- into
 //    that warp's stages of a shared-memory ring (stage s feeds warp s % 4)
@@ -337,8 +338,8 @@ struct SimtMath {
     using OutT = typename QType<Q_T>::T;
     static constexpr int kElem = KvElem<KV_T>::kBytes;
     static constexpr int kTileBytes = kBlockTokens * D * kElem;              // K or V tile
-    static constexpr int kScaleBytes = (KV_T == KV_FP8_E4M3) ? kBlockTokens * 4 : 0;
-    static constexpr int kStageBytes = 2 * kTileBytes + 2 * kScaleBytes;
+    static constexpr int kScaleBytes = (KV_T == KV_FP8_E4M3) ? 2 * kBlockTokens * 4 : 0;  // K|V
+    static constexpr int kStageBytes = 2 * kTileBytes + kScaleBytes;
     static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
     static constexpr int kRingAlign = 128;
     static constexpr int kChunkElems = 16 / kElem;                           // per 16-byte load
@@ -369,11 +370,8 @@ struct SimtMath {
         mbar_arrive_expect_tx(bar, kStageBytes);
         bulk_copy_g2s(st, p.k_pool + off, kTileBytes, bar);
         bulk_copy_g2s(st + kTileBytes, p.v_pool + off, kTileBytes, bar);
-        if constexpr (KV_T == KV_FP8_E4M3) {
-            bulk_copy_g2s(st + 2 * kTileBytes, p.k_scales + tile * kBlockTokens, kScaleBytes, bar);
-            bulk_copy_g2s(st + 2 * kTileBytes + kScaleBytes, p.v_scales + tile * kBlockTokens,
-                          kScaleBytes, bar);
-        }
+        if constexpr (KV_T == KV_FP8_E4M3)
+            bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
     }
 
     // ---- consumer side
@@ -585,8 +583,8 @@ struct MmaMath {
     static constexpr int kBoxes = kRowBytes / 128;
     static constexpr int kBoxBytes = kBlockTokens * 128;
     static constexpr int kTileBytes = kBlockTokens * kRowBytes;
-    static constexpr int kScaleBytes = kF16 ? kBlockTokens * 4 : 0;
-    static constexpr int kStageBytes = (2 * kTileBytes + 2 * kScaleBytes + 1023) / 1024 * 1024;
+    static constexpr int kScaleBytes = kF16 ? 2 * kBlockTokens * 4 : 0;  // K then V row scales
+    static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
     static constexpr int kStages = kF16 ? 12 : 8;                 // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr int kWarpScratch = 0;
@@ -596,17 +594,14 @@ struct MmaMath {
     __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
                                  const TmaMaps& maps) {
         const int32_t row = static_cast<int32_t>(tile * kBlockTokens);
-        mbar_arrive_expect_tx(bar, 2 * kTileBytes + 2 * kScaleBytes);
+        mbar_arrive_expect_tx(bar, 2 * kTileBytes + kScaleBytes);
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
             tma_load_2d(st + bx * kBoxBytes, &maps.k, bx * kBoxCols, row, bar);
             tma_load_2d(st + kTileBytes + bx * kBoxBytes, &maps.v, bx * kBoxCols, row, bar);
         }
-        if constexpr (kF16) {
-            bulk_copy_g2s(st + 2 * kTileBytes, p.k_scales + tile * kBlockTokens, kScaleBytes, bar);
-            bulk_copy_g2s(st + 2 * kTileBytes + kScaleBytes, p.v_scales + tile * kBlockTokens,
-                          kScaleBytes, bar);
-        }
+        if constexpr (kF16)
+            bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
     }
 
     // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile.

@@ -37,7 +37,7 @@ cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, con
                               int32_t* dev_error, cudaStream_t stream);
 
 cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, void* v_pool,
-                             float* k_scales, float* v_scales, const void* k_new,
+                             float* scales, const void* k_new,
                              const void* v_new, const int64_t* slots, int32_t num_tokens,
                              int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
                              cudaStream_t stream);
@@ -48,8 +48,7 @@ struct DecodeParams {
     const void* q;                // [B][Hq][D]
     const uint8_t* k_pool;        // [NB][Hkv][16][D]
     const uint8_t* v_pool;
-    const float* k_scales;        // [NB][Hkv][16] (FP8 only)
-    const float* v_scales;
+    const float* scales;          // [NB][Hkv][2][16]: K then V row scales (FP8 only)
     const int32_t* block_table;   // [B][max_blocks]
     const int32_t* context_lens;  // [B]
     int32_t* ws_seq_start;        // [B + 1]: first tile of each sequence, total tiles at [B]

@@ -50,7 +50,7 @@ extern "C" {
 
 KV_API kv_status paged_decode_attention_static_workspace(
     const kv_pool_desc* pool, void* out, const void* q, kv_dtype q_dtype, const void* k_pool,
-    const void* v_pool, const float* k_scales, const float* v_scales, const int32_t* block_table,
+    const void* v_pool, const float* scales, const int32_t* block_table,
     int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
     int32_t max_context_len, float scale, int32_t partition_tokens, int32_t* dev_error,
     kv_stream_t stream) {
@@ -69,7 +69,7 @@ KV_API kv_status paged_decode_attention_static_workspace(
     }
     // Every partial the merge reads is written earlier in the same call, so
     // nothing in the array needs clearing between calls.
-    return paged_decode_attention(pool, out, q, q_dtype, k_pool, v_pool, k_scales, v_scales,
+    return paged_decode_attention(pool, out, q, q_dtype, k_pool, v_pool, scales,
                                   block_table, max_blocks_per_seq, context_lens, batch,
                                   num_q_heads, max_context_len, scale, partition_tokens, ws,
                                   need > 0 ? KV_STATIC_WORKSPACE_BYTES : 0, dev_error, stream);

@@ -52,7 +52,7 @@ def test_cache_copy_bitexact(dtype, D):
     slots[5] = -1                       # padding
     slots[6] = NB * 16 + 3              # out of range: skipped, reported
     before = {id(cache.k_pool): _bits(cache.k_pool), id(cache.v_pool): _bits(cache.v_pool)}
-    pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, None, None, k.to(DEV),
+    pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, None, k.to(DEV),
                          v.to(DEV), torch.from_numpy(slots).to(DEV), cache.dev_error)
     slots_ok = slots.copy()
     slots_ok[6] = -1
@@ -88,16 +88,14 @@ def test_cache_fp8_bitexact(src, D):
     slots = rng.permutation(NB * 16)[:T].astype(np.int64)
     slots[9] = -1
     cache = PagedKVCache(NB, Hkv, D, "fp8", DEV, poison=True)
-    pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, cache.k_scales,
-                         cache.v_scales, k.to(DEV), v.to(DEV), torch.from_numpy(slots).to(DEV),
-                         cache.dev_error)
-    for pool, spool, src_t in ((cache.k_pool, cache.k_scales, k),
-                               (cache.v_pool, cache.v_scales, v)):
+    pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, cache.scales, k.to(DEV),
+                         v.to(DEV), torch.from_numpy(slots).to(DEV), cache.dev_error)
+    want_scales = np.full(tuple(cache.scales.shape), np.nan, np.float32)
+    for which, (pool, src_t) in enumerate(((cache.k_pool, k), (cache.v_pool, v))):
         codes, scales = oracle.quantize_rows(src_t.float().numpy())
         want_codes = oracle.scatter_to_pool(np.full(tuple(pool.shape), 0x7F, np.uint8), codes,
                                             slots)
-        nan_scales = np.full(tuple(spool.shape), np.nan, np.float32)
-        want_scales = oracle.scatter_scales_to_pool(nan_scales, scales, slots)
+        want_scales = oracle.scatter_scales_to_pool(want_scales, scales, slots, which)
         assert (pool.cpu().numpy() == want_codes).all()
-        assert (_bits(spool) == want_scales.view(np.int32)).all()
+    assert (_bits(cache.scales) == want_scales.view(np.int32)).all()
     assert cache.errors() == 0

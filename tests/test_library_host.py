@@ -56,7 +56,7 @@ def test_pool_geometry_llama_shape():
     assert d.kv_bytes == 8192 * 8 * 16 * 128 * 2 == 256 * 2**20
     assert d.scale_bytes == 0 and d.elem_bytes == 2
     f = pk.kv_pool_create(100, 16, 8, 64, pk.KV_FP8_E4M3)
-    assert f.kv_bytes == 100 * 8 * 16 * 64 and f.scale_bytes == 100 * 8 * 16 * 4
+    assert f.kv_bytes == 100 * 8 * 16 * 64 and f.scale_bytes == 100 * 8 * 2 * 16 * 4
 
 
 @pytest.mark.parametrize("args,status", [
@@ -93,14 +93,14 @@ def test_workspace_bytes_and_ranges():
 def _call_decode(desc, **kw):
     lib = pk.library()
     args = dict(out=4096, q=8192, q_dtype=pk.KV_BF16, k_pool=1 << 20, v_pool=2 << 20,
-                k_scales=None, v_scales=None, block_table=3 << 20, max_blocks=256,
+                scales=None, block_table=3 << 20, max_blocks=256,
                 context_lens=4 << 20, batch=32, num_q_heads=32, max_context_len=4096,
                 scale=0.088, partition=512, workspace=5 << 20, workspace_bytes=1 << 30,
                 dev_error=None, stream=None)
     args.update(kw)
     return lib.paged_decode_attention(
         ctypes.byref(desc), args["out"], args["q"], args["q_dtype"], args["k_pool"],
-        args["v_pool"], args["k_scales"], args["v_scales"], args["block_table"],
+        args["v_pool"], args["scales"], args["block_table"],
         args["max_blocks"], args["context_lens"], args["batch"], args["num_q_heads"],
         args["max_context_len"], args["scale"], args["partition"], args["workspace"],
         args["workspace_bytes"], args["dev_error"], args["stream"])
@@ -118,7 +118,7 @@ def _call_decode(desc, **kw):
      pk.KV_ERR_UNSUPPORTED),                                        # tile list >= 2^31
     (dict(q=8192 + 8), pk.KV_ERR_INVALID_ARGUMENT),                # misaligned
     (dict(k_pool=None), pk.KV_ERR_INVALID_ARGUMENT),
-    (dict(k_scales=6 << 20, v_scales=7 << 20), pk.KV_ERR_INVALID_ARGUMENT),  # scales on bf16
+    (dict(scales=6 << 20), pk.KV_ERR_INVALID_ARGUMENT),            # scales on a bf16 pool
     (dict(workspace_bytes=100), pk.KV_ERR_INVALID_ARGUMENT),       # too small
     (dict(workspace=None), pk.KV_ERR_INVALID_ARGUMENT),
     (dict(scale=float("nan")), pk.KV_ERR_INVALID_ARGUMENT),
@@ -131,7 +131,7 @@ def test_decode_host_validation(kw, status):
 def test_decode_fp8_pool_requires_scales():
     d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_FP8_E4M3)
     assert _call_decode(d) == pk.KV_ERR_INVALID_ARGUMENT
-    assert _call_decode(d, k_scales=6 << 20) == pk.KV_ERR_INVALID_ARGUMENT
+    assert _call_decode(d, scales=(6 << 20) + 4) == pk.KV_ERR_INVALID_ARGUMENT  # misaligned
 
 
 def test_decode_needs_a_workspace_even_for_one_range():
@@ -149,22 +149,22 @@ def test_cache_write_host_validation():
     lib = pk.library()
     d = pk.kv_pool_create(64, 16, 8, 128, pk.KV_BF16)
     f = pk.kv_pool_create(64, 16, 8, 128, pk.KV_FP8_E4M3)
-    ok = dict(kp=1 << 20, vp=2 << 20, ks=None, vs=None, kn=3 << 20, vn=4 << 20,
+    ok = dict(kp=1 << 20, vp=2 << 20, sc=None, kn=3 << 20, vn=4 << 20,
               src=pk.KV_BF16, slots=5 << 20, n=4)
 
     def call(desc, **kw):
         a = dict(ok)
         a.update(kw)
-        return lib.reshape_and_cache(ctypes.byref(desc), a["kp"], a["vp"], a["ks"], a["vs"],
-                                     a["kn"], a["vn"], a["src"], a["slots"], a["n"], None, None)
+        return lib.reshape_and_cache(ctypes.byref(desc), a["kp"], a["vp"], a["sc"], a["kn"],
+                                     a["vn"], a["src"], a["slots"], a["n"], None, None)
 
     assert call(d, n=0) == pk.KV_OK                                   # nothing to do
     assert call(d, src=pk.KV_F32) == pk.KV_ERR_UNSUPPORTED            # no conversion on copy
     assert call(d, kn=(3 << 20) + 4) == pk.KV_ERR_INVALID_ARGUMENT    # misaligned
-    assert call(d, ks=6 << 20) == pk.KV_ERR_INVALID_ARGUMENT          # scales on a bf16 pool
+    assert call(d, sc=6 << 20) == pk.KV_ERR_INVALID_ARGUMENT          # scales on a bf16 pool
     assert call(d, n=-1) == pk.KV_ERR_INVALID_ARGUMENT
     assert call(f) == pk.KV_ERR_INVALID_ARGUMENT                      # fp8 needs scales
-    assert call(f, ks=6 << 20, vs=7 << 20, src=pk.KV_FP8_E4M3) == pk.KV_ERR_UNSUPPORTED
+    assert call(f, sc=6 << 20, src=pk.KV_FP8_E4M3) == pk.KV_ERR_UNSUPPORTED
 
 
 def test_slot_mapping_host_validation():

@@ -37,7 +37,7 @@ def _static_call(st, partition):
     ptr = lambda t: None if t is None else t.data_ptr()  # noqa: E731
     status = lib.paged_decode_attention_static_workspace(
         ctypes.byref(c.desc), out.data_ptr(), st.q.data_ptr(), pk.kv_dtype_of(st.q),
-        c.k_pool.data_ptr(), c.v_pool.data_ptr(), ptr(c.k_scales), ptr(c.v_scales),
+        c.k_pool.data_ptr(), c.v_pool.data_ptr(), ptr(c.scales),
         st.block_table.data_ptr(), st.block_table.shape[1], st.context_lens.data_ptr(),
         st.q.shape[0], st.q.shape[1], st.max_context_len, st.inp.spec.scale, partition,
         c.dev_error.data_ptr(), torch.cuda.current_stream().cuda_stream)
@@ -82,6 +82,6 @@ def test_static_workspace_refuses_oversized_requests():
     dummy = torch.empty(16, dtype=torch.uint8, device="cuda")
     p = dummy.data_ptr()
     status = pk.library().paged_decode_attention_static_workspace(
-        ctypes.byref(desc), p, p, pk.KV_BF16, p, p, None, None, p, 4096, p, 64, 32, 1 << 16,
+        ctypes.byref(desc), p, p, pk.KV_BF16, p, p, None, p, 4096, p, 64, 32, 1 << 16,
         0.1, 256, None, torch.cuda.current_stream().cuda_stream)
     assert status == pk.KV_ERR_INVALID_ARGUMENT
