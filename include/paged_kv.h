@@ -54,7 +54,8 @@ typedef enum {
     KV_OK = 0,
     KV_ERR_INVALID_ARGUMENT = 1,
     KV_ERR_UNSUPPORTED = 2,
-    KV_ERR_CUDA = 3
+    KV_ERR_CUDA = 3,
+    KV_ERR_OUT_OF_BLOCKS = 4   /* block manager: no free block / sequence slot left */
 } kv_status;
 
 typedef enum {
@@ -253,6 +254,78 @@ KV_API kv_status paged_decode_attention_static_workspace(
     int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
     int32_t max_context_len, float scale, int32_t partition_tokens, int32_t* dev_error,
     kv_stream_t stream);
+
+/*
+ * Copy whole physical blocks: for i < num_copies, block copy_dst[i] of the K
+ * pool, the V pool and (FP8) the scale pool becomes a copy of block
+ * copy_src[i], every kv head ("KV Cache 深度解析" §三: blocks shared by
+ * several sequences; a sequence that writes into a shared, partly filled
+ * block first gets its own copy -- see kv_block_manager_append_slots).
+ *   copy_src, copy_dst : device int32 [num_copies]; a pair with an id outside
+ *   [0, num_blocks) is skipped with KV_DEVERR_BAD_BLOCK_ID.  Destinations
+ *   must be distinct and not also sources in the same call.
+ */
+KV_API kv_status paged_kv_copy_blocks(const kv_pool_desc* pool, void* k_pool, void* v_pool,
+                                      float* scales, const int32_t* copy_src,
+                                      const int32_t* copy_dst, int32_t num_copies,
+                                      int32_t* dev_error, kv_stream_t stream);
+
+/*
+ * Host block manager (host memory only; no device work).  Follows "KV Cache
+ * 深度解析" §三 (16-token blocks allocated on demand, at most one partly used
+ * block per sequence, physical blocks shared between sequences), "大模型推理为何
+ * 这么慢" (PagedAttention section: a finished request's blocks are freed at
+ * once) and the "llm-inference-optimization" notes §二 (a sequence takes a new
+ * block when it has none or its last one is full).  Sharing is by reference
+ * count; appending into a shared block that still has free slots first moves
+ * the sequence to a private copy (copy-on-write).  Policies: free blocks are a
+ * LIFO stack that initially yields 0, 1, 2, ...; a new sequence gets the
+ * lowest unused id.  Not thread-safe: one manager per caller thread.
+ */
+typedef struct kv_block_manager kv_block_manager;
+
+/* num_blocks physical blocks, up to max_seqs live sequences of up to
+ * max_blocks_per_seq blocks.  KV_ERR_INVALID_ARGUMENT for non-positive sizes. */
+KV_API kv_status kv_block_manager_create(int32_t num_blocks, int32_t max_seqs,
+                                         int32_t max_blocks_per_seq, kv_block_manager** out);
+KV_API void kv_block_manager_destroy(kv_block_manager* manager);
+KV_API int32_t kv_block_manager_num_free_blocks(const kv_block_manager* manager);
+/* Reference count of a physical block (0 = free), -1 for an invalid id. */
+KV_API int32_t kv_block_manager_refcount(const kv_block_manager* manager, int32_t block);
+
+/* A new empty sequence (KV_ERR_OUT_OF_BLOCKS when max_seqs are live). */
+KV_API kv_status kv_block_manager_add_sequence(kv_block_manager* manager, int32_t* seq_id);
+
+/* A new sequence sharing every block of `parent` (same length). */
+KV_API kv_status kv_block_manager_fork(kv_block_manager* manager, int32_t parent,
+                                       int32_t* child);
+
+/* Release a sequence: its blocks' counts drop, blocks reaching 0 are freed. */
+KV_API kv_status kv_block_manager_free_sequence(kv_block_manager* manager, int32_t seq_id);
+
+/*
+ * Reserve the slots of num_tokens new tokens, token i appended to sequence
+ * seq_ids[i] (several tokens of one sequence are taken in order):
+ *   slots[i]  : host int64, the token's slot (block * 16 + offset)
+ *   copy_src / copy_dst : host int32 of capacity >= num_tokens; on return the
+ *   first *num_copies pairs are the copy-on-write block copies to perform
+ *   (paged_kv_copy_blocks) BEFORE writing the new tokens.
+ * A batch that needs more free blocks than exist, or grows a sequence past
+ * max_blocks_per_seq, returns KV_ERR_OUT_OF_BLOCKS and changes nothing.
+ */
+KV_API kv_status kv_block_manager_append_slots(kv_block_manager* manager,
+                                               const int32_t* seq_ids, int32_t num_tokens,
+                                               int64_t* slots, int32_t* copy_src,
+                                               int32_t* copy_dst, int32_t* num_copies);
+
+/*
+ * Block table and context lengths of every sequence id in [0, max_seqs):
+ *   block_table  : host int32 [max_seqs][max_blocks_per_seq]; entries past a
+ *                  sequence's last block hold 0x7fffffff
+ *   context_lens : host int32 [max_seqs] (0 for ids not in use)
+ */
+KV_API kv_status kv_block_manager_export(const kv_block_manager* manager, int32_t* block_table,
+                                         int32_t* context_lens);
 
 /* Static, human-readable name of a status code. */
 KV_API const char* kv_status_string(kv_status status);

@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
 
 KV_F32, KV_BF16, KV_FP8_E4M3 = 0, 1, 2
 KV_OK, KV_ERR_INVALID_ARGUMENT, KV_ERR_UNSUPPORTED, KV_ERR_CUDA = 0, 1, 2, 3
+KV_ERR_OUT_OF_BLOCKS = 4
 KV_DEVERR_BAD_SLOT = 0x1
 KV_DEVERR_BAD_CONTEXT_LEN = 0x2
 KV_DEVERR_BAD_BLOCK_ID = 0x4
@@ -29,7 +30,11 @@ BLOCK_SIZE = 16
 EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
             "paged_decode_num_ranges", "paged_decode_workspace_bytes",
             "paged_decode_attention", "paged_decode_attention_static_workspace",
-            "kv_status_string")
+            "paged_kv_copy_blocks", "kv_block_manager_create", "kv_block_manager_destroy",
+            "kv_block_manager_num_free_blocks", "kv_block_manager_refcount",
+            "kv_block_manager_add_sequence", "kv_block_manager_fork",
+            "kv_block_manager_free_sequence", "kv_block_manager_append_slots",
+            "kv_block_manager_export", "kv_status_string")
 KV_STATIC_WORKSPACE_BYTES = 16 * 1024 * 1024
 
 
@@ -73,6 +78,16 @@ def _load() -> ctypes.CDLL:
             "paged_decode_attention_static_workspace": (
                 _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
                        ctypes.c_float, _I32, _P, _P]),
+            "paged_kv_copy_blocks": (_I32, [desc_p, _P, _P, _P, _P, _P, _I32, _P, _P]),
+            "kv_block_manager_create": (_I32, [_I32, _I32, _I32, _P]),
+            "kv_block_manager_destroy": (None, [_P]),
+            "kv_block_manager_num_free_blocks": (_I32, [_P]),
+            "kv_block_manager_refcount": (_I32, [_P, _I32]),
+            "kv_block_manager_add_sequence": (_I32, [_P, _P]),
+            "kv_block_manager_fork": (_I32, [_P, _I32, _P]),
+            "kv_block_manager_free_sequence": (_I32, [_P, _I32]),
+            "kv_block_manager_append_slots": (_I32, [_P, _P, _I32, _P, _P, _P, _P]),
+            "kv_block_manager_export": (_I32, [_P, _P, _P]),
             "kv_status_string": (ctypes.c_char_p, [_I32]),
         }
         for name, (res, args) in sig.items():
@@ -216,3 +231,76 @@ def paged_decode_attention_static_workspace(
                block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
                float(scale), partition_tokens, _ptr(dev_error), _stream(stream)))
     return out
+
+
+# ---------------------------------------------------------------- block manager
+def paged_kv_copy_blocks(pool: KvPoolDesc, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                         scales: torch.Tensor | None, copy_src: torch.Tensor,
+                         copy_dst: torch.Tensor, dev_error: torch.Tensor | None = None,
+                         stream=None) -> None:
+    _check("paged_kv_copy_blocks", _load().paged_kv_copy_blocks(
+        ctypes.byref(pool), _ptr(k_pool), _ptr(v_pool), _ptr(scales), _ptr(copy_src),
+        _ptr(copy_dst), copy_src.numel(), _ptr(dev_error), _stream(stream)))
+
+
+class BlockManager:
+    """Host block manager (kv_block_manager_* in include/paged_kv.h)."""
+
+    def __init__(self, num_blocks: int, max_seqs: int, max_blocks_per_seq: int):
+        lib = _load()
+        self.num_blocks, self.max_seqs, self.max_blocks_per_seq = (num_blocks, max_seqs,
+                                                                   max_blocks_per_seq)
+        self._h = ctypes.c_void_p()
+        _check("kv_block_manager_create", lib.kv_block_manager_create(
+            num_blocks, max_seqs, max_blocks_per_seq, ctypes.byref(self._h)))
+
+    def __del__(self):
+        if getattr(self, "_h", None) and self._h.value and _lib is not None:
+            _lib.kv_block_manager_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    @property
+    def num_free_blocks(self) -> int:
+        return int(_load().kv_block_manager_num_free_blocks(self._h))
+
+    def refcount(self, block: int) -> int:
+        return int(_load().kv_block_manager_refcount(self._h, block))
+
+    def add_sequence(self) -> int:
+        s = ctypes.c_int32()
+        _check("kv_block_manager_add_sequence",
+               _load().kv_block_manager_add_sequence(self._h, ctypes.byref(s)))
+        return s.value
+
+    def fork(self, parent: int) -> int:
+        c = ctypes.c_int32()
+        _check("kv_block_manager_fork", _load().kv_block_manager_fork(self._h, parent,
+                                                                       ctypes.byref(c)))
+        return c.value
+
+    def free_sequence(self, seq: int) -> None:
+        _check("kv_block_manager_free_sequence", _load().kv_block_manager_free_sequence(self._h,
+                                                                                         seq))
+
+    def append_slots(self, seq_ids):
+        """-> (slots int64 [n], copies [(src, dst), ...]) as numpy / list."""
+        import numpy as np
+        ids = np.ascontiguousarray(seq_ids, dtype=np.int32)
+        n = ids.size
+        slots = np.empty(n, dtype=np.int64)
+        src = np.empty(max(n, 1), dtype=np.int32)
+        dst = np.empty(max(n, 1), dtype=np.int32)
+        nc = ctypes.c_int32()
+        _check("kv_block_manager_append_slots", _load().kv_block_manager_append_slots(
+            self._h, ids.ctypes.data, n, slots.ctypes.data, src.ctypes.data, dst.ctypes.data,
+            ctypes.byref(nc)))
+        return slots, list(zip(src[:nc.value].tolist(), dst[:nc.value].tolist()))
+
+    def export(self):
+        """-> (block_table int32 [max_seqs][max_blocks_per_seq], context_lens int32 [max_seqs])."""
+        import numpy as np
+        table = np.empty((self.max_seqs, self.max_blocks_per_seq), dtype=np.int32)
+        lens = np.empty(self.max_seqs, dtype=np.int32)
+        _check("kv_block_manager_export", _load().kv_block_manager_export(
+            self._h, table.ctypes.data, lens.ctypes.data))
+        return table, lens

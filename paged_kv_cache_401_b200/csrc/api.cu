@@ -154,6 +154,25 @@ kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
+kv_status paged_kv_copy_blocks(const kv_pool_desc* pool, void* k_pool, void* v_pool,
+                               float* scales, const int32_t* copy_src, const int32_t* copy_dst,
+                               int32_t num_copies, int32_t* dev_error, kv_stream_t stream) {
+    if (!valid_pool(pool) || num_copies < 0) return KV_ERR_INVALID_ARGUMENT;
+    if (num_copies == 0) return KV_OK;
+    if (k_pool == nullptr || v_pool == nullptr || copy_src == nullptr || copy_dst == nullptr)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k_pool) || !aligned16(v_pool)) return KV_ERR_INVALID_ARGUMENT;
+    const bool fp8 = pool->dtype == KV_FP8_E4M3;
+    if (fp8 != (scales != nullptr) || (fp8 && !aligned16(scales))) return KV_ERR_INVALID_ARGUMENT;
+    const int64_t block_bytes = pool->stride_block * pool->elem_bytes;
+    const int64_t scale_bytes = fp8 ? static_cast<int64_t>(pool->num_kv_heads) * 2 * kBlockTokens * 4 : 0;
+    cudaError_t e = pkv::launch_copy_blocks(k_pool, v_pool, scales, copy_src, copy_dst,
+                                            num_copies, block_bytes, scale_bytes,
+                                            pool->num_blocks, dev_error,
+                                            reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
 int32_t paged_decode_num_ranges(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
                                 int32_t max_context_len, int32_t partition_tokens) {
     if (!valid_pool(pool) || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0 ||
@@ -285,6 +304,7 @@ const char* kv_status_string(kv_status status) {
         case KV_ERR_INVALID_ARGUMENT: return "KV_ERR_INVALID_ARGUMENT";
         case KV_ERR_UNSUPPORTED: return "KV_ERR_UNSUPPORTED";
         case KV_ERR_CUDA: return "KV_ERR_CUDA";
+        case KV_ERR_OUT_OF_BLOCKS: return "KV_ERR_OUT_OF_BLOCKS";
         default: return "KV_STATUS_UNKNOWN";
     }
 }

@@ -5,6 +5,8 @@
 // kv head h goes to block slot/16, row slot%16.  HBM-bound scatter: every
 // thread moves one 16-byte vector (bf16/fp32) or one warp quantises one row
 // (FP8), so loads and stores are full 32-byte sectors.
+#include <algorithm>
+
 #include "kernels.cuh"
 
 namespace pkv {
@@ -125,7 +127,49 @@ __global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restri
         scales[((blk * num_kv_heads + h) * 2 + which) * kBlockTokens + off] = (a == 0.0f) ? 0.0f : s;
 }
 
+// Whole-block copies (copy-on-write of shared blocks): CTA (pair, part) moves
+// 16-byte vectors of the K block, the V block and the FP8 scale line.
+__global__ void copy_blocks_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
+                                   uint8_t* __restrict__ scales, const int32_t* __restrict__ src,
+                                   const int32_t* __restrict__ dst, int64_t block_bytes,
+                                   int64_t scale_bytes, int32_t num_blocks, int32_t* dev_error) {
+    pdl_wait();
+    pdl_trigger();
+    const int32_t pair = blockIdx.y;
+    const int32_t s = src[pair], d = dst[pair];
+    if (s < 0 || s >= num_blocks || d < 0 || d >= num_blocks) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) report(dev_error, KV_DEVERR_BAD_BLOCK_ID);
+        return;
+    }
+    const int64_t vecs = block_bytes / 16;
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < vecs;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t so = s * block_bytes + i * 16, dof = d * block_bytes + i * 16;
+        *reinterpret_cast<uint4*>(k_pool + dof) = *reinterpret_cast<const uint4*>(k_pool + so);
+        *reinterpret_cast<uint4*>(v_pool + dof) = *reinterpret_cast<const uint4*>(v_pool + so);
+    }
+    if (scales != nullptr) {
+        for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+             i < scale_bytes / 16; i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+            *reinterpret_cast<uint4*>(scales + d * scale_bytes + i * 16) =
+                *reinterpret_cast<const uint4*>(scales + s * scale_bytes + i * 16);
+    }
+}
+
 // ---- launchers ------------------------------------------------------------------
+cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, float* scales, const int32_t* src,
+                               const int32_t* dst, int32_t num_copies, int64_t block_bytes,
+                               int64_t scale_bytes, int32_t num_blocks, int32_t* dev_error,
+                               cudaStream_t stream) {
+    const int threads = 256;
+    const int64_t vecs = block_bytes / 16;
+    const unsigned parts = static_cast<unsigned>(std::min<int64_t>(8, (vecs + threads - 1) / threads));
+    return launch_pdl(copy_blocks_kernel, dim3(parts, static_cast<unsigned>(num_copies)),
+                      dim3(threads), 0, stream, static_cast<uint8_t*>(k_pool),
+                      static_cast<uint8_t*>(v_pool), reinterpret_cast<uint8_t*>(scales), src, dst,
+                      block_bytes, scale_bytes, num_blocks, dev_error);
+}
+
 cudaError_t launch_slot_mapping(const int32_t* block_table, int32_t batch, int32_t max_blocks,
                                 const int32_t* seq_ids, const int32_t* positions,
                                 int32_t num_tokens, int64_t* slots, int32_t* dev_error,

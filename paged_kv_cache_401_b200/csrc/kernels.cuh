@@ -42,6 +42,11 @@ cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, 
                              int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
                              cudaStream_t stream);
 
+cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, float* scales, const int32_t* src,
+                               const int32_t* dst, int32_t num_copies, int64_t block_bytes,
+                               int64_t scale_bytes, int32_t num_blocks, int32_t* dev_error,
+                               cudaStream_t stream);
+
 // Everything the decode kernel and its merge need for one launch.
 struct DecodeParams {
     void* out;                    // [B][Hq][D] in q dtype
