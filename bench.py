@@ -273,22 +273,43 @@ def run_reference(args, inp):
 
 
 # ---------------------------------------------------------------- GPU arm
-def stage_on_device(inp, device):
-    """Fill the paged pool with every sequence's history through the library."""
+def stage_on_device(inp, device, query_tokens: int = 1):
+    """Fill the paged pool with every sequence's history (all but its last
+    `query_tokens` tokens, which each step appends) through the library."""
     from paged_kv_cache_401_b200.cache import PagedKVCache
     spec = inp.spec
     cache = PagedKVCache(inp.num_blocks, spec.num_kv_heads, spec.head_dim, spec.kv_dtype,
                          device)
     bt = torch.from_numpy(inp.block_table).to(device)
+    keep = inp.fill_positions < inp.context_lens[inp.fill_seq_ids] - query_tokens
+    f_rows, f_sids, f_pos = (inp.fill_rows[keep], inp.fill_seq_ids[keep],
+                             inp.fill_positions[keep])
     chunk = 1 << 17
-    for c0 in range(0, len(inp.fill_rows), chunk):
-        c1 = min(len(inp.fill_rows), c0 + chunk)
-        rows = torch.from_numpy(inp.fill_rows[c0:c1])
-        cache.append(bt, torch.from_numpy(inp.fill_seq_ids[c0:c1]).to(device),
-                     torch.from_numpy(inp.fill_positions[c0:c1]).to(device),
+    for c0 in range(0, len(f_rows), chunk):
+        c1 = min(len(f_rows), c0 + chunk)
+        rows = torch.from_numpy(f_rows[c0:c1])
+        cache.append(bt, torch.from_numpy(f_sids[c0:c1]).to(device),
+                     torch.from_numpy(f_pos[c0:c1]).to(device),
                      inp.k[rows].to(device), inp.v[rows].to(device))
     torch.cuda.synchronize(device)
     return cache, bt
+
+
+def step_tokens(inp, query_tokens: int):
+    """The tokens a step appends: the last `query_tokens` of every sequence
+    (rows into inp.k / inp.v, sequence ids, positions), and the step's q:
+    [B][Hq][D] for one token, else [B][Q][Hq][D] drawn with seed 401 + 100."""
+    B = inp.q.shape[0]
+    Q = query_tokens
+    pos = (inp.context_lens[:, None] - Q + np.arange(Q)[None, :]).astype(np.int32)   # [B][Q]
+    rows = (inp.seq_offsets[:, None] + pos).reshape(-1)
+    sids = np.repeat(np.arange(B, dtype=np.int32), Q)
+    if Q == 1:
+        q = inp.q
+    else:
+        g = torch.Generator(device="cpu").manual_seed(401 + 100)
+        q = torch.randn((B, Q) + tuple(inp.q.shape[1:]), generator=g).to(inp.q.dtype)
+    return torch.from_numpy(rows), sids, pos.reshape(-1), q
 
 
 def run_gpu(args, inp):
@@ -299,27 +320,37 @@ def run_gpu(args, inp):
     dist_init(world, "nccl", device)
     spec = inp.spec
     B = inp.q.shape[0]
-    cache, bt = stage_on_device(inp, device)
+    Q = args.query_tokens
+    cache, bt = stage_on_device(inp, device, Q)
     lens = torch.from_numpy(inp.context_lens).to(device)
-    q = inp.q.to(device)
-    app = torch.from_numpy(inp.append_rows)
+    app, sids_np, pos_np, q_host = step_tokens(inp, Q)
+    q = q_host.to(device)
     k_new, v_new = inp.k[app].to(device), inp.v[app].to(device)
-    seq_ids = torch.arange(B, dtype=torch.int32, device=device)
-    positions = torch.from_numpy(inp.append_positions).to(device)
-    slots = torch.empty(B, dtype=torch.int64, device=device)
+    seq_ids = torch.from_numpy(sids_np).to(device)
+    positions = torch.from_numpy(pos_np).to(device)
+    slots = torch.empty(B * Q, dtype=torch.int64, device=device)
     out = torch.empty_like(q)
     P = args.partition
     ranges = pk.paged_decode_num_ranges(cache.desc, B, spec.num_q_heads, inp.max_context_len, P)
-    ws = cache.alloc_workspace(B, spec.num_q_heads, inp.max_context_len, P)
+    ws_bytes = pk.paged_attention_workspace_bytes(cache.desc, B, spec.num_q_heads, Q,
+                                                  inp.max_context_len, P)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
     launches_per_step = 4   # slot mapping, cache write, decode, merge
 
     def append():
         cache.append(bt, seq_ids, positions, k_new, v_new, slots=slots)
 
+    def attend(qq, tbl, ln):
+        if Q == 1:
+            cache.decode(qq, tbl, ln, inp.max_context_len, spec.scale, out=out,
+                         partition_tokens=P, workspace=ws)
+        else:
+            cache.attend(qq, tbl, ln, inp.max_context_len, spec.scale, out=out,
+                         partition_tokens=P, workspace=ws)
+
     def decode():
-        cache.decode(q, bt, lens, inp.max_context_len, spec.scale, out=out,
-                     partition_tokens=P, workspace=ws)
+        attend(q, bt, lens)
 
     for _ in range(args.warmup):
         append()
@@ -356,7 +387,7 @@ def run_gpu(args, inp):
     # block table, context lengths, each 256-byte aligned) copied to a device
     # staging buffer every step; the calls take views of it; the output is
     # copied back.  Both copies are inside the timed region.
-    parts = [inp.q, inp.k[app], inp.v[app], torch.from_numpy(inp.block_table),
+    parts = [q_host, inp.k[app], inp.v[app], torch.from_numpy(inp.block_table),
              torch.from_numpy(inp.context_lens)]
     offs, total = [], 0
     for t in parts:
@@ -370,15 +401,14 @@ def run_gpu(args, inp):
         h_stage[o:o + nb].copy_(t.contiguous().view(-1).view(torch.uint8))
         views.append(d_stage[o:o + nb].view(t.dtype).view(t.shape))
     e_q, e_k, e_v, e_bt, e_lens = views
-    h_out = torch.empty_like(inp.q).pin_memory()
+    h_out = torch.empty_like(q_host).pin_memory()
     h2d = total
     d2h = h_out.numel() * h_out.element_size()
 
     def e2e_step():
         d_stage.copy_(h_stage, non_blocking=True)
         cache.append(e_bt, seq_ids, positions, e_k, e_v, slots=slots)
-        cache.decode(e_q, e_bt, e_lens, inp.max_context_len, spec.scale, out=out,
-                     partition_tokens=P, workspace=ws)
+        attend(e_q, e_bt, e_lens)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -426,7 +456,7 @@ def run_gpu(args, inp):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": spec.kv_dtype if spec.kv_dtype != "fp8" else "fp8_e4m3",
         "data": "synthetic (seeded N(0,1) q/K/V, random block permutation)",
-        "config": dict(describe(inp, P), num_ranges=ranges),
+        "config": dict(describe(inp, P), num_ranges=ranges, query_tokens=Q),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(max_e2e_ms / args.steps, 5)},
@@ -459,6 +489,9 @@ def main(argv=None):
     ap.add_argument("--reference-seqs", type=int, default=8,
                     help="sequences in the oracle's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--query-tokens", type=int, default=1,
+                    help="query tokens per sequence per step (1 = decode; >1 = speculative "
+                         "verification of that many appended tokens)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, reported as run
     inp = make_inputs(args.workload)

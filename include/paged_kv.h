@@ -214,6 +214,35 @@ KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, con
                                  kv_stream_t stream);
 
 /*
+ * Multi-query paged attention: Q = num_query_tokens new tokens per sequence
+ * attend to the cache at once -- the verification of Q speculative tokens, or a
+ * chunk of a chunked prefill ("KV Cache 深度解析" §五 chunked prefill; "大模型推理为何
+ * 这么慢", speculative decoding).  The Q tokens are the LAST Q tokens of each
+ * sequence's context and must already be in the cache: query token i of
+ * sequence b sits at position L - Q + i (L = context_lens[b]) and attends to
+ * positions 0 .. L - Q + i (causal), with the softmax of paged_decode_attention.
+ *   q, out : device [batch][Q][num_q_heads][head_dim] (q_dtype; out in q_dtype)
+ * Everything else as paged_decode_attention (Q = 1 is exactly that call).
+ * Supported shapes: bf16 or FP8 KV, head_dim 128, bf16 q, and
+ * (num_q_heads / num_kv_heads) * Q <= 16, else KV_ERR_UNSUPPORTED.  A context
+ * length below Q is invalid (zeros, KV_DEVERR_BAD_CONTEXT_LEN).
+ */
+KV_API size_t paged_attention_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
+                                              int32_t num_q_heads, int32_t num_query_tokens,
+                                              int32_t max_context_len, int32_t partition_tokens);
+
+KV_API kv_status paged_attention_multi_query(const kv_pool_desc* pool, void* out, const void* q,
+                                             kv_dtype q_dtype, int32_t num_query_tokens,
+                                             const void* k_pool, const void* v_pool,
+                                             const float* scales, const int32_t* block_table,
+                                             int32_t max_blocks_per_seq,
+                                             const int32_t* context_lens, int32_t batch,
+                                             int32_t num_q_heads, int32_t max_context_len,
+                                             float scale, int32_t partition_tokens,
+                                             void* workspace, size_t workspace_bytes,
+                                             int32_t* dev_error, kv_stream_t stream);
+
+/*
  * Bytes of device memory the library holds on every GPU that loads it, for
  * paged_decode_attention_static_workspace (16 MiB: enough for the default
  * split of e.g. 256 sequences x 8 kv heads x 4 query heads per group at

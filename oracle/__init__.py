@@ -20,6 +20,9 @@ restatement, in double precision, of every step of the decode hot path:
 * ``decode_attention``    -- softmax(q·Kᵀ·scale)·V over a CONTIGUOUS per-sequence
                              copy, GQA head grouping, two passes in double
                              (C, OpenMP); "KV Cache 深度解析", §一 and §六.
+* ``multi_query_attention`` -- Q query tokens per sequence, the last Q of its
+                             context, each attending causally ("KV Cache 深度解析"
+                             §五 chunked prefill; speculative verification).
 * ``decode_attention_bruteforce`` -- the same in numpy, one (sequence, head) at
                              a time, following the page's §六 step(): tiny inputs.
 * ``decode_attention_split`` -- the blockwise online-softmax update of the
@@ -64,6 +67,12 @@ def _load():
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
             ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
             ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32]
+        lib.oracle_multi_query_attention.restype = ctypes.c_int
+        lib.oracle_multi_query_attention.argtypes = [
+            ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_double,
+            ctypes.c_void_p]
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
     return _lib
@@ -205,6 +214,32 @@ def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offsets: n
     if rc != 0:
         raise ValueError("oracle_decode_attention: invalid arguments")
     return (out, weights) if return_weights else out
+
+
+def multi_query_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offsets: np.ndarray,
+                          lens: np.ndarray, scale: float, num_kv_heads: int, kv_dtype: str,
+                          q_dtype: str, k_scale: np.ndarray | None = None,
+                          v_scale: np.ndarray | None = None) -> np.ndarray:
+    """Causal multi-query attention (C oracle): q [B][Q][Hq][D]; query token i of
+    sequence b sees positions 0 .. L_b - Q + i.  Returns out [B][Q][Hq][D] float64."""
+    lib = _load()
+    b, nq, hq, d = q.shape
+    q = np.ascontiguousarray(q)
+    k = np.ascontiguousarray(k)
+    v = np.ascontiguousarray(v)
+    seq_offsets = np.ascontiguousarray(seq_offsets, dtype=np.int64)
+    lens = np.ascontiguousarray(lens, dtype=np.int32)
+    if kv_dtype == "fp8":
+        k_scale = np.ascontiguousarray(k_scale, dtype=np.float32)
+        v_scale = np.ascontiguousarray(v_scale, dtype=np.float32)
+    out = np.empty((b, nq, hq, d), dtype=np.float64)
+    rc = lib.oracle_multi_query_attention(_DTYPE_CODES[kv_dtype], _DTYPE_CODES[q_dtype], nq,
+                                          _ptr(q), _ptr(k), _ptr(v), _ptr(k_scale), _ptr(v_scale),
+                                          _ptr(seq_offsets), _ptr(lens), b, hq, num_kv_heads, d,
+                                          float(scale), _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_multi_query_attention: invalid arguments")
+    return out
 
 
 def widen(x: np.ndarray, dtype: str, scales: np.ndarray | None = None) -> np.ndarray:

@@ -239,3 +239,69 @@ int oracle_num_threads(void) {
 #endif
     return n;
 }
+
+/*
+ * Causal multi-query attention over CONTIGUOUS per-sequence K/V: Q query
+ * tokens per sequence are the last Q tokens of its context ("KV Cache 深度解析"
+ * §五 chunked prefill; speculative verification).  Query token i of sequence b
+ * sits at position L_b - Q + i and attends to positions 0 .. L_b - Q + i:
+ *   s_t = scale * q[b,i,h,:] . K[b,t,g,:],  t <= L_b - Q + i
+ *   out[b,i,h,:] = sum_t softmax(s)_t V[b,t,g,:]
+ *   q, out : [B][Q][Hq][D] (q in q_dtype, out double); K/V as oracle_decode_attention.
+ * Each (b, i, h) row is evaluated exactly like oracle_decode_attention with a
+ * context of L_b - Q + i + 1 tokens.  Returns -1 when some L_b < Q.
+ */
+int oracle_multi_query_attention(int32_t kv_dtype, int32_t q_dtype, int32_t num_query_tokens,
+                                 const void* q, const void* k, const void* v,
+                                 const float* k_scale, const float* v_scale,
+                                 const int64_t* seq_offsets, const int32_t* lens,
+                                 int32_t batch, int32_t num_q_heads, int32_t num_kv_heads,
+                                 int32_t head_dim, double scale, double* out) {
+    int32_t group, b;
+    const int32_t Q = num_query_tokens;
+    if (num_kv_heads <= 0 || num_q_heads % num_kv_heads != 0 || Q < 1) return -1;
+    group = num_q_heads / num_kv_heads;
+    for (b = 0; b < batch; ++b)
+        if (lens[b] < Q) return -1;
+
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t row = 0; row < (int64_t)batch * Q * num_q_heads; ++row) {
+        int32_t bb = (int32_t)(row / ((int64_t)Q * num_q_heads));
+        int32_t i = (int32_t)((row / num_q_heads) % Q);
+        int32_t h = (int32_t)(row % num_q_heads);
+        int32_t g = h / group;
+        int32_t L = lens[bb] - Q + i + 1;          /* keys this query token sees */
+        int64_t t0 = seq_offsets[bb];
+        double* s = (double*)malloc(sizeof(double) * (size_t)L);
+        double* qd = (double*)malloc(sizeof(double) * (size_t)head_dim);
+        double m = -INFINITY, Z = 0.0;
+        int32_t t, d;
+        for (d = 0; d < head_dim; ++d) {
+            int64_t qi = row * head_dim + d;
+            qd[d] = (q_dtype == ORC_F32) ? (double)((const float*)q)[qi]
+                                         : bf16_bits_to_double(((const uint16_t*)q)[qi]);
+        }
+        for (t = 0; t < L; ++t) {
+            int64_t r = (t0 + t) * num_kv_heads + g;
+            double acc = 0.0;
+            for (d = 0; d < head_dim; ++d)
+                acc += qd[d] * load_elem(k, kv_dtype, r * head_dim + d, k_scale, r);
+            s[t] = scale * acc;
+            if (s[t] > m) m = s[t];
+        }
+        for (t = 0; t < L; ++t) {
+            s[t] = exp(s[t] - m);
+            Z += s[t];
+        }
+        for (d = 0; d < head_dim; ++d) out[row * head_dim + d] = 0.0;
+        for (t = 0; t < L; ++t) {
+            int64_t r = (t0 + t) * num_kv_heads + g;
+            double w = s[t] / Z;
+            for (d = 0; d < head_dim; ++d)
+                out[row * head_dim + d] += w * load_elem(v, kv_dtype, r * head_dim + d, v_scale, r);
+        }
+        free(s);
+        free(qd);
+    }
+    return 0;
+}

@@ -30,6 +30,7 @@ BLOCK_SIZE = 16
 EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
             "paged_decode_num_ranges", "paged_decode_workspace_bytes",
             "paged_decode_attention", "paged_decode_attention_static_workspace",
+            "paged_attention_workspace_bytes", "paged_attention_multi_query",
             "paged_kv_copy_blocks", "kv_block_manager_create", "kv_block_manager_destroy",
             "kv_block_manager_num_free_blocks", "kv_block_manager_refcount",
             "kv_block_manager_add_sequence", "kv_block_manager_fork",
@@ -78,6 +79,10 @@ def _load() -> ctypes.CDLL:
             "paged_decode_attention_static_workspace": (
                 _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
                        ctypes.c_float, _I32, _P, _P]),
+            "paged_attention_workspace_bytes": (_SZ, [desc_p, _I32, _I32, _I32, _I32, _I32]),
+            "paged_attention_multi_query": (_I32, [desc_p, _P, _P, _I32, _I32, _P, _P, _P, _P,
+                                                   _I32, _P, _I32, _I32, _I32, ctypes.c_float,
+                                                   _I32, _P, _SZ, _P, _P]),
             "paged_kv_copy_blocks": (_I32, [desc_p, _P, _P, _P, _P, _P, _I32, _P, _P]),
             "kv_block_manager_create": (_I32, [_I32, _I32, _I32, _P]),
             "kv_block_manager_destroy": (None, [_P]),
@@ -230,6 +235,32 @@ def paged_decode_attention_static_workspace(
                _ptr(v_pool), _ptr(scales), _ptr(block_table),
                block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
                float(scale), partition_tokens, _ptr(dev_error), _stream(stream)))
+    return out
+
+
+def paged_attention_workspace_bytes(pool: KvPoolDesc, batch: int, num_q_heads: int,
+                                    num_query_tokens: int, max_context_len: int,
+                                    partition_tokens: int = 0) -> int:
+    return int(_load().paged_attention_workspace_bytes(ctypes.byref(pool), batch, num_q_heads,
+                                                       num_query_tokens, max_context_len,
+                                                       partition_tokens))
+
+
+def paged_attention_multi_query(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
+                                k_pool: torch.Tensor, v_pool: torch.Tensor,
+                                scales: torch.Tensor | None, block_table: torch.Tensor,
+                                context_lens: torch.Tensor, max_context_len: int, scale: float,
+                                partition_tokens: int = 0, workspace: torch.Tensor | None = None,
+                                dev_error: torch.Tensor | None = None,
+                                stream=None) -> torch.Tensor:
+    """q, out: [batch][num_query_tokens][num_q_heads][head_dim]."""
+    batch, nq, num_q_heads, _ = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("paged_attention_multi_query", _load().paged_attention_multi_query(
+        ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), nq, _ptr(k_pool), _ptr(v_pool),
+        _ptr(scales), _ptr(block_table), block_table.shape[1], _ptr(context_lens), batch,
+        num_q_heads, max_context_len, float(scale), partition_tokens, _ptr(workspace), ws_bytes,
+        _ptr(dev_error), _stream(stream)))
     return out
 
 

@@ -10,8 +10,8 @@ from __future__ import annotations
 import torch
 
 from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, compute_slot_mapping, empty_pool,
-               kv_pool_create, paged_decode_attention, paged_decode_workspace_bytes,
-               reshape_and_cache)
+               kv_pool_create, paged_attention_multi_query, paged_attention_workspace_bytes,
+               paged_decode_attention, paged_decode_workspace_bytes, reshape_and_cache)
 
 _DTYPES = {"f32": KV_F32, "bf16": KV_BF16, "fp8": KV_FP8_E4M3}
 
@@ -70,3 +70,20 @@ class PagedKVCache:
 
     def clear_errors(self) -> None:
         self.dev_error.zero_()
+
+    # ---- several query tokens per sequence (speculative verification, prefill chunk)
+    def attend(self, q: torch.Tensor, block_table: torch.Tensor, context_lens: torch.Tensor,
+               max_context_len: int, scale: float, out: torch.Tensor | None = None,
+               partition_tokens: int = 0, workspace: torch.Tensor | None = None,
+               stream=None) -> torch.Tensor:
+        """q: [batch][Q][num_q_heads][head_dim]; the Q tokens are the last Q of each context."""
+        if out is None:
+            out = torch.empty_like(q)
+        if workspace is None:
+            n = paged_attention_workspace_bytes(self.desc, q.shape[0], q.shape[2], q.shape[1],
+                                                max_context_len, partition_tokens)
+            workspace = torch.empty(n, dtype=torch.uint8, device=self.device)
+        return paged_attention_multi_query(self.desc, out, q, self.k_pool, self.v_pool,
+                                           self.scales, block_table, context_lens,
+                                           max_context_len, scale, partition_tokens, workspace,
+                                           self.dev_error, stream)

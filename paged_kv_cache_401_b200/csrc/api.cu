@@ -173,16 +173,22 @@ kv_status paged_kv_copy_blocks(const kv_pool_desc* pool, void* k_pool, void* v_p
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
-int32_t paged_decode_num_ranges(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
-                                int32_t max_context_len, int32_t partition_tokens) {
+}  // extern "C"
+
+namespace {
+
+// Consumer ranges of the tile list (see paged_decode_num_ranges).
+int32_t num_ranges_for(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
+                       int32_t query_tokens, int32_t max_context_len, int32_t partition_tokens) {
     if (!valid_pool(pool) || batch <= 0 || num_q_heads <= 0 || max_context_len <= 0 ||
-        num_q_heads % pool->num_kv_heads != 0 || partition_tokens < 0 ||
+        query_tokens < 1 || num_q_heads % pool->num_kv_heads != 0 || partition_tokens < 0 ||
         partition_tokens % kBlockTokens != 0)
         return 0;
     const int32_t group = num_q_heads / pool->num_kv_heads;
     if (partition_tokens == 0) {
         // persistent: one range per consumer warp of every CTA the GPU holds at once
-        return current_sm_count() * pkv::decode_ctas_per_sm(pool->dtype, pool->head_dim, group) * 4;
+        return current_sm_count() *
+               pkv::decode_ctas_per_sm(pool->dtype, pool->head_dim, group, query_tokens) * 4;
     }
     // ranges of at most partition_tokens tokens over the largest possible tile list
     const int64_t max_tiles = static_cast<int64_t>(batch) * pool->num_kv_heads *
@@ -192,51 +198,53 @@ int32_t paged_decode_num_ranges(const kv_pool_desc* pool, int32_t batch, int32_t
     return static_cast<int32_t>(n < 1 ? 1 : (n > (1 << 28) ? (1 << 28) : n));
 }
 
-namespace {
-// Workspace layout: [B + 1] int32 sequence starts | [pieces][G] float2 (m, l) |
-// [pieces][G][D] float partial outputs; pieces = B * Hkv + num_ranges.
+// Workspace layout: [B + 1] int32 sequence starts | [pieces][R] float2 (m, l) |
+// [pieces][R][D] float partial outputs; pieces = B * Hkv + num_ranges, R = G * Q
+// query rows per (sequence, kv head) pair.
 struct WsLayout {
     size_t ml_off, o_off, total;
 };
 WsLayout ws_layout(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
-                   int32_t num_ranges) {
+                   int32_t query_tokens, int32_t num_ranges) {
     auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-    const size_t group = static_cast<size_t>(num_q_heads / pool->num_kv_heads);
+    const size_t rows = static_cast<size_t>(num_q_heads / pool->num_kv_heads) * query_tokens;
     const size_t pieces = static_cast<size_t>(batch) * pool->num_kv_heads + num_ranges;
     WsLayout w{};
     w.ml_off = up(sizeof(int32_t) * (static_cast<size_t>(batch) + 1));
-    w.o_off = w.ml_off + up(pieces * group * sizeof(float2));
-    w.total = w.o_off + pieces * group * pool->head_dim * sizeof(float);
+    w.o_off = w.ml_off + up(pieces * rows * sizeof(float2));
+    w.total = w.o_off + pieces * rows * pool->head_dim * sizeof(float);
     return w;
 }
-}  // namespace
 
-size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
-                                    int32_t num_q_heads, int32_t max_context_len,
-                                    int32_t partition_tokens) {
-    const int32_t ranges =
-        paged_decode_num_ranges(pool, batch, num_q_heads, max_context_len, partition_tokens);
+size_t workspace_bytes_for(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
+                           int32_t query_tokens, int32_t max_context_len,
+                           int32_t partition_tokens) {
+    const int32_t ranges = num_ranges_for(pool, batch, num_q_heads, query_tokens,
+                                          max_context_len, partition_tokens);
     if (ranges <= 0) return 0;
-    return ws_layout(pool, batch, num_q_heads, ranges).total;
+    return ws_layout(pool, batch, num_q_heads, query_tokens, ranges).total;
 }
 
-kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
-                                 kv_dtype q_dtype, const void* k_pool, const void* v_pool,
-                                 const float* scales,
-                                 const int32_t* block_table, int32_t max_blocks_per_seq,
-                                 const int32_t* context_lens, int32_t batch,
-                                 int32_t num_q_heads, int32_t max_context_len, float scale,
-                                 int32_t partition_tokens, void* workspace,
-                                 size_t workspace_bytes, int32_t* dev_error,
-                                 kv_stream_t stream) {
-    if (!valid_pool(pool) || batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0)
+kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_dtype q_dtype,
+                         int32_t query_tokens, const void* k_pool, const void* v_pool,
+                         const float* scales, const int32_t* block_table,
+                         int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
+                         int32_t num_q_heads, int32_t max_context_len, float scale,
+                         int32_t partition_tokens, void* workspace, size_t workspace_bytes,
+                         int32_t* dev_error, kv_stream_t stream) {
+    if (!valid_pool(pool) || batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0 ||
+        query_tokens < 1)
         return KV_ERR_INVALID_ARGUMENT;
     if (q_dtype != KV_F32 && q_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
     if (num_q_heads % pool->num_kv_heads != 0) return KV_ERR_INVALID_ARGUMENT;
     const int32_t group = num_q_heads / pool->num_kv_heads;
     if (group != 1 && group != 2 && group != 4 && group != 8) return KV_ERR_UNSUPPORTED;
+    // several query tokens: tensor-core shapes, at most 16 query rows per kv head
+    if (query_tokens > 1 && (!pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim) ||
+                             group * query_tokens > 16))
+        return KV_ERR_UNSUPPORTED;
     if (batch == 0) return KV_OK;
-    if (max_context_len <= 0 ||
+    if (max_context_len < query_tokens ||
         static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens)
         return KV_ERR_INVALID_ARGUMENT;
     if (partition_tokens < 0 || partition_tokens % kBlockTokens != 0)
@@ -255,10 +263,10 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     if (fp8 != (scales != nullptr)) return KV_ERR_INVALID_ARGUMENT;
     if (fp8 && !aligned16(scales)) return KV_ERR_INVALID_ARGUMENT;
 
-    const int32_t ranges =
-        paged_decode_num_ranges(pool, batch, num_q_heads, max_context_len, partition_tokens);
+    const int32_t ranges = num_ranges_for(pool, batch, num_q_heads, query_tokens,
+                                          max_context_len, partition_tokens);
     if (ranges <= 0) return KV_ERR_INVALID_ARGUMENT;
-    const WsLayout wl = ws_layout(pool, batch, num_q_heads, ranges);
+    const WsLayout wl = ws_layout(pool, batch, num_q_heads, query_tokens, ranges);
     if (workspace == nullptr || workspace_bytes < wl.total || !aligned16(workspace))
         return KV_ERR_INVALID_ARGUMENT;
 
@@ -277,6 +285,7 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     p.num_blocks = pool->num_blocks;
     p.max_blocks = max_blocks_per_seq;
     p.max_context_len = max_context_len;
+    p.num_query_tokens = query_tokens;
     p.num_ranges = ranges;
     p.scale_log2 = scale * 1.4426950408889634f;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -296,6 +305,57 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     cudaError_t e = pkv::launch_paged_decode(p, maps, pool->dtype, q_dtype, pool->head_dim,
                                              group, reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int32_t paged_decode_num_ranges(const kv_pool_desc* pool, int32_t batch, int32_t num_q_heads,
+                                int32_t max_context_len, int32_t partition_tokens) {
+    return num_ranges_for(pool, batch, num_q_heads, 1, max_context_len, partition_tokens);
+}
+
+size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
+                                    int32_t num_q_heads, int32_t max_context_len,
+                                    int32_t partition_tokens) {
+    return workspace_bytes_for(pool, batch, num_q_heads, 1, max_context_len, partition_tokens);
+}
+
+size_t paged_attention_workspace_bytes(const kv_pool_desc* pool, int32_t batch,
+                                       int32_t num_q_heads, int32_t num_query_tokens,
+                                       int32_t max_context_len, int32_t partition_tokens) {
+    return workspace_bytes_for(pool, batch, num_q_heads, num_query_tokens, max_context_len,
+                               partition_tokens);
+}
+
+kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
+                                 kv_dtype q_dtype, const void* k_pool, const void* v_pool,
+                                 const float* scales, const int32_t* block_table,
+                                 int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                 int32_t batch, int32_t num_q_heads, int32_t max_context_len,
+                                 float scale, int32_t partition_tokens, void* workspace,
+                                 size_t workspace_bytes, int32_t* dev_error,
+                                 kv_stream_t stream) {
+    return attention_impl(pool, out, q, q_dtype, 1, k_pool, v_pool, scales, block_table,
+                          max_blocks_per_seq, context_lens, batch, num_q_heads, max_context_len,
+                          scale, partition_tokens, workspace, workspace_bytes, dev_error, stream);
+}
+
+kv_status paged_attention_multi_query(const kv_pool_desc* pool, void* out, const void* q,
+                                      kv_dtype q_dtype, int32_t num_query_tokens,
+                                      const void* k_pool, const void* v_pool,
+                                      const float* scales, const int32_t* block_table,
+                                      int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                      int32_t batch, int32_t num_q_heads,
+                                      int32_t max_context_len, float scale,
+                                      int32_t partition_tokens, void* workspace,
+                                      size_t workspace_bytes, int32_t* dev_error,
+                                      kv_stream_t stream) {
+    return attention_impl(pool, out, q, q_dtype, num_query_tokens, k_pool, v_pool, scales,
+                          block_table, max_blocks_per_seq, context_lens, batch, num_q_heads,
+                          max_context_len, scale, partition_tokens, workspace, workspace_bytes,
+                          dev_error, stream);
 }
 
 const char* kv_status_string(kv_status status) {

@@ -233,9 +233,12 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 }
 
 // ---- tile list bookkeeping ----------------------------------------------------------
-// Tiles of a sequence with context length L: ceil(L/16), or 0 when L is invalid.
-__device__ __forceinline__ int32_t seq_tiles(int32_t L, int32_t max_context_len) {
-    return (L >= 1 && L <= max_context_len) ? (L + kBlockTokens - 1) / kBlockTokens : 0;
+// Tiles of a sequence with context length L: ceil(L/16), or 0 when L is invalid
+// (shorter than the query tokens it must hold, or longer than max_context_len).
+__device__ __forceinline__ int32_t seq_tiles(int32_t L, const DecodeParams& p) {
+    return (L >= p.num_query_tokens && L >= 1 && L <= p.max_context_len)
+               ? (L + kBlockTokens - 1) / kBlockTokens
+               : 0;
 }
 
 // First tile of consumer range W (ranges are equal cuts of the T-tile list).
@@ -260,7 +263,7 @@ __device__ __forceinline__ int64_t warp_sum_i64(int64_t x) {
 __device__ int64_t total_tiles(const DecodeParams& p, int lane) {
     int64_t t = 0;
     for (int b = lane; b < p.batch; b += 32)
-        t += static_cast<int64_t>(p.num_kv_heads) * seq_tiles(p.context_lens[b], p.max_context_len);
+        t += static_cast<int64_t>(p.num_kv_heads) * seq_tiles(p.context_lens[b], p);
     return warp_sum_i64(t);
 }
 
@@ -283,7 +286,7 @@ __device__ Cursor locate_tile(const DecodeParams& p, int64_t x, int lane, int32_
     for (int b0 = 0; b0 < p.batch; b0 += 32) {
         const int b = b0 + lane;
         const int32_t L = b < p.batch ? p.context_lens[b] : 0;
-        const int32_t nt = b < p.batch ? seq_tiles(L, p.max_context_len) : 0;
+        const int32_t nt = b < p.batch ? seq_tiles(L, p) : 0;
         const int64_t cnt = static_cast<int64_t>(p.num_kv_heads) * nt;
         int64_t incl = cnt;
 #pragma unroll
@@ -325,7 +328,7 @@ __device__ __forceinline__ void advance(Cursor& c, const DecodeParams& p) {
     do {
         ++c.b;
         c.L = c.b < p.batch ? p.context_lens[c.b] : 0;
-        c.nt = c.b < p.batch ? seq_tiles(c.L, p.max_context_len) : 0;
+        c.nt = c.b < p.batch ? seq_tiles(c.L, p) : 0;
     } while (c.b < p.batch && c.nt == 0);
 }
 
@@ -418,7 +421,8 @@ struct SimtMath {
             for (int i = 0; i < kDPL / 2; ++i) o2[g][i] = make_float2(0.0f, 0.0f);
     }
 
-    __device__ void tile(const uint8_t* kt, int32_t nvalid, const DecodeParams&) {
+    __device__ void tile(const uint8_t* kt, int32_t jb, int32_t L, const DecodeParams&) {
+        const int32_t nvalid = min(kBlockTokens, L - jb * kBlockTokens);
         const uint8_t* vt = kt + kTileBytes;
         const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
         const float* vsc = ksc + kBlockTokens;
@@ -555,28 +559,34 @@ struct SimtMath {
 // A tile is 16 tokens x 128 dims.  K and V land in shared memory as [16 rows]
 // x [128-byte] boxes written by TMA with the 128-byte swizzle (16-byte chunk
 // c of row r stored at chunk c ^ (r & 7)), so every ldmatrix row set hits 32
-// distinct banks.  Per tile and warp (gid = lane / 4, tig = lane % 4):
-//   S   = Q.K^T      m16n8k16, rows = query heads of the group (G <= 8 real),
-//                    2 token tiles x 8 dim steps; fp32 accumulators.
-//   softmax on the accumulator fragments: row gid holds tokens 2tig,2tig+1
-//                    and 8+2tig,9+2tig; max/sum across the 4 lanes of a row.
-//   O^T += V^T.P^T   m16n8k16, rows = 16 head dims, columns = 8 heads; the P
-//                    fragment of the score accumulators is exactly the B
-//                    operand, so P never leaves registers.
+// distinct banks.  The rows of the MMAs are the query rows of a (sequence, kv
+// head) pair: row r = i * G + g is query token i (of Q) and head g (of G) of
+// the group, R = G * Q <= 16 rows.  Per tile and warp (gid = lane / 4, tig =
+// lane % 4):
+//   S   = Q.K^T      m16n8k16, 2 token tiles x 8 dim steps; fp32 accumulators;
+//                    lane holds rows gid and gid + 8 ("row sets" 0 and 1).
+//   softmax on the accumulator fragments: a row holds tokens 2tig,2tig+1 and
+//                    8+2tig,9+2tig; max/sum across the 4 lanes of the row.
+//                    Query token i sits at position L - Q + i and sees
+//                    positions <= L - Q + i (causal).
+//   O^T += V^T.P^T   m16n8k16, rows = 16 head dims, columns = 8 query rows per
+//                    row set; the P fragment of the score accumulators is
+//                    exactly the B operand, so P never leaves registers.
 // bf16 KV: bf16 MMAs, P rounded to bf16.  FP8 KV: codes widened to f16 in
 // registers (exact), f16 MMAs with q rounded to f16 and P (times the V row
 // scale) rounded to f16; the K row scale multiplies the scores.  Element
 // orders inside a k-step are permuted consistently between the two operands
 // (a dot product does not depend on the order of its terms), which is what
-// lets FP8 rows be read with 16-bit ldmatrix.
+// lets FP8 rows be read with 16-bit ldmatrix.  WIDE = more than 8 query rows.
 // ======================================================================================
-template <int KV_T, int G>
+template <int KV_T, int G, bool WIDE>
 struct MmaMath {
     static_assert(KV_T == KV_BF16 || KV_T == KV_FP8_E4M3, "bf16 or FP8 KV");
-    static_assert(G <= 8, "one m16n8 column per query head");
+    static_assert(G <= 8, "a row set holds 8 query rows");
     using OutT = uint16_t;                                        // bf16 output
     static constexpr bool kF16 = KV_T == KV_FP8_E4M3;
     static constexpr int D = 128;
+    static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
     static constexpr int kElem = KvElem<KV_T>::kBytes;
     static constexpr int kRowBytes = D * kElem;                   // 256 (bf16) / 128 (fp8)
     static constexpr int kBoxCols = 128 / kElem;                  // elements per 128-byte box row
@@ -588,9 +598,9 @@ struct MmaMath {
     static constexpr int kStages = kF16 ? 12 : 8;                 // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr int kWarpScratch = 0;
-    static constexpr int kMinBlocks = 3;
+    static constexpr int kMinBlocks = WIDE ? 2 : 3;
 
-    // ---- producer side: TMA boxes of K and V (+ FP8 row scales by bulk copy)
+    // ---- producer side: TMA boxes of K and V (+ the FP8 scale line by bulk copy)
     __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
                                  const TmaMaps& maps) {
         const int32_t row = static_cast<int32_t>(tile * kBlockTokens);
@@ -616,10 +626,11 @@ struct MmaMath {
     }
 
     // ---- consumer side
-    int32_t lane, gid, tig;
-    uint32_t qa[8][2];  // A fragments of q per 16-dim k-step: rows gid (< G), cols {lo, hi}
-    float o[8][4];      // O^T: m-tile mi = 16 dims; c0,c1 = (dim row gid, heads 2tig, 2tig+1)
-    float m_run, l_run; // running max (base 2) and this lane's part of the sum, row gid
+    int32_t lane, gid, tig, nq, rows;
+    int32_t qtok[kSets];        // query token of row gid + 8k (>= nq: padding row)
+    uint32_t qa[kSets][8][2];   // A fragments of q per 16-dim k-step, row gid + 8k: {k lo, k hi}
+    float o[kSets][8][4];       // O^T: [set][m-tile][c]; c0,c1 = (dim gid, rows 8k+2tig, +1)
+    float m_run[kSets], l_run[kSets];  // running max (base 2), lane part of the sum, row gid+8k
 
     __device__ void init(int32_t lane_, uint8_t*) {
         lane = lane_;
@@ -628,51 +639,70 @@ struct MmaMath {
     }
 
     __device__ void load_q(const DecodeParams& p, int32_t b, int32_t kvh) {
-        const uint16_t* q = static_cast<const uint16_t*>(p.q) +
-                            (static_cast<int64_t>(b) * p.num_q_heads + kvh * G + gid) * D;
+        nq = p.num_query_tokens;
+        rows = G * nq;
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            if (gid >= G) {
-                qa[ks][0] = qa[ks][1] = 0u;
-            } else if constexpr (!kF16) {
-                // k index 2tig+{0,1} -> dim 16ks+2tig+{0,1}; 8+2tig+{0,1} -> dim 16ks+8+2tig+{0,1}
-                qa[ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
-                qa[ks][1] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 8 + 2 * tig);
-            } else {
-                // FP8 rows are read 4 codes per lane: k 2tig+{0,1} -> dim 16ks+4tig+{0,1},
-                // k 8+2tig+{0,1} -> dim 16ks+4tig+{2,3}
-                const uint2 w = *reinterpret_cast<const uint2*>(q + 16 * ks + 4 * tig);
-                qa[ks][0] = pack2<true>(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xffff0000u));
-                qa[ks][1] = pack2<true>(__uint_as_float(w.y << 16), __uint_as_float(w.y & 0xffff0000u));
+        for (int k = 0; k < kSets; ++k) {
+            const int32_t r = gid + 8 * k;
+            qtok[k] = r < rows ? r / G : nq;
+            const uint16_t* q = static_cast<const uint16_t*>(p.q) +
+                                ((static_cast<int64_t>(b) * nq + (r / G)) * p.num_q_heads +
+                                 kvh * G + r % G) * D;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+                if (r >= rows) {
+                    qa[k][ks][0] = qa[k][ks][1] = 0u;
+                } else if constexpr (!kF16) {
+                    // k index 2tig+{0,1} -> dim 16ks+2tig+{0,1}; 8+2tig+{0,1} -> 16ks+8+2tig+{0,1}
+                    qa[k][ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
+                    qa[k][ks][1] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 8 + 2 * tig);
+                } else {
+                    // FP8 rows are read 4 codes per lane: k 2tig+{0,1} -> dim 16ks+4tig+{0,1},
+                    // k 8+2tig+{0,1} -> dim 16ks+4tig+{2,3}
+                    const uint2 w = *reinterpret_cast<const uint2*>(q + 16 * ks + 4 * tig);
+                    qa[k][ks][0] = pack2<true>(__uint_as_float(w.x << 16),
+                                               __uint_as_float(w.x & 0xffff0000u));
+                    qa[k][ks][1] = pack2<true>(__uint_as_float(w.y << 16),
+                                               __uint_as_float(w.y & 0xffff0000u));
+                }
             }
         }
     }
 
     __device__ void reset() {
-        m_run = -INFINITY;
-        l_run = 0.0f;
 #pragma unroll
-        for (int mi = 0; mi < 8; ++mi)
+        for (int k = 0; k < kSets; ++k) {
+            m_run[k] = -INFINITY;
+            l_run[k] = 0.0f;
 #pragma unroll
-            for (int j = 0; j < 4; ++j) o[mi][j] = 0.0f;
+            for (int mi = 0; mi < 8; ++mi)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) o[k][mi][j] = 0.0f;
+        }
     }
 
-    __device__ void tile(const uint8_t* kt, int32_t nvalid, const DecodeParams& p) {
+    __device__ void tile(const uint8_t* kt, int32_t jb, int32_t L, const DecodeParams& p) {
         const uint32_t k_s = smem_addr(kt);
         const uint32_t v_s = k_s + kTileBytes;
         const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
         const float* vsc = ksc + kBlockTokens;
-        const int32_t mtx = lane >> 3, r = lane & 7;  // ldmatrix: matrix and row this lane addresses
+        const int32_t pos0 = jb * kBlockTokens;            // position of the tile's token 0
+        const int32_t nvalid = min(kBlockTokens, L - pos0);
+        const int32_t mtx = lane >> 3, r = lane & 7;       // ldmatrix: matrix and row this lane addresses
 
-        // ---- S = Q.K^T: s[nt] holds rows gid (c0, c1) and gid + 8 (c2, c3, unused)
+        // ---- S = Q.K^T: s[nt] = rows gid (c0, c1) and gid + 8 (c2, c3)
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        auto a_hi = [&](int ks, int h) -> uint32_t {
+            if constexpr (WIDE) return qa[1][ks][h];
+            return 0u;
+        };
         if constexpr (!kF16) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 uint32_t b[4];  // {nt0 dims lo, nt0 dims hi, nt1 dims lo, nt1 dims hi}
                 ldsm_x4(b, k_s + swz(8 * (mtx >> 1) + r, 2 * ks + (mtx & 1)));
-                mma_16816<false>(s[0], qa[ks][0], 0u, qa[ks][1], 0u, b[0], b[1]);
-                mma_16816<false>(s[1], qa[ks][0], 0u, qa[ks][1], 0u, b[2], b[3]);
+                mma_16816<false>(s[0], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b[0], b[1]);
+                mma_16816<false>(s[1], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b[2], b[3]);
             }
         } else {
 #pragma unroll
@@ -685,67 +715,88 @@ struct MmaMath {
                     uint32_t b0, b1, b2, b3;
                     e4m3x4_to_f16x2x2(w[h], b0, b1);
                     e4m3x4_to_f16x2x2(w[2 + h], b2, b3);
-                    mma_16816<true>(s[0], qa[ks][0], 0u, qa[ks][1], 0u, b0, b1);
-                    mma_16816<true>(s[1], qa[ks][0], 0u, qa[ks][1], 0u, b2, b3);
+                    mma_16816<true>(s[0], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b0, b1);
+                    mma_16816<true>(s[1], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b2, b3);
                 }
             }
         }
 
-        // ---- online softmax on row gid: tokens 8nt + 2tig + j
-        float mx = -INFINITY;
+        // ---- online softmax per row set: row gid + 8k holds tokens 8nt + 2tig + j
+        float pr[kSets][2][2];
+        float corr[kSets];
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int t = 8 * nt + 2 * tig + j;
-                float v = s[nt][j] * p.scale_log2;
-                if constexpr (kF16) v *= ksc[t];
-                s[nt][j] = (t < nvalid) ? v : -INFINITY;
-                mx = fmaxf(mx, s[nt][j]);
-            }
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-        const float m_new = fmaxf(m_run, mx);
-        const float corr = exp2f(m_run - m_new);
-        float pr[2][2];
-        float psum = 0.0f;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                pr[nt][j] = exp2f(s[nt][j] - m_new);
-                psum += pr[nt][j];
-            }
-        l_run = l_run * corr + psum;
-        m_run = m_new;
-
-        // rescale O^T columns (heads 2tig, 2tig+1): head h's factor is on lanes gid == h
-        const float ca = __shfl_sync(0xffffffffu, corr, 8 * tig);
-        const float cb = __shfl_sync(0xffffffffu, corr, 8 * tig + 4);
-        if (__any_sync(0xffffffffu, ca != 1.0f || cb != 1.0f)) {
-#pragma unroll
-            for (int mi = 0; mi < 8; ++mi) {
-                o[mi][0] *= ca;
-                o[mi][1] *= cb;
-                o[mi][2] *= ca;
-                o[mi][3] *= cb;
-            }
-        }
-
-        // ---- P^T fragment (B operand: k = token, n = head gid).  Tokens past the
-        // context end have p = 0; their V rows and scales may hold anything (NaN
-        // included), so they are removed by select, never multiplied.
-        if constexpr (kF16) {
+        for (int k = 0; k < kSets; ++k) {
+            const int32_t last = L - nq + qtok[k];         // last position this row sees
+            float mx = -INFINITY;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int t = 8 * nt + 2 * tig + j;
-                    pr[nt][j] = (t < nvalid) ? pr[nt][j] * vsc[t] : 0.0f;
+                    float v = s[nt][2 * k + j] * p.scale_log2;
+                    if constexpr (kF16) v *= ksc[t];
+                    pr[k][nt][j] = (pos0 + t <= last) ? v : -INFINITY;
+                    mx = fmaxf(mx, pr[k][nt][j]);
                 }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            const float m_new = fmaxf(m_run[k], mx);
+            // a row that has seen nothing yet keeps max -inf; exponentiate against 0 then
+            const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+            corr[k] = exp2f(m_run[k] - m_use);
+            float psum = 0.0f;
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    pr[k][nt][j] = exp2f(pr[k][nt][j] - m_use);
+                    psum += pr[k][nt][j];
+                }
+            l_run[k] = l_run[k] * corr[k] + psum;
+            m_run[k] = m_new;
         }
-        const uint32_t pb0 = pack2<kF16>(pr[0][0], pr[0][1]);
-        const uint32_t pb1 = pack2<kF16>(pr[1][0], pr[1][1]);
+
+        // rescale O^T columns: column 8k + 2tig + j is row gid' = 2tig + j of set k
+        {
+            float cf[kSets][2];
+            bool any = false;
+#pragma unroll
+            for (int k = 0; k < kSets; ++k) {
+                cf[k][0] = __shfl_sync(0xffffffffu, corr[k], 8 * tig);
+                cf[k][1] = __shfl_sync(0xffffffffu, corr[k], 8 * tig + 4);
+                any = any || cf[k][0] != 1.0f || cf[k][1] != 1.0f;
+            }
+            if (__any_sync(0xffffffffu, any)) {
+#pragma unroll
+                for (int k = 0; k < kSets; ++k)
+#pragma unroll
+                    for (int mi = 0; mi < 8; ++mi) {
+                        o[k][mi][0] *= cf[k][0];
+                        o[k][mi][1] *= cf[k][1];
+                        o[k][mi][2] *= cf[k][0];
+                        o[k][mi][3] *= cf[k][1];
+                    }
+            }
+        }
+
+        // ---- P^T fragments (B operand: k = token, n = row gid of set k).  Tokens
+        // past the context end have p = 0; their V rows and scales may hold
+        // anything (NaN included), so they are removed by select, never multiplied.
+        uint32_t pb[kSets][2];
+#pragma unroll
+        for (int k = 0; k < kSets; ++k) {
+            if constexpr (kF16) {
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int t = 8 * nt + 2 * tig + j;
+                        pr[k][nt][j] = (t < nvalid) ? pr[k][nt][j] * vsc[t] : 0.0f;
+                    }
+            }
+            pb[k][0] = pack2<kF16>(pr[k][0][0], pr[k][0][1]);
+            pb[k][1] = pack2<kF16>(pr[k][1][0], pr[k][1][1]);
+        }
         // V^T fragment halves of tokens 2tig, 2tig+1 (mask_a) and 8+2tig, 9+2tig (mask_b)
         const bool partial = nvalid < kBlockTokens;
         const uint32_t mask_a = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
@@ -763,7 +814,9 @@ struct MmaMath {
                     a[2] &= mask_b;
                     a[3] &= mask_b;
                 }
-                mma_16816<false>(o[mi], a[0], a[1], a[2], a[3], pb0, pb1);
+#pragma unroll
+                for (int k = 0; k < kSets; ++k)
+                    mma_16816<false>(o[k][mi], a[0], a[1], a[2], a[3], pb[k][0], pb[k][1]);
             }
         } else {
 #pragma unroll
@@ -783,7 +836,9 @@ struct MmaMath {
                         lo1 &= mask_b;
                         hi1 &= mask_b;
                     }
-                    mma_16816<true>(o[2 * mq + h], lo0, hi0, lo1, hi1, pb0, pb1);
+#pragma unroll
+                    for (int k = 0; k < kSets; ++k)
+                        mma_16816<true>(o[k][2 * mq + h], lo0, hi0, lo1, hi1, pb[k][0], pb[k][1]);
                 }
             }
         }
@@ -791,34 +846,40 @@ struct MmaMath {
 
     __device__ void finish(const DecodeParams& p, int32_t b, int32_t kvh, bool whole,
                            int64_t pid) {
-        float l = l_run;  // row gid's sum over its 4 lanes
-        l += __shfl_xor_sync(0xffffffffu, l, 1);
-        l += __shfl_xor_sync(0xffffffffu, l, 2);
-        const float la = __shfl_sync(0xffffffffu, l, 8 * tig);      // head 2tig
-        const float lb = __shfl_sync(0xffffffffu, l, 8 * tig + 4);  // head 2tig + 1
-        const int64_t bh0 = static_cast<int64_t>(b) * p.num_q_heads + kvh * G;
 #pragma unroll
-        for (int j = 0; j < 2; ++j) {
-            const int h = 2 * tig + j;
-            if (h >= G) continue;
-            const float lh = j ? lb : la;
-            if (whole) {
-                uint16_t* out = static_cast<uint16_t*>(p.out) + (bh0 + h) * D;
+        for (int k = 0; k < kSets; ++k) {
+            float l = l_run[k];  // row gid + 8k's sum over its 4 lanes
+            l += __shfl_xor_sync(0xffffffffu, l, 1);
+            l += __shfl_xor_sync(0xffffffffu, l, 2);
+            const float lr[2] = {__shfl_sync(0xffffffffu, l, 8 * tig),        // row 8k + 2tig
+                                 __shfl_sync(0xffffffffu, l, 8 * tig + 4)};   // row 8k + 2tig + 1
 #pragma unroll
-                for (int mi = 0; mi < 8; ++mi) {
-                    out[dim_of(mi, gid)] = out_cast<uint16_t>(lh > 0.0f ? o[mi][j] / lh : 0.0f);
-                    out[dim_of(mi, gid + 8)] = out_cast<uint16_t>(lh > 0.0f ? o[mi][2 + j] / lh : 0.0f);
-                }
-            } else {
-                float* ws = p.ws_o + (pid * G + h) * D;
+            for (int j = 0; j < 2; ++j) {
+                const int32_t row = 8 * k + 2 * tig + j;
+                if (row >= rows) continue;
+                const int32_t i = row / G, g = row % G;
+                const float lh = lr[j];
+                if (whole) {
+                    uint16_t* out = static_cast<uint16_t*>(p.out) +
+                                    ((static_cast<int64_t>(b) * nq + i) * p.num_q_heads + kvh * G + g) * D;
 #pragma unroll
-                for (int mi = 0; mi < 8; ++mi) {
-                    ws[dim_of(mi, gid)] = o[mi][j];
-                    ws[dim_of(mi, gid + 8)] = o[mi][2 + j];
+                    for (int mi = 0; mi < 8; ++mi) {
+                        out[dim_of(mi, gid)] = out_cast<uint16_t>(lh > 0.0f ? o[k][mi][j] / lh : 0.0f);
+                        out[dim_of(mi, gid + 8)] =
+                            out_cast<uint16_t>(lh > 0.0f ? o[k][mi][2 + j] / lh : 0.0f);
+                    }
+                } else {
+                    float* ws = p.ws_o + (pid * rows + row) * D;
+#pragma unroll
+                    for (int mi = 0; mi < 8; ++mi) {
+                        ws[dim_of(mi, gid)] = o[k][mi][j];
+                        ws[dim_of(mi, gid + 8)] = o[k][mi][2 + j];
+                    }
                 }
             }
+            if (!whole && tig == 0 && gid + 8 * k < rows)
+                p.ws_ml[pid * rows + gid + 8 * k] = make_float2(m_run[k], l);
         }
-        if (!whole && gid < G && tig == 0) p.ws_ml[pid * G + gid] = make_float2(m_run, l);
     }
 };
 
@@ -974,8 +1035,7 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
             *abort_flag = 1;
         }
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return;  // output invalid (reported)
-        if (stage_ok[s])
-            math.tile(ring + s * M::kStageBytes, min(kBlockTokens, cur.L - cur.jb * kBlockTokens), p);
+        if (stage_ok[s]) math.tile(ring + s * M::kStageBytes, cur.jb, cur.L, p);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
@@ -1010,17 +1070,22 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
     pdl_wait();
     pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
+    // one warp per output row (sequence b, query token i, head h): out is [B][Q][Hq][D]
     const int64_t bh = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
-    if (bh >= static_cast<int64_t>(p.batch) * p.num_q_heads) return;
-    const int32_t b = static_cast<int32_t>(bh / p.num_q_heads);
+    const int32_t nq = p.num_query_tokens;
+    if (bh >= static_cast<int64_t>(p.batch) * nq * p.num_q_heads) return;
+    const int32_t b = static_cast<int32_t>(bh / (static_cast<int64_t>(nq) * p.num_q_heads));
     const int32_t h = static_cast<int32_t>(bh % p.num_q_heads);
+    const int32_t qi = static_cast<int32_t>((bh / p.num_q_heads) % nq);
     const int32_t G = p.num_q_heads / p.num_kv_heads;
-    const int32_t kvh = h / G, g = h % G;
+    const int32_t kvh = h / G;
+    const int32_t R = G * nq;          // query rows of a (sequence, kv head) pair
+    const int32_t g = qi * G + h % G;  // this warp's row within the pair
     // three independent loads in one round trip
     const int32_t L = p.context_lens[b];
     const int64_t T = p.ws_seq_start[p.batch];
     const int64_t seq0 = p.ws_seq_start[b];
-    const int32_t nt = seq_tiles(L, p.max_context_len);
+    const int32_t nt = seq_tiles(L, p);
     OutT* out = static_cast<OutT*>(p.out) + bh * D + lane * kDPL;
     if (nt == 0) {
 #pragma unroll
@@ -1051,7 +1116,7 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
         // lane i: piece i0+i's (m, l); every lane: this round's first kBatch partial
         // outputs -- both sets of loads are in flight together
         const int64_t pl = (i0 + lane < npieces) ? piece_id(i0 + lane) : -1;
-        const float2 ml = pl >= 0 ? p.ws_ml[pl * G + g] : make_float2(-INFINITY, 0.0f);
+        const float2 ml = pl >= 0 ? p.ws_ml[pl * R + g] : make_float2(-INFINITY, 0.0f);
         const int cnt = min(32, npieces - i0);
         float v[kBatch][kDPL];
         int64_t pids[kBatch];
@@ -1059,7 +1124,7 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
         for (int u = 0; u < kBatch; ++u) {
             pids[u] = __shfl_sync(0xffffffffu, pl, u);
             const bool use = u < cnt && pids[u] >= 0;
-            const float* src = p.ws_o + ((use ? pids[u] : 0) * G + g) * D + lane * kDPL;
+            const float* src = p.ws_o + ((use ? pids[u] : 0) * R + g) * D + lane * kDPL;
 #pragma unroll
             for (int j = 0; j < kDPL; ++j) v[u][j] = use ? src[j] : 0.0f;
         }
@@ -1088,7 +1153,7 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
                 const int i = (u0 + u) & 31;
                 pids[u] = __shfl_sync(0xffffffffu, pl, i);
                 const bool use = u0 + u < cnt && pids[u] >= 0;
-                const float* src = p.ws_o + ((use ? pids[u] : 0) * G + g) * D + lane * kDPL;
+                const float* src = p.ws_o + ((use ? pids[u] : 0) * R + g) * D + lane * kDPL;
 #pragma unroll
                 for (int j = 0; j < kDPL; ++j) v[u][j] = use ? src[j] : 0.0f;
             }
@@ -1127,7 +1192,7 @@ static cudaError_t launch_one(const DecodeParams& p, const TmaMaps& maps, cudaSt
     e = launch_pdl(paged_decode_kernel<M, Q_T>, dim3(grid), dim3(kThreads), S::kBytes, stream, p,
                    maps);
     if (e != cudaSuccess) return e;
-    const int64_t warps = static_cast<int64_t>(p.batch) * p.num_q_heads;
+    const int64_t warps = static_cast<int64_t>(p.batch) * p.num_query_tokens * p.num_q_heads;
     return launch_pdl(paged_decode_merge_kernel<Q_T, D>,
                       dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, stream, p);
 }
@@ -1143,15 +1208,22 @@ static cudaError_t dispatch_g(const DecodeParams& p, const TmaMaps& maps, int32_
     }
 }
 
+template <int KV_T, bool WIDE>
+static cudaError_t dispatch_mma_g(const DecodeParams& p, const TmaMaps& maps, int32_t group,
+                                  cudaStream_t s) {
+    switch (group) {
+        case 1: return launch_one<MmaMath<KV_T, 1, WIDE>, KV_BF16, 128>(p, maps, s);
+        case 2: return launch_one<MmaMath<KV_T, 2, WIDE>, KV_BF16, 128>(p, maps, s);
+        case 4: return launch_one<MmaMath<KV_T, 4, WIDE>, KV_BF16, 128>(p, maps, s);
+        default: return launch_one<MmaMath<KV_T, 8, WIDE>, KV_BF16, 128>(p, maps, s);
+    }
+}
+
 template <int KV_T>
 static cudaError_t dispatch_mma(const DecodeParams& p, const TmaMaps& maps, int32_t group,
                                 cudaStream_t s) {
-    switch (group) {
-        case 1: return launch_one<MmaMath<KV_T, 1>, KV_BF16, 128>(p, maps, s);
-        case 2: return launch_one<MmaMath<KV_T, 2>, KV_BF16, 128>(p, maps, s);
-        case 4: return launch_one<MmaMath<KV_T, 4>, KV_BF16, 128>(p, maps, s);
-        default: return launch_one<MmaMath<KV_T, 8>, KV_BF16, 128>(p, maps, s);
-    }
+    return group * p.num_query_tokens > 8 ? dispatch_mma_g<KV_T, true>(p, maps, group, s)
+                                          : dispatch_mma_g<KV_T, false>(p, maps, group, s);
 }
 
 template <int KV_T, int Q_T>
@@ -1186,6 +1258,8 @@ cudaError_t launch_paged_decode(const DecodeParams& p, const TmaMaps& maps, int3
     }
 }
 
-int32_t decode_ctas_per_sm(int32_t, int32_t, int32_t) { return 3; }
+int32_t decode_ctas_per_sm(int32_t, int32_t, int32_t group, int32_t query_tokens) {
+    return group * query_tokens > 8 ? 2 : 3;
+}
 
 }  // namespace pkv

@@ -57,11 +57,12 @@ struct DecodeParams {
     const int32_t* block_table;   // [B][max_blocks]
     const int32_t* context_lens;  // [B]
     int32_t* ws_seq_start;        // [B + 1]: first tile of each sequence, total tiles at [B]
-    float2* ws_ml;                // [pieces][G]: (running max in base-2 units, running sum)
-    float* ws_o;                  // [pieces][G][D]: unnormalised partial outputs
+    float2* ws_ml;                // [pieces][G*Q]: (running max in base-2 units, running sum)
+    float* ws_o;                  // [pieces][G*Q][D]: unnormalised partial outputs
     int32_t* dev_error;
     int32_t batch, num_q_heads, num_kv_heads, num_blocks, max_blocks;
     int32_t max_context_len;
+    int32_t num_query_tokens;     // Q: query tokens per sequence (1 for decode)
     int32_t num_ranges;           // consumer-warp ranges the tile list is cut into
     float scale_log2;             // scale * log2(e): scores are kept in base-2 units
 };
@@ -74,7 +75,8 @@ struct TmaMaps {
 };
 
 // Resident decode CTAs per SM the kernels are built for (their register budget).
-int32_t decode_ctas_per_sm(int32_t kv_dtype, int32_t head_dim, int32_t group);
+int32_t decode_ctas_per_sm(int32_t kv_dtype, int32_t head_dim, int32_t group,
+                           int32_t query_tokens);
 
 // Whether this shape runs the tensor-core tile arithmetic (and needs TmaMaps).
 bool decode_uses_tensor_cores(int32_t kv_dtype, int32_t q_dtype, int32_t head_dim);

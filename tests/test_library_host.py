@@ -175,3 +175,38 @@ def test_slot_mapping_host_validation():
                                     None) == pk.KV_ERR_UNSUPPORTED
     assert lib.compute_slot_mapping(None, 2, 4, 16, 2 << 20, 3 << 20, 5, 4 << 20, None,
                                     None) == pk.KV_ERR_INVALID_ARGUMENT
+
+
+def _call_mq(desc, q_tokens, **kw):
+    lib = pk.library()
+    a = dict(out=4096, q=8192, q_dtype=pk.KV_BF16, k_pool=1 << 20, v_pool=2 << 20, scales=None,
+             block_table=3 << 20, max_blocks=256, context_lens=4 << 20, batch=4, num_q_heads=32,
+             max_context_len=4096, scale=0.088, partition=0, workspace=None, workspace_bytes=0)
+    a.update(kw)
+    return lib.paged_attention_multi_query(
+        ctypes.byref(desc), a["out"], a["q"], a["q_dtype"], q_tokens, a["k_pool"], a["v_pool"],
+        a["scales"], a["block_table"], a["max_blocks"], a["context_lens"], a["batch"],
+        a["num_q_heads"], a["max_context_len"], a["scale"], a["partition"], a["workspace"],
+        a["workspace_bytes"], None, None)
+
+
+def test_multi_query_host_validation():
+    bf = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_BF16)
+    f32 = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_F32)
+    d64 = pk.kv_pool_create(8192, 16, 8, 64, pk.KV_BF16)
+    assert _call_mq(bf, 5) == pk.KV_ERR_UNSUPPORTED                  # 4 heads x 5 tokens > 16
+    assert _call_mq(f32, 2) == pk.KV_ERR_UNSUPPORTED                 # fp32 KV: one token only
+    assert _call_mq(d64, 2) == pk.KV_ERR_UNSUPPORTED                 # head_dim 64: one token only
+    assert _call_mq(bf, 2, q_dtype=pk.KV_F32) == pk.KV_ERR_UNSUPPORTED
+    assert _call_mq(bf, 0) == pk.KV_ERR_INVALID_ARGUMENT
+    assert _call_mq(bf, 4, max_context_len=3) == pk.KV_ERR_INVALID_ARGUMENT
+    assert _call_mq(bf, 4) == pk.KV_ERR_INVALID_ARGUMENT             # no workspace
+    # one query token is the decode; 4 heads x 4 tokens = 16 rows per kv head run
+    # 2 CTAs per SM (the wide tile), so 148 * 2 * 4 ranges
+    w1 = pk.paged_attention_workspace_bytes(bf, 32, 32, 1, 4096, 0)
+    assert w1 == pk.paged_decode_workspace_bytes(bf, 32, 32, 4096, 0)
+    assert pk.paged_decode_num_ranges(bf, 32, 32, 4096, 0) == 148 * 3 * 4
+    pieces, rows = 32 * 8 + 148 * 2 * 4, 16
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    want = up(4 * 33) + up(pieces * rows * 8) + pieces * rows * 128 * 4
+    assert pk.paged_attention_workspace_bytes(bf, 32, 32, 4, 4096, 0) == want

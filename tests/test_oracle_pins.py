@@ -341,3 +341,51 @@ def test_scatter_then_gather_round_trip():
     # negative slots are padding
     skipped = oracle.scatter_to_pool(poison, rows[:2], np.array([-1, slots[1]]))
     assert np.isnan(skipped).sum() == (nb * 16 - 1) * hkv * d
+
+
+# ---------------------------------------------------------------- multi-query (causal)
+def test_multi_query_one_token_is_decode():
+    rng = np.random.default_rng(21)
+    q, k, v, offs, lens = _rand_case(rng, 3, 8, 2, 64, [5, 40, 1])
+    mq = oracle.multi_query_attention(q[:, None], k, v, offs, lens, 0.2, 2, "f32", "f32")
+    dec = oracle.decode_attention(q, k, v, offs, lens, 0.2, 2, "f32", "f32")
+    assert (mq[:, 0] == dec).all()
+
+
+def test_multi_query_rows_are_decodes_of_shorter_contexts():
+    rng = np.random.default_rng(22)
+    nq = 4
+    _, k, v, offs, lens = _rand_case(rng, 3, 8, 2, 32, [4, 19, 50])
+    q = rng.normal(size=(3, nq, 8, 32)).astype(np.float32)
+    mq = oracle.multi_query_attention(q, k, v, offs, lens, 0.3, 2, "f32", "f32")
+    for i in range(nq):
+        dec = oracle.decode_attention(np.ascontiguousarray(q[:, i]), k, v, offs, lens - nq + i + 1,
+                                      0.3, 2, "f32", "f32")
+        assert np.abs(mq[:, i] - dec).max() <= 1e-12
+
+
+def test_multi_query_matches_torch_sdpa_with_causal_offset_mask():
+    rng = np.random.default_rng(23)
+    nq, hq, hkv, d = 3, 4, 2, 16
+    _, k, v, offs, lens = _rand_case(rng, 2, hq, hkv, d, [3, 11])
+    q = rng.normal(size=(2, nq, hq, d)).astype(np.float32)
+    mq = oracle.multi_query_attention(q, k, v, offs, lens, 0.25, hkv, "f32", "f32")
+    for s in range(2):
+        o, n = int(offs[s]), int(lens[s])
+        qq = torch.from_numpy(q[s].astype(np.float64)).permute(1, 0, 2)[None]     # [1,Hq,Q,D]
+        kk = torch.from_numpy(k[o:o + n].astype(np.float64)).permute(1, 0, 2)[None]
+        vv = torch.from_numpy(v[o:o + n].astype(np.float64)).permute(1, 0, 2)[None]
+        pos = torch.arange(n)[None, :]
+        limit = (n - nq + torch.arange(nq))[:, None]
+        mask = pos <= limit                                                        # [Q, n]
+        ref = torch.nn.functional.scaled_dot_product_attention(qq, kk, vv, attn_mask=mask,
+                                                               scale=0.25, enable_gqa=True)
+        assert np.abs(mq[s] - ref[0].permute(1, 0, 2).numpy()).max() <= 1e-12
+
+
+def test_multi_query_rejects_short_context():
+    rng = np.random.default_rng(24)
+    _, k, v, offs, lens = _rand_case(rng, 2, 4, 1, 16, [2, 9])
+    q = rng.normal(size=(2, 3, 4, 16)).astype(np.float32)
+    with pytest.raises(ValueError):
+        oracle.multi_query_attention(q, k, v, offs, lens, 1.0, 1, "f32", "f32")
