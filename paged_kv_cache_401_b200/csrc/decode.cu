@@ -577,10 +577,16 @@ struct SimtMath {
 // scale) rounded to f16; the K row scale multiplies the scores.  Element
 // orders inside a k-step are permuted consistently between the two operands
 // (a dot product does not depend on the order of its terms), which is what
-// lets FP8 rows be read with 16-bit ldmatrix.  WIDE = more than 8 query rows.
+// lets FP8 rows be read with 16-bit ldmatrix.  QM: kSingle = one query token
+// (the decode: no causal bookkeeping), kNarrow = up to 8 query rows, kWide = up
+// to 16 (two row sets).
 // ======================================================================================
-template <int KV_T, int G, bool WIDE>
+enum QueryMode { kSingle = 1, kNarrow = 2, kWide = 3 };
+
+template <int KV_T, int G, int QM>
 struct MmaMath {
+    static constexpr bool WIDE = QM == kWide;
+    static constexpr bool SINGLE = QM == kSingle;
     static_assert(KV_T == KV_BF16 || KV_T == KV_FP8_E4M3, "bf16 or FP8 KV");
     static_assert(G <= 8, "a row set holds 8 query rows");
     using OutT = uint16_t;                                        // bf16 output
@@ -639,7 +645,7 @@ struct MmaMath {
     }
 
     __device__ void load_q(const DecodeParams& p, int32_t b, int32_t kvh) {
-        nq = p.num_query_tokens;
+        nq = SINGLE ? 1 : p.num_query_tokens;
         rows = G * nq;
 #pragma unroll
         for (int k = 0; k < kSets; ++k) {
@@ -726,7 +732,8 @@ struct MmaMath {
         float corr[kSets];
 #pragma unroll
         for (int k = 0; k < kSets; ++k) {
-            const int32_t last = L - nq + qtok[k];         // last position this row sees
+            // last position this row sees (one query token: the context's last, for every row)
+            const int32_t last = SINGLE ? L - 1 : L - nq + qtok[k];
             float mx = -INFINITY;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
@@ -741,8 +748,9 @@ struct MmaMath {
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
             const float m_new = fmaxf(m_run[k], mx);
-            // a row that has seen nothing yet keeps max -inf; exponentiate against 0 then
-            const float m_use = m_new == -INFINITY ? 0.0f : m_new;
+            // with several query tokens a row may have seen nothing yet (max -inf):
+            // exponentiate against 0 then; one query token always sees a token
+            const float m_use = (!SINGLE && m_new == -INFINITY) ? 0.0f : m_new;
             corr[k] = exp2f(m_run[k] - m_use);
             float psum = 0.0f;
 #pragma unroll
@@ -1208,22 +1216,23 @@ static cudaError_t dispatch_g(const DecodeParams& p, const TmaMaps& maps, int32_
     }
 }
 
-template <int KV_T, bool WIDE>
+template <int KV_T, int QM>
 static cudaError_t dispatch_mma_g(const DecodeParams& p, const TmaMaps& maps, int32_t group,
                                   cudaStream_t s) {
     switch (group) {
-        case 1: return launch_one<MmaMath<KV_T, 1, WIDE>, KV_BF16, 128>(p, maps, s);
-        case 2: return launch_one<MmaMath<KV_T, 2, WIDE>, KV_BF16, 128>(p, maps, s);
-        case 4: return launch_one<MmaMath<KV_T, 4, WIDE>, KV_BF16, 128>(p, maps, s);
-        default: return launch_one<MmaMath<KV_T, 8, WIDE>, KV_BF16, 128>(p, maps, s);
+        case 1: return launch_one<MmaMath<KV_T, 1, QM>, KV_BF16, 128>(p, maps, s);
+        case 2: return launch_one<MmaMath<KV_T, 2, QM>, KV_BF16, 128>(p, maps, s);
+        case 4: return launch_one<MmaMath<KV_T, 4, QM>, KV_BF16, 128>(p, maps, s);
+        default: return launch_one<MmaMath<KV_T, 8, QM>, KV_BF16, 128>(p, maps, s);
     }
 }
 
 template <int KV_T>
 static cudaError_t dispatch_mma(const DecodeParams& p, const TmaMaps& maps, int32_t group,
                                 cudaStream_t s) {
-    return group * p.num_query_tokens > 8 ? dispatch_mma_g<KV_T, true>(p, maps, group, s)
-                                          : dispatch_mma_g<KV_T, false>(p, maps, group, s);
+    if (p.num_query_tokens == 1) return dispatch_mma_g<KV_T, kSingle>(p, maps, group, s);
+    return group * p.num_query_tokens > 8 ? dispatch_mma_g<KV_T, kWide>(p, maps, group, s)
+                                          : dispatch_mma_g<KV_T, kNarrow>(p, maps, group, s);
 }
 
 template <int KV_T, int Q_T>
