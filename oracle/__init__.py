@@ -16,7 +16,10 @@ restatement, in double precision, of every step of the decode hot path:
                              a pool laid out [block][kv_head][slot][dim].
 * ``e4m3_decode`` / ``e4m3_encode`` / ``quantize_rows`` -- the FP8-E4M3 codec
                              and per-(token, kv head) absmax/448 scales
-                             ("KV Cache 深度解析", §四 KV Cache 量化).
+                             ("KV Cache 深度解析", §四 KV Cache 量化);
+                             ``quantize_rows(x, "int8")`` the INT8 cache, symmetric
+                             absmax/127 (k1-blog "KV Cache 量化", freetools
+                             "KV Cache量化": INT8 halves the cache like FP8).
 * ``decode_attention``    -- softmax(q·Kᵀ·scale)·V over a CONTIGUOUS per-sequence
                              copy, GQA head grouping, two passes in double
                              (C, OpenMP); "KV Cache 深度解析", §一 and §六.
@@ -43,8 +46,9 @@ import numpy as np
 
 from . import build as _build
 
-F32, BF16, FP8_E4M3 = 0, 1, 2
-_DTYPE_CODES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3}
+F32, BF16, FP8_E4M3, INT8 = 0, 1, 2, 3
+_DTYPE_CODES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3, "int8": INT8}
+QUANTIZED = ("fp8", "int8")
 
 _lib = None
 
@@ -61,6 +65,8 @@ def _load():
         lib.oracle_quantize_rows.restype = None
         lib.oracle_quantize_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32,
                                              ctypes.c_void_p, ctypes.c_void_p]
+        lib.oracle_quantize_rows_int8.restype = None
+        lib.oracle_quantize_rows_int8.argtypes = lib.oracle_quantize_rows.argtypes
         lib.oracle_decode_attention.restype = ctypes.c_int
         lib.oracle_decode_attention.argtypes = [
             ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -167,14 +173,24 @@ def e4m3_encode(x: np.ndarray) -> np.ndarray:
     return out.reshape(np.shape(x))
 
 
-def quantize_rows(x: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
-    """x: [..., D] float32 -> (codes uint8 [..., D], scales float32 [...])."""
+def quantize_rows(x: np.ndarray, kind: str = "fp8") -> tuple[np.ndarray, np.ndarray]:
+    """x: [..., D] float32 -> (codes [..., D], scales float32 [...]).
+
+    kind "fp8": uint8 E4M3 codes, scale absmax/448; "int8": int8 codes,
+    scale absmax/127, round to nearest (ties to even), clamp to +-127."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     d = x.shape[-1]
     rows = x.size // d
-    codes = np.empty(x.shape, dtype=np.uint8)
     scales = np.empty(x.shape[:-1], dtype=np.float32)
-    _load().oracle_quantize_rows(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
+    lib = _load()
+    if kind == "int8":
+        codes = np.empty(x.shape, dtype=np.int8)
+        lib.oracle_quantize_rows_int8(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
+    elif kind == "fp8":
+        codes = np.empty(x.shape, dtype=np.uint8)
+        lib.oracle_quantize_rows(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
+    else:
+        raise ValueError(f"unknown quantisation {kind!r}")
     return codes, scales
 
 
@@ -188,10 +204,10 @@ def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offsets: n
     """Double-precision decode attention (C oracle).
 
     q     : [B][Hq][D]   float32 (q_dtype "f32") or uint16 bf16 bits ("bf16")
-    k, v  : [T][Hkv][D]  float32 / uint16 bf16 bits / uint8 E4M3 codes
+    k, v  : [T][Hkv][D]  float32 / uint16 bf16 bits / uint8 E4M3 codes / int8 codes
     seq_offsets : [B] int64, first token of each sequence in k/v
     lens  : [B] int32 context lengths (>= 1)
-    k_scale, v_scale : [T][Hkv] float32 for kv_dtype "fp8"
+    k_scale, v_scale : [T][Hkv] float32 for kv_dtype "fp8" / "int8"
     Returns out [B][Hq][D] float64 (and weights [B][Hq][max(lens)] if asked).
     """
     lib = _load()
@@ -201,7 +217,7 @@ def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offsets: n
     v = np.ascontiguousarray(v)
     seq_offsets = np.ascontiguousarray(seq_offsets, dtype=np.int64)
     lens = np.ascontiguousarray(lens, dtype=np.int32)
-    if kv_dtype == "fp8":
+    if kv_dtype in QUANTIZED:
         k_scale = np.ascontiguousarray(k_scale, dtype=np.float32)
         v_scale = np.ascontiguousarray(v_scale, dtype=np.float32)
     out = np.empty((b, hq, d), dtype=np.float64)
@@ -229,7 +245,7 @@ def multi_query_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offse
     v = np.ascontiguousarray(v)
     seq_offsets = np.ascontiguousarray(seq_offsets, dtype=np.int64)
     lens = np.ascontiguousarray(lens, dtype=np.int32)
-    if kv_dtype == "fp8":
+    if kv_dtype in QUANTIZED:
         k_scale = np.ascontiguousarray(k_scale, dtype=np.float32)
         v_scale = np.ascontiguousarray(v_scale, dtype=np.float32)
     out = np.empty((b, nq, hq, d), dtype=np.float64)
@@ -244,12 +260,15 @@ def multi_query_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offse
 
 def widen(x: np.ndarray, dtype: str, scales: np.ndarray | None = None) -> np.ndarray:
     """Stored values -> float64, exactly (bf16 bits shifted into binary32;
-    E4M3 codes decoded and multiplied by their row scale)."""
+    E4M3 / INT8 codes decoded and multiplied by their row scale)."""
     if dtype == "f32":
         return np.asarray(x, dtype=np.float32).astype(np.float64)
     if dtype == "bf16":
         return (np.asarray(x, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32) \
             .astype(np.float64)
+    if dtype == "int8":
+        return np.asarray(x, dtype=np.int8).astype(np.float64) * \
+            np.asarray(scales, dtype=np.float64)[..., None]
     return e4m3_decode(x) * np.asarray(scales, dtype=np.float64)[..., None]
 
 

@@ -15,6 +15,9 @@
  *    subtract the max, exponentiate, normalise, weight V).
  *  - "KV Cache 深度解析", §四 (fp16 → fp8 E4M3 KV quantisation with a
  *    per-token scale to hold outliers) for the FP8 codec and scales.
+ *  - k1-blog 2026-07-13 "AI", "KV Cache 量化" (FP8 and INT8 both halve the
+ *    fp16 cache) and "大模型推理为何这么慢", "KV Cache量化" (INT8 among the
+ *    lower-precision KV formats) for the INT8 cache.
  *  - "大模型推理为何这么慢？从内存带宽瓶颈到KV Cache优化的技术突围"
  *    (freetools), section on GQA (H query heads share G groups of K/V).
  *
@@ -24,7 +27,11 @@
  *  - the FP8 scale of a (token, kv head) row is absmax/448 computed in
  *    IEEE fp32, the code is E4M3(x / scale) with round-to-nearest-even and
  *    saturation to ±448, and an all-zero row has scale 0 and codes 0x00;
- *  - FP8 attention dequantises exactly: value(code) * scale, in double.
+ *  - FP8 attention dequantises exactly: value(code) * scale, in double;
+ *  - the INT8 cache follows the FP8 design: symmetric, scale = absmax/127 in
+ *    IEEE fp32, code = x / scale (fp32 division) rounded to the nearest
+ *    integer, ties to even, clamped to [-127, 127]; an all-zero row has scale
+ *    0 and codes 0; dequantisation is code * scale in double.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math).
  */
@@ -37,7 +44,7 @@
 #endif
 
 /* Stored element types of K/V and q, as the callers of this file pass them. */
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2, ORC_INT8 = 3 };
 
 /* ---- exact widening of stored values ------------------------------------ */
 
@@ -136,7 +143,41 @@ void oracle_quantize_rows(const float* x, int64_t rows, int32_t d,
     }
 }
 
-/* Value of element i of a stored row, widened to double (FP8 dequantised). */
+/*
+ * INT8 quantisation of `rows` rows of length d (fp32 values, already rounded
+ * to the source dtype by the caller), symmetric per (token, kv head):
+ *   a = max |x|;  s = a / 127 (fp32 division);  y = x / s (fp32 division);
+ *   code = the integer nearest y (ties to the even one), clamped to
+ *   [-127, 127]; or s = 0 and every code 0 when a == 0.
+ */
+static int8_t round_half_even_clamped(float y) {
+    double f = floor((double)y);
+    double r = (double)y - f;                  /* exact: y and f are close */
+    double n = (r > 0.5) ? f + 1.0 : (r < 0.5) ? f : (fmod(f, 2.0) == 0.0 ? f : f + 1.0);
+    if (n > 127.0) n = 127.0;
+    if (n < -127.0) n = -127.0;
+    return (int8_t)n;
+}
+
+void oracle_quantize_rows_int8(const float* x, int64_t rows, int32_t d,
+                               int8_t* codes, float* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* xr = x + r * d;
+        float a = 0.0f, s;
+        int32_t i;
+        for (i = 0; i < d; ++i) {
+            float v = fabsf(xr[i]);
+            if (v > a) a = v;
+        }
+        s = a / 127.0f;
+        scales[r] = (a == 0.0f) ? 0.0f : s;
+        for (i = 0; i < d; ++i)
+            codes[r * d + i] = (a == 0.0f) ? 0 : round_half_even_clamped(xr[i] / s);
+    }
+}
+
+/* Value of element i of a stored row, widened to double (8-bit codes dequantised). */
 static double load_elem(const void* base, int dtype, int64_t idx, const float* scales,
                         int64_t scale_idx) {
     switch (dtype) {
@@ -144,6 +185,8 @@ static double load_elem(const void* base, int dtype, int64_t idx, const float* s
         return (double)((const float*)base)[idx];
     case ORC_BF16:
         return bf16_bits_to_double(((const uint16_t*)base)[idx]);
+    case ORC_INT8:
+        return (double)((const int8_t*)base)[idx] * (double)scales[scale_idx];
     default:
         return oracle_e4m3_decode(((const uint8_t*)base)[idx]) * (double)scales[scale_idx];
     }
@@ -155,7 +198,7 @@ static double load_elem(const void* base, int dtype, int64_t idx, const float* s
  *   q    : [B][Hq][D] in q_dtype (F32 or BF16)
  *   k, v : [total_tokens][Hkv][D] in kv_dtype, sequence b occupying tokens
  *          [seq_offsets[b], seq_offsets[b] + lens[b])
- *   k_scale, v_scale : [total_tokens][Hkv] fp32, FP8 only (else NULL)
+ *   k_scale, v_scale : [total_tokens][Hkv] fp32, FP8 / INT8 only (else NULL)
  *   out  : [B][Hq][D] double
  *   weights (nullable): [B][Hq][max_len] double, the softmax weights
  *

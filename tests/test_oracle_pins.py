@@ -3,6 +3,8 @@
 * printed values on the pages (tests/golden/kv_sizes.txt);
 * library routines (torch scaled_dot_product_attention in float64, torch's
   float8_e4m3fn conversion);
+* hand-computed INT8 rows with exact binary scales, and a brute-force
+  nearest-integer search for the INT8 codes;
 * closed forms and special cases (length 1, identical keys, dominant key,
   weights summing to one, key-order invariance);
 * brute force on tiny inputs (numpy, one head at a time) and an independent
@@ -145,6 +147,68 @@ def test_quantize_rows_closed_form():
     assert (err <= bound).all()
 
 
+# ---------------------------------------------------------------- INT8 rows
+def test_int8_quantize_hand_examples():
+    # scales that are exact binary numbers, so every y = x / s is exact and the
+    # codes follow by hand: ties go to the even integer, |code| <= 127
+    x = np.array([[127, -0.5, 1.5, 2.5, -3.5, 0.49, 126.5, -127],
+                  [254, 3, -5, 1, -254, 0.5, 253, -1],
+                  [0, 0, 0, 0, 0, 0, 0, 0],
+                  [-63.5, 0.25, 0.75, -0.25, 31.75, 0, 0, 0]], dtype=np.float32)
+    codes, scales = oracle.quantize_rows(x, "int8")
+    assert codes.dtype == np.int8
+    assert scales.tolist() == [1.0, 2.0, 0.0, 0.5]
+    assert codes.tolist() == [[127, 0, 2, 2, -4, 0, 126, -127],
+                              [127, 2, -2, 0, -127, 0, 126, 0],
+                              [0, 0, 0, 0, 0, 0, 0, 0],
+                              [-127, 0, 2, 0, 64, 0, 0, 0]]
+
+
+def test_int8_quantize_bruteforce_nearest_even():
+    # each code is the integer of [-127, 127] nearest the exact value of the
+    # fp32 quotient x / s (ties to even), searched over all 255 candidates
+    rng = np.random.default_rng(21)
+    x = (rng.standard_t(3, size=(24, 64)) * rng.uniform(0.01, 30, size=(24, 1))).astype(np.float32)
+    codes, scales = oracle.quantize_rows(x, "int8")
+    for r in range(x.shape[0]):
+        s = np.float32(np.abs(x[r]).max()) / np.float32(127.0)
+        assert scales[r] == s
+        for i in range(x.shape[1]):
+            y = Fraction(float(np.float32(x[r, i]) / s))
+            best = min(abs(y - c) for c in range(-127, 128))
+            cands = [c for c in range(-127, 128) if abs(y - c) == best]
+            want = cands[0] if len(cands) == 1 else [c for c in cands if c % 2 == 0][0]
+            assert codes[r, i] == want, (r, i, float(y), codes[r, i], want)
+
+
+def test_int8_quantize_invariants():
+    rng = np.random.default_rng(5)
+    x = rng.normal(size=(96, 128)).astype(np.float32)
+    x[3] = 0.0
+    x[7, :] = 0.0
+    x[7, 100] = 1e-30                                   # tiny but nonzero row
+    x[9] *= 1e6                                         # large row
+    codes, scales = oracle.quantize_rows(x, "int8")
+    amax = np.abs(x).max(axis=1)
+    assert (codes[3] == 0).all() and scales[3] == 0
+    for r in range(x.shape[0]):
+        if amax[r] == 0:
+            continue
+        i = int(np.abs(x[r]).argmax())
+        assert abs(int(codes[r, i])) == 127              # the largest element maps to +-127
+    assert int(np.abs(codes.astype(np.int32)).max()) == 127
+    # round to nearest: the error is at most half a step (plus the fp32 rounding of x / s)
+    deq = codes.astype(np.float64) * scales[:, None].astype(np.float64)
+    err = np.abs(deq - x.astype(np.float64))
+    assert (err <= scales[:, None].astype(np.float64) * (0.5 + 1e-5)).all()
+    # symmetric: negating the row negates the codes and keeps the scale
+    c2, s2 = oracle.quantize_rows(-x, "int8")
+    assert (c2 == -codes).all() and (s2 == scales).all()
+    # a power-of-two factor scales the scale and leaves the codes
+    c3, s3 = oracle.quantize_rows(x * np.float32(2.0 ** -7), "int8")
+    assert (c3 == codes).all() and (s3 == scales * np.float32(2.0 ** -7)).all()
+
+
 # ---------------------------------------------------------------- attention
 def _rand_case(rng, b, hq, hkv, d, lens, kv_dtype="f32"):
     total = int(sum(lens))
@@ -172,9 +236,9 @@ def test_attention_matches_bruteforce_numpy(hq, hkv):
     assert np.abs(ours - brute).max() <= 1e-12
 
 
-@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "fp8"])
+@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "fp8", "int8"])
 def test_attention_matches_torch_sdpa_float64(kv_dtype):
-    rng = np.random.default_rng({"f32": 1, "bf16": 2, "fp8": 3}[kv_dtype])
+    rng = np.random.default_rng({"f32": 1, "bf16": 2, "fp8": 3, "int8": 4}[kv_dtype])
     hq, hkv, d = 8, 2, 64
     lens = [3, 33, 64]
     q, k, v, offs, lens = _rand_case(rng, 3, hq, hkv, d, lens)
@@ -186,6 +250,12 @@ def test_attention_matches_torch_sdpa_float64(kv_dtype):
     elif kv_dtype == "bf16":
         kst, vst = _bf16_bits(k), _bf16_bits(v)
         k64, v64 = oracle.widen(kst, "bf16"), oracle.widen(vst, "bf16")
+    elif kv_dtype == "int8":
+        kst, ks = oracle.quantize_rows(k, "int8")
+        vst, vs = oracle.quantize_rows(v, "int8")
+        # dequantise independently of the oracle: code * scale in float64 (exact)
+        k64 = kst.astype(np.float64) * ks.astype(np.float64)[..., None]
+        v64 = vst.astype(np.float64) * vs.astype(np.float64)[..., None]
     else:
         kst, ks = oracle.quantize_rows(k)
         vst, vs = oracle.quantize_rows(v)
