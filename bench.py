@@ -147,13 +147,19 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- workload bytes
+def kv_row_bytes(spec) -> int:
+    """Bytes of one stored K or V row of one KV head (plus its fp32 scale for
+    an 8-bit cache)."""
+    elem = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[spec.kv_dtype]
+    return spec.head_dim * elem + (4 if spec.kv_dtype in ("fp8", "int8") else 0)
+
+
 def kv_bytes_per_step(inp) -> int:
     """Algorithmic KV bytes one decode step reads: every context token's K and V
-    row of every KV head (plus the fp32 per-row scales of an FP8 cache)."""
+    row of every KV head (plus the fp32 per-row scales of an FP8 / INT8 cache)."""
     spec = inp.spec
     tokens = int(inp.context_lens.astype(np.int64).sum())
-    elem = {"f32": 4, "bf16": 2, "fp8": 1}[spec.kv_dtype]
-    per_row = spec.head_dim * elem + (4 if spec.kv_dtype == "fp8" else 0)
+    per_row = kv_row_bytes(spec)
     return tokens * spec.num_kv_heads * 2 * per_row
 
 
@@ -164,8 +170,7 @@ def unique_kv_bytes_per_step(inp) -> int:
     nshare = min(spec.shared_prefix_seqs, inp.q.shape[0])
     if nshare <= 1:
         return kv_bytes_per_step(inp)
-    elem = {"f32": 4, "bf16": 2, "fp8": 1}[spec.kv_dtype]
-    per_row = spec.head_dim * elem + (4 if spec.kv_dtype == "fp8" else 0)
+    per_row = kv_row_bytes(spec)
     dup = (nshare - 1) * spec.shared_prefix_tokens
     return kv_bytes_per_step(inp) - dup * spec.num_kv_heads * 2 * per_row
 
@@ -224,19 +229,18 @@ def time_oracle(inp, max_seqs: int, repeats: int = 1):
     lens = inp.context_lens[seqs]
     args = dict(seq_offsets=inp.seq_offsets[seqs], lens=lens, scale=spec.scale,
                 num_kv_heads=spec.num_kv_heads, q_dtype=spec.q_dtype)
-    if spec.kv_dtype == "fp8":
+    if spec.kv_dtype in ("fp8", "int8"):
         rows = slice(int(inp.seq_offsets[0]), int(inp.seq_offsets[n - 1] + lens[-1]))
-        kc, ks = oracle.quantize_rows(inp.k[rows].float().numpy())
-        vc, vs = oracle.quantize_rows(inp.v[rows].float().numpy())
-        kv = dict(k=kc, v=vc, kv_dtype="fp8", k_scale=ks, v_scale=vs)
+        kc, ks = oracle.quantize_rows(inp.k[rows].float().numpy(), spec.kv_dtype)
+        vc, vs = oracle.quantize_rows(inp.v[rows].float().numpy(), spec.kv_dtype)
+        kv = dict(k=kc, v=vc, kv_dtype=spec.kv_dtype, k_scale=ks, v_scale=vs)
     else:
         kv = dict(k=storage_view(inp.k), v=storage_view(inp.v), kv_dtype=spec.kv_dtype)
     t0 = time.perf_counter()
     for _ in range(repeats):
         oracle.decode_attention(q, **kv, **args)
     dt = (time.perf_counter() - t0) / repeats
-    elem = {"f32": 4, "bf16": 2, "fp8": 1}[spec.kv_dtype]
-    per_row = spec.head_dim * elem + (4 if spec.kv_dtype == "fp8" else 0)
+    per_row = kv_row_bytes(spec)
     nbytes = int(lens.astype(np.int64).sum()) * spec.num_kv_heads * 2 * per_row
     desc = (f"oracle (C, double, OpenMP) over {n} of {inp.q.shape[0]} sequences "
             f"({int(lens.sum())} tokens, {nbytes / 2**20:.0f} MiB of KV) x {repeats}")

@@ -61,7 +61,8 @@ typedef enum {
 typedef enum {
     KV_F32 = 0,        /* IEEE binary32 */
     KV_BF16 = 1,       /* bfloat16 */
-    KV_FP8_E4M3 = 2    /* OCP FP8 E4M3 codes (KV pools only) with fp32 row scales */
+    KV_FP8_E4M3 = 2,   /* OCP FP8 E4M3 codes (KV pools only) with fp32 row scales */
+    KV_INT8 = 3        /* signed 8-bit codes (KV pools only) with fp32 row scales */
 } kv_dtype;
 
 /* Bits ORed into *dev_error by the kernels. */
@@ -76,9 +77,10 @@ typedef enum {
  *
  * Layout of each pool, row-major: [num_blocks][num_kv_heads][block_size][head_dim]
  * so the 16 tokens of one (physical block, kv head) pair are one contiguous
- * span of block_size*head_dim elements.  An FP8 cache also has ONE fp32 scale
- * pool laid out [num_blocks][num_kv_heads][2][block_size]: for each (block,
- * kv head) the 16 K row scales then the 16 V row scales, 128 contiguous bytes.
+ * span of block_size*head_dim elements.  A quantised cache (FP8 or INT8) also
+ * has ONE fp32 scale pool laid out [num_blocks][num_kv_heads][2][block_size]:
+ * for each (block, kv head) the 16 K row scales then the 16 V row scales, 128
+ * contiguous bytes.
  */
 typedef struct {
     int32_t num_blocks;
@@ -88,7 +90,7 @@ typedef struct {
     int32_t dtype;           /* kv_dtype */
     int32_t elem_bytes;      /* 4, 2 or 1 */
     uint64_t kv_bytes;       /* bytes of ONE pool (K or V) */
-    uint64_t scale_bytes;    /* bytes of the scale pool (FP8 only, else 0) */
+    uint64_t scale_bytes;    /* bytes of the scale pool (FP8 / INT8 only, else 0) */
     int64_t stride_block;    /* elements between consecutive physical blocks */
     int64_t stride_head;     /* elements between consecutive kv heads of a block */
     int64_t stride_slot;     /* elements between consecutive tokens of a block */
@@ -135,8 +137,13 @@ KV_API kv_status compute_slot_mapping(const int32_t* block_table, int32_t batch,
  *     a = max |x| (fp32),  scale = a / 448 (IEEE fp32 division),
  *     code = E4M3(x / scale) (IEEE division, round to nearest even,
  *            saturating to ±448),  and scale = 0, codes 0x00 when a == 0;
+ * INT8 pools ("k1-blog" KV 量化 and "大模型推理为何这么慢" KV Cache量化: 8-bit KV
+ * halves the cache like FP8): src_dtype F32 or BF16; for each row
+ *     a = max |x|,  scale = a / 127 (IEEE fp32 division),
+ *     code = clamp(round_to_nearest_even(x / scale), -127, 127),
+ *     and scale = 0, codes 0 when a == 0.
  *   scales : device fp32 scale pool [num_blocks][num_kv_heads][2][16] (K row
- *   scales, then V row scales), NULL for non-FP8 pools.  Rows must be finite.
+ *   scales, then V row scales), NULL for F32/BF16 pools.  Rows must be finite.
  * Two tokens given the same slot race (last writer unspecified).
  */
 KV_API kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool,
@@ -187,7 +194,7 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  *   out          : device [batch][num_q_heads][head_dim] in q_dtype
  *   q            : device [batch][num_q_heads][head_dim], q_dtype F32 or BF16
  *   k_pool/v_pool: device pools (layout above)
- *   scales       : device fp32 scale pool (layout above), non-NULL iff the pool is FP8
+ *   scales       : device fp32 scale pool (layout above), non-NULL iff the pool is FP8/INT8
  *   block_table  : device int32 [batch][max_blocks_per_seq]; entries past
  *                  ceil(L/16) are never read
  *   context_lens : device int32 [batch], each in [1, max_context_len]
@@ -223,7 +230,7 @@ KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, con
  * positions 0 .. L - Q + i (causal), with the softmax of paged_decode_attention.
  *   q, out : device [batch][Q][num_q_heads][head_dim] (q_dtype; out in q_dtype)
  * Everything else as paged_decode_attention (Q = 1 is exactly that call).
- * Supported shapes: bf16 or FP8 KV, head_dim 128, bf16 q, and
+ * Supported shapes: bf16, FP8 or INT8 KV, head_dim 128, bf16 q, and
  * (num_q_heads / num_kv_heads) * Q <= 16, else KV_ERR_UNSUPPORTED.  A context
  * length below Q is invalid (zeros, KV_DEVERR_BAD_CONTEXT_LEN).
  */

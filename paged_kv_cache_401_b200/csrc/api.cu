@@ -18,6 +18,7 @@ int32_t elem_bytes(int32_t dtype) {
         case KV_F32: return 4;
         case KV_BF16: return 2;
         case KV_FP8_E4M3: return 1;
+        case KV_INT8: return 1;
         default: return 0;
     }
 }
@@ -40,6 +41,9 @@ bool valid_pool(const kv_pool_desc* d) {
 }
 
 int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
+
+// Pools of codes with a per-(token, kv head) fp32 scale.
+bool quantized(int32_t dtype) { return dtype == KV_FP8_E4M3 || dtype == KV_INT8; }
 
 // The driver's tensor-map encoder, looked up once through the runtime (no libcuda link).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -100,7 +104,7 @@ kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_
     d.stride_head = static_cast<int64_t>(block_size) * head_dim;
     d.stride_block = d.stride_head * num_kv_heads;
     d.kv_bytes = static_cast<uint64_t>(d.stride_block) * num_blocks * d.elem_bytes;
-    d.scale_bytes = dtype == KV_FP8_E4M3
+    d.scale_bytes = quantized(dtype)
                         ? static_cast<uint64_t>(num_blocks) * num_kv_heads * 2u * block_size * 4u
                         : 0u;
     *out = d;
@@ -138,10 +142,10 @@ kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool
     const int64_t num_slots = static_cast<int64_t>(pool->num_blocks) * kBlockTokens;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
-    if (pool->dtype == KV_FP8_E4M3) {
+    if (quantized(pool->dtype)) {
         if (src_dtype != KV_F32 && src_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
         if (scales == nullptr) return KV_ERR_INVALID_ARGUMENT;
-        e = pkv::launch_cache_fp8(src_dtype, pool->head_dim, k_pool, v_pool, scales,
+        e = pkv::launch_cache_quant(pool->dtype, src_dtype, pool->head_dim, k_pool, v_pool, scales,
                                   k_new, v_new, slot_mapping, num_tokens, pool->num_kv_heads,
                                   num_slots, dev_error, s);
     } else {
@@ -162,7 +166,7 @@ kv_status paged_kv_copy_blocks(const kv_pool_desc* pool, void* k_pool, void* v_p
     if (k_pool == nullptr || v_pool == nullptr || copy_src == nullptr || copy_dst == nullptr)
         return KV_ERR_INVALID_ARGUMENT;
     if (!aligned16(k_pool) || !aligned16(v_pool)) return KV_ERR_INVALID_ARGUMENT;
-    const bool fp8 = pool->dtype == KV_FP8_E4M3;
+    const bool fp8 = quantized(pool->dtype);  // FP8 or INT8: a scale pool
     if (fp8 != (scales != nullptr) || (fp8 && !aligned16(scales))) return KV_ERR_INVALID_ARGUMENT;
     const int64_t block_bytes = pool->stride_block * pool->elem_bytes;
     const int64_t scale_bytes = fp8 ? static_cast<int64_t>(pool->num_kv_heads) * 2 * kBlockTokens * 4 : 0;
@@ -259,7 +263,7 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
         return KV_ERR_INVALID_ARGUMENT;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
         return KV_ERR_INVALID_ARGUMENT;
-    const bool fp8 = pool->dtype == KV_FP8_E4M3;
+    const bool fp8 = quantized(pool->dtype);  // FP8 or INT8: a scale pool
     if (fp8 != (scales != nullptr)) return KV_ERR_INVALID_ARGUMENT;
     if (fp8 && !aligned16(scales)) return KV_ERR_INVALID_ARGUMENT;
 

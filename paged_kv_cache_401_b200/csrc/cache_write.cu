@@ -64,16 +64,19 @@ __global__ void cache_copy_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restr
     }
 }
 
-// FP8 quantising write: one warp per (token, kv head, K|V) row of D elements.
-//   a = max|x|; scale = a / 448 (IEEE fp32 division); code = E4M3(x / scale)
-//   (IEEE division, RNE, saturating); a == 0 -> scale 0 and codes 0.
-template <int SRC_T, int D>
-__global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
-                                 float* __restrict__ scales,
-                                 const void* __restrict__ k_new, const void* __restrict__ v_new,
-                                 const int64_t* __restrict__ slots, int32_t num_tokens,
-                                 int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error) {
+// Quantising write: one warp per (token, kv head, K|V) row of D elements.
+//   FP8 : a = max|x|; scale = a / 448 (IEEE fp32 division); code = E4M3(x / scale)
+//         (IEEE division, RNE, saturating)
+//   INT8: a = max|x|; scale = a / 127; code = clamp(rint(x / scale), -127, 127)
+//   a == 0 -> scale 0 and codes 0.
+template <int KV_T, int SRC_T, int D>
+__global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
+                                   float* __restrict__ scales,
+                                   const void* __restrict__ k_new, const void* __restrict__ v_new,
+                                   const int64_t* __restrict__ slots, int32_t num_tokens,
+                                   int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error) {
     constexpr int kPer = D / 32;  // elements per lane (4 or 2)
+    constexpr float kMaxCode = KV_T == KV_INT8 ? 127.0f : 448.0f;
     pdl_wait();
     pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
@@ -106,12 +109,20 @@ __global__ void cache_fp8_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restri
     for (int e = 0; e < kPer; ++e) a = fmaxf(a, fabsf(x[e]));
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
-    const float s = __fdiv_rn(a, 448.0f);
+    const float s = __fdiv_rn(a, kMaxCode);
     uint32_t codes = 0;
 #pragma unroll
     for (int e = 0; e < kPer; e += 2) {
         uint32_t pair = 0;
-        if (a != 0.0f) pair = float2_to_e4m3x2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s));
+        if (a != 0.0f) {
+            if constexpr (KV_T == KV_INT8) {
+                const int c0 = max(-127, min(127, __float2int_rn(__fdiv_rn(x[e], s))));
+                const int c1 = max(-127, min(127, __float2int_rn(__fdiv_rn(x[e + 1], s))));
+                pair = (static_cast<uint32_t>(c0) & 0xffu) | ((static_cast<uint32_t>(c1) & 0xffu) << 8);
+            } else {
+                pair = float2_to_e4m3x2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s));
+            }
+        }
         codes |= pair << (8 * e);
     }
     const int64_t blk = slot / kBlockTokens, off = slot % kBlockTokens;
@@ -195,11 +206,11 @@ cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, con
                       slots, num_tokens, num_kv_heads, row_bytes, num_slots, dev_error);
 }
 
-cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, void* v_pool,
-                             float* scales, const void* k_new,
-                             const void* v_new, const int64_t* slots, int32_t num_tokens,
-                             int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
-                             cudaStream_t stream) {
+cudaError_t launch_cache_quant(int32_t kv_dtype, int32_t src_dtype, int32_t head_dim,
+                               void* k_pool, void* v_pool, float* scales, const void* k_new,
+                               const void* v_new, const int64_t* slots, int32_t num_tokens,
+                               int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
+                               cudaStream_t stream) {
     const int threads = 256;
     const int64_t rows = 2ll * num_tokens * num_kv_heads;
     const int64_t blocks = (rows * 32 + threads - 1) / threads;
@@ -207,13 +218,20 @@ cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, 
     auto* vp = static_cast<uint8_t*>(v_pool);
     auto go = [&](auto kernel) {
         return launch_pdl(kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream,
-                          kp, vp, scales, k_new, v_new, slots, num_tokens,
-                          num_kv_heads, num_slots, dev_error);
+                          kp, vp, scales, k_new, v_new, slots, num_tokens, num_kv_heads,
+                          num_slots, dev_error);
     };
-    if (src_dtype == KV_F32 && head_dim == 128) return go(cache_fp8_kernel<KV_F32, 128>);
-    if (src_dtype == KV_F32 && head_dim == 64) return go(cache_fp8_kernel<KV_F32, 64>);
-    if (src_dtype == KV_BF16 && head_dim == 128) return go(cache_fp8_kernel<KV_BF16, 128>);
-    return go(cache_fp8_kernel<KV_BF16, 64>);
+    const bool f32 = src_dtype == KV_F32, d128 = head_dim == 128;
+    if (kv_dtype == KV_INT8) {
+        if (f32) return d128 ? go(cache_quant_kernel<KV_INT8, KV_F32, 128>)
+                             : go(cache_quant_kernel<KV_INT8, KV_F32, 64>);
+        return d128 ? go(cache_quant_kernel<KV_INT8, KV_BF16, 128>)
+                    : go(cache_quant_kernel<KV_INT8, KV_BF16, 64>);
+    }
+    if (f32) return d128 ? go(cache_quant_kernel<KV_FP8_E4M3, KV_F32, 128>)
+                         : go(cache_quant_kernel<KV_FP8_E4M3, KV_F32, 64>);
+    return d128 ? go(cache_quant_kernel<KV_FP8_E4M3, KV_BF16, 128>)
+                : go(cache_quant_kernel<KV_FP8_E4M3, KV_BF16, 64>);
 }
 
 }  // namespace pkv

@@ -114,6 +114,17 @@ __device__ __forceinline__ float2 e4m3x2_to_float2(uint32_t w16) {
     return __half22float2(h);
 }
 
+// Two signed 8-bit codes (low 16 bits of w16, low byte first) -> two floats,
+// exact.  Each code c is flipped to the biased byte c + 128, placed in the
+// mantissa of 2^23 (bit pattern 0x4B0000xx = 2^23 + c + 128) and the bias
+// subtracted.
+__device__ __forceinline__ float2 i8x2_to_float2(uint32_t w16) {
+    const uint32_t u = w16 ^ 0x8080u;
+    const float bias = 8388608.0f + 128.0f;
+    return make_float2(__uint_as_float(__byte_perm(u, 0x4B000000u, 0x7650)) - bias,
+                       __uint_as_float(__byte_perm(u, 0x4B000000u, 0x7651)) - bias);
+}
+
 // Two fp32 -> two E4M3 codes (round to nearest even, finite overflow saturates
 // to +-448), low byte = first argument.
 __device__ __forceinline__ uint32_t float2_to_e4m3x2(float lo, float hi) {

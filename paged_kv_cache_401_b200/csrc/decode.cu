@@ -23,19 +23,19 @@
 //  * a CTA is one producer warp and four consumer warps; by default the grid
 //    is the number of CTAs resident on the GPU (persistent), so the tile
 //    stream never stalls between work items;
-//  * FP8 row scales of a tile (16 K then 16 V) are one 128-byte line;
+//  * FP8 / INT8 row scales of a tile (16 K then 16 V) are one 128-byte line;
 //  * producer lane w walks consumer warp w's range and stages each (block,
 //    kv head) K and V tile -- one contiguous 16-row span of the pool -- into
 //    that warp's stages of a shared-memory ring (stage s feeds warp s % 4)
 //    through the TMA engine (no multicast), completing on mbarriers; block
 //    ids are fetched 4 tiles ahead, and no warp's refill waits behind another;
 //  * the per-tile arithmetic is a policy:
-//      MmaMath  (bf16 or FP8 KV, head_dim 128, bf16 q): tiles land in shared
+//      MmaMath  (bf16, FP8 or INT8 KV, head_dim 128, bf16 q): tiles land in shared
 //               memory 128-byte swizzled by 2-D TMA tensor copies; the group's
 //               scores S = Q.K^T come from mma.m16n8k16 (query heads as rows,
 //               fp32 accumulate), the softmax runs on the accumulator
 //               fragments, and P feeds O^T = V^T.P^T straight from registers;
-//               FP8 codes are widened to f16 in registers (exact);
+//               8-bit codes are widened to f16 in registers (exact);
 //      SimtMath (every other shape and fp32): 1-D bulk copies; q.K with
 //               packed fp32x2 FMAs and a shuffle reduce-scatter, P.V with each
 //               lane owning D/32 output columns, all in fp32;
@@ -59,6 +59,21 @@ template <>
 struct KvElem<KV_FP8_E4M3> {
     static constexpr int kBytes = 1;
 };
+template <>
+struct KvElem<KV_INT8> {
+    static constexpr int kBytes = 1;
+};
+
+// 8-bit code pools carry a per-(token, kv head) fp32 scale line.
+template <int KV_T>
+inline constexpr bool kQuantized = KV_T == KV_FP8_E4M3 || KV_T == KV_INT8;
+
+// Two 8-bit codes (low 16 bits) -> two floats (code values, before the row scale).
+template <int KV_T>
+__device__ __forceinline__ float2 codes2_to_float2(uint32_t w16) {
+    if constexpr (KV_T == KV_INT8) return i8x2_to_float2(w16);
+    else return e4m3x2_to_float2(w16);
+}
 
 // ---- small vector helpers --------------------------------------------------------
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
@@ -78,8 +93,8 @@ __device__ __forceinline__ void decode_chunk(const uint4 c, float2* out) {
         const uint32_t w[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            out[2 * i] = e4m3x2_to_float2(w[i] & 0xffffu);
-            out[2 * i + 1] = e4m3x2_to_float2(w[i] >> 16);
+            out[2 * i] = codes2_to_float2<KV_T>(w[i] & 0xffffu);
+            out[2 * i + 1] = codes2_to_float2<KV_T>(w[i] >> 16);
         }
     }
 }
@@ -107,10 +122,10 @@ __device__ __forceinline__ void load_v(const uint8_t* p, float2* out) {
     } else {
         if constexpr (kBytes == 4) {
             const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
-            out[0] = e4m3x2_to_float2(w & 0xffffu);
-            out[1] = e4m3x2_to_float2(w >> 16);
+            out[0] = codes2_to_float2<KV_T>(w & 0xffffu);
+            out[1] = codes2_to_float2<KV_T>(w >> 16);
         } else {
-            out[0] = e4m3x2_to_float2(*reinterpret_cast<const uint16_t*>(p));
+            out[0] = codes2_to_float2<KV_T>(*reinterpret_cast<const uint16_t*>(p));
         }
     }
 }
@@ -219,6 +234,34 @@ __device__ __forceinline__ void e4m3x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint
         "cvt.rn.f16x2.e4m3x2 %0, a;\n\tcvt.rn.f16x2.e4m3x2 %1, b;\n\t}"
         : "=r"(lo), "=r"(hi)
         : "r"(w));
+}
+
+// Four signed 8-bit codes -> two f16x2, exact.  Each code c becomes the biased
+// byte c + 128 in the low mantissa byte of f16 1024 (0x64xx = 1024 + c + 128),
+// then 1152 is subtracted.  SEL_LO / SEL_HI pick which two bytes of w go to the
+// low and high halves of lo and hi (byte_perm selectors over {w, 0x64646464}).
+template <uint32_t SEL_LO, uint32_t SEL_HI>
+__device__ __forceinline__ void i8x4_to_f16x2x2(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const uint32_t u = w ^ 0x80808080u;
+    const uint32_t a = __byte_perm(u, 0x64646464u, SEL_LO);
+    const uint32_t b = __byte_perm(u, 0x64646464u, SEL_HI);
+    asm("add.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0xE480E480u));  // -1152
+    asm("add.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0xE480E480u));
+}
+
+// Four 8-bit K codes (one lane's ldmatrix word) -> f16x2 {codes 0,1}, {codes 2,3}.
+template <int KV_T>
+__device__ __forceinline__ void widen_k4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    if constexpr (KV_T == KV_INT8) i8x4_to_f16x2x2<0x4140u, 0x4342u>(w, lo, hi);
+    else e4m3x4_to_f16x2x2(w, lo, hi);
+}
+
+// Four 8-bit V codes from a transposed ldmatrix word, bytes [t0 d, t0 d+1,
+// t1 d, t1 d+1] -> f16x2 {t0 d, t1 d} and {t0 d+1, t1 d+1}.
+template <int KV_T>
+__device__ __forceinline__ void widen_v4(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    if constexpr (KV_T == KV_INT8) i8x4_to_f16x2x2<0x4240u, 0x4341u>(w, lo, hi);
+    else e4m3x4_to_f16x2x2(__byte_perm(w, 0u, 0x3120), lo, hi);
 }
 
 // 2-D TMA tile load (no multicast) completing on an mbarrier; x is the
@@ -341,7 +384,7 @@ struct SimtMath {
     using OutT = typename QType<Q_T>::T;
     static constexpr int kElem = KvElem<KV_T>::kBytes;
     static constexpr int kTileBytes = kBlockTokens * D * kElem;              // K or V tile
-    static constexpr int kScaleBytes = (KV_T == KV_FP8_E4M3) ? 2 * kBlockTokens * 4 : 0;  // K|V
+    static constexpr int kScaleBytes = kQuantized<KV_T> ? 2 * kBlockTokens * 4 : 0;  // K|V
     static constexpr int kStageBytes = 2 * kTileBytes + kScaleBytes;
     static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
     static constexpr int kRingAlign = 128;
@@ -366,14 +409,14 @@ struct SimtMath {
     static_assert(kStageBytes % 16 == 0, "bulk copies need 16-B alignment");
     static_assert(kQPL % 2 == 0 && kDPL % 2 == 0, "pairs for fp32x2 FMA");
 
-    // ---- producer side: one stage = K tile, V tile (+ FP8 row scales), 1-D bulk copies
+    // ---- producer side: one stage = K tile, V tile (+ 8-bit row scales), 1-D bulk copies
     __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
                                  const TmaMaps&) {
         const int64_t off = tile * kTileBytes;
         mbar_arrive_expect_tx(bar, kStageBytes);
         bulk_copy_g2s(st, p.k_pool + off, kTileBytes, bar);
         bulk_copy_g2s(st + kTileBytes, p.v_pool + off, kTileBytes, bar);
-        if constexpr (KV_T == KV_FP8_E4M3)
+        if constexpr (kQuantized<KV_T>)
             bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
     }
 
@@ -456,7 +499,7 @@ struct SimtMath {
             const int idx = (kNV >= kLPR) ? c * kVPL + v : c / (kLPR / kNV);
             const int t = r0 + kRPI * (idx / G);
             float sc = acc[v];
-            if constexpr (KV_T == KV_FP8_E4M3) sc *= ksc[t];
+            if constexpr (kQuantized<KV_T>) sc *= ksc[t];
             s_buf[t * G + (idx % G)] = sc;
         }
         __syncwarp();
@@ -482,7 +525,7 @@ struct SimtMath {
             const float pr = exp2f(sv[i] - m_new);
             l_run += pr;
             float pv = pr;
-            if constexpr (KV_T == KV_FP8_E4M3) pv *= vsc[t];
+            if constexpr (kQuantized<KV_T>) pv *= vsc[t];
             if (lane < kSMLanes) p_buf[t * G + sm_g] = make_float2(pv, pv);
         }
         m_run = m_new;
@@ -554,7 +597,7 @@ struct SimtMath {
 };
 
 // ======================================================================================
-// MmaMath: tensor-core tile arithmetic for bf16 or FP8 KV, head_dim 128, bf16 q.
+// MmaMath: tensor-core tile arithmetic for bf16, FP8 or INT8 KV, head_dim 128, bf16 q.
 //
 // A tile is 16 tokens x 128 dims.  K and V land in shared memory as [16 rows]
 // x [128-byte] boxes written by TMA with the 128-byte swizzle (16-byte chunk
@@ -572,12 +615,12 @@ struct SimtMath {
 //   O^T += V^T.P^T   m16n8k16, rows = 16 head dims, columns = 8 query rows per
 //                    row set; the P fragment of the score accumulators is
 //                    exactly the B operand, so P never leaves registers.
-// bf16 KV: bf16 MMAs, P rounded to bf16.  FP8 KV: codes widened to f16 in
+// bf16 KV: bf16 MMAs, P rounded to bf16.  FP8 / INT8 KV: codes widened to f16 in
 // registers (exact), f16 MMAs with q rounded to f16 and P (times the V row
 // scale) rounded to f16; the K row scale multiplies the scores.  Element
 // orders inside a k-step are permuted consistently between the two operands
 // (a dot product does not depend on the order of its terms), which is what
-// lets FP8 rows be read with 16-bit ldmatrix.  QM: kSingle = one query token
+// lets 8-bit rows be read with 16-bit ldmatrix.  QM: kSingle = one query token
 // (the decode: no causal bookkeeping), kNarrow = up to 8 query rows, kWide = up
 // to 16 (two row sets).
 // ======================================================================================
@@ -587,14 +630,14 @@ template <int KV_T, int G, int QM>
 struct MmaMath {
     static constexpr bool WIDE = QM == kWide;
     static constexpr bool SINGLE = QM == kSingle;
-    static_assert(KV_T == KV_BF16 || KV_T == KV_FP8_E4M3, "bf16 or FP8 KV");
+    static_assert(KV_T == KV_BF16 || kQuantized<KV_T>, "bf16, FP8 or INT8 KV");
     static_assert(G <= 8, "a row set holds 8 query rows");
     using OutT = uint16_t;                                        // bf16 output
-    static constexpr bool kF16 = KV_T == KV_FP8_E4M3;
+    static constexpr bool kF16 = kQuantized<KV_T>;              // 8-bit codes widened to f16
     static constexpr int D = 128;
     static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
     static constexpr int kElem = KvElem<KV_T>::kBytes;
-    static constexpr int kRowBytes = D * kElem;                   // 256 (bf16) / 128 (fp8)
+    static constexpr int kRowBytes = D * kElem;                   // 256 (bf16) / 128 (8-bit)
     static constexpr int kBoxCols = 128 / kElem;                  // elements per 128-byte box row
     static constexpr int kBoxes = kRowBytes / 128;
     static constexpr int kBoxBytes = kBlockTokens * 128;
@@ -606,7 +649,7 @@ struct MmaMath {
     static constexpr int kWarpScratch = 0;
     static constexpr int kMinBlocks = WIDE ? 2 : 3;
 
-    // ---- producer side: TMA boxes of K and V (+ the FP8 scale line by bulk copy)
+    // ---- producer side: TMA boxes of K and V (+ the scale line of 8-bit codes by bulk copy)
     __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
                                  const TmaMaps& maps) {
         const int32_t row = static_cast<int32_t>(tile * kBlockTokens);
@@ -625,7 +668,7 @@ struct MmaMath {
         return (chunk >> 3) * kBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
     }
 
-    // head-dim of row r (0..15) of output m-tile mi: FP8 tiles interleave even/odd dims
+    // head-dim of row r (0..15) of output m-tile mi: 8-bit tiles interleave even/odd dims
     __device__ static __forceinline__ int32_t dim_of(int32_t mi, int32_t r) {
         if constexpr (kF16) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
         return 16 * mi + r;
@@ -663,7 +706,7 @@ struct MmaMath {
                     qa[k][ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
                     qa[k][ks][1] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 8 + 2 * tig);
                 } else {
-                    // FP8 rows are read 4 codes per lane: k 2tig+{0,1} -> dim 16ks+4tig+{0,1},
+                    // 8-bit rows are read 4 codes per lane: k 2tig+{0,1} -> dim 16ks+4tig+{0,1},
                     // k 8+2tig+{0,1} -> dim 16ks+4tig+{2,3}
                     const uint2 w = *reinterpret_cast<const uint2*>(q + 16 * ks + 4 * tig);
                     qa[k][ks][0] = pack2<true>(__uint_as_float(w.x << 16),
@@ -719,8 +762,8 @@ struct MmaMath {
                 for (int h = 0; h < 2; ++h) {
                     const int ks = 2 * kq + h;
                     uint32_t b0, b1, b2, b3;
-                    e4m3x4_to_f16x2x2(w[h], b0, b1);
-                    e4m3x4_to_f16x2x2(w[2 + h], b2, b3);
+                    widen_k4<KV_T>(w[h], b0, b1);
+                    widen_k4<KV_T>(w[2 + h], b2, b3);
                     mma_16816<true>(s[0], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b0, b1);
                     mma_16816<true>(s[1], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b2, b3);
                 }
@@ -836,8 +879,8 @@ struct MmaMath {
                     // bytes of w: [t0 d2g, t0 d2g+1, t1 d2g, t1 d2g+1] -> [t0 d2g, t1 d2g,
                     // t0 d2g+1, t1 d2g+1]; row gid <- even dim, row gid + 8 <- odd dim
                     uint32_t lo0, hi0, lo1, hi1;
-                    e4m3x4_to_f16x2x2(__byte_perm(w[2 * h], 0u, 0x3120), lo0, hi0);
-                    e4m3x4_to_f16x2x2(__byte_perm(w[2 * h + 1], 0u, 0x3120), lo1, hi1);
+                    widen_v4<KV_T>(w[2 * h], lo0, hi0);
+                    widen_v4<KV_T>(w[2 * h + 1], lo1, hi1);
                     if (partial) {
                         lo0 &= mask_a;
                         hi0 &= mask_a;
@@ -1250,19 +1293,25 @@ static cudaError_t dispatch_q(const DecodeParams& p, const TmaMaps& maps, int32_
 }
 
 bool decode_uses_tensor_cores(int32_t kv_dtype, int32_t q_dtype, int32_t head_dim) {
-    return (kv_dtype == KV_BF16 || kv_dtype == KV_FP8_E4M3) && q_dtype == KV_BF16 &&
+    return (kv_dtype == KV_BF16 || kv_dtype == KV_FP8_E4M3 || kv_dtype == KV_INT8) &&
+           q_dtype == KV_BF16 &&
            head_dim == 128;
 }
 
 cudaError_t launch_paged_decode(const DecodeParams& p, const TmaMaps& maps, int32_t kv_dtype,
                                 int32_t q_dtype, int32_t head_dim, int32_t group,
                                 cudaStream_t stream) {
-    if (decode_uses_tensor_cores(kv_dtype, q_dtype, head_dim))
-        return kv_dtype == KV_BF16 ? dispatch_mma<KV_BF16>(p, maps, group, stream)
-                                   : dispatch_mma<KV_FP8_E4M3>(p, maps, group, stream);
+    if (decode_uses_tensor_cores(kv_dtype, q_dtype, head_dim)) {
+        switch (kv_dtype) {
+            case KV_BF16: return dispatch_mma<KV_BF16>(p, maps, group, stream);
+            case KV_INT8: return dispatch_mma<KV_INT8>(p, maps, group, stream);
+            default: return dispatch_mma<KV_FP8_E4M3>(p, maps, group, stream);
+        }
+    }
     switch (kv_dtype) {
         case KV_F32: return dispatch_q<KV_F32>(p, maps, q_dtype, head_dim, group, stream);
         case KV_BF16: return dispatch_q<KV_BF16>(p, maps, q_dtype, head_dim, group, stream);
+        case KV_INT8: return dispatch_q<KV_INT8>(p, maps, q_dtype, head_dim, group, stream);
         default: return dispatch_q<KV_FP8_E4M3>(p, maps, q_dtype, head_dim, group, stream);
     }
 }

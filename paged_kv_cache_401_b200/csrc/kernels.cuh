@@ -36,11 +36,11 @@ cudaError_t launch_cache_copy(void* k_pool, void* v_pool, const void* k_new, con
                               int32_t row_bytes, int64_t num_slots, int32_t num_sms,
                               int32_t* dev_error, cudaStream_t stream);
 
-cudaError_t launch_cache_fp8(int32_t src_dtype, int32_t head_dim, void* k_pool, void* v_pool,
-                             float* scales, const void* k_new,
-                             const void* v_new, const int64_t* slots, int32_t num_tokens,
-                             int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
-                             cudaStream_t stream);
+cudaError_t launch_cache_quant(int32_t kv_dtype, int32_t src_dtype, int32_t head_dim,
+                               void* k_pool, void* v_pool, float* scales, const void* k_new,
+                               const void* v_new, const int64_t* slots, int32_t num_tokens,
+                               int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error,
+                               cudaStream_t stream);
 
 cudaError_t launch_copy_blocks(void* k_pool, void* v_pool, float* scales, const int32_t* src,
                                const int32_t* dst, int32_t num_copies, int64_t block_bytes,
@@ -53,7 +53,7 @@ struct DecodeParams {
     const void* q;                // [B][Hq][D]
     const uint8_t* k_pool;        // [NB][Hkv][16][D]
     const uint8_t* v_pool;
-    const float* scales;          // [NB][Hkv][2][16]: K then V row scales (FP8 only)
+    const float* scales;          // [NB][Hkv][2][16]: K then V row scales (FP8 / INT8)
     const int32_t* block_table;   // [B][max_blocks]
     const int32_t* context_lens;  // [B]
     int32_t* ws_seq_start;        // [B + 1]: first tile of each sequence, total tiles at [B]

@@ -4,7 +4,7 @@ and evaluate the oracle on the same inputs.
 GPU side: the pool is filled by the library's own slot computation and cache
 write (history tokens), then a step appends each sequence's new token and
 decodes.  Oracle side: the contiguous per-sequence K/V the generator drew
-(FP8: quantised by the oracle's own encoder), never the GPU's pool.
+(FP8 / INT8: quantised by the oracle's own encoder), never the GPU's pool.
 """
 from __future__ import annotations
 
@@ -21,6 +21,7 @@ TOL = {  # max-abs, max-rel (relative to the output's max magnitude)
     "f32": (1e-4, 1e-4),
     "bf16": (2e-2, 1e-2),
     "fp8": (5e-2, None),
+    "int8": (5e-2, None),
 }
 
 
@@ -77,20 +78,20 @@ def oracle_out(inp: Inputs, seqs=None) -> tuple[np.ndarray, np.ndarray]:
     seqs = np.arange(inp.q.shape[0]) if seqs is None else np.asarray(seqs)
     q = storage_view(inp.q)[seqs]
     lens = inp.context_lens[seqs]
-    if spec.kv_dtype == "fp8":
+    if spec.kv_dtype in oracle.QUANTIZED:
         ks, vs, kc, vc, offs, o = [], [], [], [], [], 0
         for s in seqs:
             a, n = int(inp.seq_offsets[s]), int(inp.context_lens[s])
             kf = inp.k[a:a + n].float().numpy()
             vf = inp.v[a:a + n].float().numpy()
-            c1, s1 = oracle.quantize_rows(kf)
-            c2, s2 = oracle.quantize_rows(vf)
+            c1, s1 = oracle.quantize_rows(kf, spec.kv_dtype)
+            c2, s2 = oracle.quantize_rows(vf, spec.kv_dtype)
             kc.append(c1), ks.append(s1), vc.append(c2), vs.append(s2)
             offs.append(o)
             o += n
         out = oracle.decode_attention(q, np.concatenate(kc), np.concatenate(vc),
                                       np.array(offs, np.int64), lens, spec.scale,
-                                      spec.num_kv_heads, "fp8", spec.q_dtype,
+                                      spec.num_kv_heads, spec.kv_dtype, spec.q_dtype,
                                       k_scale=np.concatenate(ks), v_scale=np.concatenate(vs))
     else:
         out = oracle.decode_attention(q, storage_view(inp.k), storage_view(inp.v),

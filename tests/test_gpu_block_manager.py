@@ -24,14 +24,16 @@ def _bits(t):
     return t.numpy()
 
 
-@pytest.mark.parametrize("kv", ["bf16", "f32", "fp8"])
+@pytest.mark.parametrize("kv", ["bf16", "f32", "fp8", "int8"])
 def test_copy_blocks_bitexact(kv):
     nb, hkv, d = 24, 2, 64 if kv == "f32" else 128
     cache = PagedKVCache(nb, hkv, d, kv, DEV)
     g = torch.Generator(device="cpu").manual_seed(3)
-    if kv == "fp8":
-        cache.k_pool.copy_(torch.randint(0, 255, cache.k_pool.shape, generator=g, dtype=torch.uint8))
-        cache.v_pool.copy_(torch.randint(0, 255, cache.v_pool.shape, generator=g, dtype=torch.uint8))
+    if kv in ("fp8", "int8"):
+        dt = cache.k_pool.dtype
+        lo, hi = (0, 255) if kv == "fp8" else (-127, 128)
+        cache.k_pool.copy_(torch.randint(lo, hi, cache.k_pool.shape, generator=g, dtype=dt))
+        cache.v_pool.copy_(torch.randint(lo, hi, cache.v_pool.shape, generator=g, dtype=dt))
         cache.scales.copy_(torch.rand(cache.scales.shape, generator=g))
     else:
         for t in (cache.k_pool, cache.v_pool):
@@ -50,7 +52,7 @@ def test_copy_blocks_bitexact(kv):
     assert cache.errors() == 0
 
 
-@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8"])
 def test_fork_copy_on_write_decode(kv):
     hq, hkv, d, nb, hist = 8, 2, 128, 32, 40
     m = pk.BlockManager(nb, 4, 16)
@@ -85,11 +87,11 @@ def test_fork_copy_on_write_decode(kv):
     k_seq = torch.cat([k_hist, k_new[:1], k_hist, k_new[1:]])
     v_seq = torch.cat([v_hist, v_new[:1], v_hist, v_new[1:]])
     offs = np.array([0, hist + 1], dtype=np.int64)
-    if kv == "fp8":
-        kc, ks = oracle.quantize_rows(k_seq.float().numpy())
-        vc, vs = oracle.quantize_rows(v_seq.float().numpy())
+    if kv in ("fp8", "int8"):
+        kc, ks = oracle.quantize_rows(k_seq.float().numpy(), kv)
+        vc, vs = oracle.quantize_rows(v_seq.float().numpy(), kv)
         ref = oracle.decode_attention(storage_view(q), kc, vc, offs, lens, 1 / math.sqrt(d), hkv,
-                                      "fp8", "bf16", k_scale=ks, v_scale=vs)
+                                      kv, "bf16", k_scale=ks, v_scale=vs)
         tol = 5e-2
     else:
         ref = oracle.decode_attention(storage_view(q), storage_view(k_seq), storage_view(v_seq),

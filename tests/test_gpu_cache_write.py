@@ -75,9 +75,10 @@ def _fp8_rows(rng, T, Hkv, D):
     return x
 
 
+@pytest.mark.parametrize("kind", ["fp8", "int8"])
 @pytest.mark.parametrize("src", ["f32", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
-def test_cache_fp8_bitexact(src, D):
+def test_cache_quant_bitexact(kind, src, D):
     rng = np.random.default_rng(3 + D)
     NB, Hkv, T = 50, 2, 400
     x_k = _fp8_rows(rng, T, Hkv, D)
@@ -87,13 +88,16 @@ def test_cache_fp8_bitexact(src, D):
     v = torch.from_numpy(x_v).to(tdt)
     slots = rng.permutation(NB * 16)[:T].astype(np.int64)
     slots[9] = -1
-    cache = PagedKVCache(NB, Hkv, D, "fp8", DEV, poison=True)
+    if kind == "int8":
+        x_k[6, 0, :] = np.arange(D) - D / 2 + 0.5   # exact half-integer quotients: ties
+        x_k[6, 0, 0] = 127.0
+    cache = PagedKVCache(NB, Hkv, D, kind, DEV, poison=True)
     pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, cache.scales, k.to(DEV),
                          v.to(DEV), torch.from_numpy(slots).to(DEV), cache.dev_error)
     want_scales = np.full(tuple(cache.scales.shape), np.nan, np.float32)
     for which, (pool, src_t) in enumerate(((cache.k_pool, k), (cache.v_pool, v))):
-        codes, scales = oracle.quantize_rows(src_t.float().numpy())
-        want_codes = oracle.scatter_to_pool(np.full(tuple(pool.shape), 0x7F, np.uint8), codes,
+        codes, scales = oracle.quantize_rows(src_t.float().numpy(), kind)
+        want_codes = oracle.scatter_to_pool(np.full(tuple(pool.shape), 0x7F, codes.dtype), codes,
                                             slots)
         want_scales = oracle.scatter_scales_to_pool(want_scales, scales, slots, which)
         assert (pool.cpu().numpy() == want_codes).all()

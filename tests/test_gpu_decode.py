@@ -1,7 +1,8 @@
 """GPU: paged decode attention against the double-precision oracle.
 
 Tolerances (max-abs, and max-abs relative to the output's largest magnitude):
-bf16 KV 2e-2 / 1e-2 and FP8 KV 5e-2 (the stated pass criteria); fp32 KV
+bf16 KV 2e-2 / 1e-2 and FP8 KV 5e-2 (the stated pass criteria), INT8 KV as
+FP8 (the same f16 tensor-core arithmetic on exactly widened codes); fp32 KV
 1e-4 / 1e-4 (fp32 accumulation over <= a few thousand terms of |x| ~ 1).
 """
 import math
@@ -28,7 +29,8 @@ LENS = [1, 2, 15, 16, 17, 63, 64, 65, 300, 1023, 1025]
 
 
 @pytest.mark.parametrize("kv,q", [("bf16", "bf16"), ("f32", "f32"), ("fp8", "bf16"),
-                                  ("bf16", "f32"), ("f32", "bf16"), ("fp8", "f32")])
+                                  ("bf16", "f32"), ("f32", "bf16"), ("fp8", "f32"),
+                                  ("int8", "bf16"), ("int8", "f32")])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_parity_shapes(kv, q, D, G):
@@ -192,13 +194,14 @@ def test_long_full_size_sampled():
     _sampled("long", [0, 3])
 
 
-def test_fp8_full_size_sampled_and_codes_bitexact():
+@pytest.mark.parametrize("kind", ["fp8", "int8"])
+def test_quantized_full_size_sampled_and_codes_bitexact(kind):
     import oracle
-    stats, inp, st = _sampled("fp8", [0, 40])
+    stats, inp, st = _sampled(kind, [0, 40])
     # codes and scales written by the GPU for sequence 40 match the oracle's encoder
     s = 40
     a, n = int(inp.seq_offsets[s]), int(inp.context_lens[s])
-    codes, scales = oracle.quantize_rows(inp.k[a:a + n].float().numpy())
+    codes, scales = oracle.quantize_rows(inp.k[a:a + n].float().numpy(), kind)
     kp = st.cache.k_pool.cpu().numpy()
     ks = st.cache.scales.cpu().numpy()[:, :, 0, :]   # K row scales
     for pos in range(0, n, 97):

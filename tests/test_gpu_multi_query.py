@@ -1,6 +1,6 @@
 """GPU: multi-query paged attention (Q causal query tokens per sequence) against
 the oracle's causal multi-query attention.  Tolerances as for decode: bf16 KV
-max-abs 2e-2 / max-rel 1e-2, FP8 KV max-abs 5e-2."""
+max-abs 2e-2 / max-rel 1e-2, FP8 and INT8 KV max-abs 5e-2."""
 import math
 
 import numpy as np
@@ -24,11 +24,11 @@ def _spec(kv, G, lens, idx=70, hkv=2):
 def _oracle(inp, qm):
     spec = inp.spec
     q = storage_view(qm)
-    if spec.kv_dtype == "fp8":
-        kc, ks = oracle.quantize_rows(inp.k.float().numpy())
-        vc, vs = oracle.quantize_rows(inp.v.float().numpy())
+    if spec.kv_dtype in oracle.QUANTIZED:
+        kc, ks = oracle.quantize_rows(inp.k.float().numpy(), spec.kv_dtype)
+        vc, vs = oracle.quantize_rows(inp.v.float().numpy(), spec.kv_dtype)
         return oracle.multi_query_attention(q, kc, vc, inp.seq_offsets, inp.context_lens,
-                                           spec.scale, spec.num_kv_heads, "fp8", "bf16",
+                                           spec.scale, spec.num_kv_heads, spec.kv_dtype, "bf16",
                                            k_scale=ks, v_scale=vs)
     return oracle.multi_query_attention(q, storage_view(inp.k), storage_view(inp.v),
                                         inp.seq_offsets, inp.context_lens, spec.scale,
@@ -44,7 +44,7 @@ def _full_cache(inp):
 CASES = [(g, q) for g in (1, 2, 4, 8) for q in (2, 3, 4, 5, 8, 16) if g * q <= 16]
 
 
-@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8"])
 @pytest.mark.parametrize("G,Q", CASES)
 def test_multi_query_parity(kv, G, Q):
     lens = [Q, Q + 1, 17, 33, 100, 1025, 2048 + 3]

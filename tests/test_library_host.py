@@ -57,6 +57,8 @@ def test_pool_geometry_llama_shape():
     assert d.scale_bytes == 0 and d.elem_bytes == 2
     f = pk.kv_pool_create(100, 16, 8, 64, pk.KV_FP8_E4M3)
     assert f.kv_bytes == 100 * 8 * 16 * 64 and f.scale_bytes == 100 * 8 * 2 * 16 * 4
+    i = pk.kv_pool_create(100, 16, 8, 64, pk.KV_INT8)
+    assert (i.kv_bytes, i.scale_bytes, i.elem_bytes) == (f.kv_bytes, f.scale_bytes, 1)
 
 
 @pytest.mark.parametrize("args,status", [
@@ -111,6 +113,7 @@ def _call_decode(desc, **kw):
     (dict(num_q_heads=30), pk.KV_ERR_INVALID_ARGUMENT),            # not a multiple of Hkv
     (dict(num_q_heads=128), pk.KV_ERR_UNSUPPORTED),                # group 16
     (dict(q_dtype=pk.KV_FP8_E4M3), pk.KV_ERR_UNSUPPORTED),
+    (dict(q_dtype=pk.KV_INT8), pk.KV_ERR_UNSUPPORTED),
     (dict(max_context_len=4097), pk.KV_ERR_INVALID_ARGUMENT),      # beyond the table
     (dict(max_context_len=0), pk.KV_ERR_INVALID_ARGUMENT),
     (dict(partition=500), pk.KV_ERR_INVALID_ARGUMENT),             # not a multiple of 16
@@ -128,8 +131,9 @@ def test_decode_host_validation(kw, status):
     assert _call_decode(d, **kw) == status
 
 
-def test_decode_fp8_pool_requires_scales():
-    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_FP8_E4M3)
+@pytest.mark.parametrize("dtype", [pk.KV_FP8_E4M3, pk.KV_INT8])
+def test_decode_quantized_pool_requires_scales(dtype):
+    d = pk.kv_pool_create(8192, 16, 8, 128, dtype)
     assert _call_decode(d) == pk.KV_ERR_INVALID_ARGUMENT
     assert _call_decode(d, scales=(6 << 20) + 4) == pk.KV_ERR_INVALID_ARGUMENT  # misaligned
 
@@ -165,6 +169,9 @@ def test_cache_write_host_validation():
     assert call(d, n=-1) == pk.KV_ERR_INVALID_ARGUMENT
     assert call(f) == pk.KV_ERR_INVALID_ARGUMENT                      # fp8 needs scales
     assert call(f, sc=6 << 20, src=pk.KV_FP8_E4M3) == pk.KV_ERR_UNSUPPORTED
+    i = pk.kv_pool_create(64, 16, 8, 128, pk.KV_INT8)
+    assert call(i) == pk.KV_ERR_INVALID_ARGUMENT                      # int8 needs scales
+    assert call(i, sc=6 << 20, src=pk.KV_INT8) == pk.KV_ERR_UNSUPPORTED
 
 
 def test_slot_mapping_host_validation():

@@ -1,5 +1,6 @@
 """CPU: the seeded generators produce the workloads' stated shapes and structure."""
 import numpy as np
+import pytest
 import torch
 
 from workloads import POISON_BLOCK, WORKLOADS, make_inputs
@@ -67,7 +68,8 @@ def test_long_has_outlier_channels():
     assert float(inp.v.float().pow(2).mean().sqrt()) < 1.1
 
 
-def test_fp8_lengths_in_range():
-    inp = make_inputs("fp8", batch=16)
+@pytest.mark.parametrize("name", ["fp8", "int8"])
+def test_quantized_lengths_in_range(name):
+    inp = make_inputs(name, batch=16)
     assert (inp.context_lens >= 1024).all() and (inp.context_lens <= 16384).all()
     assert inp.k.dtype == torch.bfloat16 and inp.q.dtype == torch.bfloat16
