@@ -92,8 +92,9 @@ def gpu_id(device) -> str:
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clocks, power and throttle reasons sampled every 20 ms; the
+    summary keeps the samples taken between mark_start() and mark_end()."""
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -101,6 +102,7 @@ class ClockSampler:
         self.gpu = gpu
         self.proc = None
         self.path = None
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         import tempfile
@@ -109,11 +111,17 @@ class ClockSampler:
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
         return self
+
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
 
     def __exit__(self, *a):
         if self.proc is not None:
@@ -124,26 +132,36 @@ class ClockSampler:
                 self.proc.kill()
 
     def summary(self):
+        import datetime
         if self.proc is None or self.path is None or not os.path.exists(self.path):
             return None
         rows = []
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            if len(parts) < 10:
                 continue
             try:
-                rows.append((float(parts[1]), float(parts[2]), parts[4:9]))
+                t = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((t, float(parts[2]), float(parts[3]), float(parts[4]), parts[5:10]))
             except ValueError:
                 continue
         os.unlink(self.path)
         if not rows:
             return None
+        inside = rows
+        if self.t0 is not None and self.t1 is not None:
+            # a sample describes the interval before it: keep those ending in the region
+            inside = [r for r in rows if self.t0 < r[0] <= self.t1 + 0.02]
+            if not inside:   # region shorter than the interval: the first sample after it
+                later = [r for r in rows if r[0] > self.t0]
+                inside = later[:1] or rows[-1:]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i in range(4)
+        reasons = sorted({names[i] for *_, r in inside for i in range(4)
                           if r[i + 1].lower() == "active"})
-        return {"sm_mhz": float(np.median([r[0] for r in rows])),
-                "sm_max_mhz": max(r[1] for r in rows), "reasons": reasons,
-                "samples": len(rows)}
+        return {"sm_mhz": float(np.median([r[1] for r in inside])),
+                "sm_max_mhz": max(r[2] for r in inside), "reasons": reasons,
+                "power_w": float(np.median([r[3] for r in inside])),
+                "samples": len(inside), "interval_ms": 20}
 
 
 # ---------------------------------------------------------------- workload bytes
@@ -340,10 +358,13 @@ def run_gpu(args, inp):
                                                   inp.max_context_len, P)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
-    launches_per_step = 4   # slot mapping, cache write, decode, merge
+    fused = args.append == "fused" and Q == 1
+    # separate: slot mapping, cache write, decode, merge; fused: decode (+append), merge
+    launches_per_step = 2 if fused else 4
 
     def append():
-        cache.append(bt, seq_ids, positions, k_new, v_new, slots=slots)
+        if not fused:   # the fused call appends inside the decode
+            cache.append(bt, seq_ids, positions, k_new, v_new, slots=slots)
 
     def attend(qq, tbl, ln):
         if Q == 1:
@@ -354,7 +375,11 @@ def run_gpu(args, inp):
                          partition_tokens=P, workspace=ws)
 
     def decode():
-        attend(q, bt, lens)
+        if fused:
+            cache.decode_append(q, k_new, v_new, bt, lens, inp.max_context_len, spec.scale,
+                                out=out, partition_tokens=P, workspace=ws)
+        else:
+            attend(q, bt, lens)
 
     for _ in range(args.warmup):
         append()
@@ -369,7 +394,8 @@ def run_gpu(args, inp):
     with ClockSampler(gpu_id(device)) as clk:
         barrier(device)
         torch.cuda.synchronize(device)
-        time.sleep(0.25)  # let the clock sampler see the loaded region start
+        time.sleep(0.1)  # the sampler is running before the region starts
+        clk.mark_start()
         start.record(stream)
         for _ in range(args.steps):
             append()
@@ -382,6 +408,7 @@ def run_gpu(args, inp):
             decode()
         d1.record(stream)
         torch.cuda.synchronize(device)
+        clk.mark_end()
         barrier(device)
     elapsed_ms = start.elapsed_time(end)
     decode_ms = d0.elapsed_time(d1) / args.steps
@@ -411,8 +438,12 @@ def run_gpu(args, inp):
 
     def e2e_step():
         d_stage.copy_(h_stage, non_blocking=True)
-        cache.append(e_bt, seq_ids, positions, e_k, e_v, slots=slots)
-        attend(e_q, e_bt, e_lens)
+        if fused:
+            cache.decode_append(e_q, e_k, e_v, e_bt, e_lens, inp.max_context_len, spec.scale,
+                                out=out, partition_tokens=P, workspace=ws)
+        else:
+            cache.append(e_bt, seq_ids, positions, e_k, e_v, slots=slots)
+            attend(e_q, e_bt, e_lens)
         h_out.copy_(out, non_blocking=True)
 
     for _ in range(max(1, args.warmup)):
@@ -460,7 +491,9 @@ def run_gpu(args, inp):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": spec.kv_dtype if spec.kv_dtype != "fp8" else "fp8_e4m3",
         "data": "synthetic (seeded N(0,1) q/K/V, random block permutation)",
-        "config": dict(describe(inp, P), num_ranges=ranges, query_tokens=Q),
+        "config": dict(describe(inp, P), num_ranges=ranges, query_tokens=Q,
+                       append="fused into the decode call" if fused
+                       else "separate slot-mapping and cache-write calls"),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(max_e2e_ms / args.steps, 5)},
@@ -493,6 +526,9 @@ def main(argv=None):
     ap.add_argument("--reference-seqs", type=int, default=8,
                     help="sequences in the oracle's bounded sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--append", default="fused", choices=["separate", "fused"],
+                    help="how a decode step stores its new tokens: separate slot-mapping and "
+                         "cache-write calls, or fused into the decode call (one query token)")
     ap.add_argument("--query-tokens", type=int, default=1,
                     help="query tokens per sequence per step (1 = decode; >1 = speculative "
                          "verification of that many appended tokens)")

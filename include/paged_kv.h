@@ -221,6 +221,42 @@ KV_API kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, con
                                  kv_stream_t stream);
 
 /*
+ * Fused append + decode: one call for a decode step's cache write and attention.
+ * "KV Cache 深度解析" §一/§六 (decode stores the new token's K/V, then scores the
+ * query against every cached key including it) and §三 (the slot of position p
+ * is block_table[b][p / 16] * 16 + p % 16).  For every sequence b with
+ * L = context_lens[b], the new rows k_new[b], v_new[b] go to the slot of
+ * position L - 1 -- stored exactly as reshape_and_cache would store them
+ * (for FP8 / INT8 pools: the same codes and scales, bit for bit) -- and
+ * paged_decode_attention is computed over positions 0 .. L - 1, new token
+ * included.  The result (pools and output) is identical to
+ * compute_slot_mapping + reshape_and_cache + paged_decode_attention.
+ *   k_new, v_new : device [batch][num_kv_heads][head_dim] in src_dtype, 16-byte
+ *                  aligned.  src_dtype: the pool dtype for F32 / BF16 pools (no
+ *                  conversion), F32 or BF16 for FP8 / INT8 pools, else
+ *                  KV_ERR_UNSUPPORTED.
+ *   k_pool, v_pool, scales : written (the slot of position L - 1) and read.
+ * Everything else as paged_decode_attention; it uses the same workspace size.
+ * The slot of position L - 1 must not be read by another sequence of the same
+ * call (a shared, partly filled last block is copied on write first).  When
+ * the block id of position L - 1 is invalid nothing is written for that pair
+ * (KV_DEVERR_BAD_BLOCK_ID); an invalid context length writes nothing for that
+ * sequence (KV_DEVERR_BAD_CONTEXT_LEN, zeros).  This entry point has no
+ * counterpart on the pages; it fuses two of their steps into one launch.
+ */
+KV_API kv_status paged_decode_attention_append(const kv_pool_desc* pool, void* out,
+                                               const void* q, kv_dtype q_dtype, void* k_pool,
+                                               void* v_pool, float* scales, const void* k_new,
+                                               const void* v_new, kv_dtype src_dtype,
+                                               const int32_t* block_table,
+                                               int32_t max_blocks_per_seq,
+                                               const int32_t* context_lens, int32_t batch,
+                                               int32_t num_q_heads, int32_t max_context_len,
+                                               float scale, int32_t partition_tokens,
+                                               void* workspace, size_t workspace_bytes,
+                                               int32_t* dev_error, kv_stream_t stream);
+
+/*
  * Multi-query paged attention: Q = num_query_tokens new tokens per sequence
  * attend to the cache at once -- the verification of Q speculative tokens, or a
  * chunk of a chunked prefill ("KV Cache 深度解析" §五 chunked prefill; "大模型推理为何

@@ -31,6 +31,7 @@ BLOCK_SIZE = 16
 EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
             "paged_decode_num_ranges", "paged_decode_workspace_bytes",
             "paged_decode_attention", "paged_decode_attention_static_workspace",
+            "paged_decode_attention_append",
             "paged_attention_workspace_bytes", "paged_attention_multi_query",
             "paged_kv_copy_blocks", "kv_block_manager_create", "kv_block_manager_destroy",
             "kv_block_manager_num_free_blocks", "kv_block_manager_refcount",
@@ -77,6 +78,9 @@ def _load() -> ctypes.CDLL:
             "paged_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P,
                                               _I32, _I32, _I32, ctypes.c_float, _I32, _P, _SZ,
                                               _P, _P]),
+            "paged_decode_attention_append": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P,
+                                                     _I32, _P, _I32, _P, _I32, _I32, _I32,
+                                                     ctypes.c_float, _I32, _P, _SZ, _P, _P]),
             "paged_decode_attention_static_workspace": (
                 _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
                        ctypes.c_float, _I32, _P, _P]),
@@ -220,6 +224,29 @@ def paged_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
         _ptr(scales), _ptr(block_table), block_table.shape[1],
         _ptr(context_lens), batch, num_q_heads, max_context_len, float(scale),
         partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error), _stream(stream)))
+    return out
+
+
+def paged_decode_attention_append(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
+                                  k_pool: torch.Tensor, v_pool: torch.Tensor,
+                                  scales: torch.Tensor | None, k_new: torch.Tensor,
+                                  v_new: torch.Tensor, block_table: torch.Tensor,
+                                  context_lens: torch.Tensor, max_context_len: int, scale: float,
+                                  partition_tokens: int = 0,
+                                  workspace: torch.Tensor | None = None,
+                                  dev_error: torch.Tensor | None = None,
+                                  stream=None) -> torch.Tensor:
+    """One decode step in one call: k_new/v_new [batch][kv_heads][head_dim] are
+    stored at position context_lens[b] - 1 of each sequence (as reshape_and_cache
+    would) and attended to along with the rest of the context."""
+    batch, num_q_heads, _ = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("paged_decode_attention_append", _load().paged_decode_attention_append(
+        ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool), _ptr(v_pool),
+        _ptr(scales), _ptr(k_new), _ptr(v_new), kv_dtype_of(k_new), _ptr(block_table),
+        block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
+        float(scale), partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error),
+        _stream(stream)))
     return out
 
 

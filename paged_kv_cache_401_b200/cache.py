@@ -11,7 +11,8 @@ import torch
 
 from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, KV_INT8, compute_slot_mapping, empty_pool,
                kv_pool_create, paged_attention_multi_query, paged_attention_workspace_bytes,
-               paged_decode_attention, paged_decode_workspace_bytes, reshape_and_cache)
+               paged_decode_attention, paged_decode_attention_append,
+               paged_decode_workspace_bytes, reshape_and_cache)
 
 _DTYPES = {"f32": KV_F32, "bf16": KV_BF16, "fp8": KV_FP8_E4M3, "int8": KV_INT8}
 
@@ -63,6 +64,24 @@ class PagedKVCache:
         return paged_decode_attention(self.desc, out, q, self.k_pool, self.v_pool, self.scales,
                                       block_table, context_lens, max_context_len,
                                       scale, partition_tokens, workspace, self.dev_error, stream)
+
+    def decode_append(self, q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                      block_table: torch.Tensor, context_lens: torch.Tensor,
+                      max_context_len: int, scale: float, out: torch.Tensor | None = None,
+                      partition_tokens: int = 0, workspace: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+        """One decode step in one launch pair: each sequence's new token (k_new/v_new
+        [batch][kv_heads][head_dim]) is stored at position context_lens[b] - 1 and
+        attended to with the rest of its context."""
+        if out is None:
+            out = torch.empty_like(q)
+        if workspace is None:
+            workspace = self.alloc_workspace(q.shape[0], q.shape[1], max_context_len,
+                                             partition_tokens)
+        return paged_decode_attention_append(self.desc, out, q, self.k_pool, self.v_pool,
+                                             self.scales, k_new, v_new, block_table,
+                                             context_lens, max_context_len, scale,
+                                             partition_tokens, workspace, self.dev_error, stream)
 
     def errors(self) -> int:
         """The device error word (KV_DEVERR_* bits); synchronises."""

@@ -229,16 +229,34 @@ size_t workspace_bytes_for(const kv_pool_desc* pool, int32_t batch, int32_t num_
     return ws_layout(pool, batch, num_q_heads, query_tokens, ranges).total;
 }
 
+// The new token rows of a fused append+decode call.
+struct AppendArgs {
+    void* k_pool;
+    void* v_pool;
+    float* scales;
+    const void* k_new;
+    const void* v_new;
+    kv_dtype src_dtype;
+};
+
 kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_dtype q_dtype,
                          int32_t query_tokens, const void* k_pool, const void* v_pool,
                          const float* scales, const int32_t* block_table,
                          int32_t max_blocks_per_seq, const int32_t* context_lens, int32_t batch,
                          int32_t num_q_heads, int32_t max_context_len, float scale,
                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
-                         int32_t* dev_error, kv_stream_t stream) {
+                         int32_t* dev_error, kv_stream_t stream,
+                         const AppendArgs* app = nullptr) {
     if (!valid_pool(pool) || batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0 ||
-        query_tokens < 1)
+        query_tokens < 1 || (app != nullptr && query_tokens != 1))
         return KV_ERR_INVALID_ARGUMENT;
+    if (app != nullptr) {
+        // no conversion for 16/32-bit pools (as reshape_and_cache); 8-bit pools quantise
+        const bool src_ok = quantized(pool->dtype)
+                                ? (app->src_dtype == KV_F32 || app->src_dtype == KV_BF16)
+                                : app->src_dtype == pool->dtype;
+        if (!src_ok) return KV_ERR_UNSUPPORTED;
+    }
     if (q_dtype != KV_F32 && q_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
     if (num_q_heads % pool->num_kv_heads != 0) return KV_ERR_INVALID_ARGUMENT;
     const int32_t group = num_q_heads / pool->num_kv_heads;
@@ -266,6 +284,9 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
     const bool fp8 = quantized(pool->dtype);  // FP8 or INT8: a scale pool
     if (fp8 != (scales != nullptr)) return KV_ERR_INVALID_ARGUMENT;
     if (fp8 && !aligned16(scales)) return KV_ERR_INVALID_ARGUMENT;
+    if (app != nullptr && (app->k_new == nullptr || app->v_new == nullptr ||
+                           !aligned16(app->k_new) || !aligned16(app->v_new)))
+        return KV_ERR_INVALID_ARGUMENT;
 
     const int32_t ranges = num_ranges_for(pool, batch, num_q_heads, query_tokens,
                                           max_context_len, partition_tokens);
@@ -296,6 +317,14 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
     p.ws_seq_start = reinterpret_cast<int32_t*>(ws);
     p.ws_ml = reinterpret_cast<float2*>(ws + wl.ml_off);
     p.ws_o = reinterpret_cast<float*>(ws + wl.o_off);
+    if (app != nullptr) {
+        p.k_new = app->k_new;
+        p.v_new = app->v_new;
+        p.k_dst = static_cast<uint8_t*>(app->k_pool);
+        p.v_dst = static_cast<uint8_t*>(app->v_pool);
+        p.scales_dst = app->scales;
+        p.append_src_dtype = app->src_dtype;
+    }
     pkv::TmaMaps maps{};
     if (pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim)) {
         // TMA row coordinates are 32-bit
@@ -344,6 +373,23 @@ kv_status paged_decode_attention(const kv_pool_desc* pool, void* out, const void
     return attention_impl(pool, out, q, q_dtype, 1, k_pool, v_pool, scales, block_table,
                           max_blocks_per_seq, context_lens, batch, num_q_heads, max_context_len,
                           scale, partition_tokens, workspace, workspace_bytes, dev_error, stream);
+}
+
+kv_status paged_decode_attention_append(const kv_pool_desc* pool, void* out, const void* q,
+                                        kv_dtype q_dtype, void* k_pool, void* v_pool,
+                                        float* scales, const void* k_new, const void* v_new,
+                                        kv_dtype src_dtype, const int32_t* block_table,
+                                        int32_t max_blocks_per_seq, const int32_t* context_lens,
+                                        int32_t batch, int32_t num_q_heads,
+                                        int32_t max_context_len, float scale,
+                                        int32_t partition_tokens, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_error,
+                                        kv_stream_t stream) {
+    const AppendArgs app{k_pool, v_pool, scales, k_new, v_new, src_dtype};
+    return attention_impl(pool, out, q, q_dtype, 1, k_pool, v_pool, scales, block_table,
+                          max_blocks_per_seq, context_lens, batch, num_q_heads, max_context_len,
+                          scale, partition_tokens, workspace, workspace_bytes, dev_error, stream,
+                          &app);
 }
 
 kv_status paged_attention_multi_query(const kv_pool_desc* pool, void* out, const void* q,

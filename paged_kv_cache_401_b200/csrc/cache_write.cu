@@ -8,6 +8,7 @@
 #include <algorithm>
 
 #include "kernels.cuh"
+#include "quant.cuh"
 
 namespace pkv {
 
@@ -64,11 +65,9 @@ __global__ void cache_copy_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restr
     }
 }
 
-// Quantising write: one warp per (token, kv head, K|V) row of D elements.
-//   FP8 : a = max|x|; scale = a / 448 (IEEE fp32 division); code = E4M3(x / scale)
-//         (IEEE division, RNE, saturating)
-//   INT8: a = max|x|; scale = a / 127; code = clamp(rint(x / scale), -127, 127)
-//   a == 0 -> scale 0 and codes 0.
+// Quantising write: one warp per (token, kv head, K|V) row of D elements; the
+// codes and scale come from quantize_row_warp (FP8: absmax/448, E4M3; INT8:
+// absmax/127, round to nearest even, clamp to 127).
 template <int KV_T, int SRC_T, int D>
 __global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
                                    float* __restrict__ scales,
@@ -76,7 +75,7 @@ __global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __rest
                                    const int64_t* __restrict__ slots, int32_t num_tokens,
                                    int32_t num_kv_heads, int64_t num_slots, int32_t* dev_error) {
     constexpr int kPer = D / 32;  // elements per lane (4 or 2)
-    constexpr float kMaxCode = KV_T == KV_INT8 ? 127.0f : 448.0f;
+    constexpr int kSrcBytes = SRC_T == KV_F32 ? 4 : 2;
     pdl_wait();
     pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
@@ -94,48 +93,15 @@ __global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __rest
         return;
     }
     float x[kPer];
-    const void* src = which ? v_new : k_new;
-    if constexpr (SRC_T == KV_F32) {
-        const float* p = static_cast<const float*>(src) + th * D + lane * kPer;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) x[e] = p[e];
-    } else {
-        const uint16_t* p = static_cast<const uint16_t*>(src) + th * D + lane * kPer;
-#pragma unroll
-        for (int e = 0; e < kPer; ++e) x[e] = __uint_as_float(static_cast<uint32_t>(p[e]) << 16);
-    }
-    float a = 0.0f;
-#pragma unroll
-    for (int e = 0; e < kPer; ++e) a = fmaxf(a, fabsf(x[e]));
-#pragma unroll
-    for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
-    const float s = __fdiv_rn(a, kMaxCode);
-    uint32_t codes = 0;
-#pragma unroll
-    for (int e = 0; e < kPer; e += 2) {
-        uint32_t pair = 0;
-        if (a != 0.0f) {
-            if constexpr (KV_T == KV_INT8) {
-                const int c0 = max(-127, min(127, __float2int_rn(__fdiv_rn(x[e], s))));
-                const int c1 = max(-127, min(127, __float2int_rn(__fdiv_rn(x[e + 1], s))));
-                pair = (static_cast<uint32_t>(c0) & 0xffu) | ((static_cast<uint32_t>(c1) & 0xffu) << 8);
-            } else {
-                pair = float2_to_e4m3x2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s));
-            }
-        }
-        codes |= pair << (8 * e);
-    }
+    const uint8_t* src = static_cast<const uint8_t*>(which ? v_new : k_new);
+    load_row_part<D>(src + th * D * kSrcBytes, SRC_T, lane, x);
+    float s;
+    const uint32_t codes = quantize_row_warp<KV_T, D>(x, &s);
     const int64_t blk = slot / kBlockTokens, off = slot % kBlockTokens;
     const int64_t rowi = (blk * num_kv_heads + h) * kBlockTokens + off;
-    uint8_t* dst = (which ? v_pool : k_pool) + rowi * D + lane * kPer;
-    if constexpr (kPer == 4) {
-        *reinterpret_cast<uint32_t*>(dst) = codes;
-    } else {
-        *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(codes);
-    }
+    store_codes<D>((which ? v_pool : k_pool) + rowi * D + lane * kPer, codes);
     // scale pool [block][head][K|V][16]: one 128-byte line per (block, head)
-    if (lane == 0)
-        scales[((blk * num_kv_heads + h) * 2 + which) * kBlockTokens + off] = (a == 0.0f) ? 0.0f : s;
+    if (lane == 0) scales[((blk * num_kv_heads + h) * 2 + which) * kBlockTokens + off] = s;
 }
 
 // Whole-block copies (copy-on-write of shared blocks): CTA (pair, part) moves

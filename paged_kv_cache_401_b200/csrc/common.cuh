@@ -84,9 +84,10 @@ __device__ __forceinline__ void bulk_copy_g2s(void* smem_dst, const void* gmem_s
 
 // ---- programmatic dependent launch -------------------------------------------
 // Every kernel of the library waits for the grid before it in the stream to
-// finish (and its writes to be visible) before touching global memory, then
-// lets the next grid start launching: with the launch attribute set, a
-// kernel's launch and prologue overlap its predecessor's tail; without it both
+// finish (and its writes to be visible) before touching global memory.  The
+// short kernels then let the next grid start launching at once, so its launch
+// and prologue overlap their tail; the persistent decode kernel does not (its
+// dependents start as it exits).  Without the launch attribute both
 // instructions are no-ops.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {

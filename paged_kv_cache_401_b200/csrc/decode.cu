@@ -42,6 +42,7 @@
 //  * every wait is bounded; bad block ids and context lengths are reported
 //    through the error word and never dereferenced.
 #include "kernels.cuh"
+#include "quant.cuh"
 
 namespace pkv {
 
@@ -382,6 +383,9 @@ __device__ __forceinline__ void advance(Cursor& c, const DecodeParams& p) {
 template <int KV_T, int Q_T, int D, int G>
 struct SimtMath {
     using OutT = typename QType<Q_T>::T;
+    static constexpr int kKv = KV_T;
+    static constexpr int kHeadDim = D;
+    static constexpr bool kCanAppend = true;                                 // one query token
     static constexpr int kElem = KvElem<KV_T>::kBytes;
     static constexpr int kTileBytes = kBlockTokens * D * kElem;              // K or V tile
     static constexpr int kScaleBytes = kQuantized<KV_T> ? 2 * kBlockTokens * 4 : 0;  // K|V
@@ -418,6 +422,11 @@ struct SimtMath {
         bulk_copy_g2s(st + kTileBytes, p.v_pool + off, kTileBytes, bar);
         if constexpr (kQuantized<KV_T>)
             bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
+    }
+
+    // Byte offset of byte `byte` of row `row` in a staged K or V tile (rows are contiguous).
+    __device__ static __forceinline__ int32_t tile_byte(int32_t row, int32_t byte) {
+        return row * D * kElem + byte;
     }
 
     // ---- consumer side
@@ -635,6 +644,9 @@ struct MmaMath {
     using OutT = uint16_t;                                        // bf16 output
     static constexpr bool kF16 = kQuantized<KV_T>;              // 8-bit codes widened to f16
     static constexpr int D = 128;
+    static constexpr int kKv = KV_T;
+    static constexpr int kHeadDim = D;
+    static constexpr bool kCanAppend = SINGLE;                    // fused append: decode only
     static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
     static constexpr int kElem = KvElem<KV_T>::kBytes;
     static constexpr int kRowBytes = D * kElem;                   // 256 (bf16) / 128 (8-bit)
@@ -661,6 +673,11 @@ struct MmaMath {
         }
         if constexpr (kF16)
             bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
+    }
+
+    // Byte offset of byte `byte` of row `row` in a staged (swizzled) K or V tile.
+    __device__ static __forceinline__ int32_t tile_byte(int32_t row, int32_t byte) {
+        return static_cast<int32_t>(swz(row, byte >> 4)) + (byte & 15);
     }
 
     // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile.
@@ -954,6 +971,90 @@ struct Smem {
     static_assert(kBytes <= 227 * 1024, "shared memory per block");
 };
 
+// Fused append: the warp that attends to the last tile of pair (b, kvh) -- the
+// tile holding position L - 1 -- writes that position's new K and V rows to the
+// pool (for 8-bit pools: quantised exactly as reshape_and_cache does, codes and
+// scales) and patches the staged copy of the tile, whose TMA read of that slot
+// may have seen the old contents.  The block id was validated by the producer.
+// Never inlined: it runs once per pair, and keeping it out of line keeps the
+// tile loop's register allocation as it is without the append.
+// What the fused append needs, passed by value so the out-of-line call does
+// not force a local copy of the kernel's parameters.
+struct AppendRow {
+    const void* k_new;
+    const void* v_new;
+    uint8_t* k_dst;
+    uint8_t* v_dst;
+    float* scales_dst;
+    const int32_t* table_row;  // block_table row of the sequence
+    int64_t src_row;           // row of k_new / v_new: b * Hkv + kvh
+    int32_t num_kv_heads, kvh, L, src_dtype;
+};
+
+// Bring the bytes of the new rows this lane will read in append_row into L1,
+// so the warp that owns the pair's last tile does not wait on them there.
+template <class M>
+__device__ __forceinline__ void prefetch_append(const DecodeParams& p, int32_t b, int32_t kvh,
+                                                int32_t lane) {
+    constexpr int D = M::kHeadDim;
+    const int64_t srow = static_cast<int64_t>(b) * p.num_kv_heads + kvh;
+    const uint8_t* k = static_cast<const uint8_t*>(p.k_new);
+    const uint8_t* v = static_cast<const uint8_t*>(p.v_new);
+    int64_t off;
+    if constexpr (kQuantized<M::kKv>) {
+        const int32_t src_bytes = p.append_src_dtype == KV_F32 ? 4 : 2;
+        off = (srow * D + lane * (D / 32)) * src_bytes;
+    } else {
+        constexpr int kRowBytes = D * KvElem<M::kKv>::kBytes;
+        off = srow * kRowBytes + (lane * 16) % kRowBytes;
+    }
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(k + off));
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(v + off));
+}
+
+template <class M>
+__device__ __noinline__ void append_row(uint8_t* st, const AppendRow a, int32_t lane) {
+    constexpr int D = M::kHeadDim;
+    constexpr int kElem = KvElem<M::kKv>::kBytes;
+    constexpr int kRowBytes = D * kElem;
+    constexpr int kTileBytes = kBlockTokens * kRowBytes;
+    const int32_t pos = a.L - 1, r = pos % kBlockTokens;
+    const int64_t blk = a.table_row[pos / kBlockTokens];
+    const int64_t rowi = (blk * a.num_kv_heads + a.kvh) * kBlockTokens + r;  // pool row
+    if constexpr (kQuantized<M::kKv>) {
+        constexpr int kPer = D / 32;
+        const int32_t src_bytes = a.src_dtype == KV_F32 ? 4 : 2;
+        float* sc_stage = reinterpret_cast<float*>(st + 2 * kTileBytes);  // K then V row scales
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const uint8_t* src = static_cast<const uint8_t*>(which ? a.v_new : a.k_new);
+            float x[kPer];
+            load_row_part<D>(src + a.src_row * D * src_bytes, a.src_dtype, lane, x);
+            float sc;
+            const uint32_t codes = quantize_row_warp<M::kKv, D>(x, &sc);
+            store_codes<D>((which ? a.v_dst : a.k_dst) + rowi * kRowBytes + lane * kPer, codes);
+            store_codes<D>(st + which * kTileBytes + M::tile_byte(r, lane * kPer), codes);
+            if (lane == 0) {
+                a.scales_dst[((blk * a.num_kv_heads + a.kvh) * 2 + which) * kBlockTokens + r] = sc;
+                sc_stage[which * kBlockTokens + r] = sc;
+            }
+        }
+    } else {
+        // same dtype as the pool: the row's bytes, 16 at a time
+        constexpr int kChunks = kRowBytes / 16;
+        for (int i = lane; i < 2 * kChunks; i += 32) {
+            const int which = i / kChunks, c = i % kChunks;
+            const uint8_t* src = static_cast<const uint8_t*>(which ? a.v_new : a.k_new);
+            const uint4 v = *reinterpret_cast<const uint4*>(src + a.src_row * kRowBytes + c * 16);
+            *reinterpret_cast<uint4*>((which ? a.v_dst : a.k_dst) + rowi * kRowBytes + c * 16) = v;
+            *reinterpret_cast<uint4*>(st + which * kTileBytes + M::tile_byte(r, c * 16)) = v;
+        }
+    }
+    // the stage is refilled by the async proxy (TMA) later: order these writes first
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncwarp();
+}
+
 template <class M, int Q_T>
 __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
     paged_decode_kernel(const DecodeParams p, const __grid_constant__ TmaMaps maps) {
@@ -971,8 +1072,10 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
 
     const int32_t warp = threadIdx.x >> 5;
     const int32_t lane = threadIdx.x & 31;
+    // No early launch_dependents here: this grid is persistent, and a dependent
+    // (the merge) launched at its start parks CTAs on the SMs for its whole
+    // duration; releasing it at exit measured 7 % faster per call.
     pdl_wait();
-    pdl_trigger();
     const int64_t T = total_tiles(p, lane);
     const int64_t W0 = static_cast<int64_t>(blockIdx.x) * kConsumerWarps;
 
@@ -1074,6 +1177,8 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
     math.init(lane, scratch + warp * M::kWarpScratch);
     math.load_q(p, cur.b, cur.kvh);
     math.reset();
+    if constexpr (M::kCanAppend)
+        if (p.k_new != nullptr) prefetch_append<M>(p, cur.b, cur.kvh, lane);
     int64_t piece_start = lo;
 
     constexpr int kPerWarp = M::kStages / kConsumerWarps;
@@ -1086,7 +1191,18 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
             *abort_flag = 1;
         }
         if (__any_sync(0xffffffffu, *abort_flag != 0)) return;  // output invalid (reported)
-        if (stage_ok[s]) math.tile(ring + s * M::kStageBytes, cur.jb, cur.L, p);
+        if (stage_ok[s]) {
+            if constexpr (M::kCanAppend) {
+                if (p.k_new != nullptr && cur.jb + 1 == cur.nt) {
+                    const AppendRow a{p.k_new, p.v_new, p.k_dst, p.v_dst, p.scales_dst,
+                                      p.block_table + static_cast<int64_t>(cur.b) * p.max_blocks,
+                                      static_cast<int64_t>(cur.b) * p.num_kv_heads + cur.kvh,
+                                      p.num_kv_heads, cur.kvh, cur.L, p.append_src_dtype};
+                    append_row<M>(ring + s * M::kStageBytes, a, lane);
+                }
+            }
+            math.tile(ring + s * M::kStageBytes, cur.jb, cur.L, p);
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
 
@@ -1101,6 +1217,8 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
                 piece_start = lo + j + 1;
                 math.load_q(p, cur.b, cur.kvh);
                 math.reset();
+                if constexpr (M::kCanAppend)
+                    if (p.k_new != nullptr) prefetch_append<M>(p, cur.b, cur.kvh, lane);
             }
         } else {
             ++cur.jb;

@@ -65,6 +65,15 @@ struct DecodeParams {
     int32_t num_query_tokens;     // Q: query tokens per sequence (1 for decode)
     int32_t num_ranges;           // consumer-warp ranges the tile list is cut into
     float scale_log2;             // scale * log2(e): scores are kept in base-2 units
+    // Fused append (one query token): every sequence's new K/V row [B][Hkv][D] in
+    // append_src_dtype is written to the slot of position L - 1 (codes and scale
+    // for 8-bit pools) by the warp that attends to it.  k_new == nullptr: no append.
+    const void* k_new;
+    const void* v_new;
+    uint8_t* k_dst;               // the pools again, writable
+    uint8_t* v_dst;
+    float* scales_dst;
+    int32_t append_src_dtype;
 };
 
 // TMA descriptors of the K and V pools as 2-D tensors [num_blocks*Hkv*16 rows][head_dim],

@@ -1,0 +1,78 @@
+// Per-row quantisation of a new K or V row by one warp, shared by the cache
+// write and the fused append+decode so both store identical codes.
+//
+// "KV Cache 深度解析" §四 (fp16 -> fp8 E4M3 with a per-token scale to hold
+// outliers); k1-blog "KV Cache 量化" (INT8 halves the cache like FP8).  For a
+// row x of D elements (one token, one kv head):
+//   FP8 : a = max|x|; scale = a / 448 (IEEE fp32 division);
+//         code = E4M3(x / scale) (IEEE division, round to nearest even, saturating)
+//   INT8: a = max|x|; scale = a / 127;
+//         code = clamp(round_to_nearest_even(x / scale), -127, 127)
+//   a == 0 -> scale 0 and every code 0.
+// Lane l holds elements [l * D/32, (l + 1) * D/32) of the row.
+#pragma once
+
+#include "common.cuh"
+
+namespace pkv {
+
+// Load a lane's D/32 consecutive source elements (fp32 or bf16) widened to fp32.
+template <int D>
+__device__ __forceinline__ void load_row_part(const void* row, int32_t src_dtype, int32_t lane,
+                                              float* x) {
+    constexpr int kPer = D / 32;
+    if (src_dtype == KV_F32) {
+        const float* p = static_cast<const float*>(row) + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) x[e] = p[e];
+    } else {
+        const uint16_t* p = static_cast<const uint16_t*>(row) + lane * kPer;
+#pragma unroll
+        for (int e = 0; e < kPer; ++e) x[e] = __uint_as_float(static_cast<uint32_t>(p[e]) << 16);
+    }
+}
+
+// Quantise the row held by the warp; returns this lane's D/32 codes packed
+// little-endian (first element in the low byte) and the row scale in *scale.
+template <int KV_T, int D>
+__device__ __forceinline__ uint32_t quantize_row_warp(const float* x, float* scale) {
+    constexpr int kPer = D / 32;
+    constexpr float kMaxCode = KV_T == KV_INT8 ? 127.0f : 448.0f;
+    static_assert(KV_T == KV_FP8_E4M3 || KV_T == KV_INT8, "8-bit codes");
+    static_assert(kPer == 2 || kPer == 4, "head_dim 64 or 128");
+    float a = 0.0f;
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) a = fmaxf(a, fabsf(x[e]));
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, m));
+    const float s = __fdiv_rn(a, kMaxCode);
+    uint32_t codes = 0;
+#pragma unroll
+    for (int e = 0; e < kPer; e += 2) {
+        uint32_t pair = 0;
+        if (a != 0.0f) {
+            if constexpr (KV_T == KV_INT8) {
+                const int c0 = max(-127, min(127, __float2int_rn(__fdiv_rn(x[e], s))));
+                const int c1 = max(-127, min(127, __float2int_rn(__fdiv_rn(x[e + 1], s))));
+                pair = (static_cast<uint32_t>(c0) & 0xffu) | ((static_cast<uint32_t>(c1) & 0xffu) << 8);
+            } else {
+                pair = float2_to_e4m3x2(__fdiv_rn(x[e], s), __fdiv_rn(x[e + 1], s));
+            }
+        }
+        codes |= pair << (8 * e);
+    }
+    *scale = (a == 0.0f) ? 0.0f : s;
+    return codes;
+}
+
+// Store a lane's packed codes (D/32 bytes) at dst.
+template <int D>
+__device__ __forceinline__ void store_codes(uint8_t* dst, uint32_t codes) {
+    if constexpr (D / 32 == 4) {
+        *reinterpret_cast<uint32_t*>(dst) = codes;
+    } else {
+        *reinterpret_cast<uint16_t*>(dst) = static_cast<uint16_t>(codes);
+    }
+}
+
+}  // namespace pkv

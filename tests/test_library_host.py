@@ -131,6 +131,36 @@ def test_decode_host_validation(kw, status):
     assert _call_decode(d, **kw) == status
 
 
+def _call_append(desc, **kw):
+    lib = pk.library()
+    args = dict(out=4096, q=8192, q_dtype=pk.KV_BF16, k_pool=1 << 20, v_pool=2 << 20,
+                scales=None, k_new=7 << 20, v_new=8 << 20, src_dtype=pk.KV_BF16,
+                block_table=3 << 20, max_blocks=256, context_lens=4 << 20, batch=32,
+                num_q_heads=32, max_context_len=4096, scale=0.088, partition=512,
+                workspace=5 << 20, workspace_bytes=1 << 30, dev_error=None, stream=None)
+    args.update(kw)
+    return lib.paged_decode_attention_append(
+        ctypes.byref(desc), args["out"], args["q"], args["q_dtype"], args["k_pool"],
+        args["v_pool"], args["scales"], args["k_new"], args["v_new"], args["src_dtype"],
+        args["block_table"], args["max_blocks"], args["context_lens"], args["batch"],
+        args["num_q_heads"], args["max_context_len"], args["scale"], args["partition"],
+        args["workspace"], args["workspace_bytes"], args["dev_error"], args["stream"])
+
+
+@pytest.mark.parametrize("pool,kw,status", [
+    (pk.KV_BF16, dict(src_dtype=pk.KV_F32), pk.KV_ERR_UNSUPPORTED),      # no conversion
+    (pk.KV_BF16, dict(k_new=None), pk.KV_ERR_INVALID_ARGUMENT),
+    (pk.KV_BF16, dict(v_new=(8 << 20) + 4), pk.KV_ERR_INVALID_ARGUMENT),  # misaligned
+    (pk.KV_BF16, dict(num_q_heads=24), pk.KV_ERR_UNSUPPORTED),          # as the decode
+    (pk.KV_FP8_E4M3, dict(scales=6 << 20, src_dtype=pk.KV_INT8), pk.KV_ERR_UNSUPPORTED),
+    (pk.KV_INT8, dict(scales=6 << 20, src_dtype=pk.KV_FP8_E4M3), pk.KV_ERR_UNSUPPORTED),
+    (pk.KV_INT8, dict(src_dtype=pk.KV_F32), pk.KV_ERR_INVALID_ARGUMENT),  # needs scales
+])
+def test_decode_append_host_validation(pool, kw, status):
+    d = pk.kv_pool_create(8192, 16, 8, 128, pool)
+    assert _call_append(d, **kw) == status
+
+
 @pytest.mark.parametrize("dtype", [pk.KV_FP8_E4M3, pk.KV_INT8])
 def test_decode_quantized_pool_requires_scales(dtype):
     d = pk.kv_pool_create(8192, 16, 8, 128, dtype)
