@@ -19,7 +19,10 @@ restatement, in double precision, of every step of the decode hot path:
                              ("KV Cache 深度解析", §四 KV Cache 量化);
                              ``quantize_rows(x, "int8")`` the INT8 cache, symmetric
                              absmax/127 (k1-blog "KV Cache 量化", freetools
-                             "KV Cache量化": INT8 halves the cache like FP8).
+                             "KV Cache量化": INT8 halves the cache like FP8);
+                             ``quantize_rows(x, "int4")`` the INT4 cache, the
+                             asymmetric 4-bit routine of the
+                             "llm-inference-optimization" notes §四 per row.
 * ``decode_attention``    -- softmax(q·Kᵀ·scale)·V over a CONTIGUOUS per-sequence
                              copy, GQA head grouping, two passes in double
                              (C, OpenMP); "KV Cache 深度解析", §一 and §六.
@@ -46,9 +49,9 @@ import numpy as np
 
 from . import build as _build
 
-F32, BF16, FP8_E4M3, INT8 = 0, 1, 2, 3
-_DTYPE_CODES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3, "int8": INT8}
-QUANTIZED = ("fp8", "int8")
+F32, BF16, FP8_E4M3, INT8, INT4 = 0, 1, 2, 3, 4
+_DTYPE_CODES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3, "int8": INT8, "int4": INT4}
+QUANTIZED = ("fp8", "int8", "int4")
 
 _lib = None
 
@@ -67,6 +70,8 @@ def _load():
                                              ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_quantize_rows_int8.restype = None
         lib.oracle_quantize_rows_int8.argtypes = lib.oracle_quantize_rows.argtypes
+        lib.oracle_quantize_rows_int4.restype = None
+        lib.oracle_quantize_rows_int4.argtypes = lib.oracle_quantize_rows.argtypes
         lib.oracle_decode_attention.restype = ctypes.c_int
         lib.oracle_decode_attention.argtypes = [
             ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -177,7 +182,9 @@ def quantize_rows(x: np.ndarray, kind: str = "fp8") -> tuple[np.ndarray, np.ndar
     """x: [..., D] float32 -> (codes [..., D], scales float32 [...]).
 
     kind "fp8": uint8 E4M3 codes, scale absmax/448; "int8": int8 codes,
-    scale absmax/127, round to nearest (ties to even), clamp to +-127."""
+    scale absmax/127, round to nearest (ties to even), clamp to +-127;
+    "int4": uint8 codes 0..15 (one per element, unpacked) and params
+    float32 [..., 2] = (scale, zero point) per row."""
     x = np.ascontiguousarray(x, dtype=np.float32)
     d = x.shape[-1]
     rows = x.size // d
@@ -186,6 +193,11 @@ def quantize_rows(x: np.ndarray, kind: str = "fp8") -> tuple[np.ndarray, np.ndar
     if kind == "int8":
         codes = np.empty(x.shape, dtype=np.int8)
         lib.oracle_quantize_rows_int8(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
+    elif kind == "int4":
+        codes = np.empty(x.shape, dtype=np.uint8)
+        params = np.empty(x.shape[:-1] + (2,), dtype=np.float32)
+        lib.oracle_quantize_rows_int4(_ptr(x), rows, d, _ptr(codes), _ptr(params))
+        return codes, params
     elif kind == "fp8":
         codes = np.empty(x.shape, dtype=np.uint8)
         lib.oracle_quantize_rows(_ptr(x), rows, d, _ptr(codes), _ptr(scales))
@@ -207,7 +219,9 @@ def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offsets: n
     k, v  : [T][Hkv][D]  float32 / uint16 bf16 bits / uint8 E4M3 codes / int8 codes
     seq_offsets : [B] int64, first token of each sequence in k/v
     lens  : [B] int32 context lengths (>= 1)
-    k_scale, v_scale : [T][Hkv] float32 for kv_dtype "fp8" / "int8"
+    k_scale, v_scale : [T][Hkv] float32 for kv_dtype "fp8" / "int8";
+                       [T][Hkv][2] (scale, zero) for "int4"
+    (int4 codes: uint8 0..15, one per element)
     Returns out [B][Hq][D] float64 (and weights [B][Hq][max(lens)] if asked).
     """
     lib = _load()
@@ -269,6 +283,9 @@ def widen(x: np.ndarray, dtype: str, scales: np.ndarray | None = None) -> np.nda
     if dtype == "int8":
         return np.asarray(x, dtype=np.int8).astype(np.float64) * \
             np.asarray(scales, dtype=np.float64)[..., None]
+    if dtype == "int4":
+        pz = np.asarray(scales, dtype=np.float64)
+        return (np.asarray(x, dtype=np.uint8).astype(np.float64) - pz[..., 1:2]) * pz[..., 0:1]
     return e4m3_decode(x) * np.asarray(scales, dtype=np.float64)[..., None]
 
 

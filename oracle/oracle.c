@@ -18,6 +18,10 @@
  *  - k1-blog 2026-07-13 "AI", "KV Cache 量化" (FP8 and INT8 both halve the
  *    fp16 cache) and "大模型推理为何这么慢", "KV Cache量化" (INT8 among the
  *    lower-precision KV formats) for the INT8 cache.
+ *  - "llm-inference-optimization" notes, §四 (the printed 4-bit group
+ *    quantiser: range / 15, a zero point rounded from -min / scale, codes
+ *    clamped to 0..15) and "大模型推理为何这么慢", "KV Cache量化" (a 4-bit
+ *    cache is 4x smaller than fp16) for the INT4 cache.
  *  - "大模型推理为何这么慢？从内存带宽瓶颈到KV Cache优化的技术突围"
  *    (freetools), section on GQA (H query heads share G groups of K/V).
  *
@@ -31,7 +35,13 @@
  *  - the INT8 cache follows the FP8 design: symmetric, scale = absmax/127 in
  *    IEEE fp32, code = x / scale (fp32 division) rounded to the nearest
  *    integer, ties to even, clamped to [-127, 127]; an all-zero row has scale
- *    0 and codes 0; dequantisation is code * scale in double.
+ *    0 and codes 0; dequantisation is code * scale in double;
+ *  - the INT4 cache applies the §四 routine to each (token, kv head) row, in
+ *    IEEE fp32 in the routine's order: scale = (max - min) / 15, zero =
+ *    rint(-min / scale), code = clamp(rint(x / scale) + zero, 0, 15); a
+ *    constant row, where the routine would divide by zero, is stored exactly
+ *    (scale |min|, zero -1 / +1 / 0, codes 0); value = (code - zero) * scale
+ *    in double.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math).
  */
@@ -44,7 +54,7 @@
 #endif
 
 /* Stored element types of K/V and q, as the callers of this file pass them. */
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2, ORC_INT8 = 3 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2, ORC_INT8 = 3, ORC_INT4 = 4 };
 
 /* ---- exact widening of stored values ------------------------------------ */
 
@@ -177,7 +187,46 @@ void oracle_quantize_rows_int8(const float* x, int64_t rows, int32_t d,
     }
 }
 
-/* Value of element i of a stored row, widened to double (8-bit codes dequantised). */
+/*
+ * INT4 quantisation of `rows` rows of length d ("llm-inference-optimization"
+ * notes §四's routine per row).  codes: one code (0..15) per element, unpacked;
+ * params: per row (scale, zero point).
+ */
+void oracle_quantize_rows_int4(const float* x, int64_t rows, int32_t d,
+                               uint8_t* codes, float* params) {
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        const float* xr = x + r * d;
+        float hi = xr[0], lo = xr[0], s, z;
+        int32_t i;
+        for (i = 1; i < d; ++i) {
+            if (xr[i] > hi) hi = xr[i];
+            if (xr[i] < lo) lo = xr[i];
+        }
+        if (hi == lo) {
+            /* the routine's scale would be 0: store the constant exactly */
+            s = fabsf(lo);
+            z = lo > 0.0f ? -1.0f : (lo < 0.0f ? 1.0f : 0.0f);
+            for (i = 0; i < d; ++i) codes[r * d + i] = 0;
+        } else {
+            float range = hi - lo;
+            s = range / 15.0f;
+            z = rintf(-lo / s);
+            for (i = 0; i < d; ++i) {
+                float q = rintf(xr[i] / s);
+                float c = q + z;
+                if (c < 0.0f) c = 0.0f;
+                if (c > 15.0f) c = 15.0f;
+                codes[r * d + i] = (uint8_t)c;
+            }
+        }
+        params[2 * r] = s;
+        params[2 * r + 1] = z;
+    }
+}
+
+/* Value of element i of a stored row, widened to double (codes dequantised).
+ * For INT4 `scales` holds (scale, zero) pairs per row. */
 static double load_elem(const void* base, int dtype, int64_t idx, const float* scales,
                         int64_t scale_idx) {
     switch (dtype) {
@@ -187,6 +236,9 @@ static double load_elem(const void* base, int dtype, int64_t idx, const float* s
         return bf16_bits_to_double(((const uint16_t*)base)[idx]);
     case ORC_INT8:
         return (double)((const int8_t*)base)[idx] * (double)scales[scale_idx];
+    case ORC_INT4:
+        return ((double)((const uint8_t*)base)[idx] - (double)scales[2 * scale_idx + 1]) *
+               (double)scales[2 * scale_idx];
     default:
         return oracle_e4m3_decode(((const uint8_t*)base)[idx]) * (double)scales[scale_idx];
     }
@@ -198,7 +250,8 @@ static double load_elem(const void* base, int dtype, int64_t idx, const float* s
  *   q    : [B][Hq][D] in q_dtype (F32 or BF16)
  *   k, v : [total_tokens][Hkv][D] in kv_dtype, sequence b occupying tokens
  *          [seq_offsets[b], seq_offsets[b] + lens[b])
- *   k_scale, v_scale : [total_tokens][Hkv] fp32, FP8 / INT8 only (else NULL)
+ *   k_scale, v_scale : [total_tokens][Hkv] fp32, FP8 / INT8 only; for INT4
+ *          [total_tokens][Hkv][2] (scale, zero); else NULL
  *   out  : [B][Hq][D] double
  *   weights (nullable): [B][Hq][max_len] double, the softmax weights
  *

@@ -3,8 +3,9 @@
 * printed values on the pages (tests/golden/kv_sizes.txt);
 * library routines (torch scaled_dot_product_attention in float64, torch's
   float8_e4m3fn conversion);
-* hand-computed INT8 rows with exact binary scales, and a brute-force
-  nearest-integer search for the INT8 codes;
+* hand-computed INT8 and INT4 rows with exact binary scales, a brute-force
+  nearest-integer search for the INT8 codes and an exact-rational re-derivation
+  of the INT4 scale, zero point and codes;
 * closed forms and special cases (length 1, identical keys, dominant key,
   weights summing to one, key-order invariance);
 * brute force on tiny inputs (numpy, one head at a time) and an independent
@@ -209,6 +210,80 @@ def test_int8_quantize_invariants():
     assert (c3 == codes).all() and (s3 == scales * np.float32(2.0 ** -7)).all()
 
 
+# ---------------------------------------------------------------- INT4 rows
+def test_int4_quantize_hand_examples():
+    # worked by hand from the 4-bit routine (range / 15, zero = round(-min / scale),
+    # code = clamp(round(x / scale) + zero, 0, 15)), scales exact in binary:
+    # row 0: hi 22.5, lo -7.5 -> scale 2, zero round(3.75) = 4;
+    #        x / 2 = 0, .75, 1.5, 2.25, 11.25, -3.75 -> 0, 1, 2 (tie to even), 2, 11, -4
+    # row 1: hi 15, lo 0 -> scale 1, zero 0; codes round(x): 7.5 -> 8, 8.5 -> 8,
+    #        0.5 -> 0, 1.5 -> 2, 2.5 -> 2, 14.5 -> 14 (ties to even)
+    # rows 2-4: constant rows are kept exactly
+    x = np.array([[0, 1.5, 3, 4.5, 22.5, -7.5, 0, 0],
+                  [0, 7.5, 8.5, 15, 0.5, 1.5, 2.5, 14.5],
+                  [2, 2, 2, 2, 2, 2, 2, 2],
+                  [-3, -3, -3, -3, -3, -3, -3, -3],
+                  [0, 0, 0, 0, 0, 0, 0, 0]], dtype=np.float32)
+    codes, pz = oracle.quantize_rows(x, "int4")
+    assert codes.tolist() == [[4, 5, 6, 6, 15, 0, 4, 4],
+                              [0, 8, 8, 15, 0, 2, 2, 14],
+                              [0] * 8, [0] * 8, [0] * 8]
+    assert pz.tolist() == [[2, 4], [1, 0], [2, -1], [3, 1], [0, 0]]
+    assert oracle.widen(codes, "int4", pz)[2:].tolist() == [[2] * 8, [-3] * 8, [0] * 8]
+
+
+def _nearest_even(y: Fraction) -> int:
+    f = y.numerator // y.denominator
+    r = y - f
+    if r > Fraction(1, 2) or (r == Fraction(1, 2) and f % 2 == 1):
+        return f + 1
+    return f
+
+
+def test_int4_quantize_exact_rationals():
+    # scale, zero and codes re-derived with exact rationals from the fp32
+    # quotients the routine forms (round to nearest, ties to even)
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((40, 128)) * rng.uniform(0.01, 50, (40, 1))
+         + rng.uniform(-5, 5, (40, 1))).astype(np.float32)
+    x[3] = np.abs(x[3]) + 10                           # all positive: negative zero point
+    x[4] = -np.abs(x[4]) - 10                          # all negative: zero point above 15
+    codes, pz = oracle.quantize_rows(x, "int4")
+    for r in range(x.shape[0]):
+        hi, lo = np.float32(x[r].max()), np.float32(x[r].min())
+        s = np.float32(np.float32(hi - lo) / np.float32(15))
+        z = _nearest_even(Fraction(float(np.float32(-lo) / s)))
+        assert pz[r, 0] == s and pz[r, 1] == z
+        for i in range(x.shape[1]):
+            k = _nearest_even(Fraction(float(np.float32(x[r, i]) / s)))
+            assert codes[r, i] == min(15, max(0, k + z)), (r, i)
+
+
+def test_int4_quantize_invariants():
+    rng = np.random.default_rng(8)
+    x = rng.normal(size=(64, 128)).astype(np.float32)
+    x[5, :] = 0.75                                     # constant rows: exact
+    x[6, :] = -1e-3
+    codes, pz = oracle.quantize_rows(x, "int4")
+    assert codes.max() <= 15 and codes.dtype == np.uint8
+    deq = oracle.widen(codes, "int4", pz)
+    s = pz[:, 0].astype(np.float64)[:, None]
+    err = np.abs(deq - x.astype(np.float64))
+    assert (err <= s * (1 + 1e-6)).all()               # within one step everywhere
+    inner = (codes > 0) & (codes < 15)
+    assert (err[inner] <= (s * np.ones_like(err))[inner] * (0.5 + 1e-5)).all()  # half a step
+    assert (deq[5] == 0.75).all() and (deq[6] == np.float32(-1e-3)).all()
+    # the extremes land on the ends of the code range (within one step)
+    for r in range(64):
+        if r in (5, 6):
+            continue
+        assert codes[r, np.argmax(x[r])] >= 14 and codes[r, np.argmin(x[r])] <= 1
+    # a power-of-two factor scales the scale and keeps codes and zero point
+    c2, p2 = oracle.quantize_rows(x * np.float32(0.25), "int4")
+    assert (c2 == codes).all() and (p2[:, 1] == pz[:, 1]).all()
+    assert (p2[:, 0] == pz[:, 0] * np.float32(0.25)).all()
+
+
 # ---------------------------------------------------------------- attention
 def _rand_case(rng, b, hq, hkv, d, lens, kv_dtype="f32"):
     total = int(sum(lens))
@@ -236,9 +311,9 @@ def test_attention_matches_bruteforce_numpy(hq, hkv):
     assert np.abs(ours - brute).max() <= 1e-12
 
 
-@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "fp8", "int8"])
+@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "fp8", "int8", "int4"])
 def test_attention_matches_torch_sdpa_float64(kv_dtype):
-    rng = np.random.default_rng({"f32": 1, "bf16": 2, "fp8": 3, "int8": 4}[kv_dtype])
+    rng = np.random.default_rng({"f32": 1, "bf16": 2, "fp8": 3, "int8": 4, "int4": 5}[kv_dtype])
     hq, hkv, d = 8, 2, 64
     lens = [3, 33, 64]
     q, k, v, offs, lens = _rand_case(rng, 3, hq, hkv, d, lens)
@@ -250,6 +325,12 @@ def test_attention_matches_torch_sdpa_float64(kv_dtype):
     elif kv_dtype == "bf16":
         kst, vst = _bf16_bits(k), _bf16_bits(v)
         k64, v64 = oracle.widen(kst, "bf16"), oracle.widen(vst, "bf16")
+    elif kv_dtype == "int4":
+        kst, ks = oracle.quantize_rows(k, "int4")
+        vst, vs = oracle.quantize_rows(v, "int4")
+        # dequantise independently of the oracle: (code - zero) * scale in float64
+        k64 = (kst.astype(np.float64) - ks[..., 1:2].astype(np.float64)) * ks[..., 0:1]
+        v64 = (vst.astype(np.float64) - vs[..., 1:2].astype(np.float64)) * vs[..., 0:1]
     elif kv_dtype == "int8":
         kst, ks = oracle.quantize_rows(k, "int8")
         vst, vs = oracle.quantize_rows(v, "int8")
