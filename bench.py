@@ -168,6 +168,8 @@ class ClockSampler:
 def kv_row_bytes(spec) -> int:
     """Bytes of one stored K or V row of one KV head (plus its fp32 scale for
     an 8-bit cache)."""
+    if spec.kv_dtype == "int4":    # two codes per byte + fp32 (scale, zero point)
+        return spec.head_dim // 2 + 8
     elem = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[spec.kv_dtype]
     return spec.head_dim * elem + (4 if spec.kv_dtype in ("fp8", "int8") else 0)
 
@@ -247,7 +249,7 @@ def time_oracle(inp, max_seqs: int, repeats: int = 1):
     lens = inp.context_lens[seqs]
     args = dict(seq_offsets=inp.seq_offsets[seqs], lens=lens, scale=spec.scale,
                 num_kv_heads=spec.num_kv_heads, q_dtype=spec.q_dtype)
-    if spec.kv_dtype in ("fp8", "int8"):
+    if spec.kv_dtype in ("fp8", "int8", "int4"):
         rows = slice(int(inp.seq_offsets[0]), int(inp.seq_offsets[n - 1] + lens[-1]))
         kc, ks = oracle.quantize_rows(inp.k[rows].float().numpy(), spec.kv_dtype)
         vc, vs = oracle.quantize_rows(inp.v[rows].float().numpy(), spec.kv_dtype)

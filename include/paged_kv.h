@@ -62,7 +62,9 @@ typedef enum {
     KV_F32 = 0,        /* IEEE binary32 */
     KV_BF16 = 1,       /* bfloat16 */
     KV_FP8_E4M3 = 2,   /* OCP FP8 E4M3 codes (KV pools only) with fp32 row scales */
-    KV_INT8 = 3        /* signed 8-bit codes (KV pools only) with fp32 row scales */
+    KV_INT8 = 3,       /* signed 8-bit codes (KV pools only) with fp32 row scales */
+    KV_INT4 = 4        /* unsigned 4-bit codes, two per byte (KV pools only, head_dim 128),
+                          with an fp32 (scale, zero point) pair per row */
 } kv_dtype;
 
 /* Bits ORed into *dev_error by the kernels. */
@@ -80,7 +82,10 @@ typedef enum {
  * span of block_size*head_dim elements.  A quantised cache (FP8 or INT8) also
  * has ONE fp32 scale pool laid out [num_blocks][num_kv_heads][2][block_size]:
  * for each (block, kv head) the 16 K row scales then the 16 V row scales, 128
- * contiguous bytes.
+ * contiguous bytes.  An INT4 pool stores a row's 128 codes in 64 bytes (dim
+ * 2i in the low nibble of byte i, dim 2i+1 in the high nibble) and has one
+ * fp32 parameter pool [num_blocks][num_kv_heads][2][block_size][2]: per row
+ * (scale, zero point), K rows then V rows, 256 bytes per (block, kv head).
  */
 typedef struct {
     int32_t num_blocks;
@@ -88,9 +93,9 @@ typedef struct {
     int32_t num_kv_heads;
     int32_t head_dim;        /* 64 or 128 */
     int32_t dtype;           /* kv_dtype */
-    int32_t elem_bytes;      /* 4, 2 or 1 */
+    int32_t elem_bytes;      /* 4, 2 or 1; 0 for 4-bit codes (two per byte) */
     uint64_t kv_bytes;       /* bytes of ONE pool (K or V) */
-    uint64_t scale_bytes;    /* bytes of the scale pool (FP8 / INT8 only, else 0) */
+    uint64_t scale_bytes;    /* bytes of the scale / parameter pool (FP8, INT8, INT4; else 0) */
     int64_t stride_block;    /* elements between consecutive physical blocks */
     int64_t stride_head;     /* elements between consecutive kv heads of a block */
     int64_t stride_slot;     /* elements between consecutive tokens of a block */
@@ -100,7 +105,7 @@ typedef struct {
  * Fill *out with the geometry of a pool (host only, no device work).
  * Errors: KV_ERR_INVALID_ARGUMENT for out == NULL or non-positive sizes;
  * KV_ERR_UNSUPPORTED for block_size != 16, head_dim not in {64, 128},
- * num_kv_heads > 256 or an unknown dtype.
+ * num_kv_heads > 256, an unknown dtype, or KV_INT4 with head_dim != 128.
  */
 KV_API kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
                          int32_t head_dim, kv_dtype dtype, kv_pool_desc* out);
@@ -142,8 +147,20 @@ KV_API kv_status compute_slot_mapping(const int32_t* block_table, int32_t batch,
  *     a = max |x|,  scale = a / 127 (IEEE fp32 division),
  *     code = clamp(round_to_nearest_even(x / scale), -127, 127),
  *     and scale = 0, codes 0 when a == 0.
+ * INT4 pools ("llm-inference-optimization" notes §四: the printed 4-bit
+ * routine, asymmetric with a zero point, applied to each row; "大模型推理为何
+ * 这么慢", KV Cache量化: a 4-bit cache is 4x smaller than fp16): src_dtype F32
+ * or BF16; for each row, in IEEE fp32
+ *     hi = max x, lo = min x,  scale = (hi - lo) / 15,
+ *     zero = round_to_nearest_even(-lo / scale),
+ *     code = clamp(round_to_nearest_even(x / scale) + zero, 0, 15),
+ *     value = (code - zero) * scale;
+ *     a constant row (hi == lo), where the routine would divide by zero, is
+ *     stored exactly: scale = |lo|, zero = -1 (lo > 0), +1 (lo < 0) or 0 (with
+ *     scale 0, lo == 0), every code 0.
  *   scales : device fp32 scale pool [num_blocks][num_kv_heads][2][16] (K row
- *   scales, then V row scales), NULL for F32/BF16 pools.  Rows must be finite.
+ *   scales, then V row scales), or for INT4 the parameter pool above; NULL for
+ *   F32/BF16 pools.  Rows must be finite.
  * Two tokens given the same slot race (last writer unspecified).
  */
 KV_API kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool,
@@ -194,7 +211,8 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  *   out          : device [batch][num_q_heads][head_dim] in q_dtype
  *   q            : device [batch][num_q_heads][head_dim], q_dtype F32 or BF16
  *   k_pool/v_pool: device pools (layout above)
- *   scales       : device fp32 scale pool (layout above), non-NULL iff the pool is FP8/INT8
+ *   scales       : device fp32 scale / parameter pool (layout above), non-NULL iff the
+ *                  pool is FP8, INT8 or INT4
  *   block_table  : device int32 [batch][max_blocks_per_seq]; entries past
  *                  ceil(L/16) are never read
  *   context_lens : device int32 [batch], each in [1, max_context_len]
@@ -205,8 +223,9 @@ KV_API size_t paged_decode_workspace_bytes(const kv_pool_desc* pool, int32_t bat
  * Host checks: num_q_heads % num_kv_heads == 0 with a group size of 1, 2, 4
  * or 8 (else KV_ERR_UNSUPPORTED); partition_tokens a multiple of 16;
  * max_context_len <= max_blocks_per_seq * 16; batch * num_kv_heads *
- * ceil(max_context_len / 16) < 2^31 (else KV_ERR_UNSUPPORTED); pointer
- * alignment; workspace size.  Device errors: KV_DEVERR_BAD_CONTEXT_LEN (that sequence's output is
+ * ceil(max_context_len / 16) < 2^31 (else KV_ERR_UNSUPPORTED); an INT4
+ * pool needs bf16 q (else KV_ERR_UNSUPPORTED); pointer alignment;
+ * workspace size.  Device errors: KV_DEVERR_BAD_CONTEXT_LEN (that sequence's output is
  * zero), KV_DEVERR_BAD_BLOCK_ID (that block's tokens are skipped),
  * KV_DEVERR_TIMEOUT.
  */
@@ -266,7 +285,7 @@ KV_API kv_status paged_decode_attention_append(const kv_pool_desc* pool, void* o
  * positions 0 .. L - Q + i (causal), with the softmax of paged_decode_attention.
  *   q, out : device [batch][Q][num_q_heads][head_dim] (q_dtype; out in q_dtype)
  * Everything else as paged_decode_attention (Q = 1 is exactly that call).
- * Supported shapes: bf16, FP8 or INT8 KV, head_dim 128, bf16 q, and
+ * Supported shapes: bf16, FP8, INT8 or INT4 KV, head_dim 128, bf16 q, and
  * (num_q_heads / num_kv_heads) * Q <= 16, else KV_ERR_UNSUPPORTED.  A context
  * length below Q is invalid (zeros, KV_DEVERR_BAD_CONTEXT_LEN).
  */

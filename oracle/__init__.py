@@ -147,9 +147,10 @@ def scatter_to_pool(pool: np.ndarray, rows: np.ndarray, slots: np.ndarray,
 
 def scatter_scales_to_pool(scale_pool: np.ndarray, scales: np.ndarray, slots: np.ndarray,
                            which: int, block_size: int = 16) -> np.ndarray:
-    """Expected FP8 scale pool after a write: the pool is laid out
+    """Expected scale pool after a write: the pool is laid out
     [num_blocks][kv_heads][2][block_size] (K row scales, then V row scales, of
-    each (block, kv head)); ``which`` is 0 for K, 1 for V.  scales: [T][kv_heads]."""
+    each (block, kv head)); ``which`` is 0 for K, 1 for V.  scales: [T][kv_heads].
+    INT4 parameter pools carry a trailing (scale, zero) axis on both."""
     out = scale_pool.copy()
     for t, slot in enumerate(slots.tolist()):
         if slot < 0:

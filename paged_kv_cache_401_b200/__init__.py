@@ -17,8 +17,9 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
 
-KV_F32, KV_BF16, KV_FP8_E4M3, KV_INT8 = 0, 1, 2, 3
-QUANTIZED = (KV_FP8_E4M3, KV_INT8)   # pools of 8-bit codes with fp32 row scales
+KV_F32, KV_BF16, KV_FP8_E4M3, KV_INT8, KV_INT4 = 0, 1, 2, 3, 4
+# pools of codes with per-row parameters: fp32 scales (8-bit), (scale, zero) pairs (4-bit)
+QUANTIZED = (KV_FP8_E4M3, KV_INT8, KV_INT4)
 KV_OK, KV_ERR_INVALID_ARGUMENT, KV_ERR_UNSUPPORTED, KV_ERR_CUDA = 0, 1, 2, 3
 KV_ERR_OUT_OF_BLOCKS = 4
 KV_DEVERR_BAD_SLOT = 0x1
@@ -157,17 +158,21 @@ def kv_pool_create(num_blocks: int, block_size: int, num_kv_heads: int, head_dim
 
 def empty_pool(desc: KvPoolDesc, device, fill: float | int | None = None):
     """Allocate (k_pool, v_pool, scales) tensors for a descriptor: pools
-    [num_blocks][kv_heads][16][head_dim]; scales [num_blocks][kv_heads][2][16]
-    fp32 (K then V row scales) for FP8 / INT8, else None.  ``fill`` poisons every
-    element (NaN, or a byte; scales get NaN)."""
-    shape = (desc.num_blocks, desc.num_kv_heads, desc.block_size, desc.head_dim)
+    [num_blocks][kv_heads][16][head_dim] (INT4: [..][head_dim / 2] bytes, two
+    codes each); scales [num_blocks][kv_heads][2][16] fp32 (K then V row
+    scales) for FP8 / INT8, [num_blocks][kv_heads][2][16][2] (scale, zero) for
+    INT4, else None.  ``fill`` poisons every element (NaN, or a byte; scales
+    get NaN)."""
+    cols = desc.head_dim // 2 if desc.dtype == KV_INT4 else desc.head_dim
+    shape = (desc.num_blocks, desc.num_kv_heads, desc.block_size, cols)
     dt = {KV_F32: torch.float32, KV_BF16: torch.bfloat16, KV_FP8_E4M3: torch.uint8,
-          KV_INT8: torch.int8}[desc.dtype]
+          KV_INT8: torch.int8, KV_INT4: torch.uint8}[desc.dtype]
     k = torch.empty(shape, dtype=dt, device=device)
     v = torch.empty(shape, dtype=dt, device=device)
     scales = None
     if desc.dtype in QUANTIZED:
-        scales = torch.empty((desc.num_blocks, desc.num_kv_heads, 2, desc.block_size),
+        extra = (2,) if desc.dtype == KV_INT4 else ()
+        scales = torch.empty((desc.num_blocks, desc.num_kv_heads, 2, desc.block_size) + extra,
                              dtype=torch.float32, device=device)
     if fill is not None:
         for t in (k, v):

@@ -9,12 +9,14 @@ from __future__ import annotations
 
 import torch
 
-from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, KV_INT8, compute_slot_mapping, empty_pool,
+from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, KV_INT4, KV_INT8, compute_slot_mapping,
+               empty_pool,
                kv_pool_create, paged_attention_multi_query, paged_attention_workspace_bytes,
                paged_decode_attention, paged_decode_attention_append,
                paged_decode_workspace_bytes, reshape_and_cache)
 
-_DTYPES = {"f32": KV_F32, "bf16": KV_BF16, "fp8": KV_FP8_E4M3, "int8": KV_INT8}
+_DTYPES = {"f32": KV_F32, "bf16": KV_BF16, "fp8": KV_FP8_E4M3, "int8": KV_INT8,
+           "int4": KV_INT4}
 
 
 class PagedKVCache:
@@ -25,7 +27,7 @@ class PagedKVCache:
         self.desc = kv_pool_create(num_blocks, BLOCK_SIZE, num_kv_heads, head_dim, _DTYPES[dtype])
         fill = None
         if poison:
-            fill = 0x7F if dtype in ("fp8", "int8") else float("nan")
+            fill = 0x7F if dtype in ("fp8", "int8", "int4") else float("nan")
         self.k_pool, self.v_pool, self.scales = empty_pool(self.desc, self.device, fill)
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
 

@@ -13,15 +13,32 @@ using pkv::kBlockTokens;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-int32_t elem_bytes(int32_t dtype) {
+// Bits of one stored K/V element; 0 for an unknown dtype.
+int32_t kv_bits(int32_t dtype) {
     switch (dtype) {
-        case KV_F32: return 4;
-        case KV_BF16: return 2;
-        case KV_FP8_E4M3: return 1;
-        case KV_INT8: return 1;
+        case KV_F32: return 32;
+        case KV_BF16: return 16;
+        case KV_FP8_E4M3: return 8;
+        case KV_INT8: return 8;
+        case KV_INT4: return 4;
         default: return 0;
     }
 }
+
+// The descriptor's elem_bytes: 0 for 4-bit codes (two per byte).
+int32_t elem_bytes(int32_t dtype) { return kv_bits(dtype) / 8; }
+
+// Bytes of one stored row (one token, one kv head) of a pool.
+int64_t row_bytes(const kv_pool_desc* d) {
+    return static_cast<int64_t>(d->head_dim) * kv_bits(d->dtype) / 8;
+}
+
+// Pools of codes with per-(token, kv head) parameters: one fp32 scale (FP8,
+// INT8) or an fp32 (scale, zero point) pair (INT4).
+bool quantized(int32_t dtype) {
+    return dtype == KV_FP8_E4M3 || dtype == KV_INT8 || dtype == KV_INT4;
+}
+int32_t param_bytes(int32_t dtype) { return dtype == KV_INT4 ? 8 : (quantized(dtype) ? 4 : 0); }
 
 // SM count of the current device; 148 (B200) when no device can be queried.
 int32_t current_sm_count() {
@@ -37,13 +54,12 @@ int32_t current_sm_count() {
 bool valid_pool(const kv_pool_desc* d) {
     return d != nullptr && d->num_blocks > 0 && d->block_size == kBlockTokens &&
            d->num_kv_heads > 0 && (d->head_dim == 64 || d->head_dim == 128) &&
-           elem_bytes(d->dtype) == d->elem_bytes;
+           kv_bits(d->dtype) != 0 && elem_bytes(d->dtype) == d->elem_bytes &&
+           (d->dtype != KV_INT4 || d->head_dim == 128);
 }
 
 int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
 
-// Pools of codes with a per-(token, kv head) fp32 scale.
-bool quantized(int32_t dtype) { return dtype == KV_FP8_E4M3 || dtype == KV_INT8; }
 
 // The driver's tensor-map encoder, looked up once through the runtime (no libcuda link).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
@@ -61,23 +77,29 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// A pool as a 2-D tensor [num_blocks*Hkv*16 rows][head_dim], 16-row x 128-byte
-// boxes, 128-byte swizzle.  Returns a kv_status.
+// A pool as a 2-D tensor [num_blocks*Hkv*16 rows][head_dim]: 16-row x 128-byte
+// boxes with the 128-byte swizzle; 4-bit pools (64-byte rows of packed codes,
+// as bytes) use 16-row x 64-byte boxes with the 64-byte swizzle.  Returns a
+// kv_status.
 kv_status encode_pool_map(CUtensorMap* map, const void* base, const kv_pool_desc* pool) {
     const PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
     if (encode == nullptr) return KV_ERR_CUDA;
     const cuuint64_t rows = static_cast<cuuint64_t>(pool->num_blocks) * pool->num_kv_heads *
                             kBlockTokens;
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pool->head_dim), rows};
-    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(pool->head_dim) * pool->elem_bytes};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / pool->elem_bytes),
+    const bool int4 = pool->dtype == KV_INT4;
+    const int64_t rb = row_bytes(pool);
+    const cuuint64_t dims[2] = {int4 ? static_cast<cuuint64_t>(rb)
+                                     : static_cast<cuuint64_t>(pool->head_dim), rows};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
+    const cuuint32_t box[2] = {int4 ? 64u : static_cast<cuuint32_t>(128 / pool->elem_bytes),
                                static_cast<cuuint32_t>(kBlockTokens)};
     const cuuint32_t elem_strides[2] = {1, 1};
     const CUtensorMapDataType type = pool->dtype == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
                                                             : CU_TENSOR_MAP_DATA_TYPE_UINT8;
     const CUresult r = encode(map, type, 2, const_cast<void*>(base), dims, strides, box,
                               elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              int4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? KV_OK : KV_ERR_INVALID_ARGUMENT;
 }
@@ -91,7 +113,7 @@ kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_
     if (out == nullptr || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
         return KV_ERR_INVALID_ARGUMENT;
     if (block_size != kBlockTokens || (head_dim != 64 && head_dim != 128) || num_kv_heads > 256 ||
-        elem_bytes(dtype) == 0)
+        kv_bits(dtype) == 0 || (dtype == KV_INT4 && head_dim != 128))
         return KV_ERR_UNSUPPORTED;
     kv_pool_desc d{};
     d.num_blocks = num_blocks;
@@ -103,10 +125,9 @@ kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_
     d.stride_slot = head_dim;
     d.stride_head = static_cast<int64_t>(block_size) * head_dim;
     d.stride_block = d.stride_head * num_kv_heads;
-    d.kv_bytes = static_cast<uint64_t>(d.stride_block) * num_blocks * d.elem_bytes;
-    d.scale_bytes = quantized(dtype)
-                        ? static_cast<uint64_t>(num_blocks) * num_kv_heads * 2u * block_size * 4u
-                        : 0u;
+    d.kv_bytes = static_cast<uint64_t>(d.stride_block) * num_blocks * kv_bits(dtype) / 8u;
+    d.scale_bytes = static_cast<uint64_t>(num_blocks) * num_kv_heads * 2u * block_size *
+                    static_cast<uint64_t>(param_bytes(dtype));
     *out = d;
     return KV_OK;
 }
@@ -152,7 +173,7 @@ kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool
         if (src_dtype != pool->dtype) return KV_ERR_UNSUPPORTED;
         if (scales != nullptr) return KV_ERR_INVALID_ARGUMENT;
         e = pkv::launch_cache_copy(k_pool, v_pool, k_new, v_new, slot_mapping, num_tokens,
-                                   pool->num_kv_heads, pool->head_dim * pool->elem_bytes,
+                                   pool->num_kv_heads, static_cast<int32_t>(row_bytes(pool)),
                                    num_slots, current_sm_count(), dev_error, s);
     }
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
@@ -166,10 +187,11 @@ kv_status paged_kv_copy_blocks(const kv_pool_desc* pool, void* k_pool, void* v_p
     if (k_pool == nullptr || v_pool == nullptr || copy_src == nullptr || copy_dst == nullptr)
         return KV_ERR_INVALID_ARGUMENT;
     if (!aligned16(k_pool) || !aligned16(v_pool)) return KV_ERR_INVALID_ARGUMENT;
-    const bool fp8 = quantized(pool->dtype);  // FP8 or INT8: a scale pool
+    const bool fp8 = quantized(pool->dtype);  // FP8, INT8 or INT4: a parameter pool
     if (fp8 != (scales != nullptr) || (fp8 && !aligned16(scales))) return KV_ERR_INVALID_ARGUMENT;
-    const int64_t block_bytes = pool->stride_block * pool->elem_bytes;
-    const int64_t scale_bytes = fp8 ? static_cast<int64_t>(pool->num_kv_heads) * 2 * kBlockTokens * 4 : 0;
+    const int64_t block_bytes = row_bytes(pool) * kBlockTokens * pool->num_kv_heads;
+    const int64_t scale_bytes =
+        static_cast<int64_t>(pool->num_kv_heads) * 2 * kBlockTokens * param_bytes(pool->dtype);
     cudaError_t e = pkv::launch_copy_blocks(k_pool, v_pool, scales, copy_src, copy_dst,
                                             num_copies, block_bytes, scale_bytes,
                                             pool->num_blocks, dev_error,
@@ -265,6 +287,9 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
     if (query_tokens > 1 && (!pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim) ||
                              group * query_tokens > 16))
         return KV_ERR_UNSUPPORTED;
+    // 4-bit codes have only the tensor-core tile (bf16 q, head_dim 128)
+    if (pool->dtype == KV_INT4 && !pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim))
+        return KV_ERR_UNSUPPORTED;
     if (batch == 0) return KV_OK;
     if (max_context_len < query_tokens ||
         static_cast<int64_t>(max_context_len) > static_cast<int64_t>(max_blocks_per_seq) * kBlockTokens)
@@ -281,7 +306,7 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
         return KV_ERR_INVALID_ARGUMENT;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
         return KV_ERR_INVALID_ARGUMENT;
-    const bool fp8 = quantized(pool->dtype);  // FP8 or INT8: a scale pool
+    const bool fp8 = quantized(pool->dtype);  // FP8, INT8 or INT4: a parameter pool
     if (fp8 != (scales != nullptr)) return KV_ERR_INVALID_ARGUMENT;
     if (fp8 && !aligned16(scales)) return KV_ERR_INVALID_ARGUMENT;
     if (app != nullptr && (app->k_new == nullptr || app->v_new == nullptr ||

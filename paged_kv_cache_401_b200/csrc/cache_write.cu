@@ -66,8 +66,9 @@ __global__ void cache_copy_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restr
 }
 
 // Quantising write: one warp per (token, kv head, K|V) row of D elements; the
-// codes and scale come from quantize_row_warp (FP8: absmax/448, E4M3; INT8:
-// absmax/127, round to nearest even, clamp to 127).
+// codes and parameters come from quant.cuh (FP8: absmax/448, E4M3; INT8:
+// absmax/127, round to nearest even, clamp to 127; INT4: asymmetric scale and
+// zero point, two codes per byte).
 template <int KV_T, int SRC_T, int D>
 __global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
                                    float* __restrict__ scales,
@@ -95,13 +96,23 @@ __global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __rest
     float x[kPer];
     const uint8_t* src = static_cast<const uint8_t*>(which ? v_new : k_new);
     load_row_part<D>(src + th * D * kSrcBytes, SRC_T, lane, x);
-    float s;
-    const uint32_t codes = quantize_row_warp<KV_T, D>(x, &s);
     const int64_t blk = slot / kBlockTokens, off = slot % kBlockTokens;
     const int64_t rowi = (blk * num_kv_heads + h) * kBlockTokens + off;
-    store_codes<D>((which ? v_pool : k_pool) + rowi * D + lane * kPer, codes);
-    // scale pool [block][head][K|V][16]: one 128-byte line per (block, head)
-    if (lane == 0) scales[((blk * num_kv_heads + h) * 2 + which) * kBlockTokens + off] = s;
+    const int64_t pidx = ((blk * num_kv_heads + h) * 2 + which) * kBlockTokens + off;
+    if constexpr (KV_T == KV_INT4) {
+        // 64-byte rows, 2 bytes per lane; parameter pool [block][head][K|V][16][scale, zero]
+        float s, z;
+        const uint32_t codes = quantize_row_int4_warp<D>(x, &s, &z);
+        *reinterpret_cast<uint16_t*>((which ? v_pool : k_pool) + rowi * (D / 2) + lane * 2) =
+            static_cast<uint16_t>(codes);
+        if (lane == 0) reinterpret_cast<float2*>(scales)[pidx] = make_float2(s, z);
+    } else {
+        float s;
+        const uint32_t codes = quantize_row_warp<KV_T, D>(x, &s);
+        store_codes<D>((which ? v_pool : k_pool) + rowi * D + lane * kPer, codes);
+        // scale pool [block][head][K|V][16]: one 128-byte line per (block, head)
+        if (lane == 0) scales[pidx] = s;
+    }
 }
 
 // Whole-block copies (copy-on-write of shared blocks): CTA (pair, part) moves
@@ -188,6 +199,9 @@ cudaError_t launch_cache_quant(int32_t kv_dtype, int32_t src_dtype, int32_t head
                           num_slots, dev_error);
     };
     const bool f32 = src_dtype == KV_F32, d128 = head_dim == 128;
+    if (kv_dtype == KV_INT4)  // head_dim 128 only
+        return f32 ? go(cache_quant_kernel<KV_INT4, KV_F32, 128>)
+                   : go(cache_quant_kernel<KV_INT4, KV_BF16, 128>);
     if (kv_dtype == KV_INT8) {
         if (f32) return d128 ? go(cache_quant_kernel<KV_INT8, KV_F32, 128>)
                              : go(cache_quant_kernel<KV_INT8, KV_F32, 64>);

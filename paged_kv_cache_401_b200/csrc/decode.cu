@@ -64,10 +64,15 @@ template <>
 struct KvElem<KV_INT8> {
     static constexpr int kBytes = 1;
 };
+template <>
+struct KvElem<KV_INT4> {  // two codes per byte: row sizes are computed from bits instead
+    static constexpr int kBytes = 0;
+};
 
-// 8-bit code pools carry a per-(token, kv head) fp32 scale line.
+// Quantised pools carry per-(token, kv head) parameters: an fp32 scale (8-bit
+// codes) or an fp32 (scale, zero point) pair (4-bit codes).
 template <int KV_T>
-inline constexpr bool kQuantized = KV_T == KV_FP8_E4M3 || KV_T == KV_INT8;
+inline constexpr bool kQuantized = KV_T == KV_FP8_E4M3 || KV_T == KV_INT8 || KV_T == KV_INT4;
 
 // Two 8-bit codes (low 16 bits) -> two floats (code values, before the row scale).
 template <int KV_T>
@@ -265,6 +270,23 @@ __device__ __forceinline__ void widen_v4(uint32_t w, uint32_t& lo, uint32_t& hi)
     else e4m3x4_to_f16x2x2(__byte_perm(w, 0u, 0x3120), lo, hi);
 }
 
+// Eight 4-bit codes c (one 32-bit word, nibble i = element i) -> four f16x2 of
+// exact values c * 2^-9: the byte 0x0c is the E4M3 code of c * 2^-9 for every c
+// in 0..15 (subnormals and the first binade share the step 2^-9).
+// out = {(e0, e2), (e4, e6), (e1, e3), (e5, e7)}.
+__device__ __forceinline__ void nib8_to_f16x2x4(uint32_t w, uint32_t* out) {
+    e4m3x4_to_f16x2x2(w & 0x0F0F0F0Fu, out[0], out[1]);
+    e4m3x4_to_f16x2x2((w >> 4) & 0x0F0F0F0Fu, out[2], out[3]);
+}
+
+// A transposed ldmatrix word of a 4-bit V tile: 16-bit units of two tokens t0
+// (low half) and t1, each four dims d0..d3 -> {(t0 d0, t1 d0), (t0 d2, t1 d2),
+// (t0 d1, t1 d1), (t0 d3, t1 d3)} as f16x2 of c * 2^-9.
+__device__ __forceinline__ void nib8t_to_f16x2x4(uint32_t w, uint32_t* out) {
+    e4m3x4_to_f16x2x2(__byte_perm(w & 0x0F0F0F0Fu, 0u, 0x3120), out[0], out[1]);
+    e4m3x4_to_f16x2x2(__byte_perm((w >> 4) & 0x0F0F0F0Fu, 0u, 0x3120), out[2], out[3]);
+}
+
 // 2-D TMA tile load (no multicast) completing on an mbarrier; x is the
 // innermost coordinate in elements (always 0 or a multiple of 16 bytes here).
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x,
@@ -387,7 +409,8 @@ struct SimtMath {
     static constexpr int kHeadDim = D;
     static constexpr bool kCanAppend = true;                                 // one query token
     static constexpr int kElem = KvElem<KV_T>::kBytes;
-    static constexpr int kTileBytes = kBlockTokens * D * kElem;              // K or V tile
+    static constexpr int kRowBytes = D * kElem;
+    static constexpr int kTileBytes = kBlockTokens * kRowBytes;              // K or V tile
     static constexpr int kScaleBytes = kQuantized<KV_T> ? 2 * kBlockTokens * 4 : 0;  // K|V
     static constexpr int kStageBytes = 2 * kTileBytes + kScaleBytes;
     static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
@@ -639,24 +662,26 @@ template <int KV_T, int G, int QM>
 struct MmaMath {
     static constexpr bool WIDE = QM == kWide;
     static constexpr bool SINGLE = QM == kSingle;
-    static_assert(KV_T == KV_BF16 || kQuantized<KV_T>, "bf16, FP8 or INT8 KV");
+    static_assert(KV_T == KV_BF16 || kQuantized<KV_T>, "bf16, FP8, INT8 or INT4 KV");
     static_assert(G <= 8, "a row set holds 8 query rows");
     using OutT = uint16_t;                                        // bf16 output
-    static constexpr bool kF16 = kQuantized<KV_T>;              // 8-bit codes widened to f16
+    static constexpr bool kF16 = kQuantized<KV_T>;              // codes widened to f16
+    static constexpr bool kI4 = KV_T == KV_INT4;                // 4-bit codes, 64-byte rows
     static constexpr int D = 128;
     static constexpr int kKv = KV_T;
     static constexpr int kHeadDim = D;
     static constexpr bool kCanAppend = SINGLE;                    // fused append: decode only
     static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
-    static constexpr int kElem = KvElem<KV_T>::kBytes;
-    static constexpr int kRowBytes = D * kElem;                   // 256 (bf16) / 128 (8-bit)
-    static constexpr int kBoxCols = 128 / kElem;                  // elements per 128-byte box row
-    static constexpr int kBoxes = kRowBytes / 128;
-    static constexpr int kBoxBytes = kBlockTokens * 128;
+    static constexpr int kRowBytes = kI4 ? D / 2 : D * KvElem<KV_T>::kBytes;  // 256 / 128 / 64
+    static constexpr int kBoxRow = kI4 ? 64 : 128;                // bytes of a TMA box row
+    static constexpr int kBoxCols = kI4 ? 64 : 128 / (KvElem<KV_T>::kBytes + kI4);  // box row, elements
+    static constexpr int kBoxes = kRowBytes / kBoxRow;
+    static constexpr int kBoxBytes = kBlockTokens * kBoxRow;
     static constexpr int kTileBytes = kBlockTokens * kRowBytes;
-    static constexpr int kScaleBytes = kF16 ? 2 * kBlockTokens * 4 : 0;  // K then V row scales
+    // K then V row parameters: fp32 scales (8-bit) or fp32 (scale, zero) pairs (4-bit)
+    static constexpr int kScaleBytes = kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0);
     static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
-    static constexpr int kStages = kF16 ? 12 : 8;                 // multiple of 4
+    static constexpr int kStages = kI4 ? 16 : (kF16 ? 12 : 8);     // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr int kWarpScratch = 0;
     static constexpr int kMinBlocks = WIDE ? 2 : 3;
@@ -672,7 +697,7 @@ struct MmaMath {
             tma_load_2d(st + kTileBytes + bx * kBoxBytes, &maps.v, bx * kBoxCols, row, bar);
         }
         if constexpr (kF16)
-            bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
+            bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * (kScaleBytes / 4), kScaleBytes, bar);
     }
 
     // Byte offset of byte `byte` of row `row` in a staged (swizzled) K or V tile.
@@ -680,13 +705,20 @@ struct MmaMath {
         return static_cast<int32_t>(swz(row, byte >> 4)) + (byte & 15);
     }
 
-    // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile.
+    // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile:
+    // the 128-byte swizzle (chunk ^ row % 8 within 128-byte rows), or for 4-bit
+    // tiles the 64-byte swizzle (chunk ^ (row / 2) % 4 within 64-byte rows).
     __device__ static __forceinline__ uint32_t swz(int32_t row, int32_t chunk) {
+        if constexpr (kI4) return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
         return (chunk >> 3) * kBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
     }
 
-    // head-dim of row r (0..15) of output m-tile mi: 8-bit tiles interleave even/odd dims
+    // head-dim of row r (0..15) of output m-tile mi: 8-bit tiles interleave even/odd
+    // dims; 4-bit m-tile (c, j) = (mi / 2, mi % 2) holds dims 32c + 4r' + 2j (+1 for
+    // r >= 8), r' = r % 8 (the nibble order of a transposed 16-bit unit)
     __device__ static __forceinline__ int32_t dim_of(int32_t mi, int32_t r) {
+        if constexpr (kI4)
+            return 32 * (mi >> 1) + 4 * (r & 7) + 2 * (mi & 1) + (r >> 3);
         if constexpr (kF16) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
         return 16 * mi + r;
     }
@@ -697,6 +729,8 @@ struct MmaMath {
     uint32_t qa[kSets][8][2];   // A fragments of q per 16-dim k-step, row gid + 8k: {k lo, k hi}
     float o[kSets][8][4];       // O^T: [set][m-tile][c]; c0,c1 = (dim gid, rows 8k+2tig, +1)
     float m_run[kSets], l_run[kSets];  // running max (base 2), lane part of the sum, row gid+8k
+    float qsum[kSets];          // 4-bit: sum of row gid+8k's q (as rounded to f16)
+    float b_run[kSets];         // 4-bit: lane part of sum_t p_t * scale_t * zero_t, row gid+8k
 
     __device__ void init(int32_t lane_, uint8_t*) {
         lane = lane_;
@@ -714,10 +748,25 @@ struct MmaMath {
             const uint16_t* q = static_cast<const uint16_t*>(p.q) +
                                 ((static_cast<int64_t>(b) * nq + (r / G)) * p.num_q_heads +
                                  kvh * G + r % G) * D;
+            float qs = 0.0f;
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 if (r >= rows) {
                     qa[k][ks][0] = qa[k][ks][1] = 0u;
+                } else if constexpr (kI4) {
+                    // 4-bit rows: a lane's ldmatrix word is dims 32c + 8tig + 0..7 of chunk c;
+                    // k-step 2c takes dims (+0,+2 | +4,+6), k-step 2c+1 (+1,+3 | +5,+7)
+                    const uint4 w = *reinterpret_cast<const uint4*>(q + 32 * (ks >> 1) + 8 * tig);
+                    const uint32_t x[4] = {w.x, w.y, w.z, w.w};  // bf16 pairs (0,1) (2,3) ...
+                    const int h = ks & 1;
+                    auto el = [&](int d) {  // element d (0..7) of the lane's 8 dims as float
+                        return __uint_as_float((d & 1) ? (x[d >> 1] & 0xffff0000u) : (x[d >> 1] << 16));
+                    };
+                    qa[k][ks][0] = pack2<true>(el(h), el(h + 2));
+                    qa[k][ks][1] = pack2<true>(el(h + 4), el(h + 6));
+                    const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
+                    const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
+                    qs += (f0.x + f0.y) + (f1.x + f1.y);
                 } else if constexpr (!kF16) {
                     // k index 2tig+{0,1} -> dim 16ks+2tig+{0,1}; 8+2tig+{0,1} -> 16ks+8+2tig+{0,1}
                     qa[k][ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
@@ -732,6 +781,11 @@ struct MmaMath {
                                                __uint_as_float(w.y & 0xffff0000u));
                 }
             }
+            if constexpr (kI4) {
+                qs += __shfl_xor_sync(0xffffffffu, qs, 1);
+                qs += __shfl_xor_sync(0xffffffffu, qs, 2);
+                qsum[k] = qs;
+            }
         }
     }
 
@@ -740,6 +794,7 @@ struct MmaMath {
         for (int k = 0; k < kSets; ++k) {
             m_run[k] = -INFINITY;
             l_run[k] = 0.0f;
+            b_run[k] = 0.0f;
 #pragma unroll
             for (int mi = 0; mi < 8; ++mi)
 #pragma unroll
@@ -762,7 +817,25 @@ struct MmaMath {
             if constexpr (WIDE) return qa[1][ks][h];
             return 0u;
         };
-        if constexpr (!kF16) {
+        if constexpr (kI4) {
+#pragma unroll
+            for (int cq = 0; cq < 2; ++cq) {
+                uint32_t w[4];  // {(tokens 0-7, chunk 2cq), (8-15, 2cq), (0-7, 2cq+1), (8-15, 2cq+1)}
+                ldsm_x4(w, k_s + swz(8 * (mtx & 1) + r, 2 * cq + (mtx >> 1)));
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * cq + cc;  // 32-dim chunk: k-steps 2c and 2c + 1
+                    uint32_t b0[4], b1[4];      // n-tiles 0 / 1: {(d0,d2), (d4,d6), (d1,d3), (d5,d7)}
+                    nib8_to_f16x2x4(w[2 * cc], b0);
+                    nib8_to_f16x2x4(w[2 * cc + 1], b1);
+                    const int ka = 2 * c, kb = 2 * c + 1;
+                    mma_16816<true>(s[0], qa[0][ka][0], a_hi(ka, 0), qa[0][ka][1], a_hi(ka, 1), b0[0], b0[1]);
+                    mma_16816<true>(s[1], qa[0][ka][0], a_hi(ka, 0), qa[0][ka][1], a_hi(ka, 1), b1[0], b1[1]);
+                    mma_16816<true>(s[0], qa[0][kb][0], a_hi(kb, 0), qa[0][kb][1], a_hi(kb, 1), b0[2], b0[3]);
+                    mma_16816<true>(s[1], qa[0][kb][0], a_hi(kb, 0), qa[0][kb][1], a_hi(kb, 1), b1[2], b1[3]);
+                }
+            }
+        } else if constexpr (!kF16) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 uint32_t b[4];  // {nt0 dims lo, nt0 dims hi, nt1 dims lo, nt1 dims hi}
@@ -800,8 +873,15 @@ struct MmaMath {
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int t = 8 * nt + 2 * tig + j;
-                    float v = s[nt][2 * k + j] * p.scale_log2;
-                    if constexpr (kF16) v *= ksc[t];
+                    float v;
+                    if constexpr (kI4) {
+                        // (c - zero) * scale: sum_d q_d (c_d 2^-9) 512 - zero * sum_d q_d
+                        const float2 pz = reinterpret_cast<const float2*>(ksc)[t];
+                        v = (512.0f * s[nt][2 * k + j] - pz.y * qsum[k]) * pz.x * p.scale_log2;
+                    } else {
+                        v = s[nt][2 * k + j] * p.scale_log2;
+                        if constexpr (kF16) v *= ksc[t];
+                    }
                     pr[k][nt][j] = (pos0 + t <= last) ? v : -INFINITY;
                     mx = fmaxf(mx, pr[k][nt][j]);
                 }
@@ -853,7 +933,23 @@ struct MmaMath {
         uint32_t pb[kSets][2];
 #pragma unroll
         for (int k = 0; k < kSets; ++k) {
-            if constexpr (kF16) {
+            if constexpr (kI4) {
+                // O = sum_t p_t scale_t (c_t - zero_t): P' = p * scale, and the zero
+                // term sum_t P'_t zero_t is kept per row (b_run)
+                const float2* vpz = reinterpret_cast<const float2*>(ksc) + kBlockTokens;
+                float bsum = 0.0f;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const int t = 8 * nt + 2 * tig + j;
+                        const float2 pz = vpz[t];
+                        const float pv = pr[k][nt][j] * pz.x;
+                        pr[k][nt][j] = (t < nvalid) ? pv : 0.0f;
+                        bsum += (t < nvalid) ? pv * pz.y : 0.0f;
+                    }
+                b_run[k] = b_run[k] * corr[k] + bsum;
+            } else if constexpr (kF16) {
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -871,7 +967,33 @@ struct MmaMath {
         const uint32_t mask_b = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
 
         // ---- O^T += V^T.P^T over 8 m-tiles of 16 head dims
-        if constexpr (!kF16) {
+        if constexpr (kI4) {
+#pragma unroll
+            for (int cq = 0; cq < 2; ++cq) {
+                uint32_t w[4];  // {(tok 0-7, chunk 2cq), (tok 8-15, 2cq), (0-7, 2cq+1), (8-15, 2cq+1)}
+                ldsm_x4_trans(w, v_s + swz(8 * (mtx & 1) + r, 2 * cq + (mtx >> 1)));
+#pragma unroll
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * cq + cc;
+                    uint32_t h0[4], h1[4];  // tokens 2tig,2tig+1 / 8+2tig,9+2tig: {d0, d2, d1, d3}
+                    nib8t_to_f16x2x4(w[2 * cc], h0);
+                    nib8t_to_f16x2x4(w[2 * cc + 1], h1);
+                    if (partial) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            h0[e] &= mask_a;
+                            h1[e] &= mask_b;
+                        }
+                    }
+                    // m-tile 2c: rows gid <- dim 4gid, gid+8 <- 4gid+1; m-tile 2c+1: 4gid+2, 4gid+3
+#pragma unroll
+                    for (int k = 0; k < kSets; ++k) {
+                        mma_16816<true>(o[k][2 * c], h0[0], h0[2], h1[0], h1[2], pb[k][0], pb[k][1]);
+                        mma_16816<true>(o[k][2 * c + 1], h0[1], h0[3], h1[1], h1[3], pb[k][0], pb[k][1]);
+                    }
+                }
+            }
+        } else if constexpr (!kF16) {
 #pragma unroll
             for (int mi = 0; mi < 8; ++mi) {
                 uint32_t a[4];  // {tok 0-7 dims lo, tok 0-7 dims hi, tok 8-15 lo, tok 8-15 hi}
@@ -921,6 +1043,21 @@ struct MmaMath {
             l += __shfl_xor_sync(0xffffffffu, l, 2);
             const float lr[2] = {__shfl_sync(0xffffffffu, l, 8 * tig),        // row 8k + 2tig
                                  __shfl_sync(0xffffffffu, l, 8 * tig + 4)};   // row 8k + 2tig + 1
+            // 4-bit: O = 512 * (the MMA sums of P' c 2^-9) - sum_t P'_t zero_t
+            if constexpr (kI4) {
+                float bq = b_run[k];
+                bq += __shfl_xor_sync(0xffffffffu, bq, 1);
+                bq += __shfl_xor_sync(0xffffffffu, bq, 2);
+                const float br[2] = {__shfl_sync(0xffffffffu, bq, 8 * tig),
+                                     __shfl_sync(0xffffffffu, bq, 8 * tig + 4)};
+#pragma unroll
+                for (int mi = 0; mi < 8; ++mi)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        o[k][mi][j] = 512.0f * o[k][mi][j] - br[j];
+                        o[k][mi][2 + j] = 512.0f * o[k][mi][2 + j] - br[j];
+                    }
+            }
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int32_t row = 8 * k + 2 * tig + j;
@@ -1015,13 +1152,33 @@ __device__ __forceinline__ void prefetch_append(const DecodeParams& p, int32_t b
 template <class M>
 __device__ __noinline__ void append_row(uint8_t* st, const AppendRow a, int32_t lane) {
     constexpr int D = M::kHeadDim;
-    constexpr int kElem = KvElem<M::kKv>::kBytes;
-    constexpr int kRowBytes = D * kElem;
-    constexpr int kTileBytes = kBlockTokens * kRowBytes;
+    constexpr int kRowBytes = M::kRowBytes;
+    constexpr int kTileBytes = M::kTileBytes;
     const int32_t pos = a.L - 1, r = pos % kBlockTokens;
     const int64_t blk = a.table_row[pos / kBlockTokens];
     const int64_t rowi = (blk * a.num_kv_heads + a.kvh) * kBlockTokens + r;  // pool row
-    if constexpr (kQuantized<M::kKv>) {
+    if constexpr (M::kKv == KV_INT4) {
+        // 2 bytes of packed codes per lane; (scale, zero) per row, K rows then V rows
+        const int32_t src_bytes = a.src_dtype == KV_F32 ? 4 : 2;
+        float2* pz_stage = reinterpret_cast<float2*>(st + 2 * kTileBytes);
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const uint8_t* src = static_cast<const uint8_t*>(which ? a.v_new : a.k_new);
+            float x[D / 32];
+            load_row_part<D>(src + a.src_row * D * src_bytes, a.src_dtype, lane, x);
+            float sc, zr;
+            const uint16_t codes = static_cast<uint16_t>(quantize_row_int4_warp<D>(x, &sc, &zr));
+            *reinterpret_cast<uint16_t*>((which ? a.v_dst : a.k_dst) + rowi * kRowBytes + lane * 2) =
+                codes;
+            *reinterpret_cast<uint16_t*>(st + which * kTileBytes + M::tile_byte(r, lane * 2)) = codes;
+            if (lane == 0) {
+                reinterpret_cast<float2*>(a.scales_dst)
+                    [((blk * a.num_kv_heads + a.kvh) * 2 + which) * kBlockTokens + r] =
+                    make_float2(sc, zr);
+                pz_stage[which * kBlockTokens + r] = make_float2(sc, zr);
+            }
+        }
+    } else if constexpr (kQuantized<M::kKv>) {
         constexpr int kPer = D / 32;
         const int32_t src_bytes = a.src_dtype == KV_F32 ? 4 : 2;
         float* sc_stage = reinterpret_cast<float*>(st + 2 * kTileBytes);  // K then V row scales
@@ -1411,7 +1568,8 @@ static cudaError_t dispatch_q(const DecodeParams& p, const TmaMaps& maps, int32_
 }
 
 bool decode_uses_tensor_cores(int32_t kv_dtype, int32_t q_dtype, int32_t head_dim) {
-    return (kv_dtype == KV_BF16 || kv_dtype == KV_FP8_E4M3 || kv_dtype == KV_INT8) &&
+    return (kv_dtype == KV_BF16 || kv_dtype == KV_FP8_E4M3 || kv_dtype == KV_INT8 ||
+            kv_dtype == KV_INT4) &&
            q_dtype == KV_BF16 &&
            head_dim == 128;
 }
@@ -1423,9 +1581,12 @@ cudaError_t launch_paged_decode(const DecodeParams& p, const TmaMaps& maps, int3
         switch (kv_dtype) {
             case KV_BF16: return dispatch_mma<KV_BF16>(p, maps, group, stream);
             case KV_INT8: return dispatch_mma<KV_INT8>(p, maps, group, stream);
+            case KV_INT4: return dispatch_mma<KV_INT4>(p, maps, group, stream);
             default: return dispatch_mma<KV_FP8_E4M3>(p, maps, group, stream);
         }
     }
+    // (4-bit pools have only the tensor-core tile; the host rejects other shapes)
+    if (kv_dtype == KV_INT4) return cudaErrorInvalidValue;
     switch (kv_dtype) {
         case KV_F32: return dispatch_q<KV_F32>(p, maps, q_dtype, head_dim, group, stream);
         case KV_BF16: return dispatch_q<KV_BF16>(p, maps, q_dtype, head_dim, group, stream);

@@ -65,6 +65,48 @@ __device__ __forceinline__ uint32_t quantize_row_warp(const float* x, float* sca
     return codes;
 }
 
+// INT4 ("llm-inference-optimization" notes §四: the printed 4-bit routine,
+// asymmetric with a zero point, here applied to one row), in IEEE fp32:
+//   hi = max x, lo = min x, scale = (hi - lo) / 15, zero = rint(-lo / scale),
+//   code = clamp(rint(x / scale) + zero, 0, 15); value = (code - zero) * scale.
+// A constant row (where the routine would divide by zero) is stored exactly:
+// scale = |lo|, zero = -1 / +1 / 0 for lo > 0 / < 0 / == 0, every code 0.
+// Returns this lane's 4 codes (head_dim 128) packed two per byte, the lane's
+// first element in the low nibble of the low byte.
+template <int D>
+__device__ __forceinline__ uint32_t quantize_row_int4_warp(const float* x, float* scale,
+                                                           float* zero) {
+    constexpr int kPer = D / 32;
+    static_assert(kPer == 4, "4-bit rows: head_dim 128");
+    float hi = x[0], lo = x[0];
+#pragma unroll
+    for (int e = 1; e < kPer; ++e) {
+        hi = fmaxf(hi, x[e]);
+        lo = fminf(lo, x[e]);
+    }
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) {
+        hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, m));
+        lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, m));
+    }
+    uint32_t codes = 0;
+    if (hi == lo) {
+        *scale = fabsf(lo);
+        *zero = lo > 0.0f ? -1.0f : (lo < 0.0f ? 1.0f : 0.0f);
+        return codes;
+    }
+    const float s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+    const float z = rintf(__fdiv_rn(-lo, s));
+#pragma unroll
+    for (int e = 0; e < kPer; ++e) {
+        const float c = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x[e], s)), z), 0.0f), 15.0f);
+        codes |= static_cast<uint32_t>(c) << (4 * e);
+    }
+    *scale = s;
+    *zero = z;
+    return codes;
+}
+
 // Store a lane's packed codes (D/32 bytes) at dst.
 template <int D>
 __device__ __forceinline__ void store_codes(uint8_t* dst, uint32_t codes) {

@@ -4,7 +4,7 @@ and evaluate the oracle on the same inputs.
 GPU side: the pool is filled by the library's own slot computation and cache
 write (history tokens), then a step appends each sequence's new token and
 decodes.  Oracle side: the contiguous per-sequence K/V the generator drew
-(FP8 / INT8: quantised by the oracle's own encoder), never the GPU's pool.
+(FP8 / INT8 / INT4: quantised by the oracle's own encoder), never the GPU's pool.
 """
 from __future__ import annotations
 
@@ -22,6 +22,7 @@ TOL = {  # max-abs, max-rel (relative to the output's max magnitude)
     "bf16": (2e-2, 1e-2),
     "fp8": (5e-2, None),
     "int8": (5e-2, None),
+    "int4": (5e-2, None),
 }
 
 

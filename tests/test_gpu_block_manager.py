@@ -24,14 +24,14 @@ def _bits(t):
     return t.numpy()
 
 
-@pytest.mark.parametrize("kv", ["bf16", "f32", "fp8", "int8"])
+@pytest.mark.parametrize("kv", ["bf16", "f32", "fp8", "int8", "int4"])
 def test_copy_blocks_bitexact(kv):
     nb, hkv, d = 24, 2, 64 if kv == "f32" else 128
     cache = PagedKVCache(nb, hkv, d, kv, DEV)
     g = torch.Generator(device="cpu").manual_seed(3)
-    if kv in ("fp8", "int8"):
+    if kv in ("fp8", "int8", "int4"):
         dt = cache.k_pool.dtype
-        lo, hi = (0, 255) if kv == "fp8" else (-127, 128)
+        lo, hi = (-127, 128) if kv == "int8" else (0, 255)
         cache.k_pool.copy_(torch.randint(lo, hi, cache.k_pool.shape, generator=g, dtype=dt))
         cache.v_pool.copy_(torch.randint(lo, hi, cache.v_pool.shape, generator=g, dtype=dt))
         cache.scales.copy_(torch.rand(cache.scales.shape, generator=g))
@@ -52,7 +52,7 @@ def test_copy_blocks_bitexact(kv):
     assert cache.errors() == 0
 
 
-@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8"])
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8", "int4"])
 def test_fork_copy_on_write_decode(kv):
     hq, hkv, d, nb, hist = 8, 2, 128, 32, 40
     m = pk.BlockManager(nb, 4, 16)
@@ -87,7 +87,7 @@ def test_fork_copy_on_write_decode(kv):
     k_seq = torch.cat([k_hist, k_new[:1], k_hist, k_new[1:]])
     v_seq = torch.cat([v_hist, v_new[:1], v_hist, v_new[1:]])
     offs = np.array([0, hist + 1], dtype=np.int64)
-    if kv in ("fp8", "int8"):
+    if kv in ("fp8", "int8", "int4"):
         kc, ks = oracle.quantize_rows(k_seq.float().numpy(), kv)
         vc, vs = oracle.quantize_rows(v_seq.float().numpy(), kv)
         ref = oracle.decode_attention(storage_view(q), kc, vc, offs, lens, 1 / math.sqrt(d), hkv,

@@ -72,13 +72,23 @@ def _fp8_rows(rng, T, Hkv, D):
     x[3, :, ::7] *= 50.0                         # outlier channels: subnormal codes elsewhere
     x[4] *= 3e4                                  # large magnitudes
     x[5, 1, :] = np.linspace(-1, 1, D)           # ties are likely on a regular grid
+    x[7, 0, :] = np.abs(x[7, 0, :]) + 3.0        # all positive (INT4: negative zero point)
+    x[8, 1, :] = -np.abs(x[8, 1, :]) - 3.0       # all negative (INT4: zero point above 15)
+    x[9, 0, :] = 0.625                           # constant, non-zero
     return x
 
 
-@pytest.mark.parametrize("kind", ["fp8", "int8"])
+def _pack_int4(codes):
+    """One code per element -> the pool's bytes: dim 2i low nibble, 2i+1 high."""
+    return (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+
+
+@pytest.mark.parametrize("kind", ["fp8", "int8", "int4"])
 @pytest.mark.parametrize("src", ["f32", "bf16"])
 @pytest.mark.parametrize("D", [64, 128])
 def test_cache_quant_bitexact(kind, src, D):
+    if kind == "int4" and D != 128:
+        pytest.skip("4-bit pools have head_dim 128")
     rng = np.random.default_rng(3 + D)
     NB, Hkv, T = 50, 2, 400
     x_k = _fp8_rows(rng, T, Hkv, D)
@@ -97,6 +107,8 @@ def test_cache_quant_bitexact(kind, src, D):
     want_scales = np.full(tuple(cache.scales.shape), np.nan, np.float32)
     for which, (pool, src_t) in enumerate(((cache.k_pool, k), (cache.v_pool, v))):
         codes, scales = oracle.quantize_rows(src_t.float().numpy(), kind)
+        if kind == "int4":
+            codes = _pack_int4(codes)
         want_codes = oracle.scatter_to_pool(np.full(tuple(pool.shape), 0x7F, codes.dtype), codes,
                                             slots)
         want_scales = oracle.scatter_scales_to_pool(want_scales, scales, slots, which)

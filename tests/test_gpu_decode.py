@@ -30,10 +30,12 @@ LENS = [1, 2, 15, 16, 17, 63, 64, 65, 300, 1023, 1025]
 
 @pytest.mark.parametrize("kv,q", [("bf16", "bf16"), ("f32", "f32"), ("fp8", "bf16"),
                                   ("bf16", "f32"), ("f32", "bf16"), ("fp8", "f32"),
-                                  ("int8", "bf16"), ("int8", "f32")])
+                                  ("int8", "bf16"), ("int8", "f32"), ("int4", "bf16")])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [1, 2, 4, 8])
 def test_decode_parity_shapes(kv, q, D, G):
+    if kv == "int4" and D != 128:
+        pytest.skip("4-bit pools have head_dim 128")
     inp = make_inputs(_spec(kv, q, D, G, LENS))
     st = stage(inp)
     _, ref = oracle_out(inp)
@@ -194,7 +196,7 @@ def test_long_full_size_sampled():
     _sampled("long", [0, 3])
 
 
-@pytest.mark.parametrize("kind", ["fp8", "int8"])
+@pytest.mark.parametrize("kind", ["fp8", "int8", "int4"])
 def test_quantized_full_size_sampled_and_codes_bitexact(kind):
     import oracle
     stats, inp, st = _sampled(kind, [0, 40])
@@ -202,6 +204,8 @@ def test_quantized_full_size_sampled_and_codes_bitexact(kind):
     s = 40
     a, n = int(inp.seq_offsets[s]), int(inp.context_lens[s])
     codes, scales = oracle.quantize_rows(inp.k[a:a + n].float().numpy(), kind)
+    if kind == "int4":
+        codes = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
     kp = st.cache.k_pool.cpu().numpy()
     ks = st.cache.scales.cpu().numpy()[:, :, 0, :]   # K row scales
     for pos in range(0, n, 97):

@@ -47,10 +47,12 @@ LENS = [1, 2, 15, 16, 17, 64, 65, 300, 1025]
 
 @pytest.mark.parametrize("kv,q", [("bf16", "bf16"), ("f32", "f32"), ("fp8", "bf16"),
                                   ("int8", "bf16"), ("bf16", "f32"), ("fp8", "f32"),
-                                  ("int8", "f32")])
+                                  ("int8", "f32"), ("int4", "bf16")])
 @pytest.mark.parametrize("D", [64, 128])
 @pytest.mark.parametrize("G", [1, 4, 8])
 def test_fused_equals_separate_calls(kv, q, D, G):
+    if kv == "int4" and D != 128:
+        pytest.skip("4-bit pools have head_dim 128")
     inp = make_inputs(_spec(kv, q, D, G, LENS, idx=110 + G))
     st = stage(inp)
     c = st.cache
@@ -100,7 +102,7 @@ def test_fused_steps_grow_the_context():
     assert c.errors() == 0
 
 
-@pytest.mark.parametrize("kv", ["bf16", "fp8"])
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int4"])
 def test_fused_bad_last_block_writes_nothing_for_that_sequence(kv):
     inp = make_inputs(_spec(kv, "bf16", 128, 4, [100, 200, 33], idx=121))
     st = stage(inp)

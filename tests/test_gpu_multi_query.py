@@ -1,6 +1,6 @@
 """GPU: multi-query paged attention (Q causal query tokens per sequence) against
 the oracle's causal multi-query attention.  Tolerances as for decode: bf16 KV
-max-abs 2e-2 / max-rel 1e-2, FP8 and INT8 KV max-abs 5e-2."""
+max-abs 2e-2 / max-rel 1e-2, FP8, INT8 and INT4 KV max-abs 5e-2."""
 import math
 
 import numpy as np
@@ -44,7 +44,7 @@ def _full_cache(inp):
 CASES = [(g, q) for g in (1, 2, 4, 8) for q in (2, 3, 4, 5, 8, 16) if g * q <= 16]
 
 
-@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8"])
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8", "int4"])
 @pytest.mark.parametrize("G,Q", CASES)
 def test_multi_query_parity(kv, G, Q):
     lens = [Q, Q + 1, 17, 33, 100, 1025, 2048 + 3]

@@ -59,6 +59,9 @@ def test_pool_geometry_llama_shape():
     assert f.kv_bytes == 100 * 8 * 16 * 64 and f.scale_bytes == 100 * 8 * 2 * 16 * 4
     i = pk.kv_pool_create(100, 16, 8, 64, pk.KV_INT8)
     assert (i.kv_bytes, i.scale_bytes, i.elem_bytes) == (f.kv_bytes, f.scale_bytes, 1)
+    n = pk.kv_pool_create(100, 16, 8, 128, pk.KV_INT4)      # 64-byte rows, (scale, zero) pairs
+    assert (n.kv_bytes, n.scale_bytes, n.elem_bytes) == (100 * 8 * 16 * 64, 100 * 8 * 2 * 16 * 8, 0)
+    assert n.stride_slot == 128                              # strides count codes
 
 
 @pytest.mark.parametrize("args,status", [
@@ -66,6 +69,7 @@ def test_pool_geometry_llama_shape():
     ((10, 32, 8, 128, pk.KV_BF16), pk.KV_ERR_UNSUPPORTED),
     ((10, 16, 8, 96, pk.KV_BF16), pk.KV_ERR_UNSUPPORTED),
     ((10, 16, 8, 128, 7), pk.KV_ERR_UNSUPPORTED),
+    ((10, 16, 8, 64, pk.KV_INT4), pk.KV_ERR_UNSUPPORTED),        # 4-bit: head_dim 128 only
     ((10, 16, 0, 128, pk.KV_BF16), pk.KV_ERR_INVALID_ARGUMENT),
 ])
 def test_pool_create_rejects(args, status):
@@ -161,7 +165,12 @@ def test_decode_append_host_validation(pool, kw, status):
     assert _call_append(d, **kw) == status
 
 
-@pytest.mark.parametrize("dtype", [pk.KV_FP8_E4M3, pk.KV_INT8])
+def test_decode_int4_needs_the_tensor_core_shape():
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_INT4)
+    assert _call_decode(d, q_dtype=pk.KV_F32, scales=6 << 20) == pk.KV_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("dtype", [pk.KV_FP8_E4M3, pk.KV_INT8, pk.KV_INT4])
 def test_decode_quantized_pool_requires_scales(dtype):
     d = pk.kv_pool_create(8192, 16, 8, 128, dtype)
     assert _call_decode(d) == pk.KV_ERR_INVALID_ARGUMENT

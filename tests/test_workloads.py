@@ -68,7 +68,7 @@ def test_long_has_outlier_channels():
     assert float(inp.v.float().pow(2).mean().sqrt()) < 1.1
 
 
-@pytest.mark.parametrize("name", ["fp8", "int8"])
+@pytest.mark.parametrize("name", ["fp8", "int8", "int4"])
 def test_quantized_lengths_in_range(name):
     inp = make_inputs(name, batch=16)
     assert (inp.context_lens >= 1024).all() and (inp.context_lens <= 16384).all()

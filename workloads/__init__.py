@@ -44,7 +44,8 @@ class Spec:
     num_q_heads: int
     num_kv_heads: int
     head_dim: int
-    kv_dtype: str            # "f32" | "bf16" | "fp8" | "int8" (8-bit pools are fed bf16 sources)
+    kv_dtype: str            # "f32" | "bf16" | "fp8" | "int8" | "int4" (quantised pools are fed
+                             # bf16 sources)
     q_dtype: str             # "f32" | "bf16"
     lens: tuple              # ("fixed", (L0, L1, ...)) or ("uniform", lo, hi)
     scale: float
@@ -62,7 +63,7 @@ class Spec:
 
     @property
     def source_dtype(self) -> str:
-        return "bf16" if self.kv_dtype in ("fp8", "int8") else self.kv_dtype
+        return "bf16" if self.kv_dtype in ("fp8", "int8", "int4") else self.kv_dtype
 
 
 WORKLOADS = {
@@ -84,6 +85,9 @@ WORKLOADS = {
                 scale=1.0 / math.sqrt(128.0)),
     "int8": Spec("int8", 5, batch=64, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  kv_dtype="int8", q_dtype="bf16", lens=("uniform", 1024, 16384),
+                 scale=1.0 / math.sqrt(128.0)),
+    "int4": Spec("int4", 6, batch=64, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 kv_dtype="int4", q_dtype="bf16", lens=("uniform", 1024, 16384),
                  scale=1.0 / math.sqrt(128.0)),
 }
 
