@@ -23,6 +23,9 @@ restatement, in double precision, of every step of the decode hot path:
                              ``quantize_rows(x, "int4")`` the INT4 cache, the
                              asymmetric 4-bit routine of the
                              "llm-inference-optimization" notes §四 per row.
+* ``quantize_blocks_kivi`` / ``kivi_dequantize`` -- the KIVI cache (freetools
+                             "KV Cache量化": K per channel over a block, V per
+                             token, newest tokens at full precision).
 * ``decode_attention``    -- softmax(q·Kᵀ·scale)·V over a CONTIGUOUS per-sequence
                              copy, GQA head grouping, two passes in double
                              (C, OpenMP); "KV Cache 深度解析", §一 and §六.
@@ -49,8 +52,9 @@ import numpy as np
 
 from . import build as _build
 
-F32, BF16, FP8_E4M3, INT8, INT4 = 0, 1, 2, 3, 4
-_DTYPE_CODES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3, "int8": INT8, "int4": INT4}
+F32, BF16, FP8_E4M3, INT8, INT4, F64 = 0, 1, 2, 3, 4, 5
+_DTYPE_CODES = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3, "int8": INT8, "int4": INT4,
+                "f64": F64}
 QUANTIZED = ("fp8", "int8", "int4")
 
 _lib = None
@@ -72,6 +76,11 @@ def _load():
         lib.oracle_quantize_rows_int8.argtypes = lib.oracle_quantize_rows.argtypes
         lib.oracle_quantize_rows_int4.restype = None
         lib.oracle_quantize_rows_int4.argtypes = lib.oracle_quantize_rows.argtypes
+        lib.oracle_quantize_blocks_kivi.restype = None
+        lib.oracle_quantize_blocks_kivi.argtypes = [ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_int64, ctypes.c_int32,
+                                                    ctypes.c_void_p, ctypes.c_void_p,
+                                                    ctypes.c_void_p, ctypes.c_void_p]
         lib.oracle_decode_attention.restype = ctypes.c_int
         lib.oracle_decode_attention.argtypes = [
             ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -207,6 +216,48 @@ def quantize_rows(x: np.ndarray, kind: str = "fp8") -> tuple[np.ndarray, np.ndar
     return codes, scales
 
 
+def quantize_blocks_kivi(k: np.ndarray, v: np.ndarray):
+    """KIVI quantisation of full blocks of one kv head: k, v [blocks][16][D]
+    float32 -> (k_codes [blocks][16][D] uint8, k_params [blocks][D][2],
+    v_codes [blocks][16][D] uint8, v_params [blocks][16][2]); params are
+    (scale, zero) as float32, K per channel over the block, V per token row."""
+    k = np.ascontiguousarray(k, dtype=np.float32)
+    v = np.ascontiguousarray(v, dtype=np.float32)
+    nb, bs, d = k.shape
+    assert bs == 16 and v.shape == k.shape
+    kc = np.empty(k.shape, np.uint8)
+    vc = np.empty(v.shape, np.uint8)
+    kp = np.empty((nb, d, 2), np.float32)
+    vp = np.empty((nb, 16, 2), np.float32)
+    _load().oracle_quantize_blocks_kivi(_ptr(k), _ptr(v), nb, d, _ptr(kc), _ptr(kp), _ptr(vc),
+                                        _ptr(vp))
+    return kc, kp, vc, vp
+
+
+def kivi_dequantize(k_codes, k_params, v_codes, v_params):
+    """(code - zero) * scale in float64: K with per-channel parameters, V per row."""
+    k = (k_codes.astype(np.float64) - k_params[:, None, :, 1]) * k_params[:, None, :, 0]
+    v = (v_codes.astype(np.float64) - v_params[:, :, 1:2]) * v_params[:, :, 0:1]
+    return k, v
+
+
+def kivi_sequence(k_rows: np.ndarray, v_rows: np.ndarray):
+    """One sequence's K/V [L][Hkv][D] (float32 values of the stored source rows)
+    as the KIVI cache holds them, in float64: full blocks quantised (K per
+    channel, V per token), the last L mod 16 tokens exact."""
+    L, hkv, d = k_rows.shape
+    full = L // 16
+    k64 = k_rows.astype(np.float64).copy()
+    v64 = v_rows.astype(np.float64).copy()
+    if full:
+        kb = k_rows[:full * 16].reshape(full, 16, hkv, d).transpose(0, 2, 1, 3).reshape(-1, 16, d)
+        vb = v_rows[:full * 16].reshape(full, 16, hkv, d).transpose(0, 2, 1, 3).reshape(-1, 16, d)
+        kd, vd = kivi_dequantize(*quantize_blocks_kivi(kb, vb))
+        k64[:full * 16] = kd.reshape(full, hkv, 16, d).transpose(0, 2, 1, 3).reshape(-1, hkv, d)
+        v64[:full * 16] = vd.reshape(full, hkv, 16, d).transpose(0, 2, 1, 3).reshape(-1, hkv, d)
+    return k64, v64
+
+
 # --------------------------------------------------------------------------
 # Decode attention over contiguous per-sequence K/V
 # --------------------------------------------------------------------------
@@ -217,7 +268,8 @@ def decode_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, seq_offsets: n
     """Double-precision decode attention (C oracle).
 
     q     : [B][Hq][D]   float32 (q_dtype "f32") or uint16 bf16 bits ("bf16")
-    k, v  : [T][Hkv][D]  float32 / uint16 bf16 bits / uint8 E4M3 codes / int8 codes
+    k, v  : [T][Hkv][D]  float32 / uint16 bf16 bits / uint8 E4M3 codes / int8 codes /
+                         float64 ("f64", values already dequantised)
     seq_offsets : [B] int64, first token of each sequence in k/v
     lens  : [B] int32 context lengths (>= 1)
     k_scale, v_scale : [T][Hkv] float32 for kv_dtype "fp8" / "int8";

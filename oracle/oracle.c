@@ -41,7 +41,12 @@
  *    rint(-min / scale), code = clamp(rint(x / scale) + zero, 0, 15); a
  *    constant row, where the routine would divide by zero, is stored exactly
  *    (scale |min|, zero -1 / +1 / 0, codes 0); value = (code - zero) * scale
- *    in double.
+ *    in double;
+ *  - the KIVI cache ("大模型推理为何这么慢", KV Cache量化: Key quantised per
+ *    channel, Value per token, the newest tokens kept at full precision) runs
+ *    the same routine on different groups: each channel of a full 16-token
+ *    block of K (16 values), each token row of V (head_dim values); the
+ *    tokens of a sequence's incomplete last block stay unquantised.
  *
  * Build: gcc -O2 -ffp-contract=off -fopenmp -shared -fPIC (no fast-math).
  */
@@ -54,7 +59,7 @@
 #endif
 
 /* Stored element types of K/V and q, as the callers of this file pass them. */
-enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2, ORC_INT8 = 3, ORC_INT4 = 4 };
+enum { ORC_F32 = 0, ORC_BF16 = 1, ORC_FP8_E4M3 = 2, ORC_INT8 = 3, ORC_INT4 = 4, ORC_F64 = 5 };
 
 /* ---- exact widening of stored values ------------------------------------ */
 
@@ -225,6 +230,62 @@ void oracle_quantize_rows_int4(const float* x, int64_t rows, int32_t d,
     }
 }
 
+/*
+ * The 4-bit routine on one group of n values read with a stride (the same
+ * arithmetic as oracle_quantize_rows_int4, which runs it on contiguous rows).
+ */
+static void quantize_group_int4(const float* x, int32_t n, int64_t stride, uint8_t* codes,
+                                int64_t code_stride, float* scale, float* zero) {
+    float hi = x[0], lo = x[0], s, z;
+    int32_t i;
+    for (i = 1; i < n; ++i) {
+        float v = x[i * stride];
+        if (v > hi) hi = v;
+        if (v < lo) lo = v;
+    }
+    if (hi == lo) {
+        s = fabsf(lo);
+        z = lo > 0.0f ? -1.0f : (lo < 0.0f ? 1.0f : 0.0f);
+        for (i = 0; i < n; ++i) codes[i * code_stride] = 0;
+    } else {
+        float range = hi - lo;
+        s = range / 15.0f;
+        z = rintf(-lo / s);
+        for (i = 0; i < n; ++i) {
+            float q = rintf(x[i * stride] / s);
+            float c = q + z;
+            if (c < 0.0f) c = 0.0f;
+            if (c > 15.0f) c = 15.0f;
+            codes[i * code_stride] = (uint8_t)c;
+        }
+    }
+    *scale = s;
+    *zero = z;
+}
+
+/*
+ * KIVI quantisation of `blocks` full blocks of one kv head each.
+ *   k, v   : [blocks][16][d] fp32 (already rounded to the source dtype)
+ *   k_codes, v_codes : [blocks][16][d], one code (0..15) per element
+ *   k_params : [blocks][d][2]  (scale, zero) per channel over the block's 16 tokens
+ *   v_params : [blocks][16][2] (scale, zero) per token row
+ */
+void oracle_quantize_blocks_kivi(const float* k, const float* v, int64_t blocks, int32_t d,
+                                 uint8_t* k_codes, float* k_params, uint8_t* v_codes,
+                                 float* v_params) {
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < blocks; ++b) {
+        const int64_t base = b * 16 * d;
+        int32_t c, t;
+        for (c = 0; c < d; ++c)
+            quantize_group_int4(k + base + c, 16, d, k_codes + base + c, d,
+                                &k_params[(b * d + c) * 2], &k_params[(b * d + c) * 2 + 1]);
+        for (t = 0; t < 16; ++t)
+            quantize_group_int4(v + base + (int64_t)t * d, d, 1, v_codes + base + (int64_t)t * d, 1,
+                                &v_params[(b * 16 + t) * 2], &v_params[(b * 16 + t) * 2 + 1]);
+    }
+}
+
 /* Value of element i of a stored row, widened to double (codes dequantised).
  * For INT4 `scales` holds (scale, zero) pairs per row. */
 static double load_elem(const void* base, int dtype, int64_t idx, const float* scales,
@@ -236,6 +297,8 @@ static double load_elem(const void* base, int dtype, int64_t idx, const float* s
         return bf16_bits_to_double(((const uint16_t*)base)[idx]);
     case ORC_INT8:
         return (double)((const int8_t*)base)[idx] * (double)scales[scale_idx];
+    case ORC_F64:
+        return ((const double*)base)[idx];
     case ORC_INT4:
         return ((double)((const uint8_t*)base)[idx] - (double)scales[2 * scale_idx + 1]) *
                (double)scales[2 * scale_idx];

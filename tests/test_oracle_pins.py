@@ -284,6 +284,70 @@ def test_int4_quantize_invariants():
     assert (p2[:, 0] == pz[:, 0] * np.float32(0.25)).all()
 
 
+# ---------------------------------------------------------------- KIVI blocks
+def test_kivi_hand_example():
+    # one block, one kv head, 4 channels: K groups are channels over the 16 tokens
+    k = np.zeros((1, 16, 4), np.float32)
+    k[0, :, 0] = np.arange(16)                 # hi 15, lo 0: scale 1, zero 0, codes = values
+    k[0, :, 1] = 2.5                           # constant channel: exact
+    k[0, :, 2] = np.arange(16) * -2.0          # hi 0, lo -30: scale 2, zero 15, codes 15 - t
+    k[0, :, 3] = 0.0
+    v = np.zeros((1, 16, 4), np.float32)
+    v[0, 0] = [0, 1.5, 3, 22.5]                # hi 22.5, lo 0: scale 1.5, zero 0
+    v[0, 1] = [-7.5, 0, 7.5, 0]                # hi 7.5, lo -7.5: scale 1, zero round(7.5) = 8
+    kc, kp, vc, vp = oracle.quantize_blocks_kivi(k, v)
+    assert kc[0, :, 0].tolist() == list(range(16)) and kp[0, 0].tolist() == [1, 0]
+    assert (kc[0, :, 1] == 0).all() and kp[0, 1].tolist() == [2.5, -1]
+    assert kc[0, :, 2].tolist() == list(range(15, -1, -1)) and kp[0, 2].tolist() == [2, 15]
+    assert kp[0, 3].tolist() == [0, 0]
+    assert vc[0, 0].tolist() == [0, 1, 2, 15] and vp[0, 0].tolist() == [1.5, 0]
+    assert vc[0, 1].tolist() == [0, 8, 15, 8] and vp[0, 1].tolist() == [1, 8]
+    kd, vd = oracle.kivi_dequantize(kc, kp, vc, vp)
+    assert (kd[0, :, :3] == k[0, :, :3]).all()          # these channels are exact
+    assert vd[0, 1].tolist() == [-8, 0, 7, 0]           # (c - 8) * 1
+
+
+def test_kivi_groups_exact_rationals():
+    # scale, zero and codes of every K channel and V row re-derived exactly
+    rng = np.random.default_rng(77)
+    k = (rng.standard_normal((3, 16, 64)) * rng.uniform(0.1, 20, (3, 1, 64))).astype(np.float32)
+    v = (rng.standard_normal((3, 16, 64)) * rng.uniform(0.1, 20, (3, 16, 1))).astype(np.float32)
+    k[1, :, 5] = np.abs(k[1, :, 5]) + 4         # a channel with a negative zero point
+    kc, kp, vc, vp = oracle.quantize_blocks_kivi(k, v)
+
+    def check(group, codes, params):
+        hi, lo = np.float32(group.max()), np.float32(group.min())
+        sc = np.float32(np.float32(hi - lo) / np.float32(15))
+        z = _nearest_even(Fraction(float(np.float32(-lo) / sc)))
+        assert params[0] == sc and params[1] == z
+        for x, c in zip(group.tolist(), codes.tolist()):
+            kk = _nearest_even(Fraction(float(np.float32(x) / sc)))
+            assert c == min(15, max(0, kk + z))
+
+    for b in range(3):
+        for ch in range(64):
+            check(k[b, :, ch], kc[b, :, ch], kp[b, ch])
+        for t in range(16):
+            check(v[b, t], vc[b, t], vp[b, t])
+
+
+def test_kivi_sequence_keeps_the_incomplete_block_exact():
+    rng = np.random.default_rng(5)
+    for L in (15, 16, 32, 37):
+        k = rng.normal(size=(L, 2, 32)).astype(np.float32)
+        v = rng.normal(size=(L, 2, 32)).astype(np.float32)
+        k64, v64 = oracle.kivi_sequence(k, v)
+        full = L // 16 * 16
+        assert (k64[full:] == k[full:]).all() and (v64[full:] == v[full:]).all()
+        if full:
+            assert (k64[:full] != k[:full]).any()          # quantised
+            # per-channel error bound: at most one step of that channel's block scale
+            kb = k[:full].reshape(-1, 16, 2, 32)
+            step = (kb.max(axis=1) - kb.min(axis=1)) / 15
+            err = np.abs(k64[:full] - k[:full]).reshape(-1, 16, 2, 32)
+            assert (err <= step[:, None] * (1 + 1e-5) + 1e-7).all()
+
+
 # ---------------------------------------------------------------- attention
 def _rand_case(rng, b, hq, hkv, d, lens, kv_dtype="f32"):
     total = int(sum(lens))
@@ -311,9 +375,10 @@ def test_attention_matches_bruteforce_numpy(hq, hkv):
     assert np.abs(ours - brute).max() <= 1e-12
 
 
-@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "fp8", "int8", "int4"])
+@pytest.mark.parametrize("kv_dtype", ["f32", "bf16", "fp8", "int8", "int4", "f64"])
 def test_attention_matches_torch_sdpa_float64(kv_dtype):
-    rng = np.random.default_rng({"f32": 1, "bf16": 2, "fp8": 3, "int8": 4, "int4": 5}[kv_dtype])
+    rng = np.random.default_rng({"f32": 1, "bf16": 2, "fp8": 3, "int8": 4, "int4": 5,
+                                 "f64": 6}[kv_dtype])
     hq, hkv, d = 8, 2, 64
     lens = [3, 33, 64]
     q, k, v, offs, lens = _rand_case(rng, 3, hq, hkv, d, lens)
@@ -325,6 +390,10 @@ def test_attention_matches_torch_sdpa_float64(kv_dtype):
     elif kv_dtype == "bf16":
         kst, vst = _bf16_bits(k), _bf16_bits(v)
         k64, v64 = oracle.widen(kst, "bf16"), oracle.widen(vst, "bf16")
+    elif kv_dtype == "f64":
+        k64 = k.astype(np.float64) * (1 + 2.0 ** -40)       # values no float32 can hold
+        v64 = v.astype(np.float64) * (1 - 2.0 ** -40)
+        kst, vst = k64, v64
     elif kv_dtype == "int4":
         kst, ks = oracle.quantize_rows(k, "int4")
         vst, vs = oracle.quantize_rows(v, "int4")
