@@ -170,14 +170,27 @@ def kv_row_bytes(spec) -> int:
     an 8-bit cache)."""
     if spec.kv_dtype == "int4":    # two codes per byte + fp32 (scale, zero point)
         return spec.head_dim // 2 + 8
+    if spec.kv_dtype == "kivi4":   # full blocks, per token (see kivi_bytes)
+        return spec.head_dim // 2 + (spec.head_dim + 16) * 8 // 16
     elem = {"f32": 4, "bf16": 2, "fp8": 1, "int8": 1}[spec.kv_dtype]
     return spec.head_dim * elem + (4 if spec.kv_dtype in ("fp8", "int8") else 0)
+
+
+def kivi_bytes(spec, lens) -> int:
+    """KIVI bytes of contexts `lens`: each full block is 16 rows of 64-byte K and V
+    codes plus 1152 bytes of parameters per kv head; the rest are bf16 rows."""
+    lens = np.asarray(lens, dtype=np.int64)
+    full, rest = lens // 16, lens % 16
+    per_block = 2 * 16 * spec.head_dim // 2 + (spec.head_dim + 16) * 8
+    return int((full * per_block + rest * 2 * spec.head_dim * 2).sum()) * spec.num_kv_heads
 
 
 def kv_bytes_per_step(inp) -> int:
     """Algorithmic KV bytes one decode step reads: every context token's K and V
     row of every KV head (plus the fp32 per-row scales of an FP8 / INT8 cache)."""
     spec = inp.spec
+    if spec.kv_dtype == "kivi4":
+        return kivi_bytes(spec, inp.context_lens)
     tokens = int(inp.context_lens.astype(np.int64).sum())
     per_row = kv_row_bytes(spec)
     return tokens * spec.num_kv_heads * 2 * per_row
@@ -249,7 +262,16 @@ def time_oracle(inp, max_seqs: int, repeats: int = 1):
     lens = inp.context_lens[seqs]
     args = dict(seq_offsets=inp.seq_offsets[seqs], lens=lens, scale=spec.scale,
                 num_kv_heads=spec.num_kv_heads, q_dtype=spec.q_dtype)
-    if spec.kv_dtype in ("fp8", "int8", "int4"):
+    if spec.kv_dtype == "kivi4":
+        ks, vs = [], []
+        for b in seqs:
+            a, L = int(inp.seq_offsets[b]), int(inp.context_lens[b])
+            k64, v64 = oracle.kivi_sequence(inp.k[a:a + L].float().numpy(),
+                                            inp.v[a:a + L].float().numpy())
+            ks.append(k64), vs.append(v64)
+        kv = dict(k=np.concatenate(ks), v=np.concatenate(vs), kv_dtype="f64")
+        args["seq_offsets"] = np.concatenate([[0], np.cumsum(lens)[:-1]]).astype(np.int64)
+    elif spec.kv_dtype in ("fp8", "int8", "int4"):
         rows = slice(int(inp.seq_offsets[0]), int(inp.seq_offsets[n - 1] + lens[-1]))
         kc, ks = oracle.quantize_rows(inp.k[rows].float().numpy(), spec.kv_dtype)
         vc, vs = oracle.quantize_rows(inp.v[rows].float().numpy(), spec.kv_dtype)
@@ -262,6 +284,8 @@ def time_oracle(inp, max_seqs: int, repeats: int = 1):
     dt = (time.perf_counter() - t0) / repeats
     per_row = kv_row_bytes(spec)
     nbytes = int(lens.astype(np.int64).sum()) * spec.num_kv_heads * 2 * per_row
+    if spec.kv_dtype == "kivi4":
+        nbytes = kivi_bytes(spec, lens)
     desc = (f"oracle (C, double, OpenMP) over {n} of {inp.q.shape[0]} sequences "
             f"({int(lens.sum())} tokens, {nbytes / 2**20:.0f} MiB of KV) x {repeats}")
     return nbytes / dt / 1e9, dt, desc, oracle.num_threads()
@@ -297,11 +321,39 @@ def run_reference(args, inp):
 
 
 # ---------------------------------------------------------------- GPU arm
+def stage_kivi_on_device(inp, device):
+    """A KIVI cache holding every sequence's history (all but its last token)
+    through the library: full blocks quantised, the incomplete block's rows in
+    the bf16 residual."""
+    from paged_kv_cache_401_b200.cache import PagedKVCache
+    from workloads import kivi_layout
+    spec = inp.spec
+    cache = PagedKVCache(inp.num_blocks, spec.num_kv_heads, spec.head_dim, "kivi4", device)
+    res_k, res_v = cache.alloc_residual(inp.q.shape[0])
+    lay = kivi_layout(inp)
+    chunk = 4096
+    for c0 in range(0, len(lay.block_ids), chunk):
+        n = min(chunk, len(lay.block_ids) - c0)
+        rows = torch.from_numpy(lay.block_rows[c0:c0 + n].reshape(-1))
+        shape = (n, 16, spec.num_kv_heads, spec.head_dim)
+        cache.kivi_fill(torch.from_numpy(lay.block_ids[c0:c0 + n]).to(device),
+                        inp.k[rows].reshape(shape).to(device), inp.v[rows].reshape(shape).to(device))
+    if len(lay.res_rows):
+        rr = torch.from_numpy(lay.res_rows)
+        sq, sl = torch.from_numpy(lay.res_seq).long(), torch.from_numpy(lay.res_slot).long()
+        res_k[sq, :, sl] = inp.k[rr].to(device)
+        res_v[sq, :, sl] = inp.v[rr].to(device)
+    torch.cuda.synchronize(device)
+    return cache, torch.from_numpy(inp.block_table).to(device)
+
+
 def stage_on_device(inp, device, query_tokens: int = 1):
     """Fill the paged pool with every sequence's history (all but its last
     `query_tokens` tokens, which each step appends) through the library."""
     from paged_kv_cache_401_b200.cache import PagedKVCache
     spec = inp.spec
+    if spec.kv_dtype == "kivi4":
+        return stage_kivi_on_device(inp, device)
     cache = PagedKVCache(inp.num_blocks, spec.num_kv_heads, spec.head_dim, spec.kv_dtype,
                          device)
     bt = torch.from_numpy(inp.block_table).to(device)
@@ -360,9 +412,11 @@ def run_gpu(args, inp):
                                                   inp.max_context_len, P)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream(device)
-    fused = args.append == "fused" and Q == 1
-    # separate: slot mapping, cache write, decode, merge; fused: decode (+append), merge
-    launches_per_step = 2 if fused else 4
+    kivi = spec.kv_dtype == "kivi4"   # its step always appends inside the decode call
+    fused = (args.append == "fused" and Q == 1) or kivi
+    # separate: slot mapping, cache write, decode, merge; fused: decode (+append), merge;
+    # KIVI: append (+ block flush), decode, merge
+    launches_per_step = 3 if kivi else (2 if fused else 4)
 
     def append():
         if not fused:   # the fused call appends inside the decode
@@ -376,10 +430,17 @@ def run_gpu(args, inp):
             cache.attend(qq, tbl, ln, inp.max_context_len, spec.scale, out=out,
                          partition_tokens=P, workspace=ws)
 
+    def fused_call(qq, kk, vv, tbl, ln, o):
+        if kivi:
+            cache.kivi_decode(qq, tbl, ln, inp.max_context_len, spec.scale, kk, vv, out=o,
+                              partition_tokens=P, workspace=ws)
+        else:
+            cache.decode_append(qq, kk, vv, tbl, ln, inp.max_context_len, spec.scale, out=o,
+                                partition_tokens=P, workspace=ws)
+
     def decode():
         if fused:
-            cache.decode_append(q, k_new, v_new, bt, lens, inp.max_context_len, spec.scale,
-                                out=out, partition_tokens=P, workspace=ws)
+            fused_call(q, k_new, v_new, bt, lens, out)
         else:
             attend(q, bt, lens)
 
@@ -453,8 +514,7 @@ def run_gpu(args, inp):
         stream.wait_event(ev["in"][b])
         stream.wait_event(ev["out"][b])             # step i-2's output has been read back
         if fused:
-            cache.decode_append(e_q, e_k, e_v, e_bt, e_lens, inp.max_context_len, spec.scale,
-                                out=outs[b], partition_tokens=P, workspace=ws)
+            fused_call(e_q, e_k, e_v, e_bt, e_lens, outs[b])
         else:
             cache.append(e_bt, seq_ids, positions, e_k, e_v, slots=slots)
             if Q == 1:
@@ -519,8 +579,9 @@ def run_gpu(args, inp):
         "dtype": spec.kv_dtype if spec.kv_dtype != "fp8" else "fp8_e4m3",
         "data": "synthetic (seeded N(0,1) q/K/V, random block permutation)",
         "config": dict(describe(inp, P), num_ranges=ranges, query_tokens=Q,
-                       append="fused into the decode call" if fused
-                       else "separate slot-mapping and cache-write calls"),
+                       append=("KIVI residual append (+ block flush) in the decode call" if kivi
+                               else "fused into the decode call" if fused
+                               else "separate slot-mapping and cache-write calls")),
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
                 "ms_per_step": round(max_e2e_ms / args.steps, 5)},

@@ -63,8 +63,10 @@ typedef enum {
     KV_BF16 = 1,       /* bfloat16 */
     KV_FP8_E4M3 = 2,   /* OCP FP8 E4M3 codes (KV pools only) with fp32 row scales */
     KV_INT8 = 3,       /* signed 8-bit codes (KV pools only) with fp32 row scales */
-    KV_INT4 = 4        /* unsigned 4-bit codes, two per byte (KV pools only, head_dim 128),
+    KV_INT4 = 4,       /* unsigned 4-bit codes, two per byte (KV pools only, head_dim 128),
                           with an fp32 (scale, zero point) pair per row */
+    KV_KIVI4 = 5       /* KIVI: 4-bit codes as KV_INT4, keys with a (scale, zero point) per
+                          channel of each full block, values per row; see kivi_* below */
 } kv_dtype;
 
 /* Bits ORed into *dev_error by the kernels. */
@@ -86,6 +88,10 @@ typedef enum {
  * 2i in the low nibble of byte i, dim 2i+1 in the high nibble) and has one
  * fp32 parameter pool [num_blocks][num_kv_heads][2][block_size][2]: per row
  * (scale, zero point), K rows then V rows, 256 bytes per (block, kv head).
+ * A KIVI pool (KV_KIVI4) has the INT4 code layout and a parameter pool
+ * [num_blocks][num_kv_heads][128 + 16][2] fp32: (scale, zero point) of each of
+ * the 128 key channels over the block's 16 tokens, then of each of the 16
+ * value rows, 1152 bytes per (block, kv head).
  */
 typedef struct {
     int32_t num_blocks;
@@ -95,7 +101,7 @@ typedef struct {
     int32_t dtype;           /* kv_dtype */
     int32_t elem_bytes;      /* 4, 2 or 1; 0 for 4-bit codes (two per byte) */
     uint64_t kv_bytes;       /* bytes of ONE pool (K or V) */
-    uint64_t scale_bytes;    /* bytes of the scale / parameter pool (FP8, INT8, INT4; else 0) */
+    uint64_t scale_bytes;    /* bytes of the scale / parameter pool (FP8, INT8, INT4, KIVI) */
     int64_t stride_block;    /* elements between consecutive physical blocks */
     int64_t stride_head;     /* elements between consecutive kv heads of a block */
     int64_t stride_slot;     /* elements between consecutive tokens of a block */
@@ -105,7 +111,7 @@ typedef struct {
  * Fill *out with the geometry of a pool (host only, no device work).
  * Errors: KV_ERR_INVALID_ARGUMENT for out == NULL or non-positive sizes;
  * KV_ERR_UNSUPPORTED for block_size != 16, head_dim not in {64, 128},
- * num_kv_heads > 256, an unknown dtype, or KV_INT4 with head_dim != 128.
+ * num_kv_heads > 256, an unknown dtype, or KV_INT4 / KV_KIVI4 with head_dim != 128.
  */
 KV_API kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_heads,
                          int32_t head_dim, kv_dtype dtype, kv_pool_desc* out);
@@ -274,6 +280,50 @@ KV_API kv_status paged_decode_attention_append(const kv_pool_desc* pool, void* o
                                                float scale, int32_t partition_tokens,
                                                void* workspace, size_t workspace_bytes,
                                                int32_t* dev_error, kv_stream_t stream);
+
+/*
+ * KIVI cache ("大模型推理为何这么慢", KV Cache量化: keys quantised per channel,
+ * values per token, the newest tokens kept at full precision).  The 4-bit
+ * routine is the INT4 one above (reshape_and_cache), run on a key channel's
+ * 16 values within a full block and on each value row.  A KIVI pool holds
+ * FULL blocks only; the newest L mod 16 tokens of sequence b (L its context
+ * length) live unquantised in caller-owned bf16 residual buffers
+ * res_k / res_v [batch][num_kv_heads][16][head_dim], row t holding position
+ * 16 * floor(L / 16) + t.
+ *
+ * kivi_quantize_blocks: quantise num_blocks full blocks (prefill):
+ *   k_rows, v_rows : device [num_blocks][16][num_kv_heads][head_dim], 16
+ *                    consecutive tokens per block, in src_dtype (F32 or BF16)
+ *   block_ids      : device int32 [num_blocks], the block each one goes to
+ * An out-of-range block id skips that block (KV_DEVERR_BAD_BLOCK_ID).
+ * KV_ERR_UNSUPPORTED for a pool that is not KV_KIVI4 or another src_dtype.
+ */
+KV_API kv_status kivi_quantize_blocks(const kv_pool_desc* pool, void* k_pool, void* v_pool,
+                                      float* params, const void* k_rows, const void* v_rows,
+                                      kv_dtype src_dtype, const int32_t* block_ids,
+                                      int32_t num_blocks, int32_t* dev_error, kv_stream_t stream);
+
+/*
+ * kivi_decode_attention: one decode step over a KIVI pool.  When k_new/v_new
+ * (device bf16 [batch][num_kv_heads][head_dim]) are given, each sequence's new
+ * rows are first stored at residual row (L - 1) % 16, and when that completes
+ * the block, the 16 residual rows are quantised into block
+ * block_table[b][(L - 1) / 16]; NULL for both appends nothing.  Then
+ * paged_decode_attention's result over positions 0 .. L - 1: full blocks from
+ * the pool, the last L mod 16 positions from the residual.  Arguments and
+ * workspace as paged_decode_attention; bf16 q and head_dim 128 only, else
+ * KV_ERR_UNSUPPORTED (so is a KIVI pool passed to the other entry points).
+ */
+KV_API kv_status kivi_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
+                                       kv_dtype q_dtype, void* k_pool, void* v_pool,
+                                       float* params, void* res_k, void* res_v,
+                                       const void* k_new, const void* v_new,
+                                       const int32_t* block_table, int32_t max_blocks_per_seq,
+                                       const int32_t* context_lens, int32_t batch,
+                                       int32_t num_q_heads, int32_t max_context_len, float scale,
+                                       int32_t partition_tokens, void* workspace,
+                                       size_t workspace_bytes, int32_t* dev_error,
+                                       kv_stream_t stream);
 
 /*
  * Multi-query paged attention: Q = num_query_tokens new tokens per sequence

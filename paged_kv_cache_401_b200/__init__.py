@@ -17,9 +17,9 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libpagedkv.so")
 
-KV_F32, KV_BF16, KV_FP8_E4M3, KV_INT8, KV_INT4 = 0, 1, 2, 3, 4
-# pools of codes with per-row parameters: fp32 scales (8-bit), (scale, zero) pairs (4-bit)
-QUANTIZED = (KV_FP8_E4M3, KV_INT8, KV_INT4)
+KV_F32, KV_BF16, KV_FP8_E4M3, KV_INT8, KV_INT4, KV_KIVI4 = 0, 1, 2, 3, 4, 5
+# pools of codes with parameters: fp32 scales (8-bit), (scale, zero) pairs (4-bit)
+QUANTIZED = (KV_FP8_E4M3, KV_INT8, KV_INT4, KV_KIVI4)
 KV_OK, KV_ERR_INVALID_ARGUMENT, KV_ERR_UNSUPPORTED, KV_ERR_CUDA = 0, 1, 2, 3
 KV_ERR_OUT_OF_BLOCKS = 4
 KV_DEVERR_BAD_SLOT = 0x1
@@ -32,7 +32,7 @@ BLOCK_SIZE = 16
 EXPORTED = ("kv_pool_create", "compute_slot_mapping", "reshape_and_cache",
             "paged_decode_num_ranges", "paged_decode_workspace_bytes",
             "paged_decode_attention", "paged_decode_attention_static_workspace",
-            "paged_decode_attention_append",
+            "paged_decode_attention_append", "kivi_quantize_blocks", "kivi_decode_attention",
             "paged_attention_workspace_bytes", "paged_attention_multi_query",
             "paged_kv_copy_blocks", "kv_block_manager_create", "kv_block_manager_destroy",
             "kv_block_manager_num_free_blocks", "kv_block_manager_refcount",
@@ -82,6 +82,10 @@ def _load() -> ctypes.CDLL:
             "paged_decode_attention_append": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P,
                                                      _I32, _P, _I32, _P, _I32, _I32, _I32,
                                                      ctypes.c_float, _I32, _P, _SZ, _P, _P]),
+            "kivi_quantize_blocks": (_I32, [desc_p, _P, _P, _P, _P, _P, _I32, _P, _I32, _P, _P]),
+            "kivi_decode_attention": (_I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _P, _P, _P, _P,
+                                             _I32, _P, _I32, _I32, _I32, ctypes.c_float, _I32,
+                                             _P, _SZ, _P, _P]),
             "paged_decode_attention_static_workspace": (
                 _I32, [desc_p, _P, _P, _I32, _P, _P, _P, _P, _I32, _P, _I32, _I32, _I32,
                        ctypes.c_float, _I32, _P, _P]),
@@ -163,14 +167,18 @@ def empty_pool(desc: KvPoolDesc, device, fill: float | int | None = None):
     scales) for FP8 / INT8, [num_blocks][kv_heads][2][16][2] (scale, zero) for
     INT4, else None.  ``fill`` poisons every element (NaN, or a byte; scales
     get NaN)."""
-    cols = desc.head_dim // 2 if desc.dtype == KV_INT4 else desc.head_dim
+    four_bit = desc.dtype in (KV_INT4, KV_KIVI4)
+    cols = desc.head_dim // 2 if four_bit else desc.head_dim
     shape = (desc.num_blocks, desc.num_kv_heads, desc.block_size, cols)
     dt = {KV_F32: torch.float32, KV_BF16: torch.bfloat16, KV_FP8_E4M3: torch.uint8,
-          KV_INT8: torch.int8, KV_INT4: torch.uint8}[desc.dtype]
+          KV_INT8: torch.int8, KV_INT4: torch.uint8, KV_KIVI4: torch.uint8}[desc.dtype]
     k = torch.empty(shape, dtype=dt, device=device)
     v = torch.empty(shape, dtype=dt, device=device)
     scales = None
-    if desc.dtype in QUANTIZED:
+    if desc.dtype == KV_KIVI4:    # (scale, zero) of 128 key channels, then of 16 value rows
+        scales = torch.empty((desc.num_blocks, desc.num_kv_heads, desc.head_dim + desc.block_size,
+                              2), dtype=torch.float32, device=device)
+    elif desc.dtype in QUANTIZED:
         extra = (2,) if desc.dtype == KV_INT4 else ()
         scales = torch.empty((desc.num_blocks, desc.num_kv_heads, 2, desc.block_size) + extra,
                              dtype=torch.float32, device=device)
@@ -249,6 +257,50 @@ def paged_decode_attention_append(pool: KvPoolDesc, out: torch.Tensor, q: torch.
     _check("paged_decode_attention_append", _load().paged_decode_attention_append(
         ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool), _ptr(v_pool),
         _ptr(scales), _ptr(k_new), _ptr(v_new), kv_dtype_of(k_new), _ptr(block_table),
+        block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
+        float(scale), partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error),
+        _stream(stream)))
+    return out
+
+
+def empty_residual(desc: KvPoolDesc, batch: int, device, fill: float | None = None):
+    """(res_k, res_v) bf16 [batch][kv_heads][16][head_dim]: a KIVI cache's newest
+    L mod 16 tokens per sequence, kept unquantised."""
+    shape = (batch, desc.num_kv_heads, desc.block_size, desc.head_dim)
+    res = [torch.empty(shape, dtype=torch.bfloat16, device=device) for _ in range(2)]
+    if fill is not None:
+        for t in res:
+            t.fill_(fill)
+    return res[0], res[1]
+
+
+def kivi_quantize_blocks(pool: KvPoolDesc, k_pool: torch.Tensor, v_pool: torch.Tensor,
+                         params: torch.Tensor, k_rows: torch.Tensor, v_rows: torch.Tensor,
+                         block_ids: torch.Tensor, dev_error: torch.Tensor | None = None,
+                         stream=None) -> None:
+    """k_rows, v_rows: [n][16][kv_heads][head_dim] (fp32 or bf16), full blocks that
+    go to block_ids [n] of a KIVI pool."""
+    _check("kivi_quantize_blocks", _load().kivi_quantize_blocks(
+        ctypes.byref(pool), _ptr(k_pool), _ptr(v_pool), _ptr(params), _ptr(k_rows),
+        _ptr(v_rows), kv_dtype_of(k_rows), _ptr(block_ids), block_ids.numel(), _ptr(dev_error),
+        _stream(stream)))
+
+
+def kivi_decode_attention(pool: KvPoolDesc, out: torch.Tensor, q: torch.Tensor,
+                          k_pool: torch.Tensor, v_pool: torch.Tensor, params: torch.Tensor,
+                          res_k: torch.Tensor, res_v: torch.Tensor,
+                          k_new: torch.Tensor | None, v_new: torch.Tensor | None,
+                          block_table: torch.Tensor, context_lens: torch.Tensor,
+                          max_context_len: int, scale: float, partition_tokens: int = 0,
+                          workspace: torch.Tensor | None = None,
+                          dev_error: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """A decode step over a KIVI pool; k_new/v_new (bf16 [batch][kv_heads][head_dim])
+    are appended at position context_lens[b] - 1 first (None: no append)."""
+    batch, num_q_heads, _ = q.shape
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("kivi_decode_attention", _load().kivi_decode_attention(
+        ctypes.byref(pool), _ptr(out), _ptr(q), kv_dtype_of(q), _ptr(k_pool), _ptr(v_pool),
+        _ptr(params), _ptr(res_k), _ptr(res_v), _ptr(k_new), _ptr(v_new), _ptr(block_table),
         block_table.shape[1], _ptr(context_lens), batch, num_q_heads, max_context_len,
         float(scale), partition_tokens, _ptr(workspace), ws_bytes, _ptr(dev_error),
         _stream(stream)))

@@ -9,14 +9,15 @@ from __future__ import annotations
 
 import torch
 
-from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, KV_INT4, KV_INT8, compute_slot_mapping,
-               empty_pool,
+from . import (BLOCK_SIZE, KV_BF16, KV_F32, KV_FP8_E4M3, KV_INT4, KV_INT8, KV_KIVI4,
+               compute_slot_mapping, empty_pool, empty_residual, kivi_decode_attention,
+               kivi_quantize_blocks,
                kv_pool_create, paged_attention_multi_query, paged_attention_workspace_bytes,
                paged_decode_attention, paged_decode_attention_append,
                paged_decode_workspace_bytes, reshape_and_cache)
 
 _DTYPES = {"f32": KV_F32, "bf16": KV_BF16, "fp8": KV_FP8_E4M3, "int8": KV_INT8,
-           "int4": KV_INT4}
+           "int4": KV_INT4, "kivi4": KV_KIVI4}
 
 
 class PagedKVCache:
@@ -27,7 +28,7 @@ class PagedKVCache:
         self.desc = kv_pool_create(num_blocks, BLOCK_SIZE, num_kv_heads, head_dim, _DTYPES[dtype])
         fill = None
         if poison:
-            fill = 0x7F if dtype in ("fp8", "int8", "int4") else float("nan")
+            fill = 0x7F if dtype in ("fp8", "int8", "int4", "kivi4") else float("nan")
         self.k_pool, self.v_pool, self.scales = empty_pool(self.desc, self.device, fill)
         self.dev_error = torch.zeros(1, dtype=torch.int32, device=self.device)
 
@@ -84,6 +85,33 @@ class PagedKVCache:
                                              self.scales, k_new, v_new, block_table,
                                              context_lens, max_context_len, scale,
                                              partition_tokens, workspace, self.dev_error, stream)
+
+    # ---- KIVI pools: full blocks quantised, the newest L mod 16 tokens in a bf16 residual
+    def alloc_residual(self, batch: int, poison: bool = False):
+        self.res_k, self.res_v = empty_residual(self.desc, batch, self.device,
+                                                float("nan") if poison else None)
+        return self.res_k, self.res_v
+
+    def kivi_fill(self, block_ids: torch.Tensor, k_rows: torch.Tensor, v_rows: torch.Tensor,
+                  stream=None) -> None:
+        """Quantise full blocks (k_rows/v_rows [n][16][kv_heads][head_dim])."""
+        kivi_quantize_blocks(self.desc, self.k_pool, self.v_pool, self.scales, k_rows, v_rows,
+                             block_ids, self.dev_error, stream)
+
+    def kivi_decode(self, q: torch.Tensor, block_table: torch.Tensor, context_lens: torch.Tensor,
+                    max_context_len: int, scale: float, k_new: torch.Tensor | None = None,
+                    v_new: torch.Tensor | None = None, out: torch.Tensor | None = None,
+                    partition_tokens: int = 0, workspace: torch.Tensor | None = None,
+                    stream=None) -> torch.Tensor:
+        if out is None:
+            out = torch.empty_like(q)
+        if workspace is None:
+            workspace = self.alloc_workspace(q.shape[0], q.shape[1], max_context_len,
+                                             partition_tokens)
+        return kivi_decode_attention(self.desc, out, q, self.k_pool, self.v_pool, self.scales,
+                                     self.res_k, self.res_v, k_new, v_new, block_table,
+                                     context_lens, max_context_len, scale, partition_tokens,
+                                     workspace, self.dev_error, stream)
 
     def errors(self) -> int:
         """The device error word (KV_DEVERR_* bits); synchronises."""

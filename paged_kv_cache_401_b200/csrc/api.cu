@@ -21,6 +21,7 @@ int32_t kv_bits(int32_t dtype) {
         case KV_FP8_E4M3: return 8;
         case KV_INT8: return 8;
         case KV_INT4: return 4;
+        case KV_KIVI4: return 4;
         default: return 0;
     }
 }
@@ -36,9 +37,21 @@ int64_t row_bytes(const kv_pool_desc* d) {
 // Pools of codes with per-(token, kv head) parameters: one fp32 scale (FP8,
 // INT8) or an fp32 (scale, zero point) pair (INT4).
 bool quantized(int32_t dtype) {
-    return dtype == KV_FP8_E4M3 || dtype == KV_INT8 || dtype == KV_INT4;
+    return dtype == KV_FP8_E4M3 || dtype == KV_INT8 || dtype == KV_INT4 || dtype == KV_KIVI4;
 }
-int32_t param_bytes(int32_t dtype) { return dtype == KV_INT4 ? 8 : (quantized(dtype) ? 4 : 0); }
+
+// Bytes of the scale / parameter pool per (block, kv head): fp32 scales of 16
+// K and 16 V rows (8-bit), (scale, zero) pairs of the 32 rows (INT4), or of 128
+// key channels and 16 value rows (KIVI).
+int64_t params_per_tile(int32_t dtype) {
+    switch (dtype) {
+        case KV_FP8_E4M3:
+        case KV_INT8: return 2 * kBlockTokens * 4;
+        case KV_INT4: return 2 * kBlockTokens * 8;
+        case KV_KIVI4: return (128 + kBlockTokens) * 8;
+        default: return 0;
+    }
+}
 
 // SM count of the current device; 148 (B200) when no device can be queried.
 int32_t current_sm_count() {
@@ -55,7 +68,7 @@ bool valid_pool(const kv_pool_desc* d) {
     return d != nullptr && d->num_blocks > 0 && d->block_size == kBlockTokens &&
            d->num_kv_heads > 0 && (d->head_dim == 64 || d->head_dim == 128) &&
            kv_bits(d->dtype) != 0 && elem_bytes(d->dtype) == d->elem_bytes &&
-           (d->dtype != KV_INT4 || d->head_dim == 128);
+           ((d->dtype != KV_INT4 && d->dtype != KV_KIVI4) || d->head_dim == 128);
 }
 
 int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
@@ -86,7 +99,7 @@ kv_status encode_pool_map(CUtensorMap* map, const void* base, const kv_pool_desc
     if (encode == nullptr) return KV_ERR_CUDA;
     const cuuint64_t rows = static_cast<cuuint64_t>(pool->num_blocks) * pool->num_kv_heads *
                             kBlockTokens;
-    const bool int4 = pool->dtype == KV_INT4;
+    const bool int4 = kv_bits(pool->dtype) == 4;
     const int64_t rb = row_bytes(pool);
     const cuuint64_t dims[2] = {int4 ? static_cast<cuuint64_t>(rb)
                                      : static_cast<cuuint64_t>(pool->head_dim), rows};
@@ -113,7 +126,7 @@ kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_
     if (out == nullptr || num_blocks <= 0 || block_size <= 0 || num_kv_heads <= 0 || head_dim <= 0)
         return KV_ERR_INVALID_ARGUMENT;
     if (block_size != kBlockTokens || (head_dim != 64 && head_dim != 128) || num_kv_heads > 256 ||
-        kv_bits(dtype) == 0 || (dtype == KV_INT4 && head_dim != 128))
+        kv_bits(dtype) == 0 || (kv_bits(dtype) == 4 && head_dim != 128))
         return KV_ERR_UNSUPPORTED;
     kv_pool_desc d{};
     d.num_blocks = num_blocks;
@@ -126,8 +139,8 @@ kv_status kv_pool_create(int32_t num_blocks, int32_t block_size, int32_t num_kv_
     d.stride_head = static_cast<int64_t>(block_size) * head_dim;
     d.stride_block = d.stride_head * num_kv_heads;
     d.kv_bytes = static_cast<uint64_t>(d.stride_block) * num_blocks * kv_bits(dtype) / 8u;
-    d.scale_bytes = static_cast<uint64_t>(num_blocks) * num_kv_heads * 2u * block_size *
-                    static_cast<uint64_t>(param_bytes(dtype));
+    d.scale_bytes = static_cast<uint64_t>(num_blocks) * num_kv_heads *
+                    static_cast<uint64_t>(params_per_tile(dtype));
     *out = d;
     return KV_OK;
 }
@@ -163,6 +176,7 @@ kv_status reshape_and_cache(const kv_pool_desc* pool, void* k_pool, void* v_pool
     const int64_t num_slots = static_cast<int64_t>(pool->num_blocks) * kBlockTokens;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e;
+    if (pool->dtype == KV_KIVI4) return KV_ERR_UNSUPPORTED;  // kivi_quantize_blocks / the append
     if (quantized(pool->dtype)) {
         if (src_dtype != KV_F32 && src_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
         if (scales == nullptr) return KV_ERR_INVALID_ARGUMENT;
@@ -190,8 +204,7 @@ kv_status paged_kv_copy_blocks(const kv_pool_desc* pool, void* k_pool, void* v_p
     const bool fp8 = quantized(pool->dtype);  // FP8, INT8 or INT4: a parameter pool
     if (fp8 != (scales != nullptr) || (fp8 && !aligned16(scales))) return KV_ERR_INVALID_ARGUMENT;
     const int64_t block_bytes = row_bytes(pool) * kBlockTokens * pool->num_kv_heads;
-    const int64_t scale_bytes =
-        static_cast<int64_t>(pool->num_kv_heads) * 2 * kBlockTokens * param_bytes(pool->dtype);
+    const int64_t scale_bytes = static_cast<int64_t>(pool->num_kv_heads) * params_per_tile(pool->dtype);
     cudaError_t e = pkv::launch_copy_blocks(k_pool, v_pool, scales, copy_src, copy_dst,
                                             num_copies, block_bytes, scale_bytes,
                                             pool->num_blocks, dev_error,
@@ -251,6 +264,17 @@ size_t workspace_bytes_for(const kv_pool_desc* pool, int32_t batch, int32_t num_
     return ws_layout(pool, batch, num_q_heads, query_tokens, ranges).total;
 }
 
+// The bf16 residual (newest L mod 16 tokens) of a KIVI call, and its new rows.
+struct KiviArgs {
+    void* k_pool;
+    void* v_pool;
+    float* params;
+    uint16_t* res_k;
+    uint16_t* res_v;
+    const void* k_new;  // nullable: no append
+    const void* v_new;
+};
+
 // The new token rows of a fused append+decode call.
 struct AppendArgs {
     void* k_pool;
@@ -268,10 +292,13 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
                          int32_t num_q_heads, int32_t max_context_len, float scale,
                          int32_t partition_tokens, void* workspace, size_t workspace_bytes,
                          int32_t* dev_error, kv_stream_t stream,
-                         const AppendArgs* app = nullptr) {
+                         const AppendArgs* app = nullptr, const KiviArgs* kivi = nullptr) {
     if (!valid_pool(pool) || batch < 0 || num_q_heads <= 0 || max_blocks_per_seq < 0 ||
         query_tokens < 1 || (app != nullptr && query_tokens != 1))
         return KV_ERR_INVALID_ARGUMENT;
+    // KIVI pools go through kivi_decode_attention (one query token), and only they
+    if ((pool->dtype == KV_KIVI4) != (kivi != nullptr)) return KV_ERR_UNSUPPORTED;
+    if (kivi != nullptr && query_tokens != 1) return KV_ERR_UNSUPPORTED;
     if (app != nullptr) {
         // no conversion for 16/32-bit pools (as reshape_and_cache); 8-bit pools quantise
         const bool src_ok = quantized(pool->dtype)
@@ -288,7 +315,8 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
                              group * query_tokens > 16))
         return KV_ERR_UNSUPPORTED;
     // 4-bit codes have only the tensor-core tile (bf16 q, head_dim 128)
-    if (pool->dtype == KV_INT4 && !pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim))
+    if (kv_bits(pool->dtype) == 4 &&
+        !pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim))
         return KV_ERR_UNSUPPORTED;
     if (batch == 0) return KV_OK;
     if (max_context_len < query_tokens ||
@@ -311,6 +339,11 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
     if (fp8 && !aligned16(scales)) return KV_ERR_INVALID_ARGUMENT;
     if (app != nullptr && (app->k_new == nullptr || app->v_new == nullptr ||
                            !aligned16(app->k_new) || !aligned16(app->v_new)))
+        return KV_ERR_INVALID_ARGUMENT;
+    if (kivi != nullptr &&
+        (kivi->res_k == nullptr || kivi->res_v == nullptr || !aligned16(kivi->res_k) ||
+         !aligned16(kivi->res_v) || ((kivi->k_new == nullptr) != (kivi->v_new == nullptr)) ||
+         (kivi->k_new != nullptr && (!aligned16(kivi->k_new) || !aligned16(kivi->v_new)))))
         return KV_ERR_INVALID_ARGUMENT;
 
     const int32_t ranges = num_ranges_for(pool, batch, num_q_heads, query_tokens,
@@ -350,6 +383,11 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
         p.scales_dst = app->scales;
         p.append_src_dtype = app->src_dtype;
     }
+    if (kivi != nullptr) {
+        p.kivi = 1;
+        p.res_k = kivi->res_k;
+        p.res_v = kivi->res_v;
+    }
     pkv::TmaMaps maps{};
     if (pkv::decode_uses_tensor_cores(pool->dtype, q_dtype, pool->head_dim)) {
         // TMA row coordinates are 32-bit
@@ -360,8 +398,16 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
         if (st == KV_OK) st = encode_pool_map(&maps.v, v_pool, pool);
         if (st != KV_OK) return st;
     }
-    cudaError_t e = pkv::launch_paged_decode(p, maps, pool->dtype, q_dtype, pool->head_dim,
-                                             group, reinterpret_cast<cudaStream_t>(stream));
+    cudaError_t e = cudaSuccess;
+    if (kivi != nullptr && kivi->k_new != nullptr)  // residual row, and the block it completes
+        e = pkv::launch_kivi_append(kivi->k_pool, kivi->v_pool, kivi->params, kivi->res_k,
+                                    kivi->res_v, kivi->k_new, kivi->v_new, block_table,
+                                    max_blocks_per_seq, context_lens, batch, pool->num_kv_heads,
+                                    max_context_len, pool->num_blocks, dev_error,
+                                    reinterpret_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess)
+        e = pkv::launch_paged_decode(p, maps, pool->dtype, q_dtype, pool->head_dim, group,
+                                     reinterpret_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
@@ -415,6 +461,44 @@ kv_status paged_decode_attention_append(const kv_pool_desc* pool, void* out, con
                           max_blocks_per_seq, context_lens, batch, num_q_heads, max_context_len,
                           scale, partition_tokens, workspace, workspace_bytes, dev_error, stream,
                           &app);
+}
+
+kv_status kivi_decode_attention(const kv_pool_desc* pool, void* out, const void* q,
+                                kv_dtype q_dtype, void* k_pool, void* v_pool, float* params,
+                                void* res_k, void* res_v, const void* k_new, const void* v_new,
+                                const int32_t* block_table, int32_t max_blocks_per_seq,
+                                const int32_t* context_lens, int32_t batch, int32_t num_q_heads,
+                                int32_t max_context_len, float scale, int32_t partition_tokens,
+                                void* workspace, size_t workspace_bytes, int32_t* dev_error,
+                                kv_stream_t stream) {
+    const KiviArgs kv{k_pool, v_pool, params, static_cast<uint16_t*>(res_k),
+                      static_cast<uint16_t*>(res_v), k_new, v_new};
+    return attention_impl(pool, out, q, q_dtype, 1, k_pool, v_pool, params, block_table,
+                          max_blocks_per_seq, context_lens, batch, num_q_heads, max_context_len,
+                          scale, partition_tokens, workspace, workspace_bytes, dev_error, stream,
+                          nullptr, &kv);
+}
+
+kv_status kivi_quantize_blocks(const kv_pool_desc* pool, void* k_pool, void* v_pool, float* params,
+                               const void* k_rows, const void* v_rows, kv_dtype src_dtype,
+                               const int32_t* block_ids, int32_t num_blocks, int32_t* dev_error,
+                               kv_stream_t stream) {
+    if (!valid_pool(pool) || pool->dtype != KV_KIVI4 || num_blocks < 0)
+        return pool != nullptr && valid_pool(pool) && pool->dtype != KV_KIVI4
+                   ? KV_ERR_UNSUPPORTED
+                   : KV_ERR_INVALID_ARGUMENT;
+    if (src_dtype != KV_F32 && src_dtype != KV_BF16) return KV_ERR_UNSUPPORTED;
+    if (num_blocks == 0) return KV_OK;
+    if (k_pool == nullptr || v_pool == nullptr || params == nullptr || k_rows == nullptr ||
+        v_rows == nullptr || block_ids == nullptr)
+        return KV_ERR_INVALID_ARGUMENT;
+    if (!aligned16(k_pool) || !aligned16(v_pool) || !aligned16(params) || !aligned16(k_rows) ||
+        !aligned16(v_rows))
+        return KV_ERR_INVALID_ARGUMENT;
+    const cudaError_t e = pkv::launch_kivi_quantize_blocks(
+        src_dtype, k_pool, v_pool, params, k_rows, v_rows, block_ids, num_blocks,
+        pool->num_kv_heads, pool->num_blocks, dev_error, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KV_OK : KV_ERR_CUDA;
 }
 
 kv_status paged_attention_multi_query(const kv_pool_desc* pool, void* out, const void* q,

@@ -68,11 +68,16 @@ template <>
 struct KvElem<KV_INT4> {  // two codes per byte: row sizes are computed from bits instead
     static constexpr int kBytes = 0;
 };
+template <>
+struct KvElem<KV_KIVI4> {
+    static constexpr int kBytes = 0;
+};
 
 // Quantised pools carry per-(token, kv head) parameters: an fp32 scale (8-bit
 // codes) or an fp32 (scale, zero point) pair (4-bit codes).
 template <int KV_T>
-inline constexpr bool kQuantized = KV_T == KV_FP8_E4M3 || KV_T == KV_INT8 || KV_T == KV_INT4;
+inline constexpr bool kQuantized =
+    KV_T == KV_FP8_E4M3 || KV_T == KV_INT8 || KV_T == KV_INT4 || KV_T == KV_KIVI4;
 
 // Two 8-bit codes (low 16 bits) -> two floats (code values, before the row scale).
 template <int KV_T>
@@ -270,6 +275,17 @@ __device__ __forceinline__ void widen_v4(uint32_t w, uint32_t& lo, uint32_t& hi)
     else e4m3x4_to_f16x2x2(__byte_perm(w, 0u, 0x3120), lo, hi);
 }
 
+__device__ __forceinline__ uint32_t hmul2u(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+__device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // Eight 4-bit codes c (one 32-bit word, nibble i = element i) -> four f16x2 of
 // exact values c * 2^-9: the byte 0x0c is the E4M3 code of c * 2^-9 for every c
 // in 0..15 (subnormals and the first binade share the step 2^-9).
@@ -299,12 +315,16 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
 }
 
 // ---- tile list bookkeeping ----------------------------------------------------------
-// Tiles of a sequence with context length L: ceil(L/16), or 0 when L is invalid
-// (shorter than the query tokens it must hold, or longer than max_context_len).
+// A context length is valid when it holds the query tokens and fits max_context_len.
+__device__ __forceinline__ bool seq_valid(int32_t L, const DecodeParams& p) {
+    return L >= p.num_query_tokens && L >= 1 && L <= p.max_context_len;
+}
+
+// Tiles of a sequence with context length L: ceil(L/16) -- for KIVI pools the
+// full blocks only, floor(L/16) -- or 0 when L is invalid.
 __device__ __forceinline__ int32_t seq_tiles(int32_t L, const DecodeParams& p) {
-    return (L >= p.num_query_tokens && L >= 1 && L <= p.max_context_len)
-               ? (L + kBlockTokens - 1) / kBlockTokens
-               : 0;
+    if (!seq_valid(L, p)) return 0;
+    return p.kivi ? L / kBlockTokens : (L + kBlockTokens - 1) / kBlockTokens;
 }
 
 // First tile of consumer range W (ranges are equal cuts of the T-tile list).
@@ -666,11 +686,16 @@ struct MmaMath {
     static_assert(G <= 8, "a row set holds 8 query rows");
     using OutT = uint16_t;                                        // bf16 output
     static constexpr bool kF16 = kQuantized<KV_T>;              // codes widened to f16
-    static constexpr bool kI4 = KV_T == KV_INT4;                // 4-bit codes, 64-byte rows
+    static constexpr bool kKivi = KV_T == KV_KIVI4;             // 4-bit, per-channel K params
+    static constexpr bool kI4 = KV_T == KV_INT4 || kKivi;       // 4-bit codes, 64-byte rows
+    static_assert(!kKivi || QM == kSingle, "KIVI pools: one query token");
+    // parameter block: INT4 (scale, zero) per K row then per V row; KIVI per K
+    // channel (128) then per V row (16), as float2
+    static constexpr int kVParams = kKivi ? 128 : kBlockTokens;
     static constexpr int D = 128;
     static constexpr int kKv = KV_T;
     static constexpr int kHeadDim = D;
-    static constexpr bool kCanAppend = SINGLE;                    // fused append: decode only
+    static constexpr bool kCanAppend = SINGLE && !kKivi;          // fused append: decode only
     static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
     static constexpr int kRowBytes = kI4 ? D / 2 : D * KvElem<KV_T>::kBytes;  // 256 / 128 / 64
     static constexpr int kBoxRow = kI4 ? 64 : 128;                // bytes of a TMA box row
@@ -679,7 +704,8 @@ struct MmaMath {
     static constexpr int kBoxBytes = kBlockTokens * kBoxRow;
     static constexpr int kTileBytes = kBlockTokens * kRowBytes;
     // K then V row parameters: fp32 scales (8-bit) or fp32 (scale, zero) pairs (4-bit)
-    static constexpr int kScaleBytes = kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0);
+    static constexpr int kScaleBytes =
+        kKivi ? (128 + kBlockTokens) * 8 : (kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0));
     static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
     static constexpr int kStages = kI4 ? 16 : (kF16 ? 12 : 8);     // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
@@ -764,9 +790,11 @@ struct MmaMath {
                     };
                     qa[k][ks][0] = pack2<true>(el(h), el(h + 2));
                     qa[k][ks][1] = pack2<true>(el(h + 4), el(h + 6));
-                    const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
-                    const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
-                    qs += (f0.x + f0.y) + (f1.x + f1.y);
+                    if constexpr (!kKivi) {
+                        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
+                        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
+                        qs += (f0.x + f0.y) + (f1.x + f1.y);
+                    }
                 } else if constexpr (!kF16) {
                     // k index 2tig+{0,1} -> dim 16ks+2tig+{0,1}; 8+2tig+{0,1} -> 16ks+8+2tig+{0,1}
                     qa[k][ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
@@ -781,7 +809,7 @@ struct MmaMath {
                                                __uint_as_float(w.y & 0xffff0000u));
                 }
             }
-            if constexpr (kI4) {
+            if constexpr (kI4 && !kKivi) {
                 qs += __shfl_xor_sync(0xffffffffu, qs, 1);
                 qs += __shfl_xor_sync(0xffffffffu, qs, 2);
                 qsum[k] = qs;
@@ -829,10 +857,34 @@ struct MmaMath {
                     nib8_to_f16x2x4(w[2 * cc], b0);
                     nib8_to_f16x2x4(w[2 * cc + 1], b1);
                     const int ka = 2 * c, kb = 2 * c + 1;
-                    mma_16816<true>(s[0], qa[0][ka][0], a_hi(ka, 0), qa[0][ka][1], a_hi(ka, 1), b0[0], b0[1]);
-                    mma_16816<true>(s[1], qa[0][ka][0], a_hi(ka, 0), qa[0][ka][1], a_hi(ka, 1), b1[0], b1[1]);
-                    mma_16816<true>(s[0], qa[0][kb][0], a_hi(kb, 0), qa[0][kb][1], a_hi(kb, 1), b0[2], b0[3]);
-                    mma_16816<true>(s[1], qa[0][kb][0], a_hi(kb, 0), qa[0][kb][1], a_hi(kb, 1), b1[2], b1[3]);
+                    uint32_t qa0 = qa[0][ka][0], qa1 = qa[0][ka][1], qb0 = qa[0][kb][0], qb1 = qa[0][kb][1];
+                    if constexpr (kKivi) {
+                        // key channel d: (c - zero_d) * scale_d.  q takes the scales (q' = q *
+                        // scale, f16), the codes the zero points ((c - zero) 2^-9, exact in f16)
+                        const float4* pc = reinterpret_cast<const float4*>(ksc) + 16 * c + 4 * tig;
+                        const float4 p01 = pc[0], p23 = pc[1], p45 = pc[2], p67 = pc[3];
+                        constexpr float kq = 1.0f / 512.0f;
+                        const uint32_t zA = pack2<true>(p01.y * kq, p23.y * kq);  // dims (0, 2)
+                        const uint32_t zB = pack2<true>(p45.y * kq, p67.y * kq);  // (4, 6)
+                        const uint32_t zC = pack2<true>(p01.w * kq, p23.w * kq);  // (1, 3)
+                        const uint32_t zD = pack2<true>(p45.w * kq, p67.w * kq);  // (5, 7)
+                        qa0 = hmul2u(qa0, pack2<true>(p01.x, p23.x));
+                        qa1 = hmul2u(qa1, pack2<true>(p45.x, p67.x));
+                        qb0 = hmul2u(qb0, pack2<true>(p01.z, p23.z));
+                        qb1 = hmul2u(qb1, pack2<true>(p45.z, p67.z));
+                        b0[0] = hsub2u(b0[0], zA);
+                        b0[1] = hsub2u(b0[1], zB);
+                        b0[2] = hsub2u(b0[2], zC);
+                        b0[3] = hsub2u(b0[3], zD);
+                        b1[0] = hsub2u(b1[0], zA);
+                        b1[1] = hsub2u(b1[1], zB);
+                        b1[2] = hsub2u(b1[2], zC);
+                        b1[3] = hsub2u(b1[3], zD);
+                    }
+                    mma_16816<true>(s[0], qa0, a_hi(ka, 0), qa1, a_hi(ka, 1), b0[0], b0[1]);
+                    mma_16816<true>(s[1], qa0, a_hi(ka, 0), qa1, a_hi(ka, 1), b1[0], b1[1]);
+                    mma_16816<true>(s[0], qb0, a_hi(kb, 0), qb1, a_hi(kb, 1), b0[2], b0[3]);
+                    mma_16816<true>(s[1], qb0, a_hi(kb, 0), qb1, a_hi(kb, 1), b1[2], b1[3]);
                 }
             }
         } else if constexpr (!kF16) {
@@ -874,7 +926,9 @@ struct MmaMath {
                 for (int j = 0; j < 2; ++j) {
                     const int t = 8 * nt + 2 * tig + j;
                     float v;
-                    if constexpr (kI4) {
+                    if constexpr (kKivi) {
+                        v = 512.0f * s[nt][2 * k + j] * p.scale_log2;  // parameters are in q', codes
+                    } else if constexpr (kI4) {
                         // (c - zero) * scale: sum_d q_d (c_d 2^-9) 512 - zero * sum_d q_d
                         const float2 pz = reinterpret_cast<const float2*>(ksc)[t];
                         v = (512.0f * s[nt][2 * k + j] - pz.y * qsum[k]) * pz.x * p.scale_log2;
@@ -936,7 +990,7 @@ struct MmaMath {
             if constexpr (kI4) {
                 // O = sum_t p_t scale_t (c_t - zero_t): P' = p * scale, and the zero
                 // term sum_t P'_t zero_t is kept per row (b_run)
-                const float2* vpz = reinterpret_cast<const float2*>(ksc) + kBlockTokens;
+                const float2* vpz = reinterpret_cast<const float2*>(ksc) + kVParams;
                 float bsum = 0.0f;
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
@@ -1366,7 +1420,8 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
         // ---- end of a piece: at the end of a (sequence, kv head) pair or of the range
         const bool seg_end = cur.jb + 1 == cur.nt;
         if (seg_end || j == n - 1) {
-            const bool whole = seg_end && piece_start == cur.seg_start;
+            // KIVI pairs always end in the merge, which adds the bf16 residual tokens
+            const bool whole = seg_end && piece_start == cur.seg_start && !p.kivi;
             const int64_t pid = static_cast<int64_t>(cur.b) * p.num_kv_heads + cur.kvh + W;
             math.finish(p, cur.b, cur.kvh, whole, pid);
             if (j + 1 < n) {
@@ -1413,16 +1468,17 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
     const int64_t seq0 = p.ws_seq_start[b];
     const int32_t nt = seq_tiles(L, p);
     OutT* out = static_cast<OutT*>(p.out) + bh * D + lane * kDPL;
-    if (nt == 0) {
+    if (!seq_valid(L, p)) {
 #pragma unroll
         for (int j = 0; j < kDPL; ++j) out[j] = out_cast<OutT>(0.0f);
         if (lane == 0 && g == 0 && kvh == 0) report(p.dev_error, KV_DEVERR_BAD_CONTEXT_LEN);
         return;
     }
     const int64_t a = seq0 + static_cast<int64_t>(kvh) * nt;
-    const int64_t w_first = range_of(a, T, p.num_ranges);
-    const int64_t w_last = range_of(a + nt - 1, T, p.num_ranges);
-    if (w_first == w_last) return;  // the pair was one range's: written by the decode kernel
+    const int64_t w_first = nt > 0 ? range_of(a, T, p.num_ranges) : 0;
+    const int64_t w_last = nt > 0 ? range_of(a + nt - 1, T, p.num_ranges) : -1;
+    // a pair within one range was written by the decode kernel (KIVI: never)
+    if (!p.kivi && w_first == w_last) return;
     const int64_t s = static_cast<int64_t>(b) * p.num_kv_heads + kvh;
     const int32_t npieces = static_cast<int32_t>(w_last - w_first + 1);
     // pieces are (pair s, range W) for the non-empty ranges W in [w_first, w_last],
@@ -1491,6 +1547,35 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
             }
         }
     }
+    if (p.kivi) {
+        // KIVI: the newest L mod 16 tokens, kept in bf16 at res_k / res_v
+        // [batch][Hkv][16][D], join the softmax (same base-2 scores)
+        const int32_t nres = L % kBlockTokens;
+        float qf[kDPL];
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) qf[j] = load_q_elem<Q_T>(p.q, bh * D + lane * kDPL + j);
+        const int64_t rbase = ((static_cast<int64_t>(b) * p.num_kv_heads + kvh) * kBlockTokens) * D +
+                              lane * kDPL;
+        for (int r = 0; r < nres; ++r) {
+            const uint16_t* kr = p.res_k + rbase + r * D;
+            const uint16_t* vr = p.res_v + rbase + r * D;
+            float dot = 0.0f;
+#pragma unroll
+            for (int j = 0; j < kDPL; ++j)
+                dot = fmaf(qf[j], __uint_as_float(static_cast<uint32_t>(kr[j]) << 16), dot);
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
+            const float sc = dot * p.scale_log2;
+            const float M_new = fmaxf(M, sc);
+            const float c = exp2f(M - M_new);
+            const float w = exp2f(sc - M_new);
+            M = M_new;
+            l = l * c + (lane == 0 ? w : 0.0f);  // l is lane-partial: count the token once
+#pragma unroll
+            for (int j = 0; j < kDPL; ++j)
+                o[j] = fmaf(w, __uint_as_float(static_cast<uint32_t>(vr[j]) << 16), o[j] * c);
+        }
+    }
 #pragma unroll
     for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
 #pragma unroll
@@ -1549,8 +1634,12 @@ template <int KV_T>
 static cudaError_t dispatch_mma(const DecodeParams& p, const TmaMaps& maps, int32_t group,
                                 cudaStream_t s) {
     if (p.num_query_tokens == 1) return dispatch_mma_g<KV_T, kSingle>(p, maps, group, s);
-    return group * p.num_query_tokens > 8 ? dispatch_mma_g<KV_T, kWide>(p, maps, group, s)
-                                          : dispatch_mma_g<KV_T, kNarrow>(p, maps, group, s);
+    if constexpr (KV_T == KV_KIVI4) {
+        return cudaErrorInvalidValue;  // one query token only
+    } else {
+        return group * p.num_query_tokens > 8 ? dispatch_mma_g<KV_T, kWide>(p, maps, group, s)
+                                              : dispatch_mma_g<KV_T, kNarrow>(p, maps, group, s);
+    }
 }
 
 template <int KV_T, int Q_T>
@@ -1569,7 +1658,7 @@ static cudaError_t dispatch_q(const DecodeParams& p, const TmaMaps& maps, int32_
 
 bool decode_uses_tensor_cores(int32_t kv_dtype, int32_t q_dtype, int32_t head_dim) {
     return (kv_dtype == KV_BF16 || kv_dtype == KV_FP8_E4M3 || kv_dtype == KV_INT8 ||
-            kv_dtype == KV_INT4) &&
+            kv_dtype == KV_INT4 || kv_dtype == KV_KIVI4) &&
            q_dtype == KV_BF16 &&
            head_dim == 128;
 }
@@ -1582,11 +1671,12 @@ cudaError_t launch_paged_decode(const DecodeParams& p, const TmaMaps& maps, int3
             case KV_BF16: return dispatch_mma<KV_BF16>(p, maps, group, stream);
             case KV_INT8: return dispatch_mma<KV_INT8>(p, maps, group, stream);
             case KV_INT4: return dispatch_mma<KV_INT4>(p, maps, group, stream);
+            case KV_KIVI4: return dispatch_mma<KV_KIVI4>(p, maps, group, stream);
             default: return dispatch_mma<KV_FP8_E4M3>(p, maps, group, stream);
         }
     }
     // (4-bit pools have only the tensor-core tile; the host rejects other shapes)
-    if (kv_dtype == KV_INT4) return cudaErrorInvalidValue;
+    if (kv_dtype == KV_INT4 || kv_dtype == KV_KIVI4) return cudaErrorInvalidValue;
     switch (kv_dtype) {
         case KV_F32: return dispatch_q<KV_F32>(p, maps, q_dtype, head_dim, group, stream);
         case KV_BF16: return dispatch_q<KV_BF16>(p, maps, q_dtype, head_dim, group, stream);

@@ -74,7 +74,26 @@ struct DecodeParams {
     uint8_t* v_dst;
     float* scales_dst;
     int32_t append_src_dtype;
+    // KIVI pools: only full blocks are tiles; every pair ends in the merge, which
+    // also attends to the sequence's newest L mod 16 tokens, kept in bf16 at
+    // res_k / res_v [batch][Hkv][16][D]
+    int32_t kivi;
+    const uint16_t* res_k;
+    const uint16_t* res_v;
 };
+
+cudaError_t launch_kivi_quantize_blocks(int32_t src_dtype, void* k_pool, void* v_pool,
+                                        float* params, const void* k_rows, const void* v_rows,
+                                        const int32_t* block_ids, int32_t num_blocks,
+                                        int32_t num_kv_heads, int32_t pool_blocks,
+                                        int32_t* dev_error, cudaStream_t stream);
+
+cudaError_t launch_kivi_append(void* k_pool, void* v_pool, float* params, uint16_t* res_k,
+                               uint16_t* res_v, const void* k_new, const void* v_new,
+                               const int32_t* block_table, int32_t max_blocks,
+                               const int32_t* context_lens, int32_t batch, int32_t num_kv_heads,
+                               int32_t max_context_len, int32_t pool_blocks, int32_t* dev_error,
+                               cudaStream_t stream);
 
 // TMA descriptors of the K and V pools as 2-D tensors [num_blocks*Hkv*16 rows][head_dim],
 // boxes of 16 rows x 128 bytes with the 128-byte swizzle (tensor-core path only).

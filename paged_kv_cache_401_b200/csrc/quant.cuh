@@ -66,13 +66,32 @@ __device__ __forceinline__ uint32_t quantize_row_warp(const float* x, float* sca
 }
 
 // INT4 ("llm-inference-optimization" notes §四: the printed 4-bit routine,
-// asymmetric with a zero point, here applied to one row), in IEEE fp32:
+// asymmetric with a zero point), in IEEE fp32, on a group of values:
 //   hi = max x, lo = min x, scale = (hi - lo) / 15, zero = rint(-lo / scale),
 //   code = clamp(rint(x / scale) + zero, 0, 15); value = (code - zero) * scale.
-// A constant row (where the routine would divide by zero) is stored exactly:
+// A constant group (where the routine would divide by zero) is stored exactly:
 // scale = |lo|, zero = -1 / +1 / 0 for lo > 0 / < 0 / == 0, every code 0.
-// Returns this lane's 4 codes (head_dim 128) packed two per byte, the lane's
-// first element in the low nibble of the low byte.
+// The group is a row (INT4 pools), or for KIVI pools one channel of a full
+// block's keys and one value row.
+__device__ __forceinline__ bool int4_params(float hi, float lo, float* scale, float* zero) {
+    if (hi == lo) {
+        *scale = fabsf(lo);
+        *zero = lo > 0.0f ? -1.0f : (lo < 0.0f ? 1.0f : 0.0f);
+        return false;  // every code 0
+    }
+    const float s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+    *scale = s;
+    *zero = rintf(__fdiv_rn(-lo, s));
+    return true;
+}
+
+__device__ __forceinline__ uint32_t int4_code(float x, float s, float z) {
+    return static_cast<uint32_t>(fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x, s)), z), 0.0f), 15.0f));
+}
+
+// One row held by the warp (lane l: elements 4l .. 4l+3 of a 128-element row).
+// Returns the lane's 4 codes packed two per byte, its first element in the low
+// nibble of the low byte.
 template <int D>
 __device__ __forceinline__ uint32_t quantize_row_int4_warp(const float* x, float* scale,
                                                            float* zero) {
@@ -89,22 +108,33 @@ __device__ __forceinline__ uint32_t quantize_row_int4_warp(const float* x, float
         hi = fmaxf(hi, __shfl_xor_sync(0xffffffffu, hi, m));
         lo = fminf(lo, __shfl_xor_sync(0xffffffffu, lo, m));
     }
+    float s, z;
     uint32_t codes = 0;
-    if (hi == lo) {
-        *scale = fabsf(lo);
-        *zero = lo > 0.0f ? -1.0f : (lo < 0.0f ? 1.0f : 0.0f);
-        return codes;
-    }
-    const float s = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
-    const float z = rintf(__fdiv_rn(-lo, s));
+    if (int4_params(hi, lo, &s, &z)) {
 #pragma unroll
-    for (int e = 0; e < kPer; ++e) {
-        const float c = fminf(fmaxf(__fadd_rn(rintf(__fdiv_rn(x[e], s)), z), 0.0f), 15.0f);
-        codes |= static_cast<uint32_t>(c) << (4 * e);
+        for (int e = 0; e < kPer; ++e) codes |= int4_code(x[e], s, z) << (4 * e);
     }
     *scale = s;
     *zero = z;
     return codes;
+}
+
+// One group of 16 values held by one thread (a KIVI key channel over a block);
+// codes[t] for value t.
+__device__ __forceinline__ void quantize_group16_int4(const float* x, uint32_t* codes,
+                                                      float* scale, float* zero) {
+    float hi = x[0], lo = x[0];
+#pragma unroll
+    for (int t = 1; t < 16; ++t) {
+        hi = fmaxf(hi, x[t]);
+        lo = fminf(lo, x[t]);
+    }
+    float s, z;
+    const bool any = int4_params(hi, lo, &s, &z);
+#pragma unroll
+    for (int t = 0; t < 16; ++t) codes[t] = any ? int4_code(x[t], s, z) : 0u;
+    *scale = s;
+    *zero = z;
 }
 
 // Store a lane's packed codes (D/32 bytes) at dst.

@@ -23,6 +23,7 @@ TOL = {  # max-abs, max-rel (relative to the output's max magnitude)
     "fp8": (5e-2, None),
     "int8": (5e-2, None),
     "int4": (5e-2, None),
+    "kivi4": (5e-2, None),
 }
 
 
@@ -116,3 +117,65 @@ def check_close(gpu: torch.Tensor, ref: np.ndarray, kv_dtype: str) -> dict:
     if rtol is not None:
         assert max_rel <= rtol, f"max-rel {max_rel:.3e} > {rtol}"
     return {"max_abs": max_abs, "max_rel": max_rel}
+
+
+# ---------------------------------------------------------------- KIVI pools
+@dataclass
+class KiviStaged:
+    inp: Inputs
+    cache: PagedKVCache
+    block_table: torch.Tensor
+    context_lens: torch.Tensor
+    q: torch.Tensor
+    k_new: torch.Tensor
+    v_new: torch.Tensor
+
+    @property
+    def max_context_len(self) -> int:
+        return self.inp.max_context_len
+
+
+def stage_kivi(inp: Inputs, device="cuda", chunk: int = 4096) -> KiviStaged:
+    """History (positions 0 .. L-2) through the library: full blocks quantised by
+    kivi_quantize_blocks, the incomplete block's rows copied into the residual."""
+    from workloads import kivi_layout
+    spec = inp.spec
+    cache = PagedKVCache(inp.num_blocks, spec.num_kv_heads, spec.head_dim, "kivi4", device,
+                         poison=True)
+    res_k, res_v = cache.alloc_residual(inp.q.shape[0], poison=True)
+    lay = kivi_layout(inp)
+    for c0 in range(0, len(lay.block_ids), chunk):
+        rows = torch.from_numpy(lay.block_rows[c0:c0 + chunk].reshape(-1))
+        n = min(chunk, len(lay.block_ids) - c0)
+        shape = (n, 16, spec.num_kv_heads, spec.head_dim)
+        cache.kivi_fill(torch.from_numpy(lay.block_ids[c0:c0 + chunk]).to(device),
+                        inp.k[rows].reshape(shape).to(device), inp.v[rows].reshape(shape).to(device))
+    if len(lay.res_rows):
+        rr = torch.from_numpy(lay.res_rows)
+        sq, sl = torch.from_numpy(lay.res_seq).long(), torch.from_numpy(lay.res_slot).long()
+        res_k[sq, :, sl] = inp.k[rr].to(device)
+        res_v[sq, :, sl] = inp.v[rr].to(device)
+    app = torch.from_numpy(inp.append_rows)
+    return KiviStaged(inp=inp, cache=cache,
+                      block_table=torch.from_numpy(np.ascontiguousarray(inp.block_table)).to(device),
+                      context_lens=torch.from_numpy(inp.context_lens).to(device),
+                      q=inp.q.to(device), k_new=inp.k[app].to(device), v_new=inp.v[app].to(device))
+
+
+def oracle_out_kivi(inp: Inputs, seqs=None, lens=None) -> tuple[np.ndarray, np.ndarray]:
+    """Oracle decode over each sequence's first lens[b] tokens (default: its
+    context) as a KIVI cache holds them: full blocks quantised, the rest exact."""
+    spec = inp.spec
+    seqs = np.arange(inp.q.shape[0]) if seqs is None else np.asarray(seqs)
+    lens = inp.context_lens if lens is None else np.asarray(lens, dtype=np.int32)
+    ks, vs, offs, o = [], [], [], 0
+    for b in seqs:
+        a, n = int(inp.seq_offsets[b]), int(lens[b])
+        k64, v64 = oracle.kivi_sequence(inp.k[a:a + n].float().numpy(),
+                                        inp.v[a:a + n].float().numpy())
+        ks.append(k64), vs.append(v64), offs.append(o)
+        o += n
+    out = oracle.decode_attention(storage_view(inp.q)[seqs], np.concatenate(ks), np.concatenate(vs),
+                                  np.array(offs, np.int64), lens[seqs], spec.scale,
+                                  spec.num_kv_heads, "f64", spec.q_dtype)
+    return seqs, out

@@ -63,7 +63,7 @@ class Spec:
 
     @property
     def source_dtype(self) -> str:
-        return "bf16" if self.kv_dtype in ("fp8", "int8", "int4") else self.kv_dtype
+        return "bf16" if self.kv_dtype in ("fp8", "int8", "int4", "kivi4") else self.kv_dtype
 
 
 WORKLOADS = {
@@ -88,6 +88,9 @@ WORKLOADS = {
                  scale=1.0 / math.sqrt(128.0)),
     "int4": Spec("int4", 6, batch=64, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  kv_dtype="int4", q_dtype="bf16", lens=("uniform", 1024, 16384),
+                 scale=1.0 / math.sqrt(128.0)),
+    "kivi": Spec("kivi", 7, batch=64, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 kv_dtype="kivi4", q_dtype="bf16", lens=("uniform", 1024, 16384),
                  scale=1.0 / math.sqrt(128.0)),
 }
 
@@ -253,3 +256,35 @@ def storage_view(t: torch.Tensor) -> np.ndarray:
     if t.dtype == torch.uint8:
         return t.numpy()
     raise TypeError(t.dtype)
+
+
+@dataclass
+class KiviLayout:
+    """Where a KIVI cache keeps each history token (positions 0 .. L-2 of every
+    sequence; position L-1 is the step's new token): full blocks, 16 rows each,
+    and the rows of the incomplete last block, which stay unquantised."""
+    block_rows: np.ndarray     # int64 [n][16]: rows of k/v (token order) of each full block
+    block_ids: np.ndarray      # int32 [n]: the physical block each one goes to
+    res_seq: np.ndarray        # int32 [m]: sequence of each residual row
+    res_slot: np.ndarray       # int32 [m]: its row in the sequence's residual (0..15)
+    res_rows: np.ndarray       # int64 [m]: its row of k/v
+
+
+def kivi_layout(inp: Inputs) -> KiviLayout:
+    rows, ids, rs, rsl, rr = [], [], [], [], []
+    for b in range(inp.q.shape[0]):
+        hist = int(inp.context_lens[b]) - 1
+        full = hist // BLOCK_SIZE
+        base = int(inp.seq_offsets[b])
+        for j in range(full):
+            rows.append(base + j * BLOCK_SIZE + np.arange(BLOCK_SIZE))
+            ids.append(int(inp.block_table[b, j]))
+        n = hist - full * BLOCK_SIZE
+        rs.extend([b] * n)
+        rsl.extend(range(n))
+        rr.extend(base + full * BLOCK_SIZE + np.arange(n))
+    return KiviLayout(
+        block_rows=np.array(rows, dtype=np.int64).reshape(-1, BLOCK_SIZE),
+        block_ids=np.array(ids, dtype=np.int32),
+        res_seq=np.array(rs, dtype=np.int32), res_slot=np.array(rsl, dtype=np.int32),
+        res_rows=np.array(rr, dtype=np.int64))
