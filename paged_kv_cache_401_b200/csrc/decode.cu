@@ -287,20 +287,38 @@ __device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b) {
 }
 
 // Eight 4-bit codes c (one 32-bit word, nibble i = element i) -> four f16x2 of
-// exact values c * 2^-9: the byte 0x0c is the E4M3 code of c * 2^-9 for every c
-// in 0..15 (subnormals and the first binade share the step 2^-9).
-// out = {(e0, e2), (e4, e6), (e1, e3), (e5, e7)}.
-__device__ __forceinline__ void nib8_to_f16x2x4(uint32_t w, uint32_t* out) {
+// 1024 + c: pair k holds nibbles k and k + 4, each placed in the low mantissa
+// bits of f16 1024 (0x6400), one shift and one and-or per pair.  The offset
+// must come off before the MMAs (the KIVI keys subtract 1024 + zero exactly):
+// folded into the sums instead, it cost the fp32 accumulation the codes' low
+// bits (38x the error, measured).
+__device__ __forceinline__ void nib8_to_biased_f16x2x4(uint32_t w, uint32_t* out) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) out[k] = ((w >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
+}
+
+
+// Eight 4-bit codes -> four f16x2 of exact c * 2^-9 through the E4M3 conversion
+// (bytes 0..15 are the E4M3 codes of c * 2^-9: subnormals and the first binade
+// share the step 2^-9).  out = {(e0, e2), (e4, e6), (e1, e3), (e5, e7)}.
+__device__ __forceinline__ void nib8_to_f16x2x4_e4m3(uint32_t w, uint32_t* out) {
     e4m3x4_to_f16x2x2(w & 0x0F0F0F0Fu, out[0], out[1]);
     e4m3x4_to_f16x2x2((w >> 4) & 0x0F0F0F0Fu, out[2], out[3]);
 }
 
-// A transposed ldmatrix word of a 4-bit V tile: 16-bit units of two tokens t0
-// (low half) and t1, each four dims d0..d3 -> {(t0 d0, t1 d0), (t0 d2, t1 d2),
-// (t0 d1, t1 d1), (t0 d3, t1 d3)} as f16x2 of c * 2^-9.
-__device__ __forceinline__ void nib8t_to_f16x2x4(uint32_t w, uint32_t* out) {
+// A transposed ldmatrix word of a 4-bit V tile (16-bit units of tokens t0, t1,
+// four dims d0..d3 each) -> {(t0 d0, t1 d0), (t0 d2, t1 d2), (t0 d1, t1 d1),
+// (t0 d3, t1 d3)} as f16x2 of exact c * 2^-9.
+__device__ __forceinline__ void nib8t_to_f16x2x4_e4m3(uint32_t w, uint32_t* out) {
     e4m3x4_to_f16x2x2(__byte_perm(w & 0x0F0F0F0Fu, 0u, 0x3120), out[0], out[1]);
     e4m3x4_to_f16x2x2(__byte_perm((w >> 4) & 0x0F0F0F0Fu, 0u, 0x3120), out[2], out[3]);
+}
+
+// 2^x for x <= 0 (softmax weights), flushing results below 2^-126 to zero.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 // 2-D TMA tile load (no multicast) completing on an mbarrier; x is the
@@ -780,16 +798,23 @@ struct MmaMath {
                 if (r >= rows) {
                     qa[k][ks][0] = qa[k][ks][1] = 0u;
                 } else if constexpr (kI4) {
-                    // 4-bit rows: a lane's ldmatrix word is dims 32c + 8tig + 0..7 of chunk c;
-                    // k-step 2c takes dims (+0,+2 | +4,+6), k-step 2c+1 (+1,+3 | +5,+7)
+                    // 4-bit rows: a lane's ldmatrix word is dims 32c + 8tig + 0..7 of chunk c.
+                    // KIVI keys widen pairs (e, e+4): k-step 2c takes dims (+0,+4 | +1,+5),
+                    // 2c+1 (+2,+6 | +3,+7); INT4 keys widen pairs (e, e+2) through E4M3:
+                    // k-step 2c takes (+0,+2 | +4,+6), 2c+1 (+1,+3 | +5,+7)
                     const uint4 w = *reinterpret_cast<const uint4*>(q + 32 * (ks >> 1) + 8 * tig);
                     const uint32_t x[4] = {w.x, w.y, w.z, w.w};  // bf16 pairs (0,1) (2,3) ...
                     const int h = ks & 1;
                     auto el = [&](int d) {  // element d (0..7) of the lane's 8 dims as float
                         return __uint_as_float((d & 1) ? (x[d >> 1] & 0xffff0000u) : (x[d >> 1] << 16));
                     };
-                    qa[k][ks][0] = pack2<true>(el(h), el(h + 2));
-                    qa[k][ks][1] = pack2<true>(el(h + 4), el(h + 6));
+                    if constexpr (kKivi) {
+                        qa[k][ks][0] = pack2<true>(el(2 * h), el(2 * h + 4));
+                        qa[k][ks][1] = pack2<true>(el(2 * h + 1), el(2 * h + 5));
+                    } else {
+                        qa[k][ks][0] = pack2<true>(el(h), el(h + 2));
+                        qa[k][ks][1] = pack2<true>(el(h + 4), el(h + 6));
+                    }
                     if constexpr (!kKivi) {
                         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
                         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
@@ -853,25 +878,30 @@ struct MmaMath {
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = 2 * cq + cc;  // 32-dim chunk: k-steps 2c and 2c + 1
-                    uint32_t b0[4], b1[4];      // n-tiles 0 / 1: {(d0,d2), (d4,d6), (d1,d3), (d5,d7)}
-                    nib8_to_f16x2x4(w[2 * cc], b0);
-                    nib8_to_f16x2x4(w[2 * cc + 1], b1);
+                    uint32_t b0[4], b1[4];      // n-tiles 0 / 1
+                    if constexpr (kKivi) {        // 1024 + c of dims {(0,4), (1,5), (2,6), (3,7)}
+                        nib8_to_biased_f16x2x4(w[2 * cc], b0);
+                        nib8_to_biased_f16x2x4(w[2 * cc + 1], b1);
+                    } else {                      // c 2^-9 of dims {(0,2), (4,6), (1,3), (5,7)}
+                        nib8_to_f16x2x4_e4m3(w[2 * cc], b0);
+                        nib8_to_f16x2x4_e4m3(w[2 * cc + 1], b1);
+                    }
                     const int ka = 2 * c, kb = 2 * c + 1;
                     uint32_t qa0 = qa[0][ka][0], qa1 = qa[0][ka][1], qb0 = qa[0][kb][0], qb1 = qa[0][kb][1];
                     if constexpr (kKivi) {
                         // key channel d: (c - zero_d) * scale_d.  q takes the scales (q' = q *
-                        // scale, f16), the codes the zero points ((c - zero) 2^-9, exact in f16)
+                        // scale, f16), the codes the zero points ((1024 + c) - (1024 + zero),
+                        // exact in f16)
                         const float4* pc = reinterpret_cast<const float4*>(ksc) + 16 * c + 4 * tig;
                         const float4 p01 = pc[0], p23 = pc[1], p45 = pc[2], p67 = pc[3];
-                        constexpr float kq = 1.0f / 512.0f;
-                        const uint32_t zA = pack2<true>(p01.y * kq, p23.y * kq);  // dims (0, 2)
-                        const uint32_t zB = pack2<true>(p45.y * kq, p67.y * kq);  // (4, 6)
-                        const uint32_t zC = pack2<true>(p01.w * kq, p23.w * kq);  // (1, 3)
-                        const uint32_t zD = pack2<true>(p45.w * kq, p67.w * kq);  // (5, 7)
-                        qa0 = hmul2u(qa0, pack2<true>(p01.x, p23.x));
-                        qa1 = hmul2u(qa1, pack2<true>(p45.x, p67.x));
-                        qb0 = hmul2u(qb0, pack2<true>(p01.z, p23.z));
-                        qb1 = hmul2u(qb1, pack2<true>(p45.z, p67.z));
+                        const uint32_t zA = pack2<true>(1024.0f + p01.y, 1024.0f + p45.y);  // (0,4)
+                        const uint32_t zB = pack2<true>(1024.0f + p01.w, 1024.0f + p45.w);  // (1,5)
+                        const uint32_t zC = pack2<true>(1024.0f + p23.y, 1024.0f + p67.y);  // (2,6)
+                        const uint32_t zD = pack2<true>(1024.0f + p23.w, 1024.0f + p67.w);  // (3,7)
+                        qa0 = hmul2u(qa0, pack2<true>(p01.x, p45.x));
+                        qa1 = hmul2u(qa1, pack2<true>(p01.z, p45.z));
+                        qb0 = hmul2u(qb0, pack2<true>(p23.x, p67.x));
+                        qb1 = hmul2u(qb1, pack2<true>(p23.z, p67.z));
                         b0[0] = hsub2u(b0[0], zA);
                         b0[1] = hsub2u(b0[1], zB);
                         b0[2] = hsub2u(b0[2], zC);
@@ -927,9 +957,9 @@ struct MmaMath {
                     const int t = 8 * nt + 2 * tig + j;
                     float v;
                     if constexpr (kKivi) {
-                        v = 512.0f * s[nt][2 * k + j] * p.scale_log2;  // parameters are in q', codes
+                        v = s[nt][2 * k + j] * p.scale_log2;  // parameters are in q' and the codes
                     } else if constexpr (kI4) {
-                        // (c - zero) * scale: sum_d q_d (c_d 2^-9) 512 - zero * sum_d q_d
+                        // (c - zero) * scale, summed over d with q: 512 acc - zero * sum_d q_d
                         const float2 pz = reinterpret_cast<const float2*>(ksc)[t];
                         v = (512.0f * s[nt][2 * k + j] - pz.y * qsum[k]) * pz.x * p.scale_log2;
                     } else {
@@ -945,13 +975,13 @@ struct MmaMath {
             // with several query tokens a row may have seen nothing yet (max -inf):
             // exponentiate against 0 then; one query token always sees a token
             const float m_use = (!SINGLE && m_new == -INFINITY) ? 0.0f : m_new;
-            corr[k] = exp2f(m_run[k] - m_use);
+            corr[k] = fast_exp2(m_run[k] - m_use);
             float psum = 0.0f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    pr[k][nt][j] = exp2f(pr[k][nt][j] - m_use);
+                    pr[k][nt][j] = fast_exp2(pr[k][nt][j] - m_use);
                     psum += pr[k][nt][j];
                 }
             l_run[k] = l_run[k] * corr[k] + psum;
@@ -988,21 +1018,33 @@ struct MmaMath {
 #pragma unroll
         for (int k = 0; k < kSets; ++k) {
             if constexpr (kI4) {
-                // O = sum_t p_t scale_t (c_t - zero_t): P' = p * scale, and the zero
-                // term sum_t P'_t zero_t is kept per row (b_run)
+                // O = sum_t p_t scale_t (c_t - zero_t) = sum_t P'_t c_t - sum_t P'_t zero_t,
+                // P' = p * scale as the MMA sees it (f16); the second sum is kept per
+                // row (b_run)
                 const float2* vpz = reinterpret_cast<const float2*>(ksc) + kVParams;
-                float bsum = 0.0f;
+                float2 pz[2][2];
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const int t = 8 * nt + 2 * tig + j;
-                        const float2 pz = vpz[t];
-                        const float pv = pr[k][nt][j] * pz.x;
+                        pz[nt][j] = vpz[t];
+                        const float pv = pr[k][nt][j] * pz[nt][j].x;
                         pr[k][nt][j] = (t < nvalid) ? pv : 0.0f;
-                        bsum += (t < nvalid) ? pv * pz.y : 0.0f;
                     }
+                pb[k][0] = pack2<true>(pr[k][0][0], pr[k][0][1]);
+                pb[k][1] = pack2<true>(pr[k][1][0], pr[k][1][1]);
+                // (parameters past the context end may hold anything: select, never multiply)
+                float bsum = 0.0f;
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) {
+                    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pb[k][nt]));
+                    const int t = 8 * nt + 2 * tig;
+                    bsum += (t < nvalid) ? f.x * pz[nt][0].y : 0.0f;
+                    bsum += (t + 1 < nvalid) ? f.y * pz[nt][1].y : 0.0f;
+                }
                 b_run[k] = b_run[k] * corr[k] + bsum;
+                continue;
             } else if constexpr (kF16) {
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
@@ -1029,16 +1071,12 @@ struct MmaMath {
 #pragma unroll
                 for (int cc = 0; cc < 2; ++cc) {
                     const int c = 2 * cq + cc;
-                    uint32_t h0[4], h1[4];  // tokens 2tig,2tig+1 / 8+2tig,9+2tig: {d0, d2, d1, d3}
-                    nib8t_to_f16x2x4(w[2 * cc], h0);
-                    nib8t_to_f16x2x4(w[2 * cc + 1], h1);
-                    if (partial) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            h0[e] &= mask_a;
-                            h1[e] &= mask_b;
-                        }
-                    }
+                    // tokens 2tig,2tig+1 / 8+2tig,9+2tig: c 2^-9 of dims {d0, d2, d1, d3}.
+                    // Every code widens to a finite value, and tokens past the context end
+                    // have P' = 0, so no mask is needed
+                    uint32_t h0[4], h1[4];
+                    nib8t_to_f16x2x4_e4m3(w[2 * cc], h0);
+                    nib8t_to_f16x2x4_e4m3(w[2 * cc + 1], h1);
                     // m-tile 2c: rows gid <- dim 4gid, gid+8 <- 4gid+1; m-tile 2c+1: 4gid+2, 4gid+3
 #pragma unroll
                     for (int k = 0; k < kSets; ++k) {
@@ -1097,7 +1135,7 @@ struct MmaMath {
             l += __shfl_xor_sync(0xffffffffu, l, 2);
             const float lr[2] = {__shfl_sync(0xffffffffu, l, 8 * tig),        // row 8k + 2tig
                                  __shfl_sync(0xffffffffu, l, 8 * tig + 4)};   // row 8k + 2tig + 1
-            // 4-bit: O = 512 * (the MMA sums of P' c 2^-9) - sum_t P'_t zero_t
+            // 4-bit: O = 512 (the MMA sums of P' c 2^-9) - sum_t P'_t zero_t
             if constexpr (kI4) {
                 float bq = b_run[k];
                 bq += __shfl_xor_sync(0xffffffffu, bq, 1);
@@ -1384,10 +1422,27 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
     __syncthreads();
     if (n <= 0) return;
 
+    // When the range goes on past the current pair, bring the next pair's q rows
+    // into L1 now, so switching pairs does not wait on them (one query token).
+    auto prefetch_next_q = [&]() {
+        if (p.num_query_tokens != 1 || lo + n <= cur.seg_start + cur.nt) return;
+        const int32_t G = p.num_q_heads / p.num_kv_heads;
+        const bool same_b = cur.kvh + 1 < p.num_kv_heads;
+        const int32_t b = same_b ? cur.b : cur.b + 1, kvh = same_b ? cur.kvh + 1 : 0;
+        constexpr int kQBytes = Q_T == KV_F32 ? 4 : 2;
+        const int32_t bytes = G * M::kHeadDim * kQBytes;
+        if (b < p.batch && lane * 128 < bytes)
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(
+                static_cast<const uint8_t*>(p.q) +
+                (static_cast<int64_t>(b) * p.num_q_heads + kvh * G) * M::kHeadDim * kQBytes +
+                lane * 128));
+    };
+
     M math;
     math.init(lane, scratch + warp * M::kWarpScratch);
     math.load_q(p, cur.b, cur.kvh);
     math.reset();
+    prefetch_next_q();
     if constexpr (M::kCanAppend)
         if (p.k_new != nullptr) prefetch_append<M>(p, cur.b, cur.kvh, lane);
     int64_t piece_start = lo;
@@ -1429,6 +1484,7 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
                 piece_start = lo + j + 1;
                 math.load_q(p, cur.b, cur.kvh);
                 math.reset();
+                prefetch_next_q();
                 if constexpr (M::kCanAppend)
                     if (p.k_new != nullptr) prefetch_append<M>(p, cur.b, cur.kvh, lane);
             }
