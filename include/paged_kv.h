@@ -398,7 +398,7 @@ KV_API kv_status paged_decode_attention_static_workspace(
 
 /*
  * Copy whole physical blocks: for i < num_copies, block copy_dst[i] of the K
- * pool, the V pool and (FP8) the scale pool becomes a copy of block
+ * pool, the V pool and (quantised pools) the scale / parameter pool becomes a copy of block
  * copy_src[i], every kv head ("KV Cache 深度解析" §三: blocks shared by
  * several sequences; a sequence that writes into a shared, partly filled
  * block first gets its own copy -- see kv_block_manager_append_slots).

@@ -4,7 +4,7 @@
 // Pool layout [num_blocks][num_kv_heads][16][head_dim]: the new token's row of
 // kv head h goes to block slot/16, row slot%16.  HBM-bound scatter: every
 // thread moves one 16-byte vector (bf16/fp32) or one warp quantises one row
-// (FP8), so loads and stores are full 32-byte sectors.
+// (FP8, INT8, INT4), so loads and stores are full 32-byte sectors.
 #include <algorithm>
 
 #include "kernels.cuh"
@@ -116,7 +116,7 @@ __global__ void cache_quant_kernel(uint8_t* __restrict__ k_pool, uint8_t* __rest
 }
 
 // Whole-block copies (copy-on-write of shared blocks): CTA (pair, part) moves
-// 16-byte vectors of the K block, the V block and the FP8 scale line.
+// 16-byte vectors of the K block, the V block and its scale / parameter line.
 __global__ void copy_blocks_kernel(uint8_t* __restrict__ k_pool, uint8_t* __restrict__ v_pool,
                                    uint8_t* __restrict__ scales, const int32_t* __restrict__ src,
                                    const int32_t* __restrict__ dst, int64_t block_bytes,
