@@ -212,3 +212,21 @@ def test_quantized_full_size_sampled_and_codes_bitexact(kind):
         blk = inp.block_table[s, pos // 16]
         assert (kp[blk, :, pos % 16, :] == codes[pos]).all()
         assert (ks[blk, :, pos % 16].view(np.int32) == scales[pos].view(np.int32)).all()
+
+
+def test_workspace_needs_no_initialisation():
+    # the workspace holds only what each call writes before reading it: garbage in
+    # it must not matter, and repeated calls on one workspace give the same bits
+    inp = make_inputs(_spec("bf16", "bf16", 128, 4, [3000, 17, 900, 4096], idx=59))
+    st = stage(inp)
+    st.cache.append(st.block_table, st.seq_ids, st.positions, st.k_new, st.v_new)
+    _, ref = oracle_out(inp)
+    n = st.cache.workspace_bytes(4, 8, inp.max_context_len, 64)
+    for fill in (0xFF, 0x00, 0x5A):
+        ws = torch.full((n,), fill, dtype=torch.uint8, device="cuda")
+        outs = [st.cache.decode(st.q, st.block_table, st.context_lens, inp.max_context_len,
+                                inp.spec.scale, partition_tokens=64, workspace=ws).clone()
+                for _ in range(3)]
+        assert st.cache.errors() == 0
+        check_close(outs[0], ref, "bf16")
+        assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
