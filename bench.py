@@ -608,6 +608,10 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="llama", choices=sorted(WORKLOADS))
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (same head shapes and dtypes)")
+    ap.add_argument("--context", type=int, default=None,
+                    help="override the context lengths: every sequence this many tokens")
     ap.add_argument("--partition", type=int, default=0,
                     help="max tokens per consumer range (0 = balanced over all SMs)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -622,7 +626,11 @@ def main(argv=None):
                          "verification of that many appended tokens)")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps, reported as run
-    inp = make_inputs(args.workload)
+    lens = None
+    if args.context is not None:
+        batch = args.batch if args.batch is not None else WORKLOADS[args.workload].batch
+        lens = [args.context] * batch
+    inp = make_inputs(args.workload, batch=args.batch, lens_override=lens)
     if args.impl == "reference":
         run_reference(args, inp)
     else:
