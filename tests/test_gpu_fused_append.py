@@ -146,3 +146,32 @@ def test_fused_full_size_llama_sampled():
     assert st.cache.errors() == 0
     idx, ref = oracle_out(inp, [0, 17, 31])
     check_close(out[torch.as_tensor(idx, device=out.device)], ref, "bf16")
+
+
+def test_decode_step_replays_in_a_cuda_graph():
+    # the fused step captures into a CUDA graph (host work -- argument checks, tensor
+    # maps -- happens at capture) and every replay gives the eager call's bits
+    inp = make_inputs(_spec("bf16", "bf16", 128, 4, [300, 1025, 17], idx=123))
+    st = stage(inp)
+    c = st.cache
+    out = torch.empty_like(st.q)
+    ws = c.alloc_workspace(3, 8, st.max_context_len)
+    s = torch.cuda.Stream()
+
+    def call():
+        c.decode_append(st.q, st.k_new, st.v_new, st.block_table, st.context_lens,
+                        st.max_context_len, inp.spec.scale, out=out, workspace=ws)
+
+    with torch.cuda.stream(s):
+        call()
+        torch.cuda.synchronize()
+        eager = out.clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            call()
+    for _ in range(3):
+        out.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(out, eager)
+    assert c.errors() == 0
