@@ -944,7 +944,8 @@ struct MmaMath {
 
         // ---- online softmax per row set: row gid + 8k holds tokens 8nt + 2tig + j
         float pr[kSets][2][2];
-        float corr[kSets];
+        float corr[kSets], m_old[kSets], m_ref[kSets], psum[kSets];
+        bool grow = false;
 #pragma unroll
         for (int k = 0; k < kSets; ++k) {
             // last position this row sees (one query token: the context's last, for every row)
@@ -975,39 +976,47 @@ struct MmaMath {
             // with several query tokens a row may have seen nothing yet (max -inf):
             // exponentiate against 0 then; one query token always sees a token
             const float m_use = (!SINGLE && m_new == -INFINITY) ? 0.0f : m_new;
-            corr[k] = fast_exp2(m_run[k] - m_use);
-            float psum = 0.0f;
+            grow = grow || m_new != m_run[k];
+            m_old[k] = m_run[k];
+            m_ref[k] = m_use;
+            psum[k] = 0.0f;
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     pr[k][nt][j] = fast_exp2(pr[k][nt][j] - m_use);
-                    psum += pr[k][nt][j];
+                    psum[k] += pr[k][nt][j];
                 }
-            l_run[k] = l_run[k] * corr[k] + psum;
             m_run[k] = m_new;
         }
 
-        // rescale O^T columns: column 8k + 2tig + j is row gid' = 2tig + j of set k
-        {
+        // Corrections 2^(m_old - m_new).  While no row of the warp has a new max they
+        // are all exactly 1 and the exponentials, shuffles and rescale are skipped
+        // (the result is the same to the bit).  Otherwise rescale the O^T columns:
+        // column 8k + 2tig + j is row gid' = 2tig + j of set k.
+        if (__any_sync(0xffffffffu, grow)) {
             float cf[kSets][2];
-            bool any = false;
 #pragma unroll
             for (int k = 0; k < kSets; ++k) {
+                corr[k] = fast_exp2(m_old[k] - m_ref[k]);
+                l_run[k] = l_run[k] * corr[k] + psum[k];
                 cf[k][0] = __shfl_sync(0xffffffffu, corr[k], 8 * tig);
                 cf[k][1] = __shfl_sync(0xffffffffu, corr[k], 8 * tig + 4);
-                any = any || cf[k][0] != 1.0f || cf[k][1] != 1.0f;
             }
-            if (__any_sync(0xffffffffu, any)) {
 #pragma unroll
-                for (int k = 0; k < kSets; ++k)
+            for (int k = 0; k < kSets; ++k)
 #pragma unroll
-                    for (int mi = 0; mi < 8; ++mi) {
-                        o[k][mi][0] *= cf[k][0];
-                        o[k][mi][1] *= cf[k][1];
-                        o[k][mi][2] *= cf[k][0];
-                        o[k][mi][3] *= cf[k][1];
-                    }
+                for (int mi = 0; mi < 8; ++mi) {
+                    o[k][mi][0] *= cf[k][0];
+                    o[k][mi][1] *= cf[k][1];
+                    o[k][mi][2] *= cf[k][0];
+                    o[k][mi][3] *= cf[k][1];
+                }
+        } else {
+#pragma unroll
+            for (int k = 0; k < kSets; ++k) {
+                corr[k] = 1.0f;
+                l_run[k] += psum[k];
             }
         }
 
