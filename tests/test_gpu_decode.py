@@ -95,6 +95,29 @@ def test_identical_keys_give_mean_v():
         assert np.abs(out[s] - want).max() <= 2e-2
 
 
+def _ramp_keys(inp, rising: bool):
+    """Scale every sequence's keys by a factor ramping over its positions (0.2 -> 3 or
+    3 -> 0.2): rising, a row's running max grows in nearly every tile; falling, it
+    settles in the first tiles and the online softmax's corrections stay exactly 1."""
+    for s in range(inp.q.shape[0]):
+        a, n = int(inp.seq_offsets[s]), int(inp.context_lens[s])
+        g = torch.linspace(0.2, 3.0, n) if rising else torch.linspace(3.0, 0.2, n)
+        inp.k[a:a + n] = (inp.k[a:a + n].float() * g[:, None, None]).to(inp.k.dtype)
+
+
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8", "int4"])
+@pytest.mark.parametrize("rising", [True, False])
+def test_running_max_growth_patterns(kv, rising):
+    inp = make_inputs(_spec(kv, "bf16", 128, 4, [40, 1000, 2047, 3001], idx=57))
+    _ramp_keys(inp, rising)
+    st = stage(inp)
+    _, ref = oracle_out(inp)
+    for part in (0, 256):
+        out = step(st, partition_tokens=part)
+        check_close(out, ref, kv)
+    assert st.cache.errors() == 0
+
+
 def test_permuted_pool_is_bitwise_invariant():
     inp = make_inputs(_spec("bf16", "bf16", 128, 4, [5, 400, 1500, 3000], idx=54))
     base = step(stage(inp), partition_tokens=256).cpu()

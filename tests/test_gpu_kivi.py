@@ -81,6 +81,23 @@ def test_kivi_decode_append_parity(G):
         check_close(out, ref, "kivi4")
 
 
+@pytest.mark.parametrize("rising", [True, False])
+def test_kivi_running_max_growth_patterns(rising):
+    # keys scaled by a ramp over positions: the running max grows in nearly every
+    # tile (rising) or settles early (falling)
+    inp = make_inputs(_spec(4, [40, 1000, 2047, 3001], idx=139))
+    for s in range(inp.q.shape[0]):
+        a, n = int(inp.seq_offsets[s]), int(inp.context_lens[s])
+        g = torch.linspace(0.2, 3.0, n) if rising else torch.linspace(3.0, 0.2, n)
+        inp.k[a:a + n] = (inp.k[a:a + n].float() * g[:, None, None]).to(inp.k.dtype)
+    _, ref = oracle_out_kivi(inp)
+    st = stage_kivi(inp)
+    out = st.cache.kivi_decode(st.q, st.block_table, st.context_lens, st.max_context_len,
+                               inp.spec.scale, st.k_new, st.v_new)
+    assert st.cache.errors() == 0
+    check_close(out, ref, "kivi4")
+
+
 def test_kivi_flush_writes_the_completed_block():
     lens = [16, 32, 48, 17]                     # the first three complete a block
     inp = make_inputs(_spec(4, lens, idx=140))
