@@ -855,7 +855,18 @@ struct MmaMath {
         }
     }
 
+    // A tile whose 16 tokens every query row sees (for one query token: every tile but
+    // a pair's last) needs no position masks, and runs an instantiation without them.
     __device__ void tile(const uint8_t* kt, int32_t jb, int32_t L, const DecodeParams& p) {
+        if ((jb + 1) * kBlockTokens <= L - nq + 1)
+            tile_body<true>(kt, jb, L, p);
+        else
+            tile_body<false>(kt, jb, L, p);
+    }
+
+    template <bool FULL>
+    __device__ __forceinline__ void tile_body(const uint8_t* kt, int32_t jb, int32_t L,
+                                              const DecodeParams& p) {
         const uint32_t k_s = smem_addr(kt);
         const uint32_t v_s = k_s + kTileBytes;
         const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
@@ -967,7 +978,7 @@ struct MmaMath {
                         v = s[nt][2 * k + j] * p.scale_log2;
                         if constexpr (kF16) v *= ksc[t];
                     }
-                    pr[k][nt][j] = (pos0 + t <= last) ? v : -INFINITY;
+                    pr[k][nt][j] = (FULL || pos0 + t <= last) ? v : -INFINITY;
                     mx = fmaxf(mx, pr[k][nt][j]);
                 }
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -1039,7 +1050,7 @@ struct MmaMath {
                         const int t = 8 * nt + 2 * tig + j;
                         pz[nt][j] = vpz[t];
                         const float pv = pr[k][nt][j] * pz[nt][j].x;
-                        pr[k][nt][j] = (t < nvalid) ? pv : 0.0f;
+                        pr[k][nt][j] = (FULL || t < nvalid) ? pv : 0.0f;
                     }
                 pb[k][0] = pack2<true>(pr[k][0][0], pr[k][0][1]);
                 pb[k][1] = pack2<true>(pr[k][1][0], pr[k][1][1]);
@@ -1049,8 +1060,8 @@ struct MmaMath {
                 for (int nt = 0; nt < 2; ++nt) {
                     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pb[k][nt]));
                     const int t = 8 * nt + 2 * tig;
-                    bsum += (t < nvalid) ? f.x * pz[nt][0].y : 0.0f;
-                    bsum += (t + 1 < nvalid) ? f.y * pz[nt][1].y : 0.0f;
+                    bsum += (FULL || t < nvalid) ? f.x * pz[nt][0].y : 0.0f;
+                    bsum += (FULL || t + 1 < nvalid) ? f.y * pz[nt][1].y : 0.0f;
                 }
                 b_run[k] = b_run[k] * corr[k] + bsum;
                 continue;
@@ -1060,14 +1071,14 @@ struct MmaMath {
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
                         const int t = 8 * nt + 2 * tig + j;
-                        pr[k][nt][j] = (t < nvalid) ? pr[k][nt][j] * vsc[t] : 0.0f;
+                        pr[k][nt][j] = (FULL || t < nvalid) ? pr[k][nt][j] * vsc[t] : 0.0f;
                     }
             }
             pb[k][0] = pack2<kF16>(pr[k][0][0], pr[k][0][1]);
             pb[k][1] = pack2<kF16>(pr[k][1][0], pr[k][1][1]);
         }
         // V^T fragment halves of tokens 2tig, 2tig+1 (mask_a) and 8+2tig, 9+2tig (mask_b)
-        const bool partial = nvalid < kBlockTokens;
+        const bool partial = !FULL && nvalid < kBlockTokens;
         const uint32_t mask_a = (2 * tig < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 1 < nvalid ? 0xffff0000u : 0u);
         const uint32_t mask_b = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
 
