@@ -345,15 +345,30 @@ __device__ __forceinline__ int32_t seq_tiles(int32_t L, const DecodeParams& p) {
     return p.kivi ? L / kBlockTokens : (L + kBlockTokens - 1) / kBlockTokens;
 }
 
-// First tile of consumer range W (ranges are equal cuts of the T-tile list).
+// First tile of consumer range W (ranges are equal cuts of the T-tile list):
+// floor(W T / N), N = num_ranges.  With T = q N + r that is W q + floor(W r / N),
+// which needs only 32-bit divisions when N <= 65535 (W r < N^2 < 2^32) -- the
+// persistent grid's case; 64-bit division is a long dependent chain.
 __device__ __forceinline__ int64_t range_begin(int64_t W, int64_t T, int32_t num_ranges) {
-    return W >= num_ranges ? T : (W * T) / num_ranges;
+    if (W >= num_ranges) return T;
+    if (T <= 0x7fffffff && num_ranges <= 65535) {
+        const uint32_t n = static_cast<uint32_t>(num_ranges), t = static_cast<uint32_t>(T);
+        const uint32_t w = static_cast<uint32_t>(W);
+        const uint32_t q = t / n, r = t - q * n;
+        return static_cast<int64_t>(w) * q + (w * r) / n;
+    }
+    return (W * T) / num_ranges;
 }
 
 // The range holding tile x < T: the largest W with range_begin(W) <= x, i.e.
-// the largest W with W*T < (x+1)*num_ranges.
+// the largest W with W T < (x+1) N -- in 32 bits when T N fits them.
 __device__ __forceinline__ int64_t range_of(int64_t x, int64_t T, int32_t num_ranges) {
-    const int64_t W = ((x + 1) * num_ranges - 1) / T;
+    int64_t W;
+    if (T <= static_cast<int64_t>(0xffffffffu / static_cast<uint32_t>(num_ranges)))
+        W = (static_cast<uint32_t>(x + 1) * static_cast<uint32_t>(num_ranges) - 1u) /
+            static_cast<uint32_t>(T);
+    else
+        W = ((x + 1) * num_ranges - 1) / T;
     return W < num_ranges - 1 ? W : num_ranges - 1;
 }
 
@@ -379,15 +394,23 @@ struct Cursor {
     int64_t seg_start;
 };
 
-// Warp-cooperative search for the pair holding tile x (< T).  When `prefix`
-// is non-null the warp also writes every sequence's first tile (and T at
-// [batch]) there for the merge kernel.
-__device__ Cursor locate_tile(const DecodeParams& p, int64_t x, int lane, int32_t* prefix,
-                              int64_t T) {
-    Cursor c{p.batch, 0, 0, 0, 0, T};
-    bool found = false;
+// Warp-cooperative search for the pairs holding tiles x[0..K) (each < T; a
+// negative x is not looked for), all in one pass over the lengths.  When
+// `prefix` is non-null the warp also writes every sequence's first tile (and T
+// at [batch]) there for the merge kernel.
+template <int K>
+__device__ void locate_tiles(const DecodeParams& p, const int64_t (&x)[K], int lane,
+                             int32_t* prefix, int64_t T, Cursor (&c)[K]) {
+    bool found[K];
+    int left = 0;
+#pragma unroll
+    for (int k = 0; k < K; ++k) {
+        c[k] = Cursor{p.batch, 0, 0, 0, 0, T};
+        found[k] = x[k] < 0;
+        left += found[k] ? 0 : 1;
+    }
     int64_t base = 0;
-    for (int b0 = 0; b0 < p.batch; b0 += 32) {
+    for (int b0 = 0; b0 < p.batch && (left > 0 || prefix != nullptr); b0 += 32) {
         const int b = b0 + lane;
         const int32_t L = b < p.batch ? p.context_lens[b] : 0;
         const int32_t nt = b < p.batch ? seq_tiles(L, p) : 0;
@@ -400,26 +423,38 @@ __device__ Cursor locate_tile(const DecodeParams& p, int64_t x, int lane, int32_
         }
         const int64_t excl = base + incl - cnt;
         if (prefix != nullptr && b < p.batch) prefix[b] = static_cast<int32_t>(excl);
-        const uint32_t hit = __ballot_sync(0xffffffffu, !found && cnt > 0 && x >= excl && x < excl + cnt);
-        if (hit != 0u && !found) {
-            const int src = __ffs(hit) - 1;
-            const int64_t e = __shfl_sync(0xffffffffu, excl, src);
-            const int32_t n = __shfl_sync(0xffffffffu, nt, src);
-            const int32_t l = __shfl_sync(0xffffffffu, L, src);
-            const int64_t off = x - e;
-            c.b = b0 + src;
-            c.nt = n;
-            c.L = l;
-            c.kvh = static_cast<int32_t>(off / n);
-            c.jb = static_cast<int32_t>(off % n);
-            c.seg_start = e + static_cast<int64_t>(c.kvh) * n;
-            found = true;
-            if (prefix == nullptr) break;
+#pragma unroll
+        for (int k = 0; k < K; ++k) {
+            const uint32_t hit = __ballot_sync(
+                0xffffffffu, !found[k] && cnt > 0 && x[k] >= excl && x[k] < excl + cnt);
+            if (hit != 0u) {
+                const int src = __ffs(hit) - 1;
+                const int64_t e = __shfl_sync(0xffffffffu, excl, src);
+                const int32_t n = __shfl_sync(0xffffffffu, nt, src);
+                const int32_t l = __shfl_sync(0xffffffffu, L, src);
+                // the tile list holds fewer than 2^31 tiles (checked by the host)
+                const uint32_t off = static_cast<uint32_t>(x[k] - e);
+                c[k].b = b0 + src;
+                c[k].nt = n;
+                c[k].L = l;
+                c[k].kvh = static_cast<int32_t>(off / static_cast<uint32_t>(n));
+                c[k].jb = static_cast<int32_t>(off - static_cast<uint32_t>(c[k].kvh) * n);
+                c[k].seg_start = e + static_cast<int64_t>(c[k].kvh) * n;
+                found[k] = true;
+                --left;
+            }
         }
         base += __shfl_sync(0xffffffffu, incl, 31);
     }
     if (prefix != nullptr && lane == 0) prefix[p.batch] = static_cast<int32_t>(T);
-    return c;
+}
+
+__device__ Cursor locate_tile(const DecodeParams& p, int64_t x, int lane, int32_t* prefix,
+                              int64_t T) {
+    const int64_t xs[1] = {x};
+    Cursor c[1];
+    locate_tiles<1>(p, xs, lane, prefix, T, c);
+    return c[0];
 }
 
 // Move a cursor to the next tile of the list (single thread or warp-uniform).
@@ -453,6 +488,7 @@ struct SimtMath {
     static constexpr int kStageBytes = 2 * kTileBytes + kScaleBytes;
     static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
     static constexpr int kRingAlign = 128;
+    static constexpr bool kUsesTma = false;                                  // 1-D bulk copies
     static constexpr int kChunkElems = 16 / kElem;                           // per 16-byte load
     static constexpr int kRowChunks = D / kChunkElems;
     static constexpr int kLPR = kRowChunks >= 8 ? 8 : kRowChunks;           // lanes per row
@@ -727,6 +763,7 @@ struct MmaMath {
     static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
     static constexpr int kStages = kI4 ? 16 : (kF16 ? 12 : 8);     // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
+    static constexpr bool kUsesTma = true;                        // tensor-map tile copies
     static constexpr int kWarpScratch = 0;
     static constexpr int kMinBlocks = WIDE ? 2 : 3;
 
@@ -1344,38 +1381,37 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
     // No early launch_dependents here: this grid is persistent, and a dependent
     // (the merge) launched at its start parks CTAs on the SMs for its whole
     // duration; releasing it at exit measured 7 % faster per call.
+    // The tensor maps are parameters, not data of the preceding grid: their
+    // descriptors are fetched while it finishes.
+    if constexpr (M::kUsesTma)
+        if (threadIdx.x == kConsumerWarps * 32) {
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.k)) : "memory");
+            asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&maps.v)) : "memory");
+        }
     pdl_wait();
     const int64_t T = total_tiles(p, lane);
     const int64_t W0 = static_cast<int64_t>(blockIdx.x) * kConsumerWarps;
 
     if (warp == kConsumerWarps) {
         // ================= producer warp =================
+        // the four ranges' first tiles, found in one pass over the lengths (the first
+        // CTA also publishes every sequence's first tile for the merge)
         Cursor cur[kConsumerWarps];
         int32_t cnt[kConsumerWarps];
+        int64_t first[kConsumerWarps];
 #pragma unroll
         for (int w = 0; w < kConsumerWarps; ++w) {
             const int64_t lo = range_begin(W0 + w, T, p.num_ranges);
-            const int64_t hi = range_begin(W0 + w + 1, T, p.num_ranges);
-            cnt[w] = static_cast<int32_t>(hi - lo);
-            // the first CTA also publishes every sequence's first tile for the merge
-            int32_t* prefix = (blockIdx.x == 0 && w == 0) ? p.ws_seq_start : nullptr;
-            if (cnt[w] > 0 || prefix != nullptr) cur[w] = locate_tile(p, lo, lane, prefix, T);
+            cnt[w] = static_cast<int32_t>(range_begin(W0 + w + 1, T, p.num_ranges) - lo);
+            first[w] = cnt[w] > 0 ? lo : -1;
         }
-        if (lane == 0) {
-            for (int s = 0; s < M::kStages; ++s) {
-                mbar_init(&full[s], 1);
-                mbar_init(&empty[s], 1);
-                issued_round[s] = -1;
-            }
-            *abort_flag = 0;
-            mbar_init_fence();
-        }
-        __syncthreads();
-        if (lane >= kConsumerWarps) return;
+        locate_tiles<kConsumerWarps>(p, first, lane, blockIdx.x == 0 ? p.ws_seq_start : nullptr,
+                                     T, cur);
 
         // Lane w feeds consumer warp w: its j-th tile goes through stage
         // w + 4 * (j % kPerWarp), so no warp's stage ever waits behind another
-        // warp's; block ids are loaded kLook tiles ahead.
+        // warp's; block ids are loaded kLook tiles ahead, the first ones before
+        // the barrier setup.
         constexpr int kPerWarp = M::kStages / kConsumerWarps;
         constexpr int kLook = 4;
         Cursor c = cur[0];
@@ -1386,6 +1422,7 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
                 c = cur[w];
                 count = cnt[w];
             }
+        if (lane >= kConsumerWarps) count = 0;
         int32_t q_id[kLook];
         int32_t q_head[kLook];
         auto fetch = [&](int j, int i) {
@@ -1397,6 +1434,17 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
         };
 #pragma unroll
         for (int i = 0; i < kLook; ++i) fetch(i, i);
+        if (lane == 0) {
+            for (int s = 0; s < M::kStages; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], 1);
+                issued_round[s] = -1;
+            }
+            *abort_flag = 0;
+            mbar_init_fence();
+        }
+        __syncthreads();
+        if (lane >= kConsumerWarps) return;
         for (int j0 = 0; j0 < count; j0 += kLook) {
 #pragma unroll
             for (int i = 0; i < kLook; ++i) {
@@ -1530,10 +1578,20 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
     // one warp per output row (sequence b, query token i, head h): out is [B][Q][Hq][D]
     const int64_t bh = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
     const int32_t nq = p.num_query_tokens;
-    if (bh >= static_cast<int64_t>(p.batch) * nq * p.num_q_heads) return;
-    const int32_t b = static_cast<int32_t>(bh / (static_cast<int64_t>(nq) * p.num_q_heads));
-    const int32_t h = static_cast<int32_t>(bh % p.num_q_heads);
-    const int32_t qi = static_cast<int32_t>((bh / p.num_q_heads) % nq);
+    const int64_t rows_total = static_cast<int64_t>(p.batch) * nq * p.num_q_heads;
+    if (bh >= rows_total) return;
+    int32_t b, h, qi;
+    if (rows_total <= 0x7fffffff) {  // 32-bit divisions (64-bit ones are long chains)
+        const uint32_t x = static_cast<uint32_t>(bh), hq = static_cast<uint32_t>(p.num_q_heads);
+        const uint32_t bq = x / hq;  // b * nq + qi
+        h = static_cast<int32_t>(x - bq * hq);
+        b = static_cast<int32_t>(bq / static_cast<uint32_t>(nq));
+        qi = static_cast<int32_t>(bq) - b * nq;
+    } else {
+        b = static_cast<int32_t>(bh / (static_cast<int64_t>(nq) * p.num_q_heads));
+        h = static_cast<int32_t>(bh % p.num_q_heads);
+        qi = static_cast<int32_t>((bh / p.num_q_heads) % nq);
+    }
     const int32_t G = p.num_q_heads / p.num_kv_heads;
     const int32_t kvh = h / G;
     const int32_t R = G * nq;          // query rows of a (sequence, kv head) pair
