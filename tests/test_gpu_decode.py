@@ -208,6 +208,15 @@ def test_llama_full_size_sampled():
     _sampled("llama", [0, 13, 31])
 
 
+def test_llama_full_size_more_ranges_than_32bit_shortcuts():
+    # 16-token partitions over 32 x 4096 tokens x 8 kv heads: 65536 ranges, one
+    # tile each -- past the 32-bit shortcuts of the range arithmetic (more than
+    # 65535 ranges, tiles x ranges >= 2^32), so the 64-bit paths cut and merge
+    stats, inp, st = _sampled("llama", [0, 13, 31], part=16)
+    assert pk.paged_decode_num_ranges(st.cache.desc, inp.q.shape[0], inp.spec.num_q_heads,
+                                      inp.max_context_len, 16) == 65536
+
+
 def test_ragged_full_size_sampled():
     inp = make_inputs("ragged")
     order = np.argsort(inp.context_lens)
