@@ -88,6 +88,9 @@ def test_workspace_bytes_and_ranges():
     # explicit partition: ranges of at most 512 tokens over 32 x 8 x 256 tiles
     assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 512) == 32 * 8 * 256 // 32
     assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 500) == 0
+    # one-block partitions: one range per tile, more than the 65535 ranges the kernels'
+    # 32-bit range arithmetic covers (they switch to 64-bit there)
+    assert pk.paged_decode_num_ranges(d, 32, 32, 4096, 16) == 32 * 8 * 256
     ranges = 148 * 12
     pieces = 32 * 8 + ranges
     up = lambda x: (x + 255) // 256 * 256  # noqa: E731
