@@ -15,9 +15,13 @@ e2e      = the same metric through the binding from host memory: each step
            copies one pinned buffer holding q, the new K/V rows, the block
            table and the context lengths host->device, runs the step on views
            of it, and copies the output device->host, inside the timed region;
-roofline = the decode call (decode + merge kernels): K calls back to back timed
-           with CUDA events on their stream after the steps, against the
-           measured HBM copy bandwidth;
+roofline = the decode call (decode + merge kernels) against the measured HBM
+           copy bandwidth: per-call time from the timed steps when a step is
+           one decode call (fused append, the default), else from K decode
+           calls back to back timed the same way after the steps;
+timing   = --regions regions of exactly K steps, each bracketed by a barrier
+           and a synchronize; value and e2e report the median region and the
+           line lists every region (the default 20-step region lasts ~2 ms);
 cpu_baseline = the double-precision CPU oracle on a bounded sample (rank 0).
 ``--impl reference`` times that oracle alone as the reference arm.
 With N > 1 (torchrun), every rank runs an independent replica on its own GPU
@@ -42,7 +46,17 @@ sys.path.insert(0, ROOT)
 
 from workloads import WORKLOADS, make_inputs, storage_view  # noqa: E402
 
-PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "paged_decode_llama_b32x4k.md")
+# ncu summary of each workload's decode call (DRAM bytes per call, with the
+# hash of the decode source it was captured on)
+PROFILE_SUMMARIES = {
+    "llama": "paged_decode_llama_b32x4k.md",
+    "ragged": "paged_decode_ragged_b256.md",
+    "long": "paged_decode_long_b4x128k.md",
+    "fp8": "paged_decode_fp8_b64.md",
+    "int8": "paged_decode_int8_b64.md",
+    "int4": "paged_decode_int4_b64.md",
+    "kivi": "paged_decode_kivi_b64.md",
+}
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_401_b200", "csrc", "decode.cu")
 
 
@@ -232,23 +246,26 @@ def measured_peak():
     return 6650.0, "fallback"
 
 
-def profiled_traffic():
-    """ncu DRAM bytes per decode call, if the committed summary was taken on the
-    current decode kernel source (else None: the kernel changed since)."""
-    if not os.path.exists(PROFILE_SUMMARY):
-        return None
+def profiled_traffic(workload: str):
+    """ncu DRAM bytes per decode call of a workload, if its committed summary
+    was taken on the current decode kernel source (else None: no summary, or
+    the kernel changed since).  Returns (bytes, summary file) or (None, None)."""
+    name = PROFILE_SUMMARIES.get(workload)
+    path = os.path.join(ROOT, "profiles", name) if name else None
+    if path is None or not os.path.exists(path):
+        return None, None
     kv = {}
-    for line in open(PROFILE_SUMMARY, encoding="utf-8"):
+    for line in open(path, encoding="utf-8"):
         if ":" in line and line.lstrip().startswith("- "):
             k, _, v = line.strip()[2:].partition(":")
             kv[k.strip()] = v.strip().strip("`")
     sha = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
     if kv.get("decode_source_sha256") != sha:
-        return None
+        return None, None
     try:
-        return int(kv["dram_bytes_per_decode_call"])
+        return int(kv["dram_bytes_per_decode_call"]), "profiles/" + name
     except (KeyError, ValueError):
-        return None
+        return None, None
 
 
 # ---------------------------------------------------------------- oracle (CPU) timing
@@ -444,38 +461,50 @@ def run_gpu(args, inp):
         else:
             attend(q, bt, lens)
 
-    for _ in range(args.warmup):
+    def timed_regions(body, n_regions):
+        """n_regions back-to-back regions of exactly args.steps calls of body,
+        each bracketed by a barrier and a device synchronize, timed with CUDA
+        events on the launching stream; returns the ms of each region."""
+        ms = []
+        for _ in range(n_regions):
+            barrier(device)
+            torch.cuda.synchronize(device)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                body()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            barrier(device)
+            ms.append(e0.elapsed_time(e1))
+        return ms
+
+    def whole_step():
         append()
         decode()
-    torch.cuda.synchronize(device)
-    err0 = cache.errors()
 
-    # ---- timed region: K whole steps back to back (the kernels of consecutive
-    # calls overlap their launches), then K decode calls alone for the roofline
-    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    # ---- warm-up and timed region.  The clock sampler runs from before the
+    # warm-up, so the timed steps follow the warm-up with no idle gap.  The
+    # timed region is args.regions regions of K whole steps back to back (the
+    # kernels of consecutive calls overlap their launches); the line reports
+    # the median region and lists all.  When the step is one decode call
+    # (fused append), the roofline takes its per-call time from these same
+    # regions; otherwise K decode calls alone are timed the same way after them.
     with ClockSampler(gpu_id(device)) as clk:
-        barrier(device)
+        for _ in range(args.warmup):
+            whole_step()
         torch.cuda.synchronize(device)
-        time.sleep(0.1)  # the sampler is running before the region starts
+        err0 = cache.errors()
         clk.mark_start()
-        start.record(stream)
-        for _ in range(args.steps):
-            append()
-            decode()
-        end.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(device)
-        d0.record(stream)
-        for _ in range(args.steps):
-            decode()
-        d1.record(stream)
-        torch.cuda.synchronize(device)
+        step_ms = timed_regions(whole_step, args.regions)
+        decode_ms_regions = step_ms if fused else timed_regions(decode, args.regions)
         clk.mark_end()
-        barrier(device)
-    elapsed_ms = start.elapsed_time(end)
-    decode_ms = d0.elapsed_time(d1) / args.steps
     errs = cache.errors()
+    # per region: the slowest rank; then the median region
+    step_ms = [reduce_over_ranks(m, "max", device) for m in step_ms]
+    decode_ms_regions = [reduce_over_ranks(m, "max", device) for m in decode_ms_regions]
+    elapsed_ms = float(np.median(step_ms))
+    decode_ms = float(np.median(decode_ms_regions)) / args.steps
 
     # ---- e2e: the step's inputs live in ONE pinned host buffer (q, new K/V rows,
     # block table, context lengths, each 256-byte aligned) copied to a device
@@ -542,14 +571,16 @@ def run_gpu(args, inp):
         return e0.elapsed_time(e1)
 
     e2e_run(max(2, args.warmup))
-    barrier(device)
-    e2e_ms = e2e_run(args.steps)
+    e2e_regions = []
+    for _ in range(args.regions):
+        barrier(device)
+        e2e_regions.append(reduce_over_ranks(e2e_run(args.steps), "max", device))
     barrier(device)
 
     nbytes = kv_bytes_per_step(inp)
-    max_ms = reduce_over_ranks(elapsed_ms, "max", device)
-    max_e2e_ms = reduce_over_ranks(e2e_ms, "max", device)
-    max_decode_ms = reduce_over_ranks(decode_ms, "max", device)
+    max_ms = elapsed_ms
+    max_e2e_ms = float(np.median(e2e_regions))
+    max_decode_ms = decode_ms
     total_bytes = reduce_over_ranks(nbytes * args.steps, "sum", device)
     value = total_bytes / (max_ms * 1e-3) / 1e9
     e2e_value = total_bytes / (max_e2e_ms * 1e-3) / 1e9
@@ -569,6 +600,8 @@ def run_gpu(args, inp):
         return
     peak, peak_kind = measured_peak()
     achieved = nbytes / (max_decode_ms * 1e-3) / 1e9
+    default_shape = (args.batch is None and args.context is None and Q == 1 and P == 0)
+    traffic, traffic_src = profiled_traffic(args.workload) if default_shape else (None, None)
     line = {
         "metric": "paged GQA decode: effective KV-read HBM GB/s (% of peak), decode steps/s",
         "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -582,17 +615,28 @@ def run_gpu(args, inp):
                        append=("KIVI residual append (+ block flush) in the decode call" if kivi
                                else "fused into the decode call" if fused
                                else "separate slot-mapping and cache-write calls")),
+        "timing": {"regions": args.regions,
+                   "region": f"{args.steps} steps back to back, barrier + synchronize on "
+                             "both sides, CUDA events on the launching stream",
+                   "reported": "median region (each region: the slowest rank)",
+                   "launches_per_region": launches_per_step * args.steps,
+                   "ms_per_step_regions": [round(m / args.steps, 5) for m in step_ms],
+                   "spread_pct": round(100 * (max(step_ms) - min(step_ms)) / elapsed_ms, 2)},
         "e2e": {"value": round(e2e_value, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h,
-                "ms_per_step": round(max_e2e_ms / args.steps, 5)},
+                "ms_per_step": round(max_e2e_ms / args.steps, 5),
+                "ms_per_step_regions": [round(m / args.steps, 5) for m in e2e_regions]},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                      "unit": "GB/s", "frac": round(achieved / peak, 4),
-                     "traffic": profiled_traffic(), "kernel": "paged_decode_attention "
-                     "(decode + merge kernels, one call)", "peak_kind": peak_kind,
+                     "traffic": traffic, "traffic_source": traffic_src,
+                     "kernel": "paged_decode_attention (decode + merge kernels, one call)",
+                     "peak_kind": peak_kind,
                      "algorithmic_bytes_per_launch": nbytes,
-                     "ms_per_launch": round(max_decode_ms, 5)},
+                     "ms_per_launch": round(max_decode_ms, 5),
+                     "timed_in": "the timed steps (each step is one decode call)" if fused
+                                 else "decode calls alone, timed after the steps"},
         "cpu_baseline": cpu,
-        "gpu_launches": launches_per_step * args.steps + 2 * args.steps,
+        "gpu_launches": launches_per_step * args.steps,
         "unique_kv": {"bytes_per_step": unique_kv_bytes_per_step(inp),
                       "value": round(unique_kv_bytes_per_step(inp) * args.steps * world
                                      / (max_ms * 1e-3) / 1e9, 2), "unit": "GB/s"},
@@ -607,6 +651,8 @@ def main(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--regions", type=int, default=5,
+                    help="timed regions of --steps steps each; the median region is reported")
     ap.add_argument("--workload", default="llama", choices=sorted(WORKLOADS))
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (same head shapes and dtypes)")

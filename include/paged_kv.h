@@ -380,9 +380,11 @@ KV_API kv_status paged_attention_multi_query(const kv_pool_desc* pool, void* out
  *    arguments) exceeds KV_STATIC_WORKSPACE_BYTES return
  *    KV_ERR_INVALID_ARGUMENT before anything is enqueued; a larger
  *    partition_tokens needs less workspace.
- *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.  A failed look-up returns KV_ERR_CUDA.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress); nothing is cached, so a context that was reset
+ *    and created again is handled.  The first call on a device may load the
+ *    library's device code into the context (lazy loading): make that first
+ *    call before any stream capture.  A failed look-up returns KV_ERR_CUDA.
  *  - All calls on a device share the one array, which keeps the last call's
  *    contents: calls that may overlap on the GPU (on different streams, or
  *    from different host threads without ordering) race and must be

@@ -25,7 +25,7 @@
  *  - "大模型推理为何这么慢？从内存带宽瓶颈到KV Cache优化的技术突围"
  *    (freetools), section on GQA (H query heads share G groups of K/V).
  *
- * Readings where the pages are silent (each also listed in the design doc):
+ * Readings where the pages are silent:
  *  - query head h reads KV head floor(h / (Hq/Hkv))  (consecutive groups);
  *  - scale is caller supplied (1/sqrt(head_dim) on the pages);
  *  - the FP8 scale of a (token, kv head) row is absmax/448 computed in

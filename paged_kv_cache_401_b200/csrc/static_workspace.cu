@@ -12,37 +12,16 @@
 // The array is file-scope device memory: every GPU that loads the library holds
 // KV_STATIC_WORKSPACE_BYTES of it until the process exits, and every call on a
 // device shares it.  Host code cannot use the array's name as a device address
-// (on the host it names a stand-in object), so the device address is looked up
-// once per device with cudaGetSymbolAddress, with that device current, on the
-// first call made on it.
+// (on the host it names a stand-in object), so each call looks up the device
+// address with cudaGetSymbolAddress on the current device.  Nothing is cached
+// across calls: a context that is destroyed and created again (cudaDeviceReset)
+// loads the module again, possibly at another address, and the next call finds
+// the new one.
 #include "kernels.cuh"
 
 namespace {
 
-constexpr int kMaxDevices = 64;
-
 __device__ __align__(256) static uint8_t g_static_workspace[KV_STATIC_WORKSPACE_BYTES];
-
-// Device address of g_static_workspace on each device, filled on first use.
-void* g_workspace_addr[kMaxDevices] = {};
-
-// Returns the array's device address on the current device, or nullptr with *err set.
-void* static_workspace_address(cudaError_t* err) {
-    int dev = 0;
-    *err = cudaGetDevice(&dev);
-    if (*err != cudaSuccess) return nullptr;
-    if (dev < 0 || dev >= kMaxDevices) {
-        *err = cudaErrorInvalidDevice;
-        return nullptr;
-    }
-    if (g_workspace_addr[dev] == nullptr) {  // benign race: every caller finds the same address
-        void* p = nullptr;
-        *err = cudaGetSymbolAddress(&p, g_static_workspace);
-        if (*err != cudaSuccess) return nullptr;
-        g_workspace_addr[dev] = p;
-    }
-    return g_workspace_addr[dev];
-}
 
 }  // namespace
 
@@ -60,9 +39,9 @@ KV_API kv_status paged_decode_attention_static_workspace(
     if (need > KV_STATIC_WORKSPACE_BYTES) return KV_ERR_INVALID_ARGUMENT;
     void* ws = nullptr;
     if (need > 0) {
-        cudaError_t err = cudaSuccess;
-        ws = static_workspace_address(&err);
-        if (ws == nullptr) {
+        // the array's address in the current device's context (a host-side lookup
+        // once the module is loaded)
+        if (cudaGetSymbolAddress(&ws, g_static_workspace) != cudaSuccess || ws == nullptr) {
             cudaGetLastError();
             return KV_ERR_CUDA;
         }

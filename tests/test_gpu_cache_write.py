@@ -93,14 +93,18 @@ def test_cache_quant_bitexact(kind, src, D):
     NB, Hkv, T = 50, 2, 400
     x_k = _fp8_rows(rng, T, Hkv, D)
     x_v = rng.normal(size=(T, Hkv, D)).astype(np.float32)
+    if kind == "int8":
+        # scale 127/127 = 1 and exact half-integer quotients: every code is a tie
+        # (the values are exact in bf16 too, so both source types see the row)
+        x_k[6, 0, :] = np.arange(D) - D / 2 + 0.5
+        x_k[6, 0, 0] = 127.0
     tdt = {"f32": torch.float32, "bf16": torch.bfloat16}[src]
-    k = torch.from_numpy(x_k).to(tdt)
+    k = torch.from_numpy(x_k.copy()).to(tdt)
     v = torch.from_numpy(x_v).to(tdt)
+    if kind == "int8":
+        assert k[6, 0, 1].item() == 1 - D / 2 + 0.5 and k[6, 0, 0].item() == 127.0
     slots = rng.permutation(NB * 16)[:T].astype(np.int64)
     slots[9] = -1
-    if kind == "int8":
-        x_k[6, 0, :] = np.arange(D) - D / 2 + 0.5   # exact half-integer quotients: ties
-        x_k[6, 0, 0] = 127.0
     cache = PagedKVCache(NB, Hkv, D, kind, DEV, poison=True)
     pk.reshape_and_cache(cache.desc, cache.k_pool, cache.v_pool, cache.scales, k.to(DEV),
                          v.to(DEV), torch.from_numpy(slots).to(DEV), cache.dev_error)

@@ -138,14 +138,15 @@ def test_fused_invalid_context_length_gives_zeros_and_writes_nothing():
     check_close(out[[1]], oracle_out(inp, [1])[1], "int8")
 
 
-def test_fused_full_size_llama_sampled():
+def test_fused_full_size_llama():
+    # the step the benchmark times, on its full workload: every sequence and head
     inp = make_inputs("llama")
     st = stage(inp)
     out = st.cache.decode_append(st.q, st.k_new, st.v_new, st.block_table, st.context_lens,
                                  st.max_context_len, inp.spec.scale)
     assert st.cache.errors() == 0
-    idx, ref = oracle_out(inp, [0, 17, 31])
-    check_close(out[torch.as_tensor(idx, device=out.device)], ref, "bf16")
+    _, ref = oracle_out(inp)
+    check_close(out, ref, "bf16")
 
 
 def test_decode_step_replays_in_a_cuda_graph():

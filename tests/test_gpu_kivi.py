@@ -163,11 +163,12 @@ def test_kivi_decode_without_append_and_bad_inputs():
     assert torch.isfinite(out.float()).all()
 
 
-def test_kivi_full_size_sampled():
+def test_kivi_full_size():
+    # every sequence and query head of the 64-sequence workload against the oracle
     inp = make_inputs("kivi")
     st = stage_kivi(inp)
     out = st.cache.kivi_decode(st.q, st.block_table, st.context_lens, st.max_context_len,
                                inp.spec.scale, st.k_new, st.v_new)
     assert st.cache.errors() == 0
-    idx, ref = oracle_out_kivi(inp, [0, 21, 63])
-    check_close(out[torch.as_tensor(idx, device=out.device)], ref, "kivi4")
+    _, ref = oracle_out_kivi(inp)
+    check_close(out, ref, "kivi4")

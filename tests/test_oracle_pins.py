@@ -563,6 +563,51 @@ def test_scatter_then_gather_round_trip():
     assert np.isnan(skipped).sum() == (nb * 16 - 1) * hkv * d
 
 
+def test_scatter_scales_to_pool_flat_offsets():
+    # The scale pool's layout stated by the library header: [block][kv_head][2][16]
+    # float32, K's 16 row scales of a (block, kv head) and then V's.  The flat
+    # index of (block b, head h, which w, slot offset o) is ((b*Hkv + h)*2 + w)*16 + o;
+    # INT4 pools add a trailing (scale, zero) pair, flat index * 2 + {0, 1}.
+    nb, hkv = 5, 3
+    slots = np.array([0, 17, 79, -4, 38])            # slot 79: block 4, offset 15; -4 padding
+    hand = [(0, 0), (1, 1), (4, 15), None, (2, 6)]   # (block, offset) written out by hand
+    k_sc = np.arange(1, 16, dtype=np.float32).reshape(5, hkv)
+    v_sc = -k_sc
+    pool = np.full((nb, hkv, 2, 16), np.nan, np.float32)
+    pool = oracle.scatter_scales_to_pool(pool, k_sc, slots, which=0)
+    pool = oracle.scatter_scales_to_pool(pool, v_sc, slots, which=1)
+    flat = pool.reshape(-1)
+    want = np.full(nb * hkv * 2 * 16, np.nan, np.float32)
+    for t, bo in enumerate(hand):
+        if bo is None:
+            continue
+        b, o = bo
+        for h in range(hkv):
+            want[((b * hkv + h) * 2 + 0) * 16 + o] = k_sc[t, h]
+            want[((b * hkv + h) * 2 + 1) * 16 + o] = v_sc[t, h]
+    np.testing.assert_array_equal(flat, want)
+    assert np.isnan(flat).sum() == (nb * 16 - 4) * hkv * 2
+
+    # INT4: (scale, zero) per row, K then V
+    kp = np.stack([k_sc, k_sc + 100], axis=-1)       # [T][Hkv][2]
+    vp = np.stack([v_sc, v_sc - 100], axis=-1)
+    pool4 = np.full((nb, hkv, 2, 16, 2), np.nan, np.float32)
+    pool4 = oracle.scatter_scales_to_pool(pool4, kp, slots, which=0)
+    pool4 = oracle.scatter_scales_to_pool(pool4, vp, slots, which=1)
+    flat4 = pool4.reshape(-1)
+    want4 = np.full(nb * hkv * 2 * 16 * 2, np.nan, np.float32)
+    for t, bo in enumerate(hand):
+        if bo is None:
+            continue
+        b, o = bo
+        for h in range(hkv):
+            for w, par in ((0, kp), (1, vp)):
+                base = (((b * hkv + h) * 2 + w) * 16 + o) * 2
+                want4[base] = par[t, h, 0]
+                want4[base + 1] = par[t, h, 1]
+    np.testing.assert_array_equal(flat4, want4)
+
+
 # ---------------------------------------------------------------- multi-query (causal)
 def test_multi_query_one_token_is_decode():
     rng = np.random.default_rng(21)

@@ -3,21 +3,26 @@ cannot allocate device memory (an engine that reserved all of HBM for its KV
 pool, a plugin whose host runtime owns the allocator, a loop that cannot take
 cudaMalloc's implicit synchronisation).
 
-It is called through the C ABI twice in a row, on two different workloads, and
-each output is checked against the regular entry point's (which takes a
-caller-allocated workspace) within the parity tolerances of the other tests.
-The second call finds the first call's partials still in the shared array.
+It is called through the C ABI several times in a row, on different
+workloads, and each output is compared with the regular entry point's (which
+takes a caller-allocated workspace).  Both run the same kernels with the same
+split, and the split-K arithmetic does not depend on where the workspace
+lives, so the outputs must be equal bit for bit.  Every call after the first
+finds the previous call's partials still in the shared array.  One call uses
+the default split (partition_tokens 0) at 256 sequences x 8 kv heads x 4 query
+heads per group, the size the library's fixed array is stated to cover.
 This file is collected last so a failure here stops a -x run only after every
 other test has run; it also passes on its own in a fresh process.
 """
 import ctypes
 import math
 
+import numpy as np
 import pytest
 import torch
 
 import paged_kv_cache_401_b200 as pk
-from gpu_harness import TOL, stage
+from gpu_harness import stage
 from workloads import Spec, make_inputs
 
 pytestmark = pytest.mark.gpu
@@ -50,29 +55,24 @@ def _regular_call(st, partition):
                            st.inp.spec.scale, partition_tokens=partition)
 
 
-def _assert_close(a, b, kv):
-    atol, rtol = TOL[kv]
-    diff = (a.float() - b.float()).abs().max().item()
-    assert diff <= atol
-    if rtol is not None:
-        assert diff <= rtol * b.float().abs().max().item()
-
-
-def test_static_workspace_matches_regular_entry_two_calls():
+def test_static_workspace_matches_regular_entry_several_calls():
+    lens256 = np.random.default_rng(64).integers(1, 2049, size=256).tolist()
     runs = [
         (_workload("bf16", [4096, 1, 17, 2000, 3333, 4095], 60), 256),   # 16 partitions
         (_workload("fp8", [700, 5000, 64, 129], 61), 512),               # other sizes after it
+        (_workload("bf16", lens256, 62), 0),                             # default split, B256 G4
     ]
     for inp, partition in runs:
         st = stage(inp)
         st.cache.append(st.block_table, st.seq_ids, st.positions, st.k_new, st.v_new)
-        assert st.cache.workspace_bytes(inp.q.shape[0], 32, inp.max_context_len, partition) > 0
+        need = st.cache.workspace_bytes(inp.q.shape[0], 32, inp.max_context_len, partition)
+        assert 0 < need <= pk.KV_STATIC_WORKSPACE_BYTES
         want = _regular_call(st, partition)
-        got = _static_call(st, partition)
-        torch.cuda.synchronize()
-        assert st.cache.errors() == 0
-        assert torch.isfinite(got.float()).all()
-        _assert_close(got, want, inp.spec.kv_dtype)
+        for _ in range(2):                          # a second call over the first's partials
+            got = _static_call(st, partition)
+            torch.cuda.synchronize()
+            assert st.cache.errors() == 0
+            assert torch.equal(got, want)
 
 
 def test_static_workspace_refuses_oversized_requests():
