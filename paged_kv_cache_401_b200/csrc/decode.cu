@@ -41,6 +41,8 @@
 //               lane owning D/32 output columns, all in fp32;
 //  * every wait is bounded; bad block ids and context lengths are reported
 //    through the error word and never dereferenced.
+#include <atomic>
+
 #include "kernels.cuh"
 #include "quant.cuh"
 
@@ -1362,8 +1364,7 @@ __device__ __noinline__ void append_row(uint8_t* st, const AppendRow a, int32_t 
 }
 
 template <class M, int Q_T>
-__global__ void __launch_bounds__(kThreads, M::kMinBlocks)
-    paged_decode_kernel(const DecodeParams p, const __grid_constant__ TmaMaps maps) {
+__device__ __forceinline__ void decode_body(const DecodeParams& p, const TmaMaps& maps) {
     using S = Smem<M>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>(
@@ -1562,6 +1563,38 @@ __global__ void __launch_bounds__(kThreads, M::kMinBlocks)
     }
 }
 
+// Registers per thread for kMinBlocks resident CTAs of kThreads.
+constexpr int decode_max_regs(int min_blocks) {
+    return min_blocks >= 3 ? 128 : (min_blocks == 2 ? 168 : 255);
+}
+
+// The decode grid.  For the tensor-core tiles the registers are capped directly:
+// passing the resident CTA count to __launch_bounds__ instead gives them the same
+// register counts but 4 to 32 bytes of spills per thread, about one local load per
+// tile (removing them measured time-neutral).  The CUDA-core tiles spill less with
+// the CTA count given.
+template <class M, int Q_T>
+__global__ void __launch_bounds__(kThreads) __maxnreg__(decode_max_regs(M::kMinBlocks))
+    paged_decode_kernel(const DecodeParams p, const __grid_constant__ TmaMaps maps) {
+    decode_body<M, Q_T>(p, maps);
+}
+
+template <class M, int Q_T>
+__global__ void __launch_bounds__(kThreads, M::kMinBlocks)
+    paged_decode_kernel_simt(const DecodeParams p, const __grid_constant__ TmaMaps maps) {
+    decode_body<M, Q_T>(p, maps);
+}
+
+// The entry point of a tile type (only that one is instantiated): tensor-core tiles
+// the register-capped one, CUDA-core tiles the other.
+template <class M, int Q_T>
+constexpr auto decode_entry() {
+    if constexpr (M::kUsesTma)
+        return &paged_decode_kernel<M, Q_T>;
+    else
+        return &paged_decode_kernel_simt<M, Q_T>;
+}
+
 // ======================================================================================
 // Merge kernel: one warp per (sequence, query head).  Pairs split over several
 // consumer ranges are combined:  M = max_p m_p;  w_p = 2^(m_p - M);
@@ -1722,20 +1755,35 @@ constexpr int kMaxDevices = 64;
 template <class M, int Q_T, int D>
 static cudaError_t launch_one(const DecodeParams& p, const TmaMaps& maps, cudaStream_t stream) {
     using S = Smem<M>;
-    static bool attr_set[kMaxDevices] = {};  // benign race: every caller sets the same value
+    constexpr auto kernel = decode_entry<M, Q_T>();
+    // Whether this device's context has the kernel's dynamic shared-memory limit raised.
+    // A context destroyed and created again (cudaDeviceReset) loses it while the flag
+    // stays set; the launch then fails before anything runs, and is retried once after
+    // raising the limit again.
+    static std::atomic<bool> attr_set[kMaxDevices] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= kMaxDevices || !attr_set[dev]) {
-        e = cudaFuncSetAttribute(paged_decode_kernel<M, Q_T>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+    auto set_attr = [&]() -> cudaError_t {
+        const cudaError_t a = cudaFuncSetAttribute(
+            kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, S::kBytes);
+        if (a == cudaSuccess && dev < kMaxDevices)
+            attr_set[dev].store(true, std::memory_order_relaxed);
+        return a;
+    };
+    if (dev >= kMaxDevices || !attr_set[dev].load(std::memory_order_relaxed)) {
+        e = set_attr();
         if (e != cudaSuccess) return e;
-        if (dev < kMaxDevices) attr_set[dev] = true;
     }
     const unsigned grid =
         static_cast<unsigned>((p.num_ranges + kConsumerWarps - 1) / kConsumerWarps);
-    e = launch_pdl(paged_decode_kernel<M, Q_T>, dim3(grid), dim3(kThreads), S::kBytes, stream, p,
-                   maps);
+    e = launch_pdl(kernel, dim3(grid), dim3(kThreads), S::kBytes, stream, p, maps);
+    if (e == cudaErrorInvalidValue) {
+        cudaGetLastError();
+        e = set_attr();
+        if (e == cudaSuccess)
+            e = launch_pdl(kernel, dim3(grid), dim3(kThreads), S::kBytes, stream, p, maps);
+    }
     if (e != cudaSuccess) return e;
     const int64_t warps = static_cast<int64_t>(p.batch) * p.num_query_tokens * p.num_q_heads;
     return launch_pdl(paged_decode_merge_kernel<Q_T, D>,
