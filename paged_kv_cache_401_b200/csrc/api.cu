@@ -370,6 +370,10 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
     p.max_context_len = max_context_len;
     p.num_query_tokens = query_tokens;
     p.num_ranges = ranges;
+    // pieces per pair, at most about ranges / pairs + 1 (all contexts of the longest
+    // length): many of them -> four merge warps per output row
+    const int64_t pairs = static_cast<int64_t>(batch) * pool->num_kv_heads;
+    p.merge_warps_per_row = ranges / pairs + 1 > 16 ? 4 : 1;
     p.scale_log2 = scale * 1.4426950408889634f;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     p.ws_seq_start = reinterpret_cast<int32_t*>(ws);

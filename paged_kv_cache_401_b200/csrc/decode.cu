@@ -1568,11 +1568,14 @@ constexpr int decode_max_regs(int min_blocks) {
     return min_blocks >= 3 ? 128 : (min_blocks == 2 ? 168 : 255);
 }
 
-// The decode grid.  For the tensor-core tiles the registers are capped directly:
-// passing the resident CTA count to __launch_bounds__ instead gives them the same
-// register counts but 4 to 32 bytes of spills per thread, about one local load per
-// tile (removing them measured time-neutral).  The CUDA-core tiles spill less with
-// the CTA count given.
+// The decode grid.  The tensor-core tiles take the block size (__launch_bounds__
+// without a CTA count) and a register cap (__maxnreg__); the code needs both to be
+// spill-free.  Giving the resident CTA count to __launch_bounds__ instead yields
+// the same register counts with 4 to 32 bytes of spills per thread, about one local
+// load per tile (removing them measured time-neutral).  nvcc rejects the pair when
+// the register count is a literal; with the count depending on the tile type it
+// accepts it, and a compiler that did not would fail the build, not change the code.
+// The CUDA-core tiles spill less with the CTA count given.
 template <class M, int Q_T>
 __global__ void __launch_bounds__(kThreads) __maxnreg__(decode_max_regs(M::kMinBlocks))
     paged_decode_kernel(const DecodeParams p, const __grid_constant__ TmaMaps maps) {
@@ -1596,20 +1599,31 @@ constexpr auto decode_entry() {
 }
 
 // ======================================================================================
-// Merge kernel: one warp per (sequence, query head).  Pairs split over several
-// consumer ranges are combined:  M = max_p m_p;  w_p = 2^(m_p - M);
-// out = sum_p w_p o_p / sum_p w_p l_p.  Pairs of invalid length get zeros.
+// Merge kernel: pairs split over several consumer ranges are combined:
+//   M = max_p m_p;  w_p = 2^(m_p - M);  out = sum_p w_p o_p / sum_p w_p l_p.
+// A CTA is four warps.  With few pieces per pair each warp merges one output row
+// (sequence, query token, head); when the split gives pairs many pieces (a few
+// very long sequences) the four warps of a CTA share one row, fold a quarter of
+// its pieces each and combine the four partial (max, sum, output) in warp order.
+// Pairs of invalid length get zeros.
 // ======================================================================================
-template <int Q_T, int D>
-__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p) {
+constexpr int kMergeWarps = 4;
+
+template <int Q_T, int D, bool KIVI, int WPR>
+__global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_merge_kernel(const DecodeParams p) {
     using OutT = typename QType<Q_T>::T;
     constexpr int kDPL = D / 32;
     constexpr int kBatch = 8;  // pieces whose partial outputs are loaded together
+    __shared__ float sm_o[kMergeWarps][D];
+    __shared__ float sm_ml[kMergeWarps][2];
     pdl_wait();
     pdl_trigger();
     const int32_t lane = threadIdx.x & 31;
-    // one warp per output row (sequence b, query token i, head h): out is [B][Q][Hq][D]
-    const int64_t bh = static_cast<int64_t>(blockIdx.x) * 4 + (threadIdx.x >> 5);
+    const int32_t warp = threadIdx.x >> 5;
+    constexpr int32_t wpr = WPR;                // warps per output row: 1 or 4
+    const int32_t part = warp % wpr;            // this warp's share of the row's pieces
+    // the output row (sequence b, query token i, head h): out is [B][Q][Hq][D]
+    const int64_t bh = static_cast<int64_t>(blockIdx.x) * (kMergeWarps / wpr) + warp / wpr;
     const int32_t nq = p.num_query_tokens;
     const int64_t rows_total = static_cast<int64_t>(p.batch) * nq * p.num_q_heads;
     if (bh >= rows_total) return;
@@ -1636,16 +1650,18 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
     const int32_t nt = seq_tiles(L, p);
     OutT* out = static_cast<OutT*>(p.out) + bh * D + lane * kDPL;
     if (!seq_valid(L, p)) {
+        if (part == 0) {
 #pragma unroll
-        for (int j = 0; j < kDPL; ++j) out[j] = out_cast<OutT>(0.0f);
-        if (lane == 0 && g == 0 && kvh == 0) report(p.dev_error, KV_DEVERR_BAD_CONTEXT_LEN);
+            for (int j = 0; j < kDPL; ++j) out[j] = out_cast<OutT>(0.0f);
+            if (lane == 0 && g == 0 && kvh == 0) report(p.dev_error, KV_DEVERR_BAD_CONTEXT_LEN);
+        }
         return;
     }
     const int64_t a = seq0 + static_cast<int64_t>(kvh) * nt;
     const int64_t w_first = nt > 0 ? range_of(a, T, p.num_ranges) : 0;
     const int64_t w_last = nt > 0 ? range_of(a + nt - 1, T, p.num_ranges) : -1;
     // a pair within one range was written by the decode kernel (KIVI: never)
-    if (!p.kivi && w_first == w_last) return;
+    if (!KIVI && w_first == w_last) return;
     const int64_t s = static_cast<int64_t>(b) * p.num_kv_heads + kvh;
     const int32_t npieces = static_cast<int32_t>(w_last - w_first + 1);
     // pieces are (pair s, range W) for the non-empty ranges W in [w_first, w_last],
@@ -1656,17 +1672,20 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
         if (all_ranges_full) return s + W;
         return range_begin(W, T, p.num_ranges) < range_begin(W + 1, T, p.num_ranges) ? s + W : -1;
     };
+    // this warp's pieces [pb, pe)
+    const int32_t pb = static_cast<int32_t>((static_cast<int64_t>(npieces) * part) / wpr);
+    const int32_t pe = static_cast<int32_t>((static_cast<int64_t>(npieces) * (part + 1)) / wpr);
     float o[kDPL];
 #pragma unroll
     for (int j = 0; j < kDPL; ++j) o[j] = 0.0f;
     float l = 0.0f;
     float M = -INFINITY;
-    for (int i0 = 0; i0 < npieces; i0 += 32) {
+    for (int i0 = pb; i0 < pe; i0 += 32) {
         // lane i: piece i0+i's (m, l); every lane: this round's first kBatch partial
         // outputs -- both sets of loads are in flight together
-        const int64_t pl = (i0 + lane < npieces) ? piece_id(i0 + lane) : -1;
+        const int64_t pl = (i0 + lane < pe) ? piece_id(i0 + lane) : -1;
         const float2 ml = pl >= 0 ? p.ws_ml[pl * R + g] : make_float2(-INFINITY, 0.0f);
-        const int cnt = min(32, npieces - i0);
+        const int cnt = min(32, pe - i0);
         float v[kBatch][kDPL];
         int64_t pids[kBatch];
 #pragma unroll
@@ -1714,33 +1733,82 @@ __global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodePar
             }
         }
     }
-    if (p.kivi) {
+    if constexpr (WPR > 1) {
+        // the row's warps' (M, l, o), combined by its first warp in warp order
+#pragma unroll
+        for (int m = 16; m >= 1; m >>= 1) l += __shfl_xor_sync(0xffffffffu, l, m);
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) sm_o[warp][lane * kDPL + j] = o[j];
+        if (lane == 0) {
+            sm_ml[warp][0] = M;
+            sm_ml[warp][1] = l;
+        }
+        __syncthreads();
+        if (part != 0) return;
+        float Mt = -INFINITY;
+        for (int w = warp; w < warp + wpr; ++w) Mt = fmaxf(Mt, sm_ml[w][0]);
+        float lt = 0.0f;
+#pragma unroll
+        for (int j = 0; j < kDPL; ++j) o[j] = 0.0f;
+        for (int w = warp; w < warp + wpr; ++w) {
+            const float mw = sm_ml[w][0];
+            const float c = mw == -INFINITY ? 0.0f : exp2f(mw - Mt);
+            lt += c * sm_ml[w][1];
+#pragma unroll
+            for (int j = 0; j < kDPL; ++j) o[j] = fmaf(c, sm_o[w][lane * kDPL + j], o[j]);
+        }
+        M = Mt;
+        l = lane == 0 ? lt : 0.0f;  // lane-partial again: counted once in the sum below
+    }
+    if constexpr (KIVI) {
         // KIVI: the newest L mod 16 tokens, kept in bf16 at res_k / res_v
-        // [batch][Hkv][16][D], join the softmax (same base-2 scores)
+        // [batch][Hkv][16][D], join the softmax (same base-2 scores).  All their
+        // key rows are read and scored first (independent loads and reductions),
+        // then one rescale, then all value rows.
         const int32_t nres = L % kBlockTokens;
-        float qf[kDPL];
+        if (nres > 0) {
+            float qf[kDPL];
 #pragma unroll
-        for (int j = 0; j < kDPL; ++j) qf[j] = load_q_elem<Q_T>(p.q, bh * D + lane * kDPL + j);
-        const int64_t rbase = ((static_cast<int64_t>(b) * p.num_kv_heads + kvh) * kBlockTokens) * D +
-                              lane * kDPL;
-        for (int r = 0; r < nres; ++r) {
-            const uint16_t* kr = p.res_k + rbase + r * D;
-            const uint16_t* vr = p.res_v + rbase + r * D;
-            float dot = 0.0f;
+            for (int j = 0; j < kDPL; ++j) qf[j] = load_q_elem<Q_T>(p.q, bh * D + lane * kDPL + j);
+            const int64_t rbase =
+                ((static_cast<int64_t>(b) * p.num_kv_heads + kvh) * kBlockTokens) * D + lane * kDPL;
+            float sc[kBlockTokens];
 #pragma unroll
-            for (int j = 0; j < kDPL; ++j)
-                dot = fmaf(qf[j], __uint_as_float(static_cast<uint32_t>(kr[j]) << 16), dot);
+            for (int r = 0; r < kBlockTokens; ++r) {
+                float dot = 0.0f;
+                if (r < nres) {
+                    const uint16_t* kr = p.res_k + rbase + r * D;
 #pragma unroll
-            for (int m = 16; m >= 1; m >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, m);
-            const float sc = dot * p.scale_log2;
-            const float M_new = fmaxf(M, sc);
-            const float c = exp2f(M - M_new);
-            const float w = exp2f(sc - M_new);
+                    for (int j = 0; j < kDPL; ++j)
+                        dot = fmaf(qf[j], __uint_as_float(static_cast<uint32_t>(kr[j]) << 16), dot);
+                }
+                sc[r] = dot;
+            }
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1)
+#pragma unroll
+                for (int r = 0; r < kBlockTokens; ++r)
+                    sc[r] += __shfl_xor_sync(0xffffffffu, sc[r], m);
+            float M_new = M;
+#pragma unroll
+            for (int r = 0; r < kBlockTokens; ++r)
+                if (r < nres) M_new = fmaxf(M_new, sc[r] * p.scale_log2);
+            const float c = exp2f(M - M_new);  // 0 while nothing came before (M = -inf)
+            l *= c;
+#pragma unroll
+            for (int j = 0; j < kDPL; ++j) o[j] *= c;
+#pragma unroll
+            for (int r = 0; r < kBlockTokens; ++r) {
+                if (r < nres) {
+                    const float w = exp2f(sc[r] * p.scale_log2 - M_new);
+                    l += lane == 0 ? w : 0.0f;  // l is lane-partial: count the token once
+                    const uint16_t* vr = p.res_v + rbase + r * D;
+#pragma unroll
+                    for (int j = 0; j < kDPL; ++j)
+                        o[j] = fmaf(w, __uint_as_float(static_cast<uint32_t>(vr[j]) << 16), o[j]);
+                }
+            }
             M = M_new;
-            l = l * c + (lane == 0 ? w : 0.0f);  // l is lane-partial: count the token once
-#pragma unroll
-            for (int j = 0; j < kDPL; ++j)
-                o[j] = fmaf(w, __uint_as_float(static_cast<uint32_t>(vr[j]) << 16), o[j] * c);
         }
     }
 #pragma unroll
@@ -1785,9 +1853,23 @@ static cudaError_t launch_one(const DecodeParams& p, const TmaMaps& maps, cudaSt
             e = launch_pdl(kernel, dim3(grid), dim3(kThreads), S::kBytes, stream, p, maps);
     }
     if (e != cudaSuccess) return e;
-    const int64_t warps = static_cast<int64_t>(p.batch) * p.num_query_tokens * p.num_q_heads;
-    return launch_pdl(paged_decode_merge_kernel<Q_T, D>,
-                      dim3(static_cast<unsigned>((warps + 3) / 4)), dim3(128), 0, stream, p);
+    const int64_t rows = static_cast<int64_t>(p.batch) * p.num_query_tokens * p.num_q_heads;
+    const int64_t rows_per_cta = kMergeWarps / p.merge_warps_per_row;
+    const dim3 merge_grid(static_cast<unsigned>((rows + rows_per_cta - 1) / rows_per_cta));
+    const dim3 merge_block(kMergeWarps * 32);
+    // the KIVI merge also attends to the bf16 residual, the split one shares rows
+    // between warps: their own instantiations, so the common one keeps its smaller
+    // register footprint (and occupancy)
+    const bool split = p.merge_warps_per_row > 1;
+    if (p.kivi)
+        return split ? launch_pdl(paged_decode_merge_kernel<Q_T, D, true, kMergeWarps>,
+                                  merge_grid, merge_block, 0, stream, p)
+                     : launch_pdl(paged_decode_merge_kernel<Q_T, D, true, 1>, merge_grid,
+                                  merge_block, 0, stream, p);
+    return split ? launch_pdl(paged_decode_merge_kernel<Q_T, D, false, kMergeWarps>, merge_grid,
+                              merge_block, 0, stream, p)
+                 : launch_pdl(paged_decode_merge_kernel<Q_T, D, false, 1>, merge_grid,
+                              merge_block, 0, stream, p);
 }
 
 template <int KV_T, int Q_T, int D>

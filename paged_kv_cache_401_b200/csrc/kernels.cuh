@@ -64,6 +64,8 @@ struct DecodeParams {
     int32_t max_context_len;
     int32_t num_query_tokens;     // Q: query tokens per sequence (1 for decode)
     int32_t num_ranges;           // consumer-warp ranges the tile list is cut into
+    int32_t merge_warps_per_row;  // 1: four output rows per merge CTA; 4: one row per CTA,
+                                  // its pieces split over the four warps
     float scale_log2;             // scale * log2(e): scores are kept in base-2 units
     // Fused append (one query token): every sequence's new K/V row [B][Hkv][D] in
     // append_src_dtype is written to the slot of position L - 1 (codes and scale
