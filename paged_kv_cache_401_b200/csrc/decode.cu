@@ -211,6 +211,26 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
                  : "r"(addr));
 }
 
+// 4-bit codes staged as 16-code groups padded to 16 bytes (the TMA's 16U4_ALIGN16B
+// layout), widened to one code per byte (low nibble) by the load.  Four 8-row x
+// 16-code matrices: lane l gets row l / 4, codes 4 (l % 4) .. + 3 of each, as
+// ldmatrix .b16 gives 8-bit rows; lanes 8m .. 8m + 7 address matrix m's rows.
+__device__ __forceinline__ void ldsm_x4_u4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n16.x4.shared.b8x16.b4x16_p64 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// Two 16-row x 16-code matrices of the same layout, transposed: lane (gid, tig)
+// gets codes of rows 4 tig .. + 3 in column gid (r[0]) and column gid + 8 (r[1]),
+// then the same of the second matrix (r[2], r[3]); lanes 0-15 and 16-31 address
+// the two matrices' rows.
+__device__ __forceinline__ void ldsm_x2_trans_u4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8x16.b4x16_p64 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
 // d += A(16x16, row) * B(16x8, col), fp32 accumulate; bf16 or f16 operands.
 template <bool F16>
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
@@ -744,6 +764,10 @@ struct MmaMath {
     static constexpr bool kF16 = kQuantized<KV_T>;              // codes widened to f16
     static constexpr bool kKivi = KV_T == KV_KIVI4;             // 4-bit, per-channel K params
     static constexpr bool kI4 = KV_T == KV_INT4 || kKivi;       // 4-bit codes, 64-byte rows
+    // INT4 tiles land in shared memory as 16-code groups padded to 16 bytes (128-byte
+    // rows, 128-byte swizzle) and are widened to bytes by ldmatrix; KIVI tiles keep
+    // their packed 64-byte rows
+    static constexpr bool kU4 = KV_T == KV_INT4;
     static_assert(!kKivi || QM == kSingle, "KIVI pools: one query token");
     // parameter block: INT4 (scale, zero) per K row then per V row; KIVI per K
     // channel (128) then per V row (16), as float2
@@ -754,16 +778,17 @@ struct MmaMath {
     static constexpr bool kCanAppend = SINGLE && !kKivi;          // fused append: decode only
     static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
     static constexpr int kRowBytes = kI4 ? D / 2 : D * KvElem<KV_T>::kBytes;  // 256 / 128 / 64
-    static constexpr int kBoxRow = kI4 ? 64 : 128;                // bytes of a TMA box row
-    static constexpr int kBoxCols = kI4 ? 64 : 128 / (KvElem<KV_T>::kBytes + kI4);  // box row, elements
-    static constexpr int kBoxes = kRowBytes / kBoxRow;
+    static constexpr int kBoxRow = (kI4 && !kU4) ? 64 : 128;      // shared-memory bytes of a box row
+    static constexpr int kBoxCols = kU4 ? 128 : (kI4 ? 64 : 128 / KvElem<KV_T>::kBytes);  // elements
+    static constexpr int kBoxes = kU4 ? 1 : kRowBytes / kBoxRow;
     static constexpr int kBoxBytes = kBlockTokens * kBoxRow;
-    static constexpr int kTileBytes = kBlockTokens * kRowBytes;
+    static constexpr int kTileBytes = kBoxes * kBoxBytes;         // a K or V tile in shared memory
+    static constexpr int kTileTx = kBlockTokens * kRowBytes;      // ... and the bytes it copies
     // K then V row parameters: fp32 scales (8-bit) or fp32 (scale, zero) pairs (4-bit)
     static constexpr int kScaleBytes =
         kKivi ? (128 + kBlockTokens) * 8 : (kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0));
     static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
-    static constexpr int kStages = kI4 ? 16 : (kF16 ? 12 : 8);     // multiple of 4
+    static constexpr int kStages = kU4 ? 12 : (kI4 ? 16 : (kF16 ? 12 : 8));  // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr bool kUsesTma = true;                        // tensor-map tile copies
     static constexpr int kWarpScratch = 0;
@@ -773,7 +798,7 @@ struct MmaMath {
     __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
                                  const TmaMaps& maps) {
         const int32_t row = static_cast<int32_t>(tile * kBlockTokens);
-        mbar_arrive_expect_tx(bar, 2 * kTileBytes + kScaleBytes);
+        mbar_arrive_expect_tx(bar, 2 * kTileTx + kScaleBytes);
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
             tma_load_2d(st + bx * kBoxBytes, &maps.k, bx * kBoxCols, row, bar);
@@ -783,16 +808,18 @@ struct MmaMath {
             bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * (kScaleBytes / 4), kScaleBytes, bar);
     }
 
-    // Byte offset of byte `byte` of row `row` in a staged (swizzled) K or V tile.
+    // Byte offset of byte `byte` of row `row` (as the pool stores it) in a staged
+    // (swizzled) K or V tile; padded INT4 rows hold 8 bytes of codes per 16 bytes.
     __device__ static __forceinline__ int32_t tile_byte(int32_t row, int32_t byte) {
+        if constexpr (kU4) return static_cast<int32_t>(swz(row, byte >> 3)) + (byte & 7);
         return static_cast<int32_t>(swz(row, byte >> 4)) + (byte & 15);
     }
 
     // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile:
-    // the 128-byte swizzle (chunk ^ row % 8 within 128-byte rows), or for 4-bit
-    // tiles the 64-byte swizzle (chunk ^ (row / 2) % 4 within 64-byte rows).
+    // the 128-byte swizzle (chunk ^ row % 8 within 128-byte rows), or for packed
+    // 4-bit tiles the 64-byte swizzle (chunk ^ (row / 2) % 4 within 64-byte rows).
     __device__ static __forceinline__ uint32_t swz(int32_t row, int32_t chunk) {
-        if constexpr (kI4) return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
+        if constexpr (kI4 && !kU4) return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
         return (chunk >> 3) * kBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
     }
 
@@ -800,10 +827,20 @@ struct MmaMath {
     // dims; 4-bit m-tile (c, j) = (mi / 2, mi % 2) holds dims 32c + 4r' + 2j (+1 for
     // r >= 8), r' = r % 8 (the nibble order of a transposed 16-bit unit)
     __device__ static __forceinline__ int32_t dim_of(int32_t mi, int32_t r) {
+        if constexpr (kU4) return 16 * mi + r;  // widened rows transposed per byte
         if constexpr (kI4)
             return 32 * (mi >> 1) + 4 * (r & 7) + 2 * (mi & 1) + (r >> 3);
         if constexpr (kF16) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
         return 16 * mi + r;
+    }
+
+    // Padded INT4 tiles: the transposed byte load hands lane tig the V rows of tokens
+    // 4 tig .. 4 tig + 3, where the MMA's k pairs are 2 tig, 2 tig + 1 and 2 tig + 8,
+    // 2 tig + 9.  Score column n is therefore token tok(n) (the K rows are addressed in
+    // that order), so P's fragment matches the V fragment without moving data.
+    __device__ static __forceinline__ int32_t tok(int32_t n) {
+        if constexpr (kU4) return 4 * ((n & 7) >> 1) + (n & 1) + 2 * (n >> 3);
+        return n;
     }
 
     // ---- consumer side
@@ -836,7 +873,7 @@ struct MmaMath {
             for (int ks = 0; ks < 8; ++ks) {
                 if (r >= rows) {
                     qa[k][ks][0] = qa[k][ks][1] = 0u;
-                } else if constexpr (kI4) {
+                } else if constexpr (kI4 && !kU4) {
                     // 4-bit rows: a lane's ldmatrix word is dims 32c + 8tig + 0..7 of chunk c.
                     // KIVI keys widen pairs (e, e+4): k-step 2c takes dims (+0,+4 | +1,+5),
                     // 2c+1 (+2,+6 | +3,+7); INT4 keys widen pairs (e, e+2) through E4M3:
@@ -871,6 +908,11 @@ struct MmaMath {
                                                __uint_as_float(w.x & 0xffff0000u));
                     qa[k][ks][1] = pack2<true>(__uint_as_float(w.y << 16),
                                                __uint_as_float(w.y & 0xffff0000u));
+                    if constexpr (kU4) {  // widened INT4 codes: the row's q sum too
+                        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
+                        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
+                        qs += (f0.x + f0.y) + (f1.x + f1.y);
+                    }
                 }
             }
             if constexpr (kI4 && !kKivi) {
@@ -920,7 +962,7 @@ struct MmaMath {
             if constexpr (WIDE) return qa[1][ks][h];
             return 0u;
         };
-        if constexpr (kI4) {
+        if constexpr (kI4 && !kU4) {
 #pragma unroll
             for (int cq = 0; cq < 2; ++cq) {
                 uint32_t w[4];  // {(tokens 0-7, chunk 2cq), (8-15, 2cq), (0-7, 2cq+1), (8-15, 2cq+1)}
@@ -979,7 +1021,10 @@ struct MmaMath {
 #pragma unroll
             for (int kq = 0; kq < 4; ++kq) {
                 uint32_t w[4];  // {(ks 2kq, nt0), (2kq+1, nt0), (2kq, nt1), (2kq+1, nt1)}
-                ldsm_x4(w, k_s + swz(8 * (mtx >> 1) + r, 2 * kq + (mtx & 1)));
+                if constexpr (kU4)  // score column n is token tok(n): rows addressed in that order
+                    ldsm_x4_u4(w, k_s + swz(tok(8 * (mtx >> 1) + r), 2 * kq + (mtx & 1)));
+                else
+                    ldsm_x4(w, k_s + swz(8 * (mtx >> 1) + r, 2 * kq + (mtx & 1)));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int ks = 2 * kq + h;
@@ -1005,7 +1050,7 @@ struct MmaMath {
             for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const int t = 8 * nt + 2 * tig + j;
+                    const int t = tok(8 * nt + 2 * tig + j);  // token of this score
                     float v;
                     if constexpr (kKivi) {
                         v = s[nt][2 * k + j] * p.scale_log2;  // parameters are in q' and the codes
@@ -1086,7 +1131,7 @@ struct MmaMath {
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const int t = 8 * nt + 2 * tig + j;
+                        const int t = tok(8 * nt + 2 * tig + j);
                         pz[nt][j] = vpz[t];
                         const float pv = pr[k][nt][j] * pz[nt][j].x;
                         pr[k][nt][j] = (FULL || t < nvalid) ? pv : 0.0f;
@@ -1098,7 +1143,7 @@ struct MmaMath {
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt) {
                     const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&pb[k][nt]));
-                    const int t = 8 * nt + 2 * tig;
+                    const int t = tok(8 * nt + 2 * tig);  // tok(n + 1) = tok(n) + 1 for even n
                     bsum += (FULL || t < nvalid) ? f.x * pz[nt][0].y : 0.0f;
                     bsum += (FULL || t + 1 < nvalid) ? f.y * pz[nt][1].y : 0.0f;
                 }
@@ -1122,7 +1167,27 @@ struct MmaMath {
         const uint32_t mask_b = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
 
         // ---- O^T += V^T.P^T over 8 m-tiles of 16 head dims
-        if constexpr (kI4) {
+        if constexpr (kU4) {
+#pragma unroll
+            for (int mp = 0; mp < 4; ++mp) {
+                // chunks 2mp, 2mp + 1 (16 dims each), all 16 tokens, widened and transposed:
+                // w = {(dim gid), (dim gid + 8)} of chunk 2mp, then of chunk 2mp + 1, each
+                // the codes of tokens 4tig .. 4tig + 3 = score columns 2tig, 2tig + 1,
+                // 2tig + 8, 2tig + 9.  Every code widens to a finite value, and tokens past
+                // the context end have P' = 0, so no mask is needed
+                uint32_t w[4];
+                ldsm_x2_trans_u4(w, v_s + swz(lane & 15, 2 * mp + (lane >> 4)));
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                    uint32_t lo0, hi0, lo1, hi1;  // c 2^-9 of (dim, token pair)
+                    e4m3x4_to_f16x2x2(w[2 * m], lo0, hi0);
+                    e4m3x4_to_f16x2x2(w[2 * m + 1], lo1, hi1);
+#pragma unroll
+                    for (int k = 0; k < kSets; ++k)
+                        mma_16816<true>(o[k][2 * mp + m], lo0, lo1, hi0, hi1, pb[k][0], pb[k][1]);
+                }
+            }
+        } else if constexpr (kI4) {
 #pragma unroll
             for (int cq = 0; cq < 2; ++cq) {
                 uint32_t w[4];  // {(tok 0-7, chunk 2cq), (tok 8-15, 2cq), (0-7, 2cq+1), (8-15, 2cq+1)}
