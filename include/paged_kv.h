@@ -21,8 +21,8 @@
  *  - Every device buffer is owned by the caller.  The library allocates no
  *    device memory, keeps no state between calls and never synchronises:
  *    work is enqueued on the caller's stream (NULL = legacy default stream).
- *  - Device pointers must be 16-byte aligned (the K and V pools of an INT4 cache
- *    32-byte aligned); contiguous row-major layouts.
+ *  - Device pointers must be 16-byte aligned (the K and V pools of INT4 and KIVI
+ *    caches 32-byte aligned); contiguous row-major layouts.
  *  - Argument errors found on the host return KV_ERR_INVALID_ARGUMENT or
  *    KV_ERR_UNSUPPORTED before anything is enqueued; a failed launch returns
  *    KV_ERR_CUDA.  Nothing throws, nothing aborts the process.

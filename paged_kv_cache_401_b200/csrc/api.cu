@@ -99,28 +99,23 @@ kv_status encode_pool_map(CUtensorMap* map, const void* base, const kv_pool_desc
     if (encode == nullptr) return KV_ERR_CUDA;
     const cuuint64_t rows = static_cast<cuuint64_t>(pool->num_blocks) * pool->num_kv_heads *
                             kBlockTokens;
-    // INT4 rows are copied as 4-bit elements, each 16 of them padded to 16 bytes in
-    // shared memory (the kernel widens them to bytes as it loads them); KIVI rows as
-    // packed bytes with the 64-byte swizzle; everything else as 128-byte rows
-    const bool int4 = pool->dtype == KV_INT4;
-    const bool packed4 = pool->dtype == KV_KIVI4;
+    // 4-bit rows (INT4, KIVI) are copied as 4-bit elements, each 16 of them padded to
+    // 16 bytes in shared memory (the kernel widens them to bytes as it loads them);
+    // every row lands as 128 bytes with the 128-byte swizzle
+    const bool four_bit = kv_bits(pool->dtype) == 4;
     const int64_t rb = row_bytes(pool);
-    const cuuint64_t dims[2] = {packed4 ? static_cast<cuuint64_t>(rb)
-                                        : static_cast<cuuint64_t>(pool->head_dim), rows};
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(pool->head_dim), rows};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(rb)};
-    const cuuint32_t box[2] = {packed4 ? 64u
-                                       : (int4 ? 128u
-                                               : static_cast<cuuint32_t>(128 / pool->elem_bytes)),
+    const cuuint32_t box[2] = {four_bit ? 128u : static_cast<cuuint32_t>(128 / pool->elem_bytes),
                                static_cast<cuuint32_t>(kBlockTokens)};
     const cuuint32_t elem_strides[2] = {1, 1};
     const CUtensorMapDataType type =
         pool->dtype == KV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                               : (int4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B
-                                       : CU_TENSOR_MAP_DATA_TYPE_UINT8);
+                               : (four_bit ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B
+                                           : CU_TENSOR_MAP_DATA_TYPE_UINT8);
     const CUresult r = encode(map, type, 2, const_cast<void*>(base), dims, strides, box,
                               elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                              packed4 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
-                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? KV_OK : KV_ERR_INVALID_ARGUMENT;
 }
@@ -342,9 +337,9 @@ kv_status attention_impl(const kv_pool_desc* pool, void* out, const void* q, kv_
         return KV_ERR_INVALID_ARGUMENT;
     if (!aligned16(out) || !aligned16(q) || !aligned16(k_pool) || !aligned16(v_pool))
         return KV_ERR_INVALID_ARGUMENT;
-    // the 4-bit element copies of INT4 pools need 32-byte aligned pools
-    if (pool->dtype == KV_INT4 && ((reinterpret_cast<uintptr_t>(k_pool) & 31) != 0 ||
-                                   (reinterpret_cast<uintptr_t>(v_pool) & 31) != 0))
+    // the 4-bit element copies of INT4 and KIVI pools need 32-byte aligned pools
+    if (kv_bits(pool->dtype) == 4 && ((reinterpret_cast<uintptr_t>(k_pool) & 31) != 0 ||
+                                      (reinterpret_cast<uintptr_t>(v_pool) & 31) != 0))
         return KV_ERR_INVALID_ARGUMENT;
     const bool fp8 = quantized(pool->dtype);  // FP8, INT8 or INT4: a parameter pool
     if (fp8 != (scales != nullptr)) return KV_ERR_INVALID_ARGUMENT;

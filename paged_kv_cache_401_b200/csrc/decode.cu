@@ -308,34 +308,6 @@ __device__ __forceinline__ uint32_t hsub2u(uint32_t a, uint32_t b) {
     return r;
 }
 
-// Eight 4-bit codes c (one 32-bit word, nibble i = element i) -> four f16x2 of
-// 1024 + c: pair k holds nibbles k and k + 4, each placed in the low mantissa
-// bits of f16 1024 (0x6400), one shift and one and-or per pair.  The offset
-// must come off before the MMAs (the KIVI keys subtract 1024 + zero exactly):
-// folded into the sums instead, it cost the fp32 accumulation the codes' low
-// bits (38x the error, measured).
-__device__ __forceinline__ void nib8_to_biased_f16x2x4(uint32_t w, uint32_t* out) {
-#pragma unroll
-    for (int k = 0; k < 4; ++k) out[k] = ((w >> (4 * k)) & 0x000F000Fu) | 0x64006400u;
-}
-
-
-// Eight 4-bit codes -> four f16x2 of exact c * 2^-9 through the E4M3 conversion
-// (bytes 0..15 are the E4M3 codes of c * 2^-9: subnormals and the first binade
-// share the step 2^-9).  out = {(e0, e2), (e4, e6), (e1, e3), (e5, e7)}.
-__device__ __forceinline__ void nib8_to_f16x2x4_e4m3(uint32_t w, uint32_t* out) {
-    e4m3x4_to_f16x2x2(w & 0x0F0F0F0Fu, out[0], out[1]);
-    e4m3x4_to_f16x2x2((w >> 4) & 0x0F0F0F0Fu, out[2], out[3]);
-}
-
-// A transposed ldmatrix word of a 4-bit V tile (16-bit units of tokens t0, t1,
-// four dims d0..d3 each) -> {(t0 d0, t1 d0), (t0 d2, t1 d2), (t0 d1, t1 d1),
-// (t0 d3, t1 d3)} as f16x2 of exact c * 2^-9.
-__device__ __forceinline__ void nib8t_to_f16x2x4_e4m3(uint32_t w, uint32_t* out) {
-    e4m3x4_to_f16x2x2(__byte_perm(w & 0x0F0F0F0Fu, 0u, 0x3120), out[0], out[1]);
-    e4m3x4_to_f16x2x2(__byte_perm((w >> 4) & 0x0F0F0F0Fu, 0u, 0x3120), out[2], out[3]);
-}
-
 // 2^x for x <= 0 (softmax weights), flushing results below 2^-126 to zero.
 __device__ __forceinline__ float fast_exp2(float x) {
     float r;
@@ -764,10 +736,9 @@ struct MmaMath {
     static constexpr bool kF16 = kQuantized<KV_T>;              // codes widened to f16
     static constexpr bool kKivi = KV_T == KV_KIVI4;             // 4-bit, per-channel K params
     static constexpr bool kI4 = KV_T == KV_INT4 || kKivi;       // 4-bit codes, 64-byte rows
-    // INT4 tiles land in shared memory as 16-code groups padded to 16 bytes (128-byte
-    // rows, 128-byte swizzle) and are widened to bytes by ldmatrix; KIVI tiles keep
-    // their packed 64-byte rows
-    static constexpr bool kU4 = KV_T == KV_INT4;
+    // 4-bit tiles land in shared memory as 16-code groups padded to 16 bytes (128-byte
+    // rows, 128-byte swizzle) and are widened to bytes by ldmatrix
+    static constexpr bool kU4 = kI4;
     static_assert(!kKivi || QM == kSingle, "KIVI pools: one query token");
     // parameter block: INT4 (scale, zero) per K row then per V row; KIVI per K
     // channel (128) then per V row (16), as float2
@@ -778,8 +749,8 @@ struct MmaMath {
     static constexpr bool kCanAppend = SINGLE && !kKivi;          // fused append: decode only
     static constexpr int kSets = WIDE ? 2 : 1;                    // row sets used
     static constexpr int kRowBytes = kI4 ? D / 2 : D * KvElem<KV_T>::kBytes;  // 256 / 128 / 64
-    static constexpr int kBoxRow = (kI4 && !kU4) ? 64 : 128;      // shared-memory bytes of a box row
-    static constexpr int kBoxCols = kU4 ? 128 : (kI4 ? 64 : 128 / KvElem<KV_T>::kBytes);  // elements
+    static constexpr int kBoxRow = 128;                           // shared-memory bytes of a box row
+    static constexpr int kBoxCols = kU4 ? 128 : 128 / KvElem<KV_T>::kBytes;  // box row, elements
     static constexpr int kBoxes = kU4 ? 1 : kRowBytes / kBoxRow;
     static constexpr int kBoxBytes = kBlockTokens * kBoxRow;
     static constexpr int kTileBytes = kBoxes * kBoxBytes;         // a K or V tile in shared memory
@@ -788,7 +759,7 @@ struct MmaMath {
     static constexpr int kScaleBytes =
         kKivi ? (128 + kBlockTokens) * 8 : (kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0));
     static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
-    static constexpr int kStages = kU4 ? 12 : (kI4 ? 16 : (kF16 ? 12 : 8));  // multiple of 4
+    static constexpr int kStages = kF16 ? 12 : 8;                  // multiple of 4
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr bool kUsesTma = true;                        // tensor-map tile copies
     static constexpr int kWarpScratch = 0;
@@ -816,25 +787,20 @@ struct MmaMath {
     }
 
     // Byte offset of 16-byte chunk `chunk` of row `row` in a swizzled K or V tile:
-    // the 128-byte swizzle (chunk ^ row % 8 within 128-byte rows), or for packed
-    // 4-bit tiles the 64-byte swizzle (chunk ^ (row / 2) % 4 within 64-byte rows).
+    // the 128-byte swizzle (chunk ^ row % 8 within 128-byte rows).
     __device__ static __forceinline__ uint32_t swz(int32_t row, int32_t chunk) {
-        if constexpr (kI4 && !kU4) return row * 64 + ((chunk ^ ((row >> 1) & 3)) << 4);
         return (chunk >> 3) * kBoxBytes + row * 128 + (((chunk & 7) ^ (row & 7)) << 4);
     }
 
     // head-dim of row r (0..15) of output m-tile mi: 8-bit tiles interleave even/odd
-    // dims; 4-bit m-tile (c, j) = (mi / 2, mi % 2) holds dims 32c + 4r' + 2j (+1 for
-    // r >= 8), r' = r % 8 (the nibble order of a transposed 16-bit unit)
+    // dims (the byte order of a transposed 16-bit unit); bf16 and widened 4-bit tiles
+    // keep them in order
     __device__ static __forceinline__ int32_t dim_of(int32_t mi, int32_t r) {
-        if constexpr (kU4) return 16 * mi + r;  // widened rows transposed per byte
-        if constexpr (kI4)
-            return 32 * (mi >> 1) + 4 * (r & 7) + 2 * (mi & 1) + (r >> 3);
-        if constexpr (kF16) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
+        if constexpr (kF16 && !kU4) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
         return 16 * mi + r;
     }
 
-    // Padded INT4 tiles: the transposed byte load hands lane tig the V rows of tokens
+    // Padded 4-bit tiles: the transposed byte load hands lane tig the V rows of tokens
     // 4 tig .. 4 tig + 3, where the MMA's k pairs are 2 tig, 2 tig + 1 and 2 tig + 8,
     // 2 tig + 9.  Score column n is therefore token tok(n) (the K rows are addressed in
     // that order), so P's fragment matches the V fragment without moving data.
@@ -873,29 +839,6 @@ struct MmaMath {
             for (int ks = 0; ks < 8; ++ks) {
                 if (r >= rows) {
                     qa[k][ks][0] = qa[k][ks][1] = 0u;
-                } else if constexpr (kI4 && !kU4) {
-                    // 4-bit rows: a lane's ldmatrix word is dims 32c + 8tig + 0..7 of chunk c.
-                    // KIVI keys widen pairs (e, e+4): k-step 2c takes dims (+0,+4 | +1,+5),
-                    // 2c+1 (+2,+6 | +3,+7); INT4 keys widen pairs (e, e+2) through E4M3:
-                    // k-step 2c takes (+0,+2 | +4,+6), 2c+1 (+1,+3 | +5,+7)
-                    const uint4 w = *reinterpret_cast<const uint4*>(q + 32 * (ks >> 1) + 8 * tig);
-                    const uint32_t x[4] = {w.x, w.y, w.z, w.w};  // bf16 pairs (0,1) (2,3) ...
-                    const int h = ks & 1;
-                    auto el = [&](int d) {  // element d (0..7) of the lane's 8 dims as float
-                        return __uint_as_float((d & 1) ? (x[d >> 1] & 0xffff0000u) : (x[d >> 1] << 16));
-                    };
-                    if constexpr (kKivi) {
-                        qa[k][ks][0] = pack2<true>(el(2 * h), el(2 * h + 4));
-                        qa[k][ks][1] = pack2<true>(el(2 * h + 1), el(2 * h + 5));
-                    } else {
-                        qa[k][ks][0] = pack2<true>(el(h), el(h + 2));
-                        qa[k][ks][1] = pack2<true>(el(h + 4), el(h + 6));
-                    }
-                    if constexpr (!kKivi) {
-                        const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
-                        const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
-                        qs += (f0.x + f0.y) + (f1.x + f1.y);
-                    }
                 } else if constexpr (!kF16) {
                     // k index 2tig+{0,1} -> dim 16ks+2tig+{0,1}; 8+2tig+{0,1} -> 16ks+8+2tig+{0,1}
                     qa[k][ks][0] = *reinterpret_cast<const uint32_t*>(q + 16 * ks + 2 * tig);
@@ -908,7 +851,7 @@ struct MmaMath {
                                                __uint_as_float(w.x & 0xffff0000u));
                     qa[k][ks][1] = pack2<true>(__uint_as_float(w.y << 16),
                                                __uint_as_float(w.y & 0xffff0000u));
-                    if constexpr (kU4) {  // widened INT4 codes: the row's q sum too
+                    if constexpr (kU4 && !kKivi) {  // widened INT4 codes: the row's q sum too
                         const float2 f0 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][0]));
                         const float2 f1 = __half22float2(*reinterpret_cast<const __half2*>(&qa[k][ks][1]));
                         qs += (f0.x + f0.y) + (f1.x + f1.y);
@@ -962,54 +905,7 @@ struct MmaMath {
             if constexpr (WIDE) return qa[1][ks][h];
             return 0u;
         };
-        if constexpr (kI4 && !kU4) {
-#pragma unroll
-            for (int cq = 0; cq < 2; ++cq) {
-                uint32_t w[4];  // {(tokens 0-7, chunk 2cq), (8-15, 2cq), (0-7, 2cq+1), (8-15, 2cq+1)}
-                ldsm_x4(w, k_s + swz(8 * (mtx & 1) + r, 2 * cq + (mtx >> 1)));
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * cq + cc;  // 32-dim chunk: k-steps 2c and 2c + 1
-                    uint32_t b0[4], b1[4];      // n-tiles 0 / 1
-                    if constexpr (kKivi) {        // 1024 + c of dims {(0,4), (1,5), (2,6), (3,7)}
-                        nib8_to_biased_f16x2x4(w[2 * cc], b0);
-                        nib8_to_biased_f16x2x4(w[2 * cc + 1], b1);
-                    } else {                      // c 2^-9 of dims {(0,2), (4,6), (1,3), (5,7)}
-                        nib8_to_f16x2x4_e4m3(w[2 * cc], b0);
-                        nib8_to_f16x2x4_e4m3(w[2 * cc + 1], b1);
-                    }
-                    const int ka = 2 * c, kb = 2 * c + 1;
-                    uint32_t qa0 = qa[0][ka][0], qa1 = qa[0][ka][1], qb0 = qa[0][kb][0], qb1 = qa[0][kb][1];
-                    if constexpr (kKivi) {
-                        // key channel d: (c - zero_d) * scale_d.  q takes the scales (q' = q *
-                        // scale, f16), the codes the zero points ((1024 + c) - (1024 + zero),
-                        // exact in f16)
-                        const float4* pc = reinterpret_cast<const float4*>(ksc) + 16 * c + 4 * tig;
-                        const float4 p01 = pc[0], p23 = pc[1], p45 = pc[2], p67 = pc[3];
-                        const uint32_t zA = pack2<true>(1024.0f + p01.y, 1024.0f + p45.y);  // (0,4)
-                        const uint32_t zB = pack2<true>(1024.0f + p01.w, 1024.0f + p45.w);  // (1,5)
-                        const uint32_t zC = pack2<true>(1024.0f + p23.y, 1024.0f + p67.y);  // (2,6)
-                        const uint32_t zD = pack2<true>(1024.0f + p23.w, 1024.0f + p67.w);  // (3,7)
-                        qa0 = hmul2u(qa0, pack2<true>(p01.x, p45.x));
-                        qa1 = hmul2u(qa1, pack2<true>(p01.z, p45.z));
-                        qb0 = hmul2u(qb0, pack2<true>(p23.x, p67.x));
-                        qb1 = hmul2u(qb1, pack2<true>(p23.z, p67.z));
-                        b0[0] = hsub2u(b0[0], zA);
-                        b0[1] = hsub2u(b0[1], zB);
-                        b0[2] = hsub2u(b0[2], zC);
-                        b0[3] = hsub2u(b0[3], zD);
-                        b1[0] = hsub2u(b1[0], zA);
-                        b1[1] = hsub2u(b1[1], zB);
-                        b1[2] = hsub2u(b1[2], zC);
-                        b1[3] = hsub2u(b1[3], zD);
-                    }
-                    mma_16816<true>(s[0], qa0, a_hi(ka, 0), qa1, a_hi(ka, 1), b0[0], b0[1]);
-                    mma_16816<true>(s[1], qa0, a_hi(ka, 0), qa1, a_hi(ka, 1), b1[0], b1[1]);
-                    mma_16816<true>(s[0], qb0, a_hi(kb, 0), qb1, a_hi(kb, 1), b0[2], b0[3]);
-                    mma_16816<true>(s[1], qb0, a_hi(kb, 0), qb1, a_hi(kb, 1), b1[2], b1[3]);
-                }
-            }
-        } else if constexpr (!kF16) {
+        if constexpr (!kF16) {
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 uint32_t b[4];  // {nt0 dims lo, nt0 dims hi, nt1 dims lo, nt1 dims hi}
@@ -1031,8 +927,26 @@ struct MmaMath {
                     uint32_t b0, b1, b2, b3;
                     widen_k4<KV_T>(w[h], b0, b1);
                     widen_k4<KV_T>(w[2 + h], b2, b3);
-                    mma_16816<true>(s[0], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b0, b1);
-                    mma_16816<true>(s[1], qa[0][ks][0], a_hi(ks, 0), qa[0][ks][1], a_hi(ks, 1), b2, b3);
+                    uint32_t qa0 = qa[0][ks][0], qa1 = qa[0][ks][1];
+                    if constexpr (kKivi) {
+                        // key channel d: (c - zero_d) * scale_d.  q takes the scales (q' = q *
+                        // scale, f16), the codes the zero points: c 2^-9 - zero 2^-9 =
+                        // (c - zero) 2^-9, exact in f16 (the score takes the 2^-9 back).
+                        // This lane's dims of k-step ks: 16ks + 4tig + {0, 1} and {2, 3}
+                        constexpr uint32_t kTwoM9 = 0x18001800u;  // f16 2^-9, both halves
+                        const float4* pc = reinterpret_cast<const float4*>(ksc) + 8 * ks + 2 * tig;
+                        const float4 p01 = pc[0], p23 = pc[1];  // (scale, zero) of 2 channels each
+                        const uint32_t z01 = hmul2u(pack2<true>(p01.y, p01.w), kTwoM9);
+                        const uint32_t z23 = hmul2u(pack2<true>(p23.y, p23.w), kTwoM9);
+                        qa0 = hmul2u(qa0, pack2<true>(p01.x, p01.z));
+                        qa1 = hmul2u(qa1, pack2<true>(p23.x, p23.z));
+                        b0 = hsub2u(b0, z01);
+                        b1 = hsub2u(b1, z23);
+                        b2 = hsub2u(b2, z01);
+                        b3 = hsub2u(b3, z23);
+                    }
+                    mma_16816<true>(s[0], qa0, a_hi(ks, 0), qa1, a_hi(ks, 1), b0, b1);
+                    mma_16816<true>(s[1], qa0, a_hi(ks, 0), qa1, a_hi(ks, 1), b2, b3);
                 }
             }
         }
@@ -1053,7 +967,8 @@ struct MmaMath {
                     const int t = tok(8 * nt + 2 * tig + j);  // token of this score
                     float v;
                     if constexpr (kKivi) {
-                        v = s[nt][2 * k + j] * p.scale_log2;  // parameters are in q' and the codes
+                        // parameters are in q' and the codes; the codes carry 2^-9
+                        v = s[nt][2 * k + j] * (512.0f * p.scale_log2);
                     } else if constexpr (kI4) {
                         // (c - zero) * scale, summed over d with q: 512 acc - zero * sum_d q_d
                         const float2 pz = reinterpret_cast<const float2*>(ksc)[t];
@@ -1185,28 +1100,6 @@ struct MmaMath {
 #pragma unroll
                     for (int k = 0; k < kSets; ++k)
                         mma_16816<true>(o[k][2 * mp + m], lo0, lo1, hi0, hi1, pb[k][0], pb[k][1]);
-                }
-            }
-        } else if constexpr (kI4) {
-#pragma unroll
-            for (int cq = 0; cq < 2; ++cq) {
-                uint32_t w[4];  // {(tok 0-7, chunk 2cq), (tok 8-15, 2cq), (0-7, 2cq+1), (8-15, 2cq+1)}
-                ldsm_x4_trans(w, v_s + swz(8 * (mtx & 1) + r, 2 * cq + (mtx >> 1)));
-#pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * cq + cc;
-                    // tokens 2tig,2tig+1 / 8+2tig,9+2tig: c 2^-9 of dims {d0, d2, d1, d3}.
-                    // Every code widens to a finite value, and tokens past the context end
-                    // have P' = 0, so no mask is needed
-                    uint32_t h0[4], h1[4];
-                    nib8t_to_f16x2x4_e4m3(w[2 * cc], h0);
-                    nib8t_to_f16x2x4_e4m3(w[2 * cc + 1], h1);
-                    // m-tile 2c: rows gid <- dim 4gid, gid+8 <- 4gid+1; m-tile 2c+1: 4gid+2, 4gid+3
-#pragma unroll
-                    for (int k = 0; k < kSets; ++k) {
-                        mma_16816<true>(o[k][2 * c], h0[0], h0[2], h1[0], h1[2], pb[k][0], pb[k][1]);
-                        mma_16816<true>(o[k][2 * c + 1], h0[1], h0[3], h1[1], h1[3], pb[k][0], pb[k][1]);
-                    }
                 }
             }
         } else if constexpr (!kF16) {
