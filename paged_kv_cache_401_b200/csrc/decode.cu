@@ -30,12 +30,14 @@
 //    through the TMA engine (no multicast), completing on mbarriers; block
 //    ids are fetched 4 tiles ahead, and no warp's refill waits behind another;
 //  * the per-tile arithmetic is a policy:
-//      MmaMath  (bf16, FP8 or INT8 KV, head_dim 128, bf16 q): tiles land in shared
-//               memory 128-byte swizzled by 2-D TMA tensor copies; the group's
-//               scores S = Q.K^T come from mma.m16n8k16 (query heads as rows,
-//               fp32 accumulate), the softmax runs on the accumulator
-//               fragments, and P feeds O^T = V^T.P^T straight from registers;
-//               8-bit codes are widened to f16 in registers (exact);
+//      MmaMath  (bf16, FP8, INT8, INT4 or KIVI KV, head_dim 128, bf16 q): tiles
+//               land in shared memory 128-byte swizzled by 2-D TMA tensor copies
+//               (4-bit codes as 16-code groups padded to 16 bytes, widened to
+//               bytes by ldmatrix); the group's scores S = Q.K^T come from
+//               mma.m16n8k16 (query heads as rows, fp32 accumulate), the softmax
+//               runs on the accumulator fragments, and P feeds O^T = V^T.P^T
+//               straight from registers; codes are widened to f16 in registers
+//               (exact);
 //      SimtMath (every other shape and fp32): 1-D bulk copies; q.K with
 //               packed fp32x2 FMAs and a shuffle reduce-scatter, P.V with each
 //               lane owning D/32 output columns, all in fp32;
@@ -217,6 +219,15 @@ __device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], uint32_t addr) {
 // ldmatrix .b16 gives 8-bit rows; lanes 8m .. 8m + 7 address matrix m's rows.
 __device__ __forceinline__ void ldsm_x4_u4(uint32_t (&r)[4], uint32_t addr) {
     asm volatile("ldmatrix.sync.aligned.m8n16.x4.shared.b8x16.b4x16_p64 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+// Two 16-row x 16-byte matrices, transposed per byte: lane (gid, tig) gets bytes of
+// rows 4 tig .. + 3 in column gid (r[0]) and column gid + 8 (r[1]), then the same of
+// the second matrix (r[2], r[3]); lanes 0-15 and 16-31 address the two matrices' rows.
+__device__ __forceinline__ void ldsm_x2_trans_b8(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0,%1,%2,%3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
 }
@@ -697,7 +708,8 @@ struct SimtMath {
 };
 
 // ======================================================================================
-// MmaMath: tensor-core tile arithmetic for bf16, FP8 or INT8 KV, head_dim 128, bf16 q.
+// MmaMath: tensor-core tile arithmetic for bf16, FP8, INT8, INT4 or KIVI KV, head_dim
+// 128, bf16 q.
 //
 // A tile is 16 tokens x 128 dims.  K and V land in shared memory as [16 rows]
 // x [128-byte] boxes written by TMA with the 128-byte swizzle (16-byte chunk
@@ -720,7 +732,12 @@ struct SimtMath {
 // scale) rounded to f16; the K row scale multiplies the scores.  Element
 // orders inside a k-step are permuted consistently between the two operands
 // (a dot product does not depend on the order of its terms), which is what
-// lets 8-bit rows be read with 16-bit ldmatrix.  QM: kSingle = one query token
+// lets 8-bit rows be read with 16-bit ldmatrix.  4-bit KV (INT4, KIVI): the
+// TMA stages each 16 codes padded to 16 bytes, and ldmatrix widens them to one
+// code per byte, which the FP8 conversion turns into c * 2^-9 exactly; the row
+// (INT4) or channel (KIVI keys) parameters enter as in the comments below.
+// FP8 and 4-bit V tiles are read by a per-byte transposed ldmatrix, whose token
+// order the score columns follow (tok()).  QM: kSingle = one query token
 // (the decode: no causal bookkeeping), kNarrow = up to 8 query rows, kWide = up
 // to 16 (two row sets).
 // ======================================================================================
@@ -739,6 +756,9 @@ struct MmaMath {
     // 4-bit tiles land in shared memory as 16-code groups padded to 16 bytes (128-byte
     // rows, 128-byte swizzle) and are widened to bytes by ldmatrix
     static constexpr bool kU4 = kI4;
+    // V tiles read by the transposed byte load (4-bit and FP8 codes): the lanes then
+    // own tokens in the order tok() gives, and the K rows are addressed to match
+    static constexpr bool kByteV = kU4 || KV_T == KV_FP8_E4M3;
     static_assert(!kKivi || QM == kSingle, "KIVI pools: one query token");
     // parameter block: INT4 (scale, zero) per K row then per V row; KIVI per K
     // channel (128) then per V row (16), as float2
@@ -796,16 +816,16 @@ struct MmaMath {
     // dims (the byte order of a transposed 16-bit unit); bf16 and widened 4-bit tiles
     // keep them in order
     __device__ static __forceinline__ int32_t dim_of(int32_t mi, int32_t r) {
-        if constexpr (kF16 && !kU4) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
+        if constexpr (kF16 && !kByteV) return 16 * mi + (r < 8 ? 2 * r : 2 * (r - 8) + 1);
         return 16 * mi + r;
     }
 
-    // Padded 4-bit tiles: the transposed byte load hands lane tig the V rows of tokens
+    // Byte-transposed V tiles: the transposed byte load hands lane tig the V rows of tokens
     // 4 tig .. 4 tig + 3, where the MMA's k pairs are 2 tig, 2 tig + 1 and 2 tig + 8,
     // 2 tig + 9.  Score column n is therefore token tok(n) (the K rows are addressed in
     // that order), so P's fragment matches the V fragment without moving data.
     __device__ static __forceinline__ int32_t tok(int32_t n) {
-        if constexpr (kU4) return 4 * ((n & 7) >> 1) + (n & 1) + 2 * (n >> 3);
+        if constexpr (kByteV) return 4 * ((n & 7) >> 1) + (n & 1) + 2 * (n >> 3);
         return n;
     }
 
@@ -920,7 +940,7 @@ struct MmaMath {
                 if constexpr (kU4)  // score column n is token tok(n): rows addressed in that order
                     ldsm_x4_u4(w, k_s + swz(tok(8 * (mtx >> 1) + r), 2 * kq + (mtx & 1)));
                 else
-                    ldsm_x4(w, k_s + swz(8 * (mtx >> 1) + r, 2 * kq + (mtx & 1)));
+                    ldsm_x4(w, k_s + swz(tok(8 * (mtx >> 1) + r), 2 * kq + (mtx & 1)));
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int ks = 2 * kq + h;
@@ -1069,7 +1089,7 @@ struct MmaMath {
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const int t = 8 * nt + 2 * tig + j;
+                        const int t = tok(8 * nt + 2 * tig + j);
                         pr[k][nt][j] = (FULL || t < nvalid) ? pr[k][nt][j] * vsc[t] : 0.0f;
                     }
             }
@@ -1082,21 +1102,37 @@ struct MmaMath {
         const uint32_t mask_b = (2 * tig + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * tig + 9 < nvalid ? 0xffff0000u : 0u);
 
         // ---- O^T += V^T.P^T over 8 m-tiles of 16 head dims
-        if constexpr (kU4) {
+        if constexpr (kByteV) {
+            // FP8 codes past the context end may be NaN: masked by token when the tile is
+            // partial.  4-bit codes all widen to finite values and those tokens have
+            // P' = 0, so they need no mask
+            const bool vmask = !kU4 && partial;
+            const uint32_t m_lo = (4 * tig < nvalid ? 0x0000ffffu : 0u) |
+                                  (4 * tig + 1 < nvalid ? 0xffff0000u : 0u);
+            const uint32_t m_hi = (4 * tig + 2 < nvalid ? 0x0000ffffu : 0u) |
+                                  (4 * tig + 3 < nvalid ? 0xffff0000u : 0u);
 #pragma unroll
             for (int mp = 0; mp < 4; ++mp) {
-                // chunks 2mp, 2mp + 1 (16 dims each), all 16 tokens, widened and transposed:
-                // w = {(dim gid), (dim gid + 8)} of chunk 2mp, then of chunk 2mp + 1, each
-                // the codes of tokens 4tig .. 4tig + 3 = score columns 2tig, 2tig + 1,
-                // 2tig + 8, 2tig + 9.  Every code widens to a finite value, and tokens past
-                // the context end have P' = 0, so no mask is needed
+                // chunks 2mp, 2mp + 1 (16 dims each), all 16 tokens, transposed per byte
+                // (4-bit codes widened to bytes first): w = {(dim gid), (dim gid + 8)} of
+                // chunk 2mp, then of chunk 2mp + 1, each the codes of tokens 4tig ..
+                // 4tig + 3 = score columns 2tig, 2tig + 1, 2tig + 8, 2tig + 9
                 uint32_t w[4];
-                ldsm_x2_trans_u4(w, v_s + swz(lane & 15, 2 * mp + (lane >> 4)));
+                if constexpr (kU4)
+                    ldsm_x2_trans_u4(w, v_s + swz(lane & 15, 2 * mp + (lane >> 4)));
+                else
+                    ldsm_x2_trans_b8(w, v_s + swz(lane & 15, 2 * mp + (lane >> 4)));
 #pragma unroll
                 for (int m = 0; m < 2; ++m) {
-                    uint32_t lo0, hi0, lo1, hi1;  // c 2^-9 of (dim, token pair)
+                    uint32_t lo0, hi0, lo1, hi1;  // (dim, token pair), E4M3 -> f16 exact
                     e4m3x4_to_f16x2x2(w[2 * m], lo0, hi0);
                     e4m3x4_to_f16x2x2(w[2 * m + 1], lo1, hi1);
+                    if (vmask) {
+                        lo0 &= m_lo;
+                        lo1 &= m_lo;
+                        hi0 &= m_hi;
+                        hi1 &= m_hi;
+                    }
 #pragma unroll
                     for (int k = 0; k < kSets; ++k)
                         mma_16816<true>(o[k][2 * mp + m], lo0, lo1, hi0, hi1, pb[k][0], pb[k][1]);
