@@ -173,6 +173,24 @@ def test_decode_int4_needs_the_tensor_core_shape():
     assert _call_decode(d, q_dtype=pk.KV_F32, scales=6 << 20) == pk.KV_ERR_UNSUPPORTED
 
 
+@pytest.mark.parametrize("which", ["k_pool", "v_pool"])
+def test_decode_4bit_pools_need_32_byte_alignment(which):
+    # 4-bit pools are copied as 4-bit elements padded in shared memory, which needs
+    # 32-byte aligned sources: a 16-byte aligned pool is refused on the host
+    d = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_INT4)
+    base = {"k_pool": 1 << 20, "v_pool": 2 << 20}[which]
+    assert _call_decode(d, scales=6 << 20, **{which: base + 16}) == pk.KV_ERR_INVALID_ARGUMENT
+    dk = pk.kv_pool_create(8192, 16, 8, 128, pk.KV_KIVI4)
+    lib = pk.library()
+    ptrs = dict(k_pool=1 << 20, v_pool=2 << 20)
+    ptrs[which] += 16
+    status = lib.kivi_decode_attention(
+        ctypes.byref(dk), 4096, 8192, pk.KV_BF16, ptrs["k_pool"], ptrs["v_pool"], 6 << 20,
+        9 << 20, 10 << 20, None, None, 3 << 20, 256, 4 << 20, 32, 32, 4096, 0.088, 0,
+        5 << 20, 1 << 30, None, None)
+    assert status == pk.KV_ERR_INVALID_ARGUMENT
+
+
 @pytest.mark.parametrize("dtype", [pk.KV_FP8_E4M3, pk.KV_INT8, pk.KV_INT4])
 def test_decode_quantized_pool_requires_scales(dtype):
     d = pk.kv_pool_create(8192, 16, 8, 128, dtype)
