@@ -230,7 +230,11 @@ def unique_kv_bytes_per_step(inp) -> int:
     return kv_bytes_per_step(inp) - dup * spec.num_kv_heads * 2 * per_row
 
 
-def describe(inp, partition: int) -> dict:
+DATA = "synthetic (seeded N(0,1) q/K/V, random block permutation)"
+
+
+def describe(inp, partition: int, query_tokens: int) -> dict:
+    """The workload, the same for both arms (the implementation's own choices are not here)."""
     spec = inp.spec
     return {"workload": f"{spec.name}: paged GQA decode, batch {inp.q.shape[0]}, "
                         f"{spec.num_q_heads} q / {spec.num_kv_heads} kv heads, head_dim "
@@ -243,7 +247,8 @@ def describe(inp, partition: int) -> dict:
             "partition_tokens": partition if partition else "0 (balanced over all SMs)",
             "l2": "inputs larger than L2 (KV read per step > 126 MB), no flush"
             if kv_bytes_per_step(inp) > 126e6 else "inputs fit in L2, not flushed",
-            "parallelism": "replicas: one independent decode per GPU"}
+            "parallelism": "replicas: one independent decode per GPU",
+            "query_tokens": query_tokens}
 
 
 def measured_peak():
@@ -336,8 +341,8 @@ def run_reference(args, inp):
             "value": round(gbs, 3), "unit": "GB/s", "impl": "reference",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": describe(inp, 0),
+            "vs_baseline": None, "dtype": "f64", "data": DATA,
+            "config": describe(inp, args.partition, 1),
             "cpu_baseline": {"value": round(gbs, 3), "unit": "GB/s", "cores": cores,
                              "kind": "oracle", "sample": desc},
             "e2e": {"value": round(gbs, 3), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -618,11 +623,12 @@ def run_gpu(args, inp):
         "pct_of_peak": round(100 * value / world / peak, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": spec.kv_dtype if spec.kv_dtype != "fp8" else "fp8_e4m3",
-        "data": "synthetic (seeded N(0,1) q/K/V, random block permutation)",
-        "config": dict(describe(inp, P), num_ranges=ranges, query_tokens=Q,
-                       append=("KIVI residual append (+ block flush) in the decode call" if kivi
-                               else "fused into the decode call" if fused
-                               else "separate slot-mapping and cache-write calls")),
+        "data": DATA,
+        "config": describe(inp, P, Q),
+        "split": {"num_ranges": ranges,
+                  "append": ("KIVI residual append (+ block flush) in the decode call" if kivi
+                             else "fused into the decode call" if fused
+                             else "separate slot-mapping and cache-write calls")},
         "timing": {"regions": args.regions,
                    "region": f"{args.steps} steps back to back, barrier + synchronize on "
                              "both sides, CUDA events on the launching stream",
