@@ -780,6 +780,10 @@ struct MmaMath {
         kKivi ? (128 + kBlockTokens) * 8 : (kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0));
     static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
     static constexpr int kStages = kF16 ? 12 : 8;                  // multiple of 4
+    // KIVI: f16 key parameters (128 x {scale, zero 2^-9}) in the stage's unused tail
+    static constexpr int kKiviF16Params = 2 * kTileBytes + kScaleBytes;
+    static_assert(!kKivi || kStageBytes - kKiviF16Params >= 128 * 4, "f16 key parameters fit");
+    static_assert(kKiviF16Params % 16 == 0, "16-byte stores");
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr bool kUsesTma = true;                        // tensor-map tile copies
     static constexpr int kWarpScratch = 0;
@@ -901,7 +905,7 @@ struct MmaMath {
 
     // A tile whose 16 tokens every query row sees (for one query token: every tile but
     // a pair's last) needs no position masks, and runs an instantiation without them.
-    __device__ void tile(const uint8_t* kt, int32_t jb, int32_t L, const DecodeParams& p) {
+    __device__ void tile(uint8_t* kt, int32_t jb, int32_t L, const DecodeParams& p) {
         if ((jb + 1) * kBlockTokens <= L - nq + 1)
             tile_body<true>(kt, jb, L, p);
         else
@@ -909,7 +913,7 @@ struct MmaMath {
     }
 
     template <bool FULL>
-    __device__ __forceinline__ void tile_body(const uint8_t* kt, int32_t jb, int32_t L,
+    __device__ __forceinline__ void tile_body(uint8_t* kt, int32_t jb, int32_t L,
                                               const DecodeParams& p) {
         const uint32_t k_s = smem_addr(kt);
         const uint32_t v_s = k_s + kTileBytes;
@@ -921,6 +925,22 @@ struct MmaMath {
 
         // ---- S = Q.K^T: s[nt] = rows gid (c0, c1) and gid + 8 (c2, c3)
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        // KIVI: the 128 key channels' (scale, zero) as f16 {scale, zero 2^-9}, converted once
+        // per tile into the stage's tail, past the bytes the copies write (so no async-proxy
+        // write can meet these stores); lane l converts channels 4l .. 4l + 3
+        [[maybe_unused]] const uint4* kp16 = reinterpret_cast<const uint4*>(kt + kKiviF16Params);
+        if constexpr (kKivi) {
+            constexpr uint32_t kTwoM9 = 0x18001800u;  // f16 2^-9, both halves
+            const float4* pc = reinterpret_cast<const float4*>(ksc) + 2 * lane;
+            const float4 p01 = pc[0], p23 = pc[1];  // (scale, zero) of 2 channels each
+            uint4 h;
+            h.x = pack2<true>(p01.x, p01.z);
+            h.y = pack2<true>(p23.x, p23.z);
+            h.z = hmul2u(pack2<true>(p01.y, p01.w), kTwoM9);
+            h.w = hmul2u(pack2<true>(p23.y, p23.w), kTwoM9);
+            reinterpret_cast<uint4*>(kt + kKiviF16Params)[lane] = h;
+            __syncwarp();
+        }
         auto a_hi = [&](int ks, int h) -> uint32_t {
             if constexpr (WIDE) return qa[1][ks][h];
             return 0u;
@@ -951,19 +971,16 @@ struct MmaMath {
                     if constexpr (kKivi) {
                         // key channel d: (c - zero_d) * scale_d.  q takes the scales (q' = q *
                         // scale, f16), the codes the zero points: c 2^-9 - zero 2^-9 =
-                        // (c - zero) 2^-9, exact in f16 (the score takes the 2^-9 back).
-                        // This lane's dims of k-step ks: 16ks + 4tig + {0, 1} and {2, 3}
-                        constexpr uint32_t kTwoM9 = 0x18001800u;  // f16 2^-9, both halves
-                        const float4* pc = reinterpret_cast<const float4*>(ksc) + 8 * ks + 2 * tig;
-                        const float4 p01 = pc[0], p23 = pc[1];  // (scale, zero) of 2 channels each
-                        const uint32_t z01 = hmul2u(pack2<true>(p01.y, p01.w), kTwoM9);
-                        const uint32_t z23 = hmul2u(pack2<true>(p23.y, p23.w), kTwoM9);
-                        qa0 = hmul2u(qa0, pack2<true>(p01.x, p01.z));
-                        qa1 = hmul2u(qa1, pack2<true>(p23.x, p23.z));
-                        b0 = hsub2u(b0, z01);
-                        b1 = hsub2u(b1, z23);
-                        b2 = hsub2u(b2, z01);
-                        b3 = hsub2u(b3, z23);
+                        // (c - zero) 2^-9, exact in f16 while |c - zero| <= 2048 (the score
+                        // takes the 2^-9 back).  This lane's dims of k-step ks: 16ks + 4tig +
+                        // {0, 1} and {2, 3}, converted by lane 4ks + tig
+                        const uint4 h = kp16[4 * ks + tig];
+                        qa0 = hmul2u(qa0, h.x);
+                        qa1 = hmul2u(qa1, h.y);
+                        b0 = hsub2u(b0, h.z);
+                        b1 = hsub2u(b1, h.w);
+                        b2 = hsub2u(b2, h.z);
+                        b3 = hsub2u(b3, h.w);
                     }
                     mma_16816<true>(s[0], qa0, a_hi(ks, 0), qa1, a_hi(ks, 1), b0, b1);
                     mma_16816<true>(s[1], qa0, a_hi(ks, 0), qa1, a_hi(ks, 1), b2, b3);
