@@ -39,15 +39,29 @@ __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_addr(bar)) : "memory");
 }
 
+// One poll of an mbarrier phase.  A thread whose phase is not complete may be
+// suspended until it completes or a time limit passes: the hardware's own limit
+// (SUSPEND_NS = 0), else SUSPEND_NS nanoseconds.
+template <uint32_t SUSPEND_NS = 0>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
+    if constexpr (SUSPEND_NS == 0) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_addr(bar)), "r"(parity), "n"(SUSPEND_NS)
+            : "memory");
+    }
     return ok != 0;
 }
 
@@ -61,11 +75,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // time (or 2^30 polls) and reports false; the caller records KV_DEVERR_TIMEOUT.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+template <uint32_t SUSPEND_NS = 0>
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<SUSPEND_NS>(bar, parity)) return true;
     const uint64_t t0 = globaltimer_ns();
     for (uint32_t it = 0; it < (1u << 30); ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait<SUSPEND_NS>(bar, parity)) return true;
         if ((it & 63u) == 63u && globaltimer_ns() - t0 > kWaitLimitNs) return false;
     }
     return false;

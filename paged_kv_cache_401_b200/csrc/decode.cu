@@ -1254,6 +1254,13 @@ struct MmaMath {
 // Decode kernel: grid ceil(num_ranges / 4) CTAs of 160 threads.
 // ======================================================================================
 constexpr int kConsumerWarps = 4;
+// Poll limits of the ring's waits (0: the hardware's own).  The producer warp spends
+// most of a compute-bound call waiting for released stages; letting its polls sleep
+// up to 20 us (a completed phase still wakes it) leaves the issue slots to the
+// consumer warps.  Consumer polls keep the hardware's limit: a 20 us one measured
+// no better.
+constexpr uint32_t kConsumerSuspendNs = 0;
+constexpr uint32_t kProducerSuspendNs = 20000u;
 constexpr int kThreads = (kConsumerWarps + 1) * 32;
 
 template <class M>
@@ -1464,7 +1471,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const TmaMaps
                 if (j < count && !*abort_flag) {
                     const int s = lane + kConsumerWarps * (j % kPerWarp);
                     const int round = j / kPerWarp;
-                    if (round > 0 && !mbar_wait_bounded(&empty[s], (round - 1) & 1)) {
+                    if (round > 0 && !mbar_wait_bounded<kProducerSuspendNs>(&empty[s], (round - 1) & 1)) {
                         report(p.dev_error, KV_DEVERR_TIMEOUT);
                         *abort_flag = 1;
                     } else {
@@ -1531,12 +1538,12 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const TmaMaps
     for (int j = 0; j < n; ++j) {
         const int s = warp + kConsumerWarps * (j % kPerWarp);
         const bool arrived =
-            __all_sync(0xffffffffu, mbar_wait_bounded(&full[s], (j / kPerWarp) & 1));
-        if (!arrived) {
+            __all_sync(0xffffffffu, mbar_wait_bounded<kConsumerSuspendNs>(&full[s], (j / kPerWarp) & 1));
+        if (!arrived) {  // output invalid (reported); the producer stops at its next tile
             if (lane == 0) report(p.dev_error, KV_DEVERR_TIMEOUT);
             *abort_flag = 1;
+            return;
         }
-        if (__any_sync(0xffffffffu, *abort_flag != 0)) return;  // output invalid (reported)
         if (stage_ok[s]) {
             if constexpr (M::kCanAppend) {
                 if (p.k_new != nullptr && cur.jb + 1 == cur.nt) {
