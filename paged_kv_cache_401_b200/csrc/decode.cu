@@ -492,6 +492,7 @@ struct SimtMath {
     static constexpr int kScaleBytes = kQuantized<KV_T> ? 2 * kBlockTokens * 4 : 0;  // K|V
     static constexpr int kStageBytes = 2 * kTileBytes + kScaleBytes;
     static constexpr int kStages = (kStageBytes >= 16384) ? 4 : 8;           // multiple of 4
+    static constexpr int kParamBytes = 0;  // the row scales travel inside the stage
     static constexpr int kRingAlign = 128;
     static constexpr bool kUsesTma = false;                                  // 1-D bulk copies
     static constexpr int kChunkElems = 16 / kElem;                           // per 16-byte load
@@ -516,14 +517,14 @@ struct SimtMath {
     static_assert(kQPL % 2 == 0 && kDPL % 2 == 0, "pairs for fp32x2 FMA");
 
     // ---- producer side: one stage = K tile, V tile (+ 8-bit row scales), 1-D bulk copies
-    __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
-                                 const TmaMaps&) {
+    __device__ static void issue(uint8_t* st, uint8_t* prm, int64_t tile, uint64_t* bar,
+                                 const DecodeParams& p, const TmaMaps&) {
         const int64_t off = tile * kTileBytes;
         mbar_arrive_expect_tx(bar, kStageBytes);
         bulk_copy_g2s(st, p.k_pool + off, kTileBytes, bar);
         bulk_copy_g2s(st + kTileBytes, p.v_pool + off, kTileBytes, bar);
         if constexpr (kQuantized<KV_T>)
-            bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
+            bulk_copy_g2s(prm, p.scales + tile * 2 * kBlockTokens, kScaleBytes, bar);
     }
 
     // Byte offset of byte `byte` of row `row` in a staged K or V tile (rows are contiguous).
@@ -575,10 +576,11 @@ struct SimtMath {
             for (int i = 0; i < kDPL / 2; ++i) o2[g][i] = make_float2(0.0f, 0.0f);
     }
 
-    __device__ void tile(const uint8_t* kt, int32_t jb, int32_t L, const DecodeParams&) {
+    __device__ void tile(const uint8_t* kt, uint8_t* prm, int32_t jb, int32_t L,
+                         const DecodeParams&) {
         const int32_t nvalid = min(kBlockTokens, L - jb * kBlockTokens);
         const uint8_t* vt = kt + kTileBytes;
-        const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
+        const float* ksc = reinterpret_cast<const float*>(prm);
         const float* vsc = ksc + kBlockTokens;
 
         // scores: partial dot products over this lane's columns, then reduce-scatter
@@ -778,11 +780,16 @@ struct MmaMath {
     // K then V row parameters: fp32 scales (8-bit) or fp32 (scale, zero) pairs (4-bit)
     static constexpr int kScaleBytes =
         kKivi ? (128 + kBlockTokens) * 8 : (kI4 ? 2 * kBlockTokens * 8 : (kF16 ? 2 * kBlockTokens * 4 : 0));
-    static constexpr int kStageBytes = (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
+    // A stage holds the K and V tiles (1024-byte aligned, as the swizzle needs) and,
+    // after them, the tile's parameter line.  KIVI parameter lines sit in a ring of their
+    // own instead (measured 3 % faster; for the other tiles the same move measured no
+    // better): the line's 1152 bytes plus the f16 key parameters (128 x {scale,
+    // zero 2^-9}) that the tile converts once, past the bytes the copy writes.
+    static constexpr int kParamBytes = kKivi ? (kScaleBytes + 128 * 4 + 127) / 128 * 128 : 0;
+    static constexpr int kStageBytes =
+        kKivi ? 2 * kTileBytes : (2 * kTileBytes + kScaleBytes + 1023) / 1024 * 1024;
+    static constexpr int kKiviF16Params = kScaleBytes;
     static constexpr int kStages = kF16 ? 12 : 8;                  // multiple of 4
-    // KIVI: f16 key parameters (128 x {scale, zero 2^-9}) in the stage's unused tail
-    static constexpr int kKiviF16Params = 2 * kTileBytes + kScaleBytes;
-    static_assert(!kKivi || kStageBytes - kKiviF16Params >= 128 * 4, "f16 key parameters fit");
     static_assert(kKiviF16Params % 16 == 0, "16-byte stores");
     static constexpr int kRingAlign = 1024;                       // 128-byte swizzle atom
     static constexpr bool kUsesTma = true;                        // tensor-map tile copies
@@ -790,8 +797,8 @@ struct MmaMath {
     static constexpr int kMinBlocks = WIDE ? 2 : 3;
 
     // ---- producer side: TMA boxes of K and V (+ the scale line of 8-bit codes by bulk copy)
-    __device__ static void issue(uint8_t* st, int64_t tile, uint64_t* bar, const DecodeParams& p,
-                                 const TmaMaps& maps) {
+    __device__ static void issue(uint8_t* st, uint8_t* prm, int64_t tile, uint64_t* bar,
+                                 const DecodeParams& p, const TmaMaps& maps) {
         const int32_t row = static_cast<int32_t>(tile * kBlockTokens);
         mbar_arrive_expect_tx(bar, 2 * kTileTx + kScaleBytes);
 #pragma unroll
@@ -800,7 +807,7 @@ struct MmaMath {
             tma_load_2d(st + kTileBytes + bx * kBoxBytes, &maps.v, bx * kBoxCols, row, bar);
         }
         if constexpr (kF16)
-            bulk_copy_g2s(st + 2 * kTileBytes, p.scales + tile * (kScaleBytes / 4), kScaleBytes, bar);
+            bulk_copy_g2s(prm, p.scales + tile * (kScaleBytes / 4), kScaleBytes, bar);
     }
 
     // Byte offset of byte `byte` of row `row` (as the pool stores it) in a staged
@@ -905,19 +912,22 @@ struct MmaMath {
 
     // A tile whose 16 tokens every query row sees (for one query token: every tile but
     // a pair's last) needs no position masks, and runs an instantiation without them.
-    __device__ void tile(uint8_t* kt, int32_t jb, int32_t L, const DecodeParams& p) {
+    __device__ void tile(const uint8_t* kt, uint8_t* prm, int32_t jb, int32_t L,
+                         const DecodeParams& p) {
         if ((jb + 1) * kBlockTokens <= L - nq + 1)
-            tile_body<true>(kt, jb, L, p);
+            tile_body<true>(kt, prm, jb, L, p);
         else
-            tile_body<false>(kt, jb, L, p);
+            tile_body<false>(kt, prm, jb, L, p);
     }
 
     template <bool FULL>
-    __device__ __forceinline__ void tile_body(uint8_t* kt, int32_t jb, int32_t L,
+    __device__ __forceinline__ void tile_body(const uint8_t* kt, uint8_t* prm, int32_t jb, int32_t L,
                                               const DecodeParams& p) {
         const uint32_t k_s = smem_addr(kt);
         const uint32_t v_s = k_s + kTileBytes;
-        const float* ksc = reinterpret_cast<const float*>(kt + 2 * kTileBytes);
+        // the parameter line (in-stage lines are addressed from the stage itself)
+        if constexpr (kParamBytes == 0) prm = const_cast<uint8_t*>(kt) + 2 * kTileBytes;
+        const float* ksc = reinterpret_cast<const float*>(prm);
         const float* vsc = ksc + kBlockTokens;
         const int32_t pos0 = jb * kBlockTokens;            // position of the tile's token 0
         const int32_t nvalid = min(kBlockTokens, L - pos0);
@@ -926,9 +936,9 @@ struct MmaMath {
         // ---- S = Q.K^T: s[nt] = rows gid (c0, c1) and gid + 8 (c2, c3)
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         // KIVI: the 128 key channels' (scale, zero) as f16 {scale, zero 2^-9}, converted once
-        // per tile into the stage's tail, past the bytes the copies write (so no async-proxy
-        // write can meet these stores); lane l converts channels 4l .. 4l + 3
-        [[maybe_unused]] const uint4* kp16 = reinterpret_cast<const uint4*>(kt + kKiviF16Params);
+        // per tile into the parameter line's tail, past the bytes the copies write (so no
+        // async-proxy write can meet these stores); lane l converts channels 4l .. 4l + 3
+        [[maybe_unused]] const uint4* kp16 = reinterpret_cast<const uint4*>(prm + kKiviF16Params);
         if constexpr (kKivi) {
             constexpr uint32_t kTwoM9 = 0x18001800u;  // f16 2^-9, both halves
             const float4* pc = reinterpret_cast<const float4*>(ksc) + 2 * lane;
@@ -938,7 +948,7 @@ struct MmaMath {
             h.y = pack2<true>(p23.x, p23.z);
             h.z = hmul2u(pack2<true>(p01.y, p01.w), kTwoM9);
             h.w = hmul2u(pack2<true>(p23.y, p23.w), kTwoM9);
-            reinterpret_cast<uint4*>(kt + kKiviF16Params)[lane] = h;
+            reinterpret_cast<uint4*>(prm + kKiviF16Params)[lane] = h;
             __syncwarp();
         }
         auto a_hi = [&](int ks, int h) -> uint32_t {
@@ -1266,14 +1276,19 @@ constexpr int kThreads = (kConsumerWarps + 1) * 32;
 template <class M>
 struct Smem {
     static constexpr int kRingBytes = M::kStages * M::kStageBytes;
+    static constexpr int kParamRingBytes = M::kStages * M::kParamBytes;
     static constexpr int kScratch = kConsumerWarps * M::kWarpScratch;
     static constexpr int kFlags = (2 * M::kStages * 4 + 16 + 15) / 16 * 16;  // ok, issued, abort
     static constexpr int kBars = 2 * M::kStages * 8;
     // dynamic shared memory is only guaranteed 16-byte aligned: pad for the ring's alignment
-    static constexpr int kBytes = M::kRingAlign + kRingBytes + kScratch + kFlags + kBars;
+    static constexpr int kBytes =
+        M::kRingAlign + kRingBytes + kParamRingBytes + kScratch + kFlags + kBars;
+    static_assert(M::kParamBytes % 16 == 0, "bulk copies need 16-B alignment");
+    static_assert(M::kMinBlocks * (kBytes + 1024) <= 228 * 1024, "resident CTAs per SM");
     static_assert(M::kStages % kConsumerWarps == 0, "stage s feeds consumer warp s % 4");
     static_assert(M::kStageBytes % M::kRingAlign == 0, "stages keep the ring's alignment");
-    static_assert((kRingBytes + kScratch + kFlags) % 8 == 0, "mbarriers need 8-B alignment");
+    static_assert((kRingBytes + kParamRingBytes + kScratch + kFlags) % 8 == 0,
+                  "mbarriers need 8-B alignment");
     static_assert(kBytes <= 227 * 1024, "shared memory per block");
 };
 
@@ -1319,7 +1334,8 @@ __device__ __forceinline__ void prefetch_append(const DecodeParams& p, int32_t b
 }
 
 template <class M>
-__device__ __noinline__ void append_row(uint8_t* st, const AppendRow a, int32_t lane) {
+__device__ __noinline__ void append_row(uint8_t* st, uint8_t* prm, const AppendRow a,
+                                       int32_t lane) {
     constexpr int D = M::kHeadDim;
     constexpr int kRowBytes = M::kRowBytes;
     constexpr int kTileBytes = M::kTileBytes;
@@ -1329,7 +1345,7 @@ __device__ __noinline__ void append_row(uint8_t* st, const AppendRow a, int32_t 
     if constexpr (M::kKv == KV_INT4) {
         // 2 bytes of packed codes per lane; (scale, zero) per row, K rows then V rows
         const int32_t src_bytes = a.src_dtype == KV_F32 ? 4 : 2;
-        float2* pz_stage = reinterpret_cast<float2*>(st + 2 * kTileBytes);
+        float2* pz_stage = reinterpret_cast<float2*>(prm);
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
             const uint8_t* src = static_cast<const uint8_t*>(which ? a.v_new : a.k_new);
@@ -1350,7 +1366,7 @@ __device__ __noinline__ void append_row(uint8_t* st, const AppendRow a, int32_t 
     } else if constexpr (kQuantized<M::kKv>) {
         constexpr int kPer = D / 32;
         const int32_t src_bytes = a.src_dtype == KV_F32 ? 4 : 2;
-        float* sc_stage = reinterpret_cast<float*>(st + 2 * kTileBytes);  // K then V row scales
+        float* sc_stage = reinterpret_cast<float*>(prm);  // K then V row scales
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
             const uint8_t* src = static_cast<const uint8_t*>(which ? a.v_new : a.k_new);
@@ -1388,12 +1404,18 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const TmaMaps
     uint8_t* ring = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + M::kRingAlign - 1) &
         ~static_cast<uintptr_t>(M::kRingAlign - 1));
-    uint8_t* scratch = ring + S::kRingBytes;
+    uint8_t* params = ring + S::kRingBytes;  // parameter lines (tile types that have a ring)
+    uint8_t* scratch = params + S::kParamRingBytes;
     int32_t* stage_ok = reinterpret_cast<int32_t*>(scratch + S::kScratch);
     int32_t* issued_round = stage_ok + M::kStages;
     volatile int32_t* abort_flag = issued_round + M::kStages;
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(stage_ok) + S::kFlags);
     uint64_t* empty = full + M::kStages;
+    // stage s's parameter line: in the parameter ring, or after the stage's two tiles
+    auto param_line = [&](int s) -> uint8_t* {
+        if constexpr (M::kParamBytes > 0) return params + s * M::kParamBytes;
+        else return ring + s * M::kStageBytes + 2 * M::kTileBytes;
+    };
 
     const int32_t warp = threadIdx.x >> 5;
     const int32_t lane = threadIdx.x & 31;
@@ -1480,7 +1502,7 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const TmaMaps
                         stage_ok[s] = ok;
                         issued_round[s] = round;
                         if (ok) {
-                            M::issue(ring + s * M::kStageBytes,
+                            M::issue(ring + s * M::kStageBytes, param_line(s),
                                      static_cast<int64_t>(id) * p.num_kv_heads + q_head[i], &full[s],
                                      p, maps);
                         } else {
@@ -1551,10 +1573,10 @@ __device__ __forceinline__ void decode_body(const DecodeParams& p, const TmaMaps
                                       p.block_table + static_cast<int64_t>(cur.b) * p.max_blocks,
                                       static_cast<int64_t>(cur.b) * p.num_kv_heads + cur.kvh,
                                       p.num_kv_heads, cur.kvh, cur.L, p.append_src_dtype};
-                    append_row<M>(ring + s * M::kStageBytes, a, lane);
+                    append_row<M>(ring + s * M::kStageBytes, param_line(s), a, lane);
                 }
             }
-            math.tile(ring + s * M::kStageBytes, cur.jb, cur.L, p);
+            math.tile(ring + s * M::kStageBytes, param_line(s), cur.jb, cur.L, p);
         }
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
