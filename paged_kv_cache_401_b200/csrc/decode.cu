@@ -1683,6 +1683,19 @@ __global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_merge_kernel(co
     const int32_t kvh = h / G;
     const int32_t R = G * nq;          // query rows of a (sequence, kv head) pair
     const int32_t g = qi * G + h % G;  // this warp's row within the pair
+    // KIVI: bring all 16 residual K and V rows of the pair into L1 now, in the same
+    // round trip as the lengths, so the residual tokens at the end wait on no memory
+    // (rows past L mod 16 are fetched and not used); lane l fetches 128-byte line
+    // l % 2 of row l / 2 (D = 128: two lines per row)
+    if constexpr (KIVI) {
+        const int64_t row = (static_cast<int64_t>(b) * p.num_kv_heads + kvh) * kBlockTokens +
+                            lane / 2;
+        const int64_t e = row * D + (lane % 2) * 64;
+        if (lane / 2 < kBlockTokens && (lane % 2) * 64 < D) {
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.res_k + e));
+            asm volatile("prefetch.global.L1 [%0];" ::"l"(p.res_v + e));
+        }
+    }
     // three independent loads in one round trip
     const int32_t L = p.context_lens[b];
     const int64_t T = p.ws_seq_start[p.batch];
@@ -1802,9 +1815,8 @@ __global__ void __launch_bounds__(kMergeWarps * 32) paged_decode_merge_kernel(co
     }
     if constexpr (KIVI) {
         // KIVI: the newest L mod 16 tokens, kept in bf16 at res_k / res_v
-        // [batch][Hkv][16][D], join the softmax (same base-2 scores).  All their
-        // key rows are read and scored first (independent loads and reductions),
-        // then one rescale, then all value rows.
+        // [batch][Hkv][16][D] (fetched into L1 at the start), join the softmax (same
+        // base-2 scores): all their scores first, then one rescale, then the value rows.
         const int32_t nres = L % kBlockTokens;
         if (nres > 0) {
             float qf[kDPL];
