@@ -70,6 +70,25 @@ def test_reference_arm_only_on_rank_zero(monkeypatch, capsys):
     assert capsys.readouterr().out == ""
 
 
+def test_reference_arm_prints_the_workload_config_of_the_gpu_arm(monkeypatch, capsys):
+    # the driver compares the two arms' configs: the reference line must carry the
+    # same workload description (and data note) the GPU arm builds with describe()
+    sys.path.insert(0, ROOT)
+    import json
+    import bench
+    from workloads import make_inputs
+    monkeypatch.setenv("RANK", "0")
+    inp = make_inputs("tiny")
+    args = type("A", (), {"gpus": 1, "steps": 1, "warmup": 3, "reference_seqs": 2,
+                          "partition": 0})()
+    bench.run_reference(args, inp)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.describe(inp, 0, 1)
+    assert line["data"] == bench.DATA
+    assert "split" not in line["config"] and "num_ranges" not in line["config"]
+
+
 @pytest.mark.parametrize("workload", ["tiny", "llama"])
 def test_kv_bytes_per_step(workload):
     sys.path.insert(0, ROOT)
