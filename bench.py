@@ -21,7 +21,9 @@ roofline = the decode call (decode + merge kernels) against the measured HBM
            calls back to back timed the same way after the steps;
 timing   = --regions regions of exactly K steps, each bracketed by a barrier
            and a synchronize; value and e2e report the median region and the
-           line lists every region (the default 20-step region lasts ~2 ms);
+           line lists every region (a 20-step region lasts ~2 ms);
+config   = the workload only, the same for both arms; the split this arm chose
+           (ranges, how the new tokens are appended) is under ``split``;
 cpu_baseline = the double-precision CPU oracle on a bounded sample (rank 0).
 ``--impl reference`` times that oracle alone as the reference arm.
 With N > 1 (torchrun), every rank runs an independent replica on its own GPU
