@@ -81,6 +81,24 @@ def test_kivi_decode_append_parity(G):
         check_close(out, ref, "kivi4")
 
 
+@pytest.mark.parametrize("offset", [8.0, 120.0])
+def test_kivi_key_channels_with_large_offsets(offset):
+    # key channels that sit far from zero relative to their spread in a block (up to
+    # ~130 times the range): zero points of over a thousand codes, q times large
+    # per-channel scales.  The codes minus zero stay exact in f16 (|c - zero| <= 2048);
+    # what grows is the f16 rounding of q * scale, which stays well inside the budget
+    inp = make_inputs(_spec(4, [300, 1024, 1025, 2047], idx=150))
+    g = torch.Generator().manual_seed(7)
+    off = (torch.rand(2, 128, generator=g) * 2 - 1) * offset  # per (kv head, channel)
+    inp.k[:] = (inp.k.float() * 0.25 + off[None]).to(inp.k.dtype)
+    _, ref = oracle_out_kivi(inp)
+    st = stage_kivi(inp)
+    out = st.cache.kivi_decode(st.q, st.block_table, st.context_lens, st.max_context_len,
+                               inp.spec.scale, st.k_new, st.v_new)
+    assert st.cache.errors() == 0
+    check_close(out, ref, "kivi4")
+
+
 @pytest.mark.parametrize("rising", [True, False])
 def test_kivi_running_max_growth_patterns(rising):
     # keys scaled by a ramp over positions: the running max grows in nearly every
