@@ -46,6 +46,22 @@ def test_decode_parity_shapes(kv, q, D, G):
         assert st.cache.errors() == 0
 
 
+@pytest.mark.parametrize("kv", ["bf16", "fp8", "int8", "int4"])
+def test_decode_key_channels_with_large_offsets(kv):
+    # keys far from zero relative to their spread (per-channel offsets up to 120):
+    # large scores, large row scales and zero points.  The codes are the oracle's own,
+    # so the comparison measures the tile arithmetic
+    inp = make_inputs(_spec(kv, "bf16", 128, 4, [300, 1024, 1025, 2047], idx=152))
+    g = torch.Generator().manual_seed(8)
+    off = (torch.rand(2, 128, generator=g) * 2 - 1) * 120.0  # per (kv head, channel)
+    inp.k[:] = (inp.k.float() * 0.25 + off[None]).to(inp.k.dtype)
+    st = stage(inp)
+    _, ref = oracle_out(inp)
+    out = step(st)
+    assert st.cache.errors() == 0
+    check_close(out, ref, kv)
+
+
 @pytest.mark.parametrize("part", [16, 48, 256, 1008, 1024, 1040, 4096, 8192])
 def test_decode_partition_edges(part):
     # context lengths at partition size -1/0/+1 and at block boundaries
